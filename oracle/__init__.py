@@ -1,0 +1,163 @@
+"""CPU oracle for group-wise affine weight quantization (TEST INFRASTRUCTURE).
+
+Only the test suite, ``__graft_entry__.smoke()`` and the benchmark's
+``cpu_baseline`` / reference leg may import this package.  The product path
+(the CUDA library and its Python binding) never does, and this package never
+imports the product: the two share nothing but the seeded input generator in
+``synthetic``.
+
+The arithmetic lives in ``qz_oracle.c`` (plain scalar C, fp32 IEEE for the
+quantizer, fp64 for the matmul); this module only marshals numpy arrays.
+Every function cites the page passage it follows in the C source.
+"""
+import ctypes
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+_p = ctypes.c_void_p
+
+
+def load(path: str):
+    """Open an oracle shared library at ``path`` and declare its signatures."""
+    L = ctypes.CDLL(path)
+    L.qzo_bf16_to_f32.argtypes = [ctypes.c_uint16]
+    L.qzo_bf16_to_f32.restype = ctypes.c_float
+    L.qzo_f32_to_bf16_rne.argtypes = [ctypes.c_float]
+    L.qzo_f32_to_bf16_rne.restype = ctypes.c_uint16
+    L.qzo_f32_to_bf16_up.argtypes = [ctypes.c_float]
+    L.qzo_f32_to_bf16_up.restype = ctypes.c_uint16
+    L.qzo_code_range.argtypes = [_int, _int, ctypes.POINTER(_int), ctypes.POINTER(_int)]
+    L.qzo_code_range.restype = _int
+    L.qzo_num_groups.argtypes = [_i64, _i64, _i64]
+    L.qzo_num_groups.restype = _i64
+    L.qzo_quantize_pack.argtypes = [_p, _i64, _i64, _int, _int, _i64, _p, _p, _p]
+    L.qzo_quantize_pack.restype = _int
+    L.qzo_dequantize.argtypes = [_p, _p, _p, _i64, _i64, _int, _int, _i64, _p]
+    L.qzo_dequantize.restype = _int
+    L.qzo_matmul_f64.argtypes = [_p, _p, _i64, _i64, _i64, _p, _p]
+    L.qzo_matmul_f64.restype = _int
+    L.qzo_set_threads.argtypes = [_int]
+    L.qzo_set_threads.restype = None
+    L.qzo_max_threads.argtypes = []
+    L.qzo_max_threads.restype = _int
+    return L
+
+
+def lib():
+    """The oracle library, built from ``qz_oracle.c`` on first use."""
+    global _lib
+    if _lib is None:
+        _lib = load(_build.build())
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def set_threads(n: int) -> None:
+    lib().qzo_set_threads(int(n))
+
+
+def max_threads() -> int:
+    return int(lib().qzo_max_threads())
+
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    """Widen bf16 bit patterns to fp32 values (exact: bf16 is the top half)."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def f32_to_bf16_rne(x: float) -> int:
+    return int(lib().qzo_f32_to_bf16_rne(float(x)))
+
+
+def f32_to_bf16_up(x: float) -> int:
+    return int(lib().qzo_f32_to_bf16_up(float(x)))
+
+
+def code_range(bits: int, symmetric: bool):
+    lo, hi = _int(), _int()
+    if lib().qzo_code_range(bits, int(symmetric), ctypes.byref(lo), ctypes.byref(hi)):
+        raise ValueError("unsupported format")
+    return lo.value, hi.value
+
+
+def num_groups(N: int, K: int, group_size: int) -> int:
+    return int(lib().qzo_num_groups(N, K, group_size))
+
+
+def packed_shapes(N: int, K: int, bits: int, symmetric: bool, group_size: int):
+    """Array shapes of (codes, scales, zeros); zeros is None when symmetric."""
+    codes = (N, K // 2) if bits == 4 else (N, K)
+    if group_size == 0:
+        scales = (1,)
+    else:
+        scales = (N, K // group_size)
+    return codes, scales, (None if symmetric else scales)
+
+
+def quantize_pack(w, bits: int = 4, symmetric: bool = False, group_size: int = 128):
+    """Quantize an N x K matrix.
+
+    ``w`` is either bf16 bit patterns (uint16) or fp32 values.  Returns
+    ``(codes uint8, scales bf16-bits uint16, zeros uint8 or None)``.
+    """
+    w = np.asarray(w)
+    if w.dtype == np.uint16:
+        wf = bf16_bits_to_f32(w)
+    else:
+        wf = np.ascontiguousarray(w, dtype=np.float32)
+    if wf.ndim != 2:
+        raise ValueError("w must be 2-D")
+    N, K = wf.shape
+    cs, ss, zs = packed_shapes(N, K, bits, symmetric, group_size)
+    codes = np.zeros(cs, dtype=np.uint8)
+    scales = np.zeros(ss, dtype=np.uint16)
+    zeros = None if zs is None else np.zeros(zs, dtype=np.uint8)
+    rc = lib().qzo_quantize_pack(_ptr(wf), N, K, bits, int(symmetric), group_size,
+                                 _ptr(codes), _ptr(scales), _ptr(zeros))
+    if rc != 0:
+        raise ValueError("qzo_quantize_pack rejected the arguments")
+    return codes, scales, zeros
+
+
+def dequantize(codes, scales, zeros, N: int, K: int, bits: int = 4,
+               symmetric: bool = False, group_size: int = 128) -> np.ndarray:
+    """Return the bf16 bit patterns of w_hat = bf16(S * (q - Z)), N x K."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    if zeros is not None:
+        zeros = np.ascontiguousarray(zeros, dtype=np.uint8)
+    out = np.zeros((N, K), dtype=np.uint16)
+    rc = lib().qzo_dequantize(_ptr(codes), _ptr(scales), _ptr(zeros), N, K, bits,
+                              int(symmetric), group_size, _ptr(out))
+    if rc != 0:
+        raise ValueError("qzo_dequantize rejected the arguments")
+    return out
+
+
+def matmul_f64(a_bits, w_hat_bits):
+    """fp64 y = a @ w_hat^T and sum_k |a*w_hat| over bf16 bit-pattern inputs."""
+    a = np.ascontiguousarray(a_bits, dtype=np.uint16)
+    w = np.ascontiguousarray(w_hat_bits, dtype=np.uint16)
+    M, K = a.shape
+    N, K2 = w.shape
+    if K != K2:
+        raise ValueError("inner dimensions differ")
+    y = np.zeros((M, N), dtype=np.float64)
+    ya = np.zeros((M, N), dtype=np.float64)
+    lib().qzo_matmul_f64(_ptr(a), _ptr(w), M, N, K, _ptr(y), _ptr(ya))
+    return y, ya
+
+
+def tolerance(y_ref: np.ndarray, abs_ref: np.ndarray) -> np.ndarray:
+    """Per-element bound |y - y_ref| <= 8e-3 |y_ref| + 1e-4 sum_k |a_k w_k|."""
+    return 8e-3 * np.abs(y_ref) + 1e-4 * abs_ref

@@ -1,0 +1,325 @@
+/*
+ * qz_oracle.c -- plain, slow, scalar CPU oracle for group-wise affine weight
+ * quantization and the weight-only dequantize-matmul.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call, link or
+ * load this file: only the test suite, the smoke check and the benchmark's
+ * CPU-baseline leg use it.  It shares no code, header, table or constant with
+ * the CUDA library; the two meet only through the seeded input generator.
+ *
+ * Sources (the HF Transformers "Quantization concepts" guide, section
+ * "Mapping values to fewer bits"; the taqaniya.com "What is quantization"
+ * page, IBM absmax example; the GPTQ explainer at azimuth.plus):
+ *   scale        S = (val_max - val_min) / (q_max - q_min)
+ *   zero-point   Z = q_min - round(val_min / S)
+ *   quantize     q = round(x / S + Z)
+ *   dequantize   x ~ S * (q - Z)
+ *   symmetric    range [-a, a], Z fixed at 0, only S stored (int8: +-127)
+ *   granularity  per-tensor / per-channel (one per output row) / per-group of
+ *                consecutive values along a row (section "Choose granularity")
+ *   int4 packing two codes per byte, first in the low nibble (section
+ *                "int8 and int4", packing figure)
+ *
+ * Readings where the pages are silent (each is listed with its reason in the
+ * design notes of the repository):
+ *   - round() is round-half-to-even (rintf in the default rounding mode);
+ *   - q is clamped to [q_min, q_max];
+ *   - the asymmetric range is extended to contain 0.0, since Z is defined as
+ *     the integer that represents 0.0;
+ *   - S is computed in IEEE fp32 and stored as bf16 rounded toward +inf, and
+ *     quantization divides by that stored value (so every x/S+Z stays inside
+ *     [q_min - 1/2, q_max + 1/2]);
+ *   - S == 0 (an all-zero group) is replaced by 1.0;
+ *   - int4 asymmetric codes are unsigned [0, 15]; int4 symmetric codes are
+ *     [-7, 7]; int8 asymmetric codes are [-128, 127]; int8 symmetric [-127, 127];
+ *   - the dequantized weight is bf16, rounded to nearest-even from the exact
+ *     fp32 product S*(q - Z);
+ *   - the matmul reference is an fp64 dot product over those bf16 weights.
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fopenmp -fPIC -shared
+ * (no FMA contraction, no fast-math, no flush-to-zero).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------ */
+/* bf16 <-> fp32 bit conversions                                        */
+/* ------------------------------------------------------------------ */
+
+static float f32_of_bits(uint32_t b) { float f; memcpy(&f, &b, sizeof f); return f; }
+static uint32_t bits_of_f32(float f) { uint32_t b; memcpy(&b, &f, sizeof b); return b; }
+
+/* A bf16 value is the upper 16 bits of an fp32: widening is exact. */
+float qzo_bf16_to_f32(uint16_t h) { return f32_of_bits((uint32_t)h << 16); }
+
+/* fp32 -> bf16, round to nearest, ties to even (finite inputs; NaN kept quiet). */
+uint16_t qzo_f32_to_bf16_rne(float x)
+{
+    uint32_t b = bits_of_f32(x);
+    if ((b & 0x7F800000u) == 0x7F800000u && (b & 0x007FFFFFu) != 0)
+        return (uint16_t)((b >> 16) | 0x0040u);
+    uint32_t kept = b & 0xFFFF0000u;      /* truncated magnitude (sign-magnitude) */
+    uint32_t dropped = b & 0x0000FFFFu;   /* the 16 bits that do not fit */
+    int kept_is_odd = (kept >> 16) & 1u;
+    if (dropped > 0x8000u || (dropped == 0x8000u && kept_is_odd))
+        kept += 0x00010000u;              /* one bf16 ulp away from zero */
+    return (uint16_t)(kept >> 16);
+}
+
+/* fp32 -> bf16 rounded toward +infinity, for the non-negative scale S. */
+uint16_t qzo_f32_to_bf16_up(float s)
+{
+    uint32_t b = bits_of_f32(s);
+    uint32_t kept = b & 0xFFFF0000u;
+    if (b & 0x0000FFFFu)
+        kept += 0x00010000u;              /* next bf16 above (s > 0) */
+    return (uint16_t)(kept >> 16);
+}
+
+/* ------------------------------------------------------------------ */
+/* Code ranges (quantization concepts guide: int8 is [-128, 127], int4   */
+/* holds 16 integers; IBM example: symmetric int8 range is -127..127).   */
+/* ------------------------------------------------------------------ */
+
+int qzo_code_range(int bits, int symmetric, int *qmin, int *qmax)
+{
+    if (bits != 4 && bits != 8) return -1;
+    if (symmetric) {
+        *qmax = (1 << (bits - 1)) - 1;   /* 7 or 127 */
+        *qmin = -*qmax;
+    } else if (bits == 4) {
+        *qmin = 0;                       /* unsigned nibble */
+        *qmax = 15;
+    } else {
+        *qmin = -128;
+        *qmax = 127;
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* One group: scale, zero-point, codes.                                  */
+/* x[0..n) are consecutive values of one group (fp32, exact bf16 values). */
+/* ------------------------------------------------------------------ */
+
+static void quantize_group(const float *x, int64_t n, int bits, int symmetric,
+                           uint16_t *scale_bf16, int32_t *zero, int32_t *q)
+{
+    int qmin, qmax;
+    qzo_code_range(bits, symmetric, &qmin, &qmax);
+
+    float S;
+    float vmin = 0.0f, vmax = 0.0f;       /* the range always contains 0.0 */
+    if (symmetric) {
+        float a = 0.0f;                   /* a = max |x| */
+        for (int64_t i = 0; i < n; ++i) {
+            float m = fabsf(x[i]);
+            if (m > a) a = m;
+        }
+        S = a / (float)qmax;              /* range [-a, a] onto [-qmax, qmax] */
+    } else {
+        for (int64_t i = 0; i < n; ++i) {
+            if (x[i] < vmin) vmin = x[i];
+            if (x[i] > vmax) vmax = x[i];
+        }
+        S = (vmax - vmin) / (float)(qmax - qmin);
+    }
+    if (S == 0.0f) S = 1.0f;              /* all-zero group */
+
+    uint16_t Sb = qzo_f32_to_bf16_up(S);  /* stored scale */
+    float Sf = qzo_bf16_to_f32(Sb);       /* the value every later step uses */
+
+    int32_t Z = 0;
+    if (!symmetric)
+        Z = qmin - (int32_t)rintf(vmin / Sf);
+
+    for (int64_t i = 0; i < n; ++i) {
+        float u = x[i] / Sf + (float)Z;   /* divide, then shift by Z, in fp32 */
+        float r = rintf(u);               /* round half to even */
+        int32_t c = (int32_t)r;
+        if (c < qmin) c = qmin;
+        if (c > qmax) c = qmax;
+        q[i] = c;
+    }
+    *scale_bf16 = Sb;
+    *zero = Z;
+}
+
+/* ------------------------------------------------------------------ */
+/* Tensor layout                                                         */
+/*   w      : N x K row-major values (fp32 carrying bf16 values)         */
+/*   groups : group_size g > 0 with K % g == 0 -> groups of g consecutive */
+/*            values along each row, scales[n*(K/g) + k/g];              */
+/*            g == K is per-channel; g == 0 is per-tensor (one group).   */
+/*   codes  : bits 4 -> N x K/2 bytes, value k in the low nibble when k   */
+/*            is even, in the high nibble when k is odd;                  */
+/*            bits 8 -> N x K bytes (two's complement).                   */
+/*   zeros  : one byte per group (asymmetric only): unsigned for int4,    */
+/*            two's complement for int8.                                  */
+/* ------------------------------------------------------------------ */
+
+int64_t qzo_num_groups(int64_t N, int64_t K, int64_t g)
+{
+    if (g == 0) return 1;
+    return N * (K / g);
+}
+
+static int check_shape(int64_t N, int64_t K, int bits, int64_t g)
+{
+    if (N < 1 || K < 1) return -1;
+    if (g < 0) return -1;
+    if (g > 0 && (K % g) != 0) return -1;
+    if (bits == 4 && (K % 2) != 0) return -1;
+    return 0;
+}
+
+static void store_code(uint8_t *codes, int64_t N, int64_t K, int bits,
+                       int64_t n, int64_t k, int32_t c)
+{
+    (void)N;
+    if (bits == 8) {
+        codes[n * K + k] = (uint8_t)(int8_t)c;
+    } else {
+        uint8_t nib = (uint8_t)(c & 0xF);
+        uint8_t *byte = &codes[n * (K / 2) + k / 2];
+        if ((k & 1) == 0) *byte = (uint8_t)((*byte & 0xF0) | nib);
+        else              *byte = (uint8_t)((*byte & 0x0F) | (nib << 4));
+    }
+}
+
+static int32_t load_code(const uint8_t *codes, int64_t K, int bits, int symmetric,
+                         int64_t n, int64_t k)
+{
+    if (bits == 8)
+        return (int32_t)(int8_t)codes[n * K + k];
+    uint8_t byte = codes[n * (K / 2) + k / 2];
+    int32_t nib = (k & 1) ? (byte >> 4) : (byte & 0xF);
+    if (symmetric && nib >= 8) nib -= 16;   /* two's complement nibble */
+    return nib;
+}
+
+/* Quantize and pack.  Returns 0 on success, -1 on a bad argument. */
+int qzo_quantize_pack(const float *w, int64_t N, int64_t K, int bits, int symmetric,
+                      int64_t g, uint8_t *codes, uint16_t *scales, uint8_t *zeros)
+{
+    int qmin, qmax;
+    if (qzo_code_range(bits, symmetric, &qmin, &qmax) || check_shape(N, K, bits, g))
+        return -1;
+
+    if (g == 0) {
+        /* per-tensor: one group spanning the whole matrix */
+        int64_t total = N * K;
+        int32_t *q = (int32_t *)malloc((size_t)total * sizeof(int32_t));
+        if (!q) return -1;
+        uint16_t Sb; int32_t Z;
+        quantize_group(w, total, bits, symmetric, &Sb, &Z, q);
+        for (int64_t n = 0; n < N; ++n)
+            for (int64_t k = 0; k < K; ++k)
+                store_code(codes, N, K, bits, n, k, q[n * K + k]);
+        scales[0] = Sb;
+        if (!symmetric) zeros[0] = (uint8_t)(int8_t)Z;
+        free(q);
+        return 0;
+    }
+
+    int64_t gpr = K / g;   /* groups per row */
+    int failed = 0;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
+    for (int64_t n = 0; n < N; ++n) {
+        int32_t *q = (int32_t *)malloc((size_t)g * sizeof(int32_t));
+        if (!q) { failed = 1; continue; }
+        for (int64_t j = 0; j < gpr; ++j) {
+            uint16_t Sb; int32_t Z;
+            quantize_group(&w[n * K + j * g], g, bits, symmetric, &Sb, &Z, q);
+            for (int64_t i = 0; i < g; ++i)
+                store_code(codes, N, K, bits, n, j * g + i, q[i]);
+            scales[n * gpr + j] = Sb;
+            if (!symmetric) zeros[n * gpr + j] = (uint8_t)(int8_t)Z;
+        }
+        free(q);
+    }
+    return failed ? -1 : 0;
+}
+
+/* Dequantize: w_hat = bf16_rne( S * (q - Z) ).  The fp32 product of an
+ * 8-bit-significand scale and an integer of at most 8 bits is exact, so the
+ * only rounding is the final one to bf16. */
+int qzo_dequantize(const uint8_t *codes, const uint16_t *scales, const uint8_t *zeros,
+                   int64_t N, int64_t K, int bits, int symmetric, int64_t g,
+                   uint16_t *w_hat)
+{
+    int qmin, qmax;
+    if (qzo_code_range(bits, symmetric, &qmin, &qmax) || check_shape(N, K, bits, g))
+        return -1;
+    int64_t gpr = (g == 0) ? 0 : K / g;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            int64_t gi = (g == 0) ? 0 : n * gpr + k / g;
+            float Sf = qzo_bf16_to_f32(scales[gi]);
+            int32_t Z = 0;
+            if (!symmetric) {
+                Z = (bits == 4) ? (int32_t)zeros[gi] : (int32_t)(int8_t)zeros[gi];
+            }
+            int32_t q = load_code(codes, K, bits, symmetric, n, k);
+            float prod = Sf * (float)(q - Z);
+            w_hat[n * K + k] = qzo_f32_to_bf16_rne(prod);
+        }
+    }
+    return 0;
+}
+
+/* Reference matmul in fp64 over bf16 operands:
+ *   y[m][n]     = sum_k a[m][k] * w_hat[n][k]
+ *   abs_y[m][n] = sum_k |a[m][k] * w_hat[n][k]|   (for the tolerance bound)
+ * a is M x K, w_hat is N x K (both bf16 bits, row-major). */
+int qzo_matmul_f64(const uint16_t *a, const uint16_t *w_hat, int64_t M, int64_t N,
+                   int64_t K, double *y, double *abs_y)
+{
+    if (M < 0 || N < 0 || K < 0) return -1;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t m = 0; m < M; ++m) {
+            double s = 0.0, sa = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double p = (double)qzo_bf16_to_f32(a[m * K + k]) *
+                           (double)qzo_bf16_to_f32(w_hat[n * K + k]);
+                s += p;
+                sa += fabs(p);
+            }
+            y[m * N + n] = s;
+            if (abs_y) abs_y[m * N + n] = sa;
+        }
+    }
+    return 0;
+}
+
+/* Thread control for the timed CPU baseline. */
+void qzo_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+int qzo_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,202 @@
+/*
+ * qz.h -- C ABI of the B200 (sm_100a) weight-only quantization library libqz.so.
+ *
+ * The library quantizes bf16 weight matrices with group-wise affine
+ * quantization, packs the codes, and runs the matmuls that consume the packed
+ * weights directly (dequantizing on the fly).  Every compute step runs in the
+ * library's own CUDA kernels.
+ *
+ * Definitions (HF Transformers "Quantization concepts" guide, section
+ * "Mapping values to fewer bits", and taqaniya.com "What is quantization",
+ * IBM absmax example):
+ *   S = (val_max - val_min) / (q_max - q_min)      scale (fp32, IEEE)
+ *   Z = q_min - round(val_min / S)                  zero-point
+ *   q = clamp(round(x / S + Z), q_min, q_max)       code (round half to even)
+ *   x_hat = S * (q - Z)                             dequantized weight
+ * with these fixed readings: the range [val_min, val_max] is widened to
+ * contain 0.0; S == 0 becomes 1.0; S is stored as bf16 rounded toward +inf and
+ * the stored value is the one quantization divides by; x_hat is the exact
+ * fp32 product rounded to nearest-even bf16.
+ *
+ * Formats (argument triple bits / symmetric / group_size):
+ *   bits 4, symmetric 0   codes 0..15 (unsigned nibble), zero 0..15 (uint8)
+ *   bits 4, symmetric 1   codes -7..7 (two's-complement nibble), no zeros
+ *   bits 8, symmetric 0   codes -128..127, zero -128..127 (int8 in a byte)
+ *   bits 8, symmetric 1   codes -127..127 (absmax, range [-a, a]), no zeros
+ * Granularity (section "Choose granularity"): group_size g > 0 with K % g == 0
+ * quantizes runs of g consecutive values along each row, one scale (and zero)
+ * per run, stored at [n * (K / g) + k / g]; g == K is per-channel (one per
+ * output row); g == 0 is per-tensor (a single scale/zero).
+ *
+ * Layouts (all row-major, all device memory):
+ *   w        N x K bf16 (N = output features, K = input features)
+ *   codes    bits 4: N x K/2 bytes, value k in the low nibble of byte k/2 when
+ *            k is even and in the high nibble when k is odd (section "int8
+ *            and int4", packing figure); bits 8: N x K bytes
+ *   scales   bf16, N x K/g (g > 0) or 1 (g == 0)
+ *   zeros    uint8/int8 bytes, same shape as scales (asymmetric only)
+ *   a        M x K bf16 activations; y = a * w_hat^T, M x N bf16
+ *
+ * Conventions for every entry point:
+ *   - Pointers are DEVICE pointers and must be 16-byte aligned (scales and
+ *     zeros: 2- and 1-byte aligned).  The caller owns and allocates every
+ *     buffer, including workspaces; the library never allocates, frees or
+ *     synchronizes.  `stream` is a cudaStream_t (NULL = legacy default stream)
+ *     and all work is asynchronous on it.
+ *   - Argument errors are returned synchronously before any launch and leave
+ *     every buffer untouched.  QZ_ERR_CUDA reports a failed launch.
+ *   - Inputs must be finite; NaN/Inf inputs (or a weight range whose width
+ *     overflows fp32) give unspecified codes.
+ *   - Calls are thread-safe.  Two calls that run concurrently need distinct
+ *     workspaces.
+ */
+#ifndef QZ_H_
+#define QZ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QZ_API __attribute__((visibility("default")))
+#else
+#define QZ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QZ_OK = 0,
+    QZ_ERR_INVALID_ARG = 1,     /* null pointer, bad size or shape */
+    QZ_ERR_ALIGNMENT = 2,       /* a pointer is not aligned as required */
+    QZ_ERR_UNSUPPORTED = 3,     /* a format or shape the kernels do not cover */
+    QZ_ERR_WORKSPACE = 4,       /* workspace pointer missing or too small */
+    QZ_ERR_CUDA = 5,            /* a CUDA call or launch failed */
+    QZ_ERR_DEVICE_TIMEOUT = 6   /* a bounded device-side wait ran out */
+} qz_status;
+
+/* Operation ids for qz_workspace_bytes. */
+enum {
+    QZ_OP_QUANTIZE_PACK = 0,
+    QZ_OP_DEQUANTIZE = 1,
+    QZ_OP_W4A16_GEMV = 2,
+    QZ_OP_W4A16_GEMM = 3,
+    QZ_OP_W8A16_GEMV = 4
+};
+
+/* Static description of a status code (never NULL). */
+QZ_API const char *qz_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+QZ_API int qz_version(void);
+
+/*
+ * Sizes in bytes of the three output buffers of qz_quantize_pack for an
+ * N x K matrix in the given format (section "Choose granularity": one scale,
+ * plus one zero when asymmetric, per group).  zeros_bytes is 0 when symmetric.
+ * Host-only; never touches the GPU.
+ */
+QZ_API qz_status qz_packed_bytes(int64_t N, int64_t K, int32_t bits, int32_t symmetric,
+                          int64_t group_size, size_t *codes_bytes,
+                          size_t *scales_bytes, size_t *zeros_bytes);
+
+/*
+ * Device workspace needed by `op` for the given sizes (0 when none).  The
+ * workspace of QZ_OP_QUANTIZE_PACK (per-tensor only) and of the GEMV/GEMM
+ * split-K paths must be zero-filled once before its first use; every call
+ * leaves it zero-filled again when it completes.  Host-only.
+ */
+QZ_API qz_status qz_workspace_bytes(int32_t op, int64_t M, int64_t N, int64_t K,
+                             int64_t group_size, size_t *bytes);
+
+/*
+ * quantize_pack: w (N x K bf16) -> codes, scales (bf16), zeros.
+ * Quantization concepts guide, "Mapping values to fewer bits" (S, Z, q) and
+ * "int8 and int4" (packing).  Requirements: N >= 1; K >= 1, K % 8 == 0;
+ * group_size 0, or a divisor of K that is a multiple of 8 (the fast
+ * warp-per-group kernel covers 32, 64, 128 and 256; other sizes, including
+ * per-channel group_size == K, run one thread block per group).  `zeros`
+ * must be NULL when symmetric and non-NULL otherwise.  Per-tensor
+ * (group_size 0) needs a zero-filled workspace of qz_workspace_bytes bytes;
+ * other formats accept workspace NULL.
+ */
+QZ_API qz_status qz_quantize_pack(const void *w, int64_t N, int64_t K, int32_t bits,
+                           int32_t symmetric, int64_t group_size, void *codes,
+                           void *scales, void *zeros, void *workspace,
+                           size_t workspace_bytes, void *stream);
+
+/*
+ * dequantize: codes/scales/zeros -> w_hat (N x K bf16),
+ * w_hat = bf16_rne(S * (q - Z)) (guide: "Dequantization reverses the
+ * mapping"; the bf16 rounding is this library's fixed reading).  Same format
+ * requirements as qz_quantize_pack; no workspace.
+ */
+QZ_API qz_status qz_dequantize(const void *codes, const void *scales, const void *zeros,
+                        int64_t N, int64_t K, int32_t bits, int32_t symmetric,
+                        int64_t group_size, void *w_hat, void *stream);
+
+/*
+ * W4A16 decode GEMV: y (M x N bf16) = a (M x K bf16) * w_hat^T where w_hat is
+ * the int4 asymmetric group-wise weight (bits 4, symmetric 0) given by codes,
+ * scales, zeros.  Quantization concepts guide, "Quantize weights or
+ * activations" (weight-only: weights are dequantized to the compute dtype
+ * before each matmul; decoding one token at a time is bound by reading the
+ * weights) and the GPTQ explainer's fused dequantize-in-matmul kernels.
+ * Each w_hat is formed exactly as qz_dequantize forms it, products are
+ * accumulated in fp32, y is rounded to bf16.  Requirements: 1 <= M <= 16;
+ * N >= 1; K % 128 == 0; group_size a multiple of 32 dividing K.  Workspace:
+ * qz_workspace_bytes(QZ_OP_W4A16_GEMV, M, N, K, group_size) bytes,
+ * zero-filled before first use (0 bytes means workspace may be NULL).
+ */
+QZ_API qz_status qz_w4a16_gemv(const void *a, const void *codes, const void *scales,
+                        const void *zeros, int64_t M, int64_t N, int64_t K,
+                        int64_t group_size, void *y, void *workspace,
+                        size_t workspace_bytes, void *stream);
+
+/*
+ * W4A16 prefill GEMM: the same product as qz_w4a16_gemv for any M >= 1,
+ * dequantizing weight tiles into shared memory for the tcgen05 tensor cores
+ * (guide, "Quantize weights or activations": prefill and large batches are
+ * compute-bound).  Requirements: M >= 1; N >= 1; K % 128 == 0; group_size a
+ * multiple of 64 dividing K.  Workspace as reported by qz_workspace_bytes
+ * (currently 0).  A device-side wait that runs out (see
+ * qz_set_device_wait_limit) makes the kernel return early; the next
+ * qz_device_status call reports QZ_ERR_DEVICE_TIMEOUT.
+ */
+QZ_API qz_status qz_w4a16_gemm(const void *a, const void *codes, const void *scales,
+                        const void *zeros, int64_t M, int64_t N, int64_t K,
+                        int64_t group_size, void *y, void *workspace,
+                        size_t workspace_bytes, void *stream);
+
+/*
+ * W8A16 decode GEMV: y = a * w_hat^T for the int8 symmetric per-channel
+ * weight (bits 8, symmetric 1, group_size K; codes N x K int8, scales N bf16;
+ * taqaniya.com IBM absmax example).  w_hat = bf16_rne(S * q), fp32
+ * accumulation, bf16 y.  Requirements: 1 <= M <= 16; N >= 1; K % 128 == 0.
+ * Workspace as for qz_w4a16_gemv with QZ_OP_W8A16_GEMV.
+ */
+QZ_API qz_status qz_w8a16_gemv(const void *a, const void *codes, const void *scales,
+                        int64_t M, int64_t N, int64_t K, void *y, void *workspace,
+                        size_t workspace_bytes, void *stream);
+
+/*
+ * Device-side wait bound used by kernels that wait on mbarriers (the GEMM).
+ * `limit` counts polling iterations of one wait; 0 restores the default.
+ * Not part of the method: a safety bound so that a broken pipeline returns an
+ * error instead of hanging the GPU.  Host-only setter, applies to later calls.
+ */
+QZ_API void qz_set_device_wait_limit(uint64_t limit);
+
+/*
+ * Reads and clears the device error word of the current device (written by a
+ * kernel whose bounded wait ran out).  Synchronizes the current device.
+ * Returns QZ_OK or QZ_ERR_DEVICE_TIMEOUT (or QZ_ERR_CUDA).
+ */
+QZ_API qz_status qz_device_status(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QZ_H_ */

@@ -1,0 +1,134 @@
+"""Host-side checks of the C ABI (no GPU needed, no kernel is launched).
+
+Every entry point declared in include/qz.h must be exported by libqz.so, and
+every argument error must come back synchronously, before any launch.  The
+pointers below are fake addresses that are never dereferenced: each call is
+rejected by the host-side checks first.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import weight_only_quantization_wise_b200 as qz
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qz.h")
+
+OK, INVALID, ALIGN, UNSUP, WS = 0, 1, 2, 3, 4
+A = ctypes.c_void_p(0x10000)          # fake, 16-byte aligned "device" pointers
+B = ctypes.c_void_p(0x20000)
+C = ctypes.c_void_p(0x30000)
+D = ctypes.c_void_p(0x40000)
+Y = ctypes.c_void_p(0x50000)
+MIS = ctypes.c_void_p(0x10008)        # 8-byte aligned only
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"QZ_API\s+[\w\s\*]*?\b(qz_\w+)\s*\(", src)))
+
+
+def test_header_declarations_are_exported():
+    names = declared_functions()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(qz.lib, n), n
+    assert sorted(qz.EXPORTED_SYMBOLS) == names
+
+
+def test_status_strings_and_version():
+    for s in range(7):
+        assert qz.qz_status_string(s)
+    assert qz.qz_status_string(99) == "unknown status"
+    assert qz.qz_version() >= 100
+
+
+def test_packed_bytes_formats():
+    assert qz.qz_packed_bytes(4096, 4096, 4, False, 128) == (4096 * 2048, 4096 * 32 * 2, 4096 * 32)
+    assert qz.qz_packed_bytes(4096, 4096, 8, True, 4096) == (4096 * 4096, 4096 * 2, 0)
+    assert qz.qz_packed_bytes(10, 64, 4, True, 0) == (320, 2, 0)
+    for bad in [(0, 128, 4, False, 128), (8, 100, 4, False, 128), (8, 128, 4, False, -1)]:
+        with pytest.raises(qz.QzError):
+            qz.qz_packed_bytes(*bad)
+    with pytest.raises(qz.QzError):
+        qz.qz_packed_bytes(8, 128, 3, False, 128)
+
+
+def test_workspace_bytes():
+    assert qz.qz_workspace_bytes(qz.QZ_OP_QUANTIZE_PACK, 1, 8, 128, 128) == 0
+    assert qz.qz_workspace_bytes(qz.QZ_OP_QUANTIZE_PACK, 1, 8, 128, 0) == 8
+    assert qz.qz_workspace_bytes(qz.QZ_OP_DEQUANTIZE, 1, 8, 128, 128) == 0
+    big = qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMV, 1, 1024, 1024, 128)
+    assert big > 0 and big % 4 == 0
+    assert qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMV, 16, 1024, 1024, 128) >= big
+    with pytest.raises(qz.QzError):
+        qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMV, 17, 1024, 1024, 128)
+    with pytest.raises(qz.QzError):
+        qz.qz_workspace_bytes(99, 1, 8, 128, 128)
+
+
+def L():
+    return qz.lib
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((None, 8, 128, 4, 0, 128, B, C, D, None, 0, None), INVALID),        # null w
+    ((A, 8, 128, 4, 0, 128, B, C, None, None, 0, None), INVALID),        # asym without zeros
+    ((A, 8, 128, 4, 1, 128, B, C, D, None, 0, None), INVALID),           # sym with zeros
+    ((A, 0, 128, 4, 0, 128, B, C, D, None, 0, None), INVALID),           # N = 0
+    ((A, 8, 100, 4, 0, 100, B, C, D, None, 0, None), UNSUP),             # K % 8
+    ((A, 8, 128, 4, 0, 48, B, C, D, None, 0, None), INVALID),            # K % g
+    ((A, 8, 128, 5, 0, 128, B, C, D, None, 0, None), UNSUP),             # bits
+    ((MIS, 8, 128, 4, 0, 128, B, C, D, None, 0, None), ALIGN),           # w alignment
+    ((A, 8, 128, 4, 0, 0, B, C, D, None, 0, None), WS),                  # per-tensor needs ws
+    ((A, 8, 128, 4, 0, 0, B, C, D, Y, 4, None), WS),                     # ws too small
+])
+def test_quantize_pack_rejects(args, expect):
+    assert L().qz_quantize_pack(*args) == expect
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((None, B, C, 8, 128, 4, 0, 128, Y, None), INVALID),
+    ((A, B, None, 8, 128, 4, 0, 128, Y, None), INVALID),
+    ((A, B, C, 8, 128, 4, 0, 128, MIS, None), ALIGN),
+    ((A, B, C, 8, 130, 4, 0, 130, Y, None), UNSUP),
+])
+def test_dequantize_rejects(args, expect):
+    assert L().qz_dequantize(*args) == expect
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((A, B, C, D, 0, 64, 128, 128, Y, None, 0, None), INVALID),          # M = 0
+    ((A, B, C, D, 17, 64, 128, 128, Y, None, 0, None), UNSUP),           # M > 16
+    ((A, B, C, D, 1, 64, 192, 64, Y, None, 0, None), UNSUP),             # K % 128
+    ((A, B, C, D, 1, 64, 256, 48, Y, None, 0, None), INVALID),           # K % g
+    ((A, B, C, D, 1, 64, 256, 16, Y, None, 0, None), UNSUP),             # g % 32
+    ((A, B, C, None, 1, 64, 256, 128, Y, None, 0, None), INVALID),       # null zeros
+    ((MIS, B, C, D, 1, 64, 256, 128, Y, None, 0, None), ALIGN),
+    ((A, B, C, D, 1, 4096, 4096, 128, Y, None, 0, None), WS),            # split-K needs ws
+])
+def test_w4a16_gemv_rejects(args, expect):
+    assert L().qz_w4a16_gemv(*args) == expect
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((A, B, C, 0, 64, 128, Y, None, 0, None), INVALID),
+    ((A, B, C, 17, 64, 128, Y, None, 0, None), UNSUP),
+    ((A, B, None, 1, 64, 128, Y, None, 0, None), INVALID),
+    ((A, MIS, C, 1, 64, 128, Y, None, 0, None), ALIGN),
+    ((A, B, C, 1, 4096, 4096, Y, None, 0, None), WS),
+])
+def test_w8a16_gemv_rejects(args, expect):
+    assert L().qz_w8a16_gemv(*args) == expect
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((A, B, C, D, 0, 64, 128, 128, Y, None, 0, None), INVALID),
+    ((A, B, C, D, 64, 64, 192, 64, Y, None, 0, None), UNSUP),
+    ((A, B, C, D, 64, 64, 256, 32, Y, None, 0, None), UNSUP),           # g % 64 for the GEMM
+    ((None, B, C, D, 64, 64, 256, 128, Y, None, 0, None), INVALID),
+])
+def test_w4a16_gemm_rejects(args, expect):
+    assert L().qz_w4a16_gemm(*args) == expect

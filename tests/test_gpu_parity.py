@@ -1,0 +1,337 @@
+"""CUDA path vs the CPU oracle on the same seeded inputs (needs a B200).
+
+Bars (fixed before any kernel was written):
+  * codes, scales, zeros: bit-exact;
+  * dequantized bf16 weights: bit-exact;
+  * matmul outputs: |y - y_ref| <= 8e-3 |y_ref| + 1e-4 sum_k |a_k w_k| against
+    the oracle's fp64 product over its own bf16 dequantized weights.
+Large configurations are checked on sampled rows that the oracle computes on
+its own; everything else is compared element by element.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+import weight_only_quantization_wise_b200 as qz
+
+pytestmark = pytest.mark.gpu
+
+FORMATS = [(4, False), (4, True), (8, False), (8, True)]
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch.device("cuda:0")
+
+
+def u16(t):
+    return synthetic.bf16_bits(t)
+
+
+def u8(t):
+    return t.detach().cpu().numpy().view(np.uint8)
+
+
+def gpu_quantize(w_dev, bits, sym, g):
+    ws = qz.Workspace(w_dev.device)
+    c, s, z = qz.qz_quantize_pack(w_dev, bits, sym, g, workspace=ws)
+    torch.cuda.synchronize()
+    return u8(c), u16(s), (None if z is None else u8(z))
+
+
+def to_dev_u8(a, dev):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+
+def to_dev_bf16(bits, dev):
+    return synthetic.from_bf16_bits(bits, dev)
+
+
+def assert_quant_equal(got, ref):
+    (gc, gs, gz), (rc, rs, rz) = got, ref
+    assert np.array_equal(gs.reshape(rs.shape), rs), "scales differ"
+    if rz is None:
+        assert gz is None
+    else:
+        assert np.array_equal(gz.reshape(rz.shape), rz), "zeros differ"
+    if not np.array_equal(gc.reshape(rc.shape), rc):
+        bad = np.argwhere(gc.reshape(rc.shape) != rc)
+        raise AssertionError(f"codes differ at {len(bad)} bytes, first {bad[:5].tolist()}")
+
+
+def check_tolerance(y_gpu_bits, y_ref, abs_ref, what=""):
+    y = oracle.bf16_bits_to_f32(y_gpu_bits).astype(np.float64).reshape(y_ref.shape)
+    bound = oracle.tolerance(y_ref, abs_ref)
+    err = np.abs(y - y_ref)
+    ratio = float((err / np.maximum(bound, 1e-300)).max())
+    assert (err <= bound).all(), f"{what}: max error/bound = {ratio:.3f}"
+    return ratio
+
+
+def group_sizes(K):
+    gs = [32, 64, 128, 256, K, 0]
+    if (K // 2) % 8 == 0 and K // 2 not in gs and K % (K // 2) == 0:
+        gs.append(K // 2)
+    return [g for g in gs if g == 0 or K % g == 0]
+
+
+SHAPES = [(1, 128), (37, 384), (64, 1024), (130, 2048)]
+
+
+@pytest.mark.parametrize("bits,sym", FORMATS)
+@pytest.mark.parametrize("N,K", SHAPES)
+def test_quantize_pack_bit_exact(dev, bits, sym, N, K):
+    w = synthetic.weights(N, K, sigma=0.02, seed=N * 7 + K)
+    for g in group_sizes(K):
+        ref = oracle.quantize_pack(u16(w), bits, sym, g)
+        got = gpu_quantize(w.to(dev), bits, sym, g)
+        assert_quant_equal(got, ref)
+
+
+@pytest.mark.parametrize("bits,sym", FORMATS)
+@pytest.mark.parametrize("N,K", SHAPES)
+def test_dequantize_bit_exact(dev, bits, sym, N, K):
+    w = synthetic.weights(N, K, sigma=0.02, seed=N * 11 + K)
+    for g in group_sizes(K):
+        c, s, z = oracle.quantize_pack(u16(w), bits, sym, g)
+        ref = oracle.dequantize(c, s, z, N, K, bits, sym, g)
+        out = qz.qz_dequantize(to_dev_u8(c, dev), to_dev_bf16(s, dev),
+                               None if z is None else to_dev_u8(z, dev), N, K, bits, sym, g)
+        torch.cuda.synchronize()
+        assert np.array_equal(u16(out), ref), (bits, sym, g)
+
+
+def edge_matrix():
+    """Rows that exercise the degenerate and boundary cases of the method."""
+    K = 256
+    rows = []
+    rows.append(np.zeros(K, np.float32))                          # all zero
+    rows.append(np.full(K, 0.75, np.float32))                     # constant positive
+    rows.append(np.full(K, -3.0, np.float32))                     # constant negative
+    r = np.zeros(K, np.float32); r[:4] = [0.0, 15.0, 2.5, 3.5]; rows.append(r)   # ties (S=1)
+    r = np.zeros(K, np.float32); r[:2] = [-1.5, 13.5]; rows.append(r)           # clamp at top
+    rng = np.random.default_rng(0)
+    rows.append((rng.normal(0, 1, K) * 1e-39).astype(np.float32))              # subnormal range
+    rows.append((rng.normal(0, 1, K) * 1e30).astype(np.float32))               # huge range
+    r = (rng.normal(0, 0.02, K)).astype(np.float32); r[77] = 3.0; rows.append(r)  # one outlier
+    rows.append(np.abs(rng.normal(0, 1, K)).astype(np.float32))                # all positive
+    rows.append(-np.abs(rng.normal(0, 1, K)).astype(np.float32))               # all negative
+    r = np.zeros(K, np.float32); r[5] = -0.0; r[6] = 1e-45; rows.append(r)      # -0, min subnormal
+    m = np.stack(rows)
+    t = torch.from_numpy(m).to(torch.bfloat16)
+    return t
+
+
+@pytest.mark.parametrize("bits,sym", FORMATS)
+def test_edge_groups_bit_exact(dev, bits, sym):
+    w = edge_matrix()
+    N, K = w.shape
+    for g in (32, 128, 256, 0):
+        ref = oracle.quantize_pack(u16(w), bits, sym, g)
+        got = gpu_quantize(w.to(dev), bits, sym, g)
+        assert_quant_equal(got, ref)
+        c, s, z = ref
+        wref = oracle.dequantize(c, s, z, N, K, bits, sym, g)
+        out = qz.qz_dequantize(to_dev_u8(c, dev), to_dev_bf16(s, dev),
+                               None if z is None else to_dev_u8(z, dev), N, K, bits, sym, g)
+        torch.cuda.synchronize()
+        assert np.array_equal(u16(out), wref)
+
+
+# ---------------------------------------------------------------------------
+# GEMV
+# ---------------------------------------------------------------------------
+
+GEMV_CASES = [  # (N, K, g)
+    (1024, 1024, 128), (1000, 384, 128), (17, 128, 32), (96, 512, 64),
+    (256, 2048, 256), (64, 1024, 1024), (4100, 1152, 128),
+]
+
+
+def oracle_w4(w_bits, g):
+    N, K = w_bits.shape
+    c, s, z = oracle.quantize_pack(w_bits, 4, False, g)
+    return c, s, z, oracle.dequantize(c, s, z, N, K, 4, False, g)
+
+
+@pytest.mark.parametrize("N,K,g", GEMV_CASES)
+@pytest.mark.parametrize("M", [1, 2, 5, 8, 9, 16])
+def test_w4a16_gemv_tolerance(dev, N, K, g, M):
+    w = synthetic.weights(N, K, sigma=0.02, seed=N + K + g)
+    a = synthetic.activations(M, K, seed=M)
+    c, s, z, w_hat = oracle_w4(u16(w), g)
+    y_ref, abs_ref = oracle.matmul_f64(u16(a), w_hat)
+    y = qz.qz_w4a16_gemv(a.to(dev), to_dev_u8(c, dev), to_dev_bf16(s, dev), to_dev_u8(z, dev),
+                         N, K, g)
+    torch.cuda.synchronize()
+    check_tolerance(u16(y), y_ref, abs_ref, f"w4a16 M={M} N={N} K={K} g={g}")
+
+
+@pytest.mark.parametrize("N,K,g", [(1024, 1024, 128), (37, 384, 32), (300, 4096, 128)])
+def test_w4a16_gemv_onehot_is_exact(dev, N, K, g):
+    """With one-hot activations y[m][n] = w_hat[n][k_m]: the in-register
+    dequantization must reproduce the oracle's bf16 weights bit for bit."""
+    w = synthetic.weights(N, K, sigma=0.02, seed=5)
+    c, s, z, w_hat = oracle_w4(u16(w), g)
+    rng = np.random.default_rng(1)
+    ks = rng.choice(K, size=16, replace=False)
+    a = np.zeros((16, K), np.uint16)
+    a[np.arange(16), ks] = 0x3F80
+    y = qz.qz_w4a16_gemv(to_dev_bf16(a, dev), to_dev_u8(c, dev), to_dev_bf16(s, dev),
+                         to_dev_u8(z, dev), N, K, g)
+    torch.cuda.synchronize()
+    assert np.array_equal(u16(y), w_hat[:, ks].T)
+
+
+@pytest.mark.parametrize("N,K", [(1024, 1024), (1000, 384), (17, 128), (4100, 1152)])
+@pytest.mark.parametrize("M", [1, 3, 8, 16])
+def test_w8a16_gemv_tolerance(dev, N, K, M):
+    w = synthetic.weights(N, K, sigma=0.015, seed=N * 3 + K)
+    a = synthetic.activations(M, K, seed=M + 100)
+    c, s, _ = oracle.quantize_pack(u16(w), 8, True, K)
+    w_hat = oracle.dequantize(c, s, None, N, K, 8, True, K)
+    y_ref, abs_ref = oracle.matmul_f64(u16(a), w_hat)
+    y = qz.qz_w8a16_gemv(a.to(dev), to_dev_u8(c, dev), to_dev_bf16(s, dev), N, K)
+    torch.cuda.synchronize()
+    check_tolerance(u16(y), y_ref, abs_ref, f"w8a16 M={M} N={N} K={K}")
+    # one-hot rows reproduce w_hat exactly
+    ks = np.arange(min(16, K)) * (K // 16)
+    oh = np.zeros((16, K), np.uint16)
+    oh[np.arange(16), ks] = 0x3F80
+    y1 = qz.qz_w8a16_gemv(to_dev_bf16(oh, dev), to_dev_u8(c, dev), to_dev_bf16(s, dev), N, K)
+    torch.cuda.synchronize()
+    assert np.array_equal(u16(y1), w_hat[:, ks].T)
+
+
+def test_gemv_workspace_is_left_zeroed_and_results_repeat(dev):
+    N, K, g, M = 4096, 4096, 128, 4
+    nbytes = qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMV, M, N, K, g)
+    assert nbytes > 0
+    w = synthetic.weights(N, K, seed=9, device=dev)
+    a = synthetic.activations(M, K, seed=9, device=dev)
+    c, s, z = qz.qz_quantize_pack(w, 4, False, g)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+    y1 = qz.qz_w4a16_gemv(a, c, s, z, N, K, g, workspace=ws)
+    y2 = qz.qz_w4a16_gemv(a, c, s, z, N, K, g, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    # the counter region (after the partials) must be zero again
+    plan_partials = nbytes - ((-(-((N + 15) // 16) // 64)) * 64 * 4)
+    assert int(ws[plan_partials:].count_nonzero()) == 0
+
+
+def test_outputs_stay_inside_their_buffers(dev):
+    """Guard bands around every output must be untouched (a stand-in for a
+    memory checker, which this pool does not offer)."""
+    N, K, g, M = 300, 1024, 128, 3
+    pad = 4096
+    w = synthetic.weights(N, K, seed=4, device=dev)
+    a = synthetic.activations(M, K, seed=4, device=dev)
+
+    def guarded(nbytes):
+        buf = torch.full((nbytes + 2 * pad,), 0xA5, dtype=torch.uint8, device=dev)
+        return buf, buf[pad:pad + nbytes]
+
+    cb, sb, zb = qz.qz_packed_bytes(N, K, 4, False, g)
+    cbuf, cv = guarded(cb)
+    sbuf, sv = guarded(sb)
+    zbuf, zv = guarded(zb)
+    qz.qz_quantize_pack(w, 4, False, g, codes=cv, scales=sv.view(torch.bfloat16), zeros=zv)
+    ybuf, yv = guarded(M * N * 2)
+    qz.qz_w4a16_gemv(a, cv, sv.view(torch.bfloat16), zv, N, K, g, y=yv.view(torch.bfloat16))
+    dbuf, dv = guarded(N * K * 2)
+    qz.qz_dequantize(cv, sv.view(torch.bfloat16), zv, N, K, 4, False, g, out=dv.view(torch.bfloat16))
+    torch.cuda.synchronize()
+    for buf in (cbuf, sbuf, zbuf, ybuf, dbuf):
+        assert bool((buf[:pad] == 0xA5).all()) and bool((buf[-pad:] == 0xA5).all())
+
+
+# ---------------------------------------------------------------------------
+# Full-size configurations, checked on sampled rows
+# ---------------------------------------------------------------------------
+
+def sample_rows(N, count, seed):
+    rng = np.random.default_rng(seed)
+    rows = set(rng.choice(N, size=min(count, N), replace=False).tolist())
+    rows.update({0, N - 1})
+    return np.array(sorted(rows))
+
+
+def check_layer_sampled(dev, N, K, M, sigma, seed, bits, sym, g, rows=48):
+    w = synthetic.weights(N, K, sigma=sigma, seed=seed, device=dev)
+    a = synthetic.activations(M, K, seed=seed + 1000, device=dev)
+    ws = qz.Workspace(dev)
+    c, s, z = qz.qz_quantize_pack(w, bits, sym, g, workspace=ws)
+    if bits == 4:
+        y = qz.qz_w4a16_gemv(a, c, s, z, N, K, g, workspace=ws)
+    else:
+        y = qz.qz_w8a16_gemv(a, c, s, N, K, workspace=ws)
+    torch.cuda.synchronize()
+    idx = sample_rows(N, rows, seed)
+    ti = torch.from_numpy(idx).to(dev)
+    w_rows = u16(w.index_select(0, ti))
+    ref = oracle.quantize_pack(w_rows, bits, sym, g)
+    got = (u8(c.index_select(0, ti)), u16(s.index_select(0, ti)),
+           None if z is None else u8(z.index_select(0, ti)))
+    assert_quant_equal(got, ref)
+    w_hat = oracle.dequantize(*ref, len(idx), K, bits, sym, g)
+    y_ref, abs_ref = oracle.matmul_f64(u16(a), w_hat)
+    return check_tolerance(u16(y)[:, idx], y_ref, abs_ref, f"N={N} K={K} M={M} bits={bits}")
+
+
+def test_tiny_config_full(dev):
+    """1024 x 1024, M = 1, seed 0: every code and every output."""
+    N, K = 1024, 1024
+    w = synthetic.weights(N, K, sigma=0.02, seed=0)
+    a = synthetic.activations(1, K, seed=0)
+    ref = oracle.quantize_pack(u16(w), 4, False, 128)
+    got = gpu_quantize(w.to(dev), 4, False, 128)
+    assert_quant_equal(got, ref)
+    w_hat = oracle.dequantize(*ref, N, K, 4, False, 128)
+    y_ref, abs_ref = oracle.matmul_f64(u16(a), w_hat)
+    c, s, z = (to_dev_u8(got[0], dev), to_dev_bf16(got[1], dev), to_dev_u8(got[2], dev))
+    y = qz.qz_w4a16_gemv(a.to(dev), c, s, z, N, K, 128)
+    torch.cuda.synchronize()
+    check_tolerance(u16(y), y_ref, abs_ref, "tiny")
+
+
+@pytest.mark.parametrize("li,NK", list(enumerate(synthetic.DECODE_7B)))
+def test_decode_7b_layers(dev, li, NK):
+    N, K = NK
+    check_layer_sampled(dev, N, K, 1, 0.02, 1 + li, 4, False, 128)
+
+
+@pytest.mark.parametrize("M", synthetic.DECODE_70B_M)
+@pytest.mark.parametrize("li,NK", list(enumerate(synthetic.DECODE_70B)))
+@pytest.mark.parametrize("bits", [4, 8])
+def test_decode_70b_layers(dev, M, li, NK, bits):
+    N, K = NK
+    sym = bits == 8
+    g = 128 if bits == 4 else K
+    check_layer_sampled(dev, N, K, M, 0.015, 4 + li, bits, sym, g, rows=24)
+
+
+def test_bulk_quantization_stack(dev):
+    """32 layer sets (7.785e9 parameters) through quantize_pack, int4 g128 and
+    int8 per-channel; sampled rows of every layer checked bit-exact."""
+    total = 0
+    ws = qz.Workspace(dev)
+    for si in range(synthetic.BULK_SETS):
+        for li, (N, K) in enumerate(synthetic.BULK_LAYER_SET):
+            seed = 100 + si * 16 + li
+            w = synthetic.weights(N, K, sigma=0.02, seed=seed, device=dev)
+            idx = sample_rows(N, 2, seed)
+            ti = torch.from_numpy(idx).to(dev)
+            w_rows = u16(w.index_select(0, ti))
+            for bits, sym, g in ((4, False, 128), (8, True, K)):
+                c, s, z = qz.qz_quantize_pack(w, bits, sym, g, workspace=ws)
+                got = (u8(c.index_select(0, ti)), u16(s.index_select(0, ti)),
+                       None if z is None else u8(z.index_select(0, ti)))
+                assert_quant_equal(got, oracle.quantize_pack(w_rows, bits, sym, g))
+            total += N * K
+            del w
+    assert total == 7_784_628_224

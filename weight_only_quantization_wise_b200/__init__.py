@@ -1,0 +1,221 @@
+"""Python binding of libqz.so, the B200 weight-only quantization library.
+
+Argument marshalling only: every function below validates Python-side types,
+allocates outputs with PyTorch when the caller did not pass them, and calls
+the C entry point of the same name (declared in ``include/qz.h``) on the
+current CUDA stream.  All arithmetic runs in the library's CUDA kernels; there
+is no CPU or PyTorch fallback.  If ``libqz.so`` is missing the import fails.
+"""
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "QzError", "lib", "qz_version", "qz_status_string", "qz_packed_bytes",
+    "qz_workspace_bytes", "qz_quantize_pack", "qz_dequantize", "qz_w4a16_gemv",
+    "qz_w4a16_gemm", "qz_w8a16_gemv", "qz_set_device_wait_limit", "qz_device_status",
+    "Workspace", "QZ_OP_QUANTIZE_PACK", "QZ_OP_DEQUANTIZE", "QZ_OP_W4A16_GEMV",
+    "QZ_OP_W4A16_GEMM", "QZ_OP_W8A16_GEMV", "EXPORTED_SYMBOLS",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqz.so")
+
+QZ_OK = 0
+QZ_ERR_DEVICE_TIMEOUT = 6
+QZ_OP_QUANTIZE_PACK, QZ_OP_DEQUANTIZE, QZ_OP_W4A16_GEMV, QZ_OP_W4A16_GEMM, QZ_OP_W8A16_GEMV = range(5)
+
+_i32, _i64, _sz, _p = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p
+_SIGS = {
+    "qz_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    "qz_version": ([], ctypes.c_int),
+    "qz_packed_bytes": ([_i64, _i64, _i32, _i32, _i64, ctypes.POINTER(_sz),
+                         ctypes.POINTER(_sz), ctypes.POINTER(_sz)], ctypes.c_int),
+    "qz_workspace_bytes": ([_i32, _i64, _i64, _i64, _i64, ctypes.POINTER(_sz)], ctypes.c_int),
+    "qz_quantize_pack": ([_p, _i64, _i64, _i32, _i32, _i64, _p, _p, _p, _p, _sz, _p], ctypes.c_int),
+    "qz_dequantize": ([_p, _p, _p, _i64, _i64, _i32, _i32, _i64, _p, _p], ctypes.c_int),
+    "qz_w4a16_gemv": ([_p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p, _sz, _p], ctypes.c_int),
+    "qz_w4a16_gemm": ([_p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p, _sz, _p], ctypes.c_int),
+    "qz_w8a16_gemv": ([_p, _p, _p, _i64, _i64, _i64, _p, _p, _sz, _p], ctypes.c_int),
+    "qz_set_device_wait_limit": ([ctypes.c_uint64], None),
+    "qz_device_status": ([], ctypes.c_int),
+}
+EXPORTED_SYMBOLS = tuple(_SIGS)
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is not built; run `python -m weight_only_quantization_wise_b200.build` "
+        "(there is no fallback implementation)")
+
+lib = ctypes.CDLL(LIB_PATH)
+for _name, (_args, _res) in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.argtypes = _args
+    _f.restype = _res
+
+
+class QzError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {qz_status_string(status)} (status {status})")
+
+
+def _check(status: int, where: str) -> None:
+    if status != QZ_OK:
+        raise QzError(status, where)
+
+
+def qz_status_string(status: int) -> str:
+    return lib.qz_status_string(int(status)).decode()
+
+
+def qz_version() -> int:
+    return int(lib.qz_version())
+
+
+def qz_packed_bytes(N, K, bits=4, symmetric=False, group_size=128):
+    c, s, z = _sz(), _sz(), _sz()
+    _check(lib.qz_packed_bytes(N, K, bits, int(symmetric), group_size, ctypes.byref(c),
+                               ctypes.byref(s), ctypes.byref(z)), "qz_packed_bytes")
+    return c.value, s.value, z.value
+
+
+def qz_workspace_bytes(op, M, N, K, group_size=128) -> int:
+    b = _sz()
+    _check(lib.qz_workspace_bytes(op, M, N, K, group_size, ctypes.byref(b)), "qz_workspace_bytes")
+    return b.value
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+class Workspace:
+    """A zero-filled device workspace that grows on demand.
+
+    The library leaves split-K workspaces zero-filled after each call, so one
+    buffer serves every call issued on one stream.  Calls that may run
+    concurrently need separate Workspace objects.
+    """
+
+    def __init__(self, device=None):
+        self.device = torch.device(device if device is not None else "cuda")
+        self.buf = None
+
+    def get(self, nbytes: int):
+        if nbytes == 0:
+            return None
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=self.device)
+        return self.buf
+
+
+def _ws_args(workspace, nbytes, device):
+    if nbytes == 0:
+        return None, 0
+    if workspace is None:
+        workspace = Workspace(device).get(nbytes)
+    elif isinstance(workspace, Workspace):
+        workspace = workspace.get(nbytes)
+    return _ptr(workspace), workspace.numel() * workspace.element_size()
+
+
+def qz_quantize_pack(w, bits=4, symmetric=False, group_size=128, codes=None, scales=None,
+                     zeros=None, workspace=None, stream=None):
+    """Quantize an N x K bf16 matrix; returns (codes uint8, scales bf16, zeros uint8 | None)."""
+    if w.dtype != torch.bfloat16 or w.dim() != 2:
+        raise ValueError("w must be a 2-D bf16 tensor")
+    N, K = w.shape
+    cb, sb, zb = qz_packed_bytes(N, K, bits, symmetric, group_size)
+    dev = w.device
+    if codes is None:
+        codes = torch.empty((N, K // 2) if bits == 4 else (N, K), dtype=torch.uint8, device=dev)
+    if scales is None:
+        shape = (1,) if group_size == 0 else (N, K // group_size)
+        scales = torch.empty(shape, dtype=torch.bfloat16, device=dev)
+    if zeros is None and not symmetric:
+        shape = (1,) if group_size == 0 else (N, K // group_size)
+        zeros = torch.empty(shape, dtype=torch.uint8, device=dev)
+    ws_ptr, ws_bytes = _ws_args(workspace, qz_workspace_bytes(QZ_OP_QUANTIZE_PACK, 1, N, K,
+                                                              group_size), dev)
+    _check(lib.qz_quantize_pack(_ptr(w), N, K, bits, int(symmetric), group_size, _ptr(codes),
+                                _ptr(scales), _ptr(zeros) if not symmetric else None, ws_ptr,
+                                ws_bytes, _stream(stream, dev)), "qz_quantize_pack")
+    return codes, scales, (None if symmetric else zeros)
+
+
+def qz_dequantize(codes, scales, zeros, N, K, bits=4, symmetric=False, group_size=128,
+                  out=None, stream=None):
+    """w_hat = bf16(S * (q - Z)) as an N x K bf16 tensor."""
+    dev = codes.device
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    _check(lib.qz_dequantize(_ptr(codes), _ptr(scales), _ptr(zeros), N, K, bits,
+                             int(symmetric), group_size, _ptr(out), _stream(stream, dev)),
+           "qz_dequantize")
+    return out
+
+
+def _matmul_out(a, N, y):
+    if a.dtype != torch.bfloat16 or a.dim() != 2:
+        raise ValueError("a must be a 2-D bf16 tensor")
+    if y is None:
+        y = torch.empty((a.shape[0], N), dtype=torch.bfloat16, device=a.device)
+    return y
+
+
+def qz_w4a16_gemv(a, codes, scales, zeros, N, K, group_size=128, y=None, workspace=None,
+                  stream=None):
+    """y = a * w_hat^T for int4 asymmetric group-wise weights, M <= 16."""
+    y = _matmul_out(a, N, y)
+    M = a.shape[0]
+    ws_ptr, ws_bytes = _ws_args(workspace, qz_workspace_bytes(QZ_OP_W4A16_GEMV, M, N, K,
+                                                              group_size), a.device)
+    _check(lib.qz_w4a16_gemv(_ptr(a), _ptr(codes), _ptr(scales), _ptr(zeros), M, N, K,
+                             group_size, _ptr(y), ws_ptr, ws_bytes, _stream(stream, a.device)),
+           "qz_w4a16_gemv")
+    return y
+
+
+def qz_w4a16_gemm(a, codes, scales, zeros, N, K, group_size=128, y=None, workspace=None,
+                  stream=None):
+    """y = a * w_hat^T for int4 asymmetric group-wise weights, any M."""
+    y = _matmul_out(a, N, y)
+    M = a.shape[0]
+    ws_ptr, ws_bytes = _ws_args(workspace, qz_workspace_bytes(QZ_OP_W4A16_GEMM, M, N, K,
+                                                              group_size), a.device)
+    _check(lib.qz_w4a16_gemm(_ptr(a), _ptr(codes), _ptr(scales), _ptr(zeros), M, N, K,
+                             group_size, _ptr(y), ws_ptr, ws_bytes, _stream(stream, a.device)),
+           "qz_w4a16_gemm")
+    return y
+
+
+def qz_w8a16_gemv(a, codes, scales, N, K, y=None, workspace=None, stream=None):
+    """y = a * w_hat^T for int8 symmetric per-channel weights, M <= 16."""
+    y = _matmul_out(a, N, y)
+    M = a.shape[0]
+    ws_ptr, ws_bytes = _ws_args(workspace, qz_workspace_bytes(QZ_OP_W8A16_GEMV, M, N, K, K),
+                                a.device)
+    _check(lib.qz_w8a16_gemv(_ptr(a), _ptr(codes), _ptr(scales), M, N, K, _ptr(y), ws_ptr,
+                             ws_bytes, _stream(stream, a.device)), "qz_w8a16_gemv")
+    return y
+
+
+def qz_set_device_wait_limit(limit: int) -> None:
+    lib.qz_set_device_wait_limit(int(limit))
+
+
+def qz_device_status() -> int:
+    return int(lib.qz_device_status())

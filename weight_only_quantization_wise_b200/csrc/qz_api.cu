@@ -1,0 +1,207 @@
+// qz_api.cu -- the exported C ABI (include/qz.h): argument validation and
+// dispatch to the kernels.  Every check runs on the host before any launch.
+#include <cuda_runtime.h>
+
+#include <atomic>
+
+#include "qz_internal.cuh"
+
+namespace qz {
+
+static std::atomic<uint64_t> g_wait_limit{0};
+constexpr uint64_t kDefaultWaitLimit = uint64_t(1) << 26;
+
+uint64_t device_wait_limit() {
+    const uint64_t v = g_wait_limit.load(std::memory_order_relaxed);
+    return v ? v : kDefaultWaitLimit;
+}
+
+namespace {
+
+constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
+constexpr int64_t kMaxElems = int64_t(1) << 40;
+
+bool format_ok(int32_t bits, int32_t symmetric) {
+    return (bits == 4 || bits == 8) && (symmetric == 0 || symmetric == 1);
+}
+
+// Shape/format checks shared by quantize_pack and dequantize.
+qz_status check_matrix_format(int64_t N, int64_t K, int32_t bits, int32_t symmetric,
+                              int64_t g) {
+    if (!format_ok(bits, symmetric)) return QZ_ERR_UNSUPPORTED;
+    if (N < 1 || K < 1 || N > kMaxDim || K > kMaxDim || N * K > kMaxElems)
+        return QZ_ERR_INVALID_ARG;
+    if (g < 0) return QZ_ERR_INVALID_ARG;
+    if (g > 0 && K % g != 0) return QZ_ERR_INVALID_ARG;
+    if (K % 8 != 0) return QZ_ERR_UNSUPPORTED;
+    if (g > 0 && g % 8 != 0) return QZ_ERR_UNSUPPORTED;
+    return QZ_OK;
+}
+
+qz_status check_gemv_shape(int64_t M, int64_t N, int64_t K) {
+    if (M < 1 || N < 1 || K < 1 || N > kMaxDim || K > kMaxDim) return QZ_ERR_INVALID_ARG;
+    if (M > 16) return QZ_ERR_UNSUPPORTED;
+    if (K % 128 != 0) return QZ_ERR_UNSUPPORTED;
+    if ((int64_t)N * K > kMaxElems) return QZ_ERR_INVALID_ARG;
+    return QZ_OK;
+}
+
+qz_status check_workspace(size_t need, const void *ws, size_t ws_bytes) {
+    if (need == 0) return QZ_OK;
+    if (ws == nullptr || ws_bytes < need) return QZ_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return QZ_ERR_ALIGNMENT;
+    return QZ_OK;
+}
+
+cudaStream_t as_stream(void *s) { return static_cast<cudaStream_t>(s); }
+
+}  // namespace
+}  // namespace qz
+
+using namespace qz;
+
+extern "C" {
+
+QZ_API const char *qz_status_string(int status) {
+    switch (status) {
+    case QZ_OK: return "ok";
+    case QZ_ERR_INVALID_ARG: return "invalid argument (null pointer, size or shape)";
+    case QZ_ERR_ALIGNMENT: return "pointer not aligned as required";
+    case QZ_ERR_UNSUPPORTED: return "format or shape not supported by the kernels";
+    case QZ_ERR_WORKSPACE: return "workspace missing or too small";
+    case QZ_ERR_CUDA: return "CUDA call or kernel launch failed";
+    case QZ_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait ran out";
+    default: return "unknown status";
+    }
+}
+
+QZ_API int qz_version(void) { return 100; }
+
+QZ_API qz_status qz_packed_bytes(int64_t N, int64_t K, int32_t bits, int32_t symmetric,
+                                 int64_t group_size, size_t *codes_bytes,
+                                 size_t *scales_bytes, size_t *zeros_bytes) {
+    if (!codes_bytes || !scales_bytes || !zeros_bytes) return QZ_ERR_INVALID_ARG;
+    if (!format_ok(bits, symmetric)) return QZ_ERR_UNSUPPORTED;
+    if (N < 1 || K < 1 || group_size < 0) return QZ_ERR_INVALID_ARG;
+    if (group_size > 0 && K % group_size != 0) return QZ_ERR_INVALID_ARG;
+    if (bits == 4 && K % 2 != 0) return QZ_ERR_INVALID_ARG;
+    const int64_t groups = group_size == 0 ? 1 : N * (K / group_size);
+    *codes_bytes = (size_t)(bits == 4 ? N * (K / 2) : N * K);
+    *scales_bytes = (size_t)groups * 2;
+    *zeros_bytes = symmetric ? 0 : (size_t)groups;
+    return QZ_OK;
+}
+
+QZ_API qz_status qz_workspace_bytes(int32_t op, int64_t M, int64_t N, int64_t K,
+                                    int64_t group_size, size_t *bytes) {
+    if (!bytes) return QZ_ERR_INVALID_ARG;
+    switch (op) {
+    case QZ_OP_QUANTIZE_PACK:
+        if (group_size < 0) return QZ_ERR_INVALID_ARG;
+        *bytes = quantize_workspace_bytes(group_size);
+        return QZ_OK;
+    case QZ_OP_DEQUANTIZE:
+        *bytes = 0;
+        return QZ_OK;
+    case QZ_OP_W4A16_GEMV:
+    case QZ_OP_W8A16_GEMV: {
+        const qz_status s = check_gemv_shape(M, N, K);
+        if (s != QZ_OK) return s;
+        *bytes = gemv_plan(M, N, K).total_bytes;
+        return QZ_OK;
+    }
+    case QZ_OP_W4A16_GEMM:
+        if (M < 1 || N < 1 || K < 1) return QZ_ERR_INVALID_ARG;
+        *bytes = M <= 16 && K % 128 == 0 ? gemv_plan(M, N, K).total_bytes
+                                         : gemm_workspace_bytes(M, N, K);
+        return QZ_OK;
+    default:
+        return QZ_ERR_INVALID_ARG;
+    }
+}
+
+QZ_API qz_status qz_quantize_pack(const void *w, int64_t N, int64_t K, int32_t bits,
+                                  int32_t symmetric, int64_t group_size, void *codes,
+                                  void *scales, void *zeros, void *workspace,
+                                  size_t workspace_bytes, void *stream) {
+    qz_status s = check_matrix_format(N, K, bits, symmetric, group_size);
+    if (s != QZ_OK) return s;
+    if (!w || !codes || !scales) return QZ_ERR_INVALID_ARG;
+    if (symmetric ? (zeros != nullptr) : (zeros == nullptr)) return QZ_ERR_INVALID_ARG;
+    if (!aligned(w, 16) || !aligned(codes, 16) || !aligned(scales, 2)) return QZ_ERR_ALIGNMENT;
+    s = check_workspace(quantize_workspace_bytes(group_size), workspace, workspace_bytes);
+    if (s != QZ_OK) return s;
+    return launch_quantize_pack(w, N, K, bits, symmetric, group_size, codes, scales, zeros,
+                                workspace, as_stream(stream));
+}
+
+QZ_API qz_status qz_dequantize(const void *codes, const void *scales, const void *zeros,
+                               int64_t N, int64_t K, int32_t bits, int32_t symmetric,
+                               int64_t group_size, void *w_hat, void *stream) {
+    const qz_status s = check_matrix_format(N, K, bits, symmetric, group_size);
+    if (s != QZ_OK) return s;
+    if (!codes || !scales || !w_hat) return QZ_ERR_INVALID_ARG;
+    if (symmetric ? (zeros != nullptr) : (zeros == nullptr)) return QZ_ERR_INVALID_ARG;
+    if (!aligned(codes, 16) || !aligned(w_hat, 16) || !aligned(scales, 2)) return QZ_ERR_ALIGNMENT;
+    return launch_dequantize(codes, scales, zeros, N, K, bits, symmetric, group_size, w_hat,
+                             as_stream(stream));
+}
+
+QZ_API qz_status qz_w4a16_gemv(const void *a, const void *codes, const void *scales,
+                               const void *zeros, int64_t M, int64_t N, int64_t K,
+                               int64_t group_size, void *y, void *workspace,
+                               size_t workspace_bytes, void *stream) {
+    qz_status s = check_gemv_shape(M, N, K);
+    if (s != QZ_OK) return s;
+    if (group_size < 32 || group_size % 32 != 0 || K % group_size != 0)
+        return group_size <= 0 || K % group_size != 0 ? QZ_ERR_INVALID_ARG : QZ_ERR_UNSUPPORTED;
+    if (!a || !codes || !scales || !zeros || !y) return QZ_ERR_INVALID_ARG;
+    if (!aligned(a, 16) || !aligned(codes, 16) || !aligned(scales, 2) || !aligned(y, 2))
+        return QZ_ERR_ALIGNMENT;
+    const GemvPlan plan = gemv_plan(M, N, K);
+    s = check_workspace(plan.total_bytes, workspace, workspace_bytes);
+    if (s != QZ_OK) return s;
+    return launch_w4a16_gemv(a, codes, scales, zeros, M, N, K, group_size, y, workspace, plan,
+                             as_stream(stream));
+}
+
+QZ_API qz_status qz_w8a16_gemv(const void *a, const void *codes, const void *scales,
+                               int64_t M, int64_t N, int64_t K, void *y, void *workspace,
+                               size_t workspace_bytes, void *stream) {
+    qz_status s = check_gemv_shape(M, N, K);
+    if (s != QZ_OK) return s;
+    if (!a || !codes || !scales || !y) return QZ_ERR_INVALID_ARG;
+    if (!aligned(a, 16) || !aligned(codes, 16) || !aligned(scales, 2) || !aligned(y, 2))
+        return QZ_ERR_ALIGNMENT;
+    const GemvPlan plan = gemv_plan(M, N, K);
+    s = check_workspace(plan.total_bytes, workspace, workspace_bytes);
+    if (s != QZ_OK) return s;
+    return launch_w8a16_gemv(a, codes, scales, M, N, K, y, workspace, plan, as_stream(stream));
+}
+
+QZ_API qz_status qz_w4a16_gemm(const void *a, const void *codes, const void *scales,
+                               const void *zeros, int64_t M, int64_t N, int64_t K,
+                               int64_t group_size, void *y, void *workspace,
+                               size_t workspace_bytes, void *stream) {
+    if (M < 1 || N < 1 || K < 1 || M > kMaxDim || N > kMaxDim || K > kMaxDim)
+        return QZ_ERR_INVALID_ARG;
+    if (K % 128 != 0) return QZ_ERR_UNSUPPORTED;
+    if (group_size <= 0 || K % group_size != 0) return QZ_ERR_INVALID_ARG;
+    if (!a || !codes || !scales || !zeros || !y) return QZ_ERR_INVALID_ARG;
+    if (M <= 16)   // the decode kernel covers small M with the same arithmetic
+        return qz_w4a16_gemv(a, codes, scales, zeros, M, N, K, group_size, y, workspace,
+                             workspace_bytes, stream);
+    if (group_size % 64 != 0) return QZ_ERR_UNSUPPORTED;
+    if (!aligned(a, 16) || !aligned(codes, 16) || !aligned(scales, 2) || !aligned(y, 16))
+        return QZ_ERR_ALIGNMENT;
+    const qz_status s = check_workspace(gemm_workspace_bytes(M, N, K), workspace, workspace_bytes);
+    if (s != QZ_OK) return s;
+    return launch_w4a16_gemm(a, codes, scales, zeros, M, N, K, group_size, y, workspace,
+                             as_stream(stream));
+}
+
+QZ_API void qz_set_device_wait_limit(uint64_t limit) {
+    g_wait_limit.store(limit, std::memory_order_relaxed);
+}
+
+}  // extern "C"

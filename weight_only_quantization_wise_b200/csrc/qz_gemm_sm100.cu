@@ -1,0 +1,457 @@
+// qz_gemm_sm100.cu -- W4A16 prefill GEMM on the sm_100a (tcgen05) tensor cores,
+// and the device error word used by bounded device-side waits.
+//
+// Quantization concepts guide, "Quantize weights or activations": weight-only
+// methods dequantize the weights to the compute dtype before each matmul;
+// prefill and large batches are compute-bound, so this path must keep the
+// tensor cores busy.  The GPTQ explainer: the dequantization happens inside
+// the matmul kernel, with no separate conversion pass.
+//
+// y (M x N) = a (M x K) * w_hat^T with w_hat = bf16_rne(S * (q - Z)).
+//
+// One CTA computes a tile of 128 weight rows x 256 tokens.  The roles:
+//   warp 0      TMA producer: per 64-wide K step, the activation tile
+//               (256 tokens x 64 bf16, 128-byte swizzle) and the packed codes
+//               (128 rows x 32 bytes) into a STAGES-deep shared-memory ring.
+//   warp 1      allocates tensor memory; one lane issues tcgen05.mma.
+//   warps 2..5  dequantize: thread t of warp w owns weight row 32*(w%4)+t
+//               (the tensor-memory lane quarter that warp may access), turns
+//               its 64 codes into bf16 exactly as qz_dequantize does and
+//               stores them with tcgen05.st as the A operand of the MMA
+//               (A = weights in tensor memory, K-major, 2 bf16 per column);
+//               after the K loop they read the fp32 accumulators back with
+//               tcgen05.ld and write bf16 y.
+// The MMA is M = 128 (weight rows), N = 256 (tokens), K = 16, fp32
+// accumulation in tensor memory (256 columns); B = activations from shared
+// memory.  Each weight tile is dequantized once per 256 tokens.
+//
+// Every mbarrier wait is bounded by a caller-set iteration limit; on expiry
+// the thread records the fault in g_device_error_word and in a CTA-local
+// abort flag, every role stops issuing work, in-flight copies and MMAs are
+// drained (with bounded waits), tensor memory is released and the CTA exits.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "qz_internal.cuh"
+
+namespace qz {
+
+// Set (atomicOr) by a kernel whose bounded wait ran out.
+__device__ unsigned int g_device_error_word = 0;
+
+namespace {
+
+constexpr int kStages = 4;
+constexpr int kTileN = 128;               // weight rows per CTA (MMA M)
+constexpr int kTileM = 256;               // tokens per CTA (MMA N)
+constexpr int kTileK = 64;                // K per stage
+constexpr int kActStageBytes = kTileM * kTileK * 2;      // 32 KB
+constexpr int kPackStageBytes = kTileN * kTileK / 2;     // 4 KB
+constexpr int kAccCols = kTileM;                         // fp32 accumulator columns
+constexpr int kACols = kTileK / 2;                       // A columns per stage (bf16 pairs)
+constexpr int kTmemCols = 512;
+constexpr int kThreads = 192;
+constexpr int kSmemBytes = kStages * (kActStageBytes + kPackStageBytes) + 1024 + 256;
+
+// instruction descriptor, kind::f16: D f32, A bf16, B bf16, both K-major,
+// N = 256 (>>3), M = 128 (>>4)
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                            ((uint32_t)(kTileM >> 3) << 17) | ((uint32_t)(kTileN >> 4) << 24);
+
+struct SmemLayout {
+    // offsets from the 1024-aligned base
+    static constexpr uint32_t act = 0;
+    static constexpr uint32_t pack = act + kStages * kActStageBytes;
+    static constexpr uint32_t bars = pack + kStages * kPackStageBytes;
+    // barriers: full[S], empty[S], afull[S], accum, drain
+    static constexpr uint32_t full = bars;
+    static constexpr uint32_t empty = full + 8 * kStages;
+    static constexpr uint32_t afull = empty + 8 * kStages;
+    static constexpr uint32_t accum = afull + 8 * kStages;
+    static constexpr uint32_t drain = accum + 8;
+    static constexpr uint32_t tmem_slot = drain + 8;
+    static constexpr uint32_t abort_flag = tmem_slot + 4;
+    static constexpr uint32_t end = abort_flag + 4;
+};
+static_assert(SmemLayout::end + 1024 <= kSmemBytes, "shared memory layout");
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: true when the phase completed, false when the limit ran out
+// or another thread of the CTA aborted (then the caller unwinds).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit,
+                                          volatile uint32_t *abort_flag) {
+    for (uint64_t i = 0; i < limit; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+    }
+    *abort_flag = 1u;
+    atomicOr(&g_device_error_word, 1u);
+    return false;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (stride byte offset), leading byte offset unused (1),
+// descriptor version 1.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1u << 16;                 // leading byte offset (16 B units)
+    d |= (uint64_t)(1024u >> 4) << 32;       // stride byte offset
+    d |= (uint64_t)1u << 46;                 // version
+    d |= (uint64_t)2u << 61;                 // 128-byte swizzle
+    return d;
+}
+
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(kIdesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {"
+        "%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+        "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {"
+        "%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Natural-order bf16 pair (k = 2i, 2i+1) of a packed code word: byte i of
+// `w` holds q_{2i} in its low nibble, byte i of `w >> 4` holds q_{2i+1}.
+__device__ __forceinline__ uint32_t dequant_pair_nat(uint32_t w, uint32_t w4, int i,
+                                                     uint32_t s2, uint32_t z2) {
+    const uint32_t sel = (uint32_t)i | ((uint32_t)(4 + i) << 8);
+    const uint32_t t = dev::prmt(w, w4, sel);
+    const uint32_t x = (t & 0x000F000Fu) | 0x43004300u;          // bf16(128 + q)
+    return dev::bf16x2_mul(dev::bf16x2_sub(x, z2), s2);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+w4a16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
+                   const __grid_constant__ CUtensorMap pack_map,
+                   const uint16_t *__restrict__ scales, const uint8_t *__restrict__ zeros,
+                   int M, int N, int K, int group_size, uint16_t *__restrict__ y,
+                   uint64_t wait_limit) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + SmemLayout::abort_flag);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SmemLayout::tmem_slot);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * kTileN;
+    const int m0 = blockIdx.y * kTileM;
+    const int KT = K / kTileK;
+
+    auto full_bar = [&](int s) { return sbase + SmemLayout::full + 8 * s; };
+    auto empty_bar = [&](int s) { return sbase + SmemLayout::empty + 8 * s; };
+    auto afull_bar = [&](int s) { return sbase + SmemLayout::afull + 8 * s; };
+    const uint32_t accum_bar = sbase + SmemLayout::accum;
+    const uint32_t drain_bar = sbase + SmemLayout::drain;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1 + 4);     // MMA commit + 4 dequant warps
+            mbar_init(afull_bar(s), 4);         // 4 dequant warps
+        }
+        mbar_init(accum_bar, 1);
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&act_map)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&pack_map)) : "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const uint32_t tmem_acc = tmem_base;                // columns [0, 256)
+    const uint32_t tmem_a = tmem_base + kAccCols;       // A slots: kStages x 32 columns
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            int issued_round[kStages];
+            for (int s = 0; s < kStages; ++s) issued_round[s] = -1;
+            for (int kt = 0; kt < KT; ++kt) {
+                const int s = kt % kStages, r = kt / kStages;
+                if (r > 0 && !mbar_wait(empty_bar(s), (r - 1) & 1, wait_limit, abort_flag)) break;
+                mbar_arrive_expect_tx(full_bar(s), kActStageBytes + kPackStageBytes);
+                tma_load_2d(sbase + SmemLayout::act + s * kActStageBytes, &act_map, kt * kTileK,
+                            m0, full_bar(s));
+                tma_load_2d(sbase + SmemLayout::pack + s * kPackStageBytes, &pack_map,
+                            kt * (kTileK / 2), n0, full_bar(s));
+                issued_round[s] = r;
+            }
+            // drain: every issued copy must have landed before the CTA may exit
+            for (int s = 0; s < kStages; ++s)
+                if (issued_round[s] >= 0) {
+                    volatile uint32_t never = 0;
+                    mbar_wait(full_bar(s), issued_round[s] & 1, wait_limit, &never);
+                }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            bool ok = true;
+            for (int kt = 0; kt < KT && ok; ++kt) {
+                const int s = kt % kStages, r = kt / kStages;
+                ok = mbar_wait(full_bar(s), r & 1, wait_limit, abort_flag) &&
+                     mbar_wait(afull_bar(s), r & 1, wait_limit, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t act_addr = sbase + SmemLayout::act + s * kActStageBytes;
+#pragma unroll
+                for (int j = 0; j < kTileK / 16; ++j) {
+                    mma_ts(tmem_acc, tmem_a + s * kACols + j * 8,
+                           smem_desc_sw128(act_addr + j * 32), (kt > 0 || j > 0) ? 1u : 0u);
+                }
+                mma_commit(empty_bar(s));
+            }
+            if (ok) {
+                mma_commit(accum_bar);
+            } else {
+                // let every issued MMA finish before tensor memory is released
+                mma_commit(drain_bar);
+                volatile uint32_t never = 0;
+                mbar_wait(drain_bar, 0, wait_limit, &never);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------- dequantize + epilogue (warps 2..5) ----------------
+        const int quarter = warp & 3;                // tensor-memory lane quarter
+        const int row_local = quarter * 32 + lane;
+        const int n = n0 + row_local;
+        const bool valid = n < N;
+        const int gpr = K / group_size;
+        const uint16_t *srow = scales + (int64_t)(valid ? n : 0) * gpr;
+        const uint8_t *zrow = zeros + (int64_t)(valid ? n : 0) * gpr;
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        bool ok = true;
+        uint32_t s_next = valid ? __ldg(&srow[0]) : 0u;
+        uint32_t z_next = valid ? __ldg(&zrow[0]) : 0u;
+        for (int kt = 0; kt < KT; ++kt) {
+            const int s = kt % kStages, r = kt / kStages;
+            const uint32_t sb = s_next, zb = z_next;
+            if (kt + 1 < KT && valid) {
+                const int gi = ((kt + 1) * kTileK) / group_size;
+                s_next = __ldg(&srow[gi]);
+                z_next = __ldg(&zrow[gi]);
+            }
+            if (!mbar_wait(full_bar(s), r & 1, wait_limit, abort_flag)) { ok = false; break; }
+            const uint4 *src = reinterpret_cast<const uint4 *>(
+                smem + SmemLayout::pack + s * kPackStageBytes + row_local * (kTileK / 2));
+            const uint4 p0 = src[0], p1 = src[1];
+            const uint32_t s2 = sb | (sb << 16);
+            const uint32_t z2 = (0x4300u + zb) * 0x00010001u;
+            const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+            uint32_t a[32];
+#pragma unroll
+            for (int wi = 0; wi < 8; ++wi) {
+                const uint32_t w = words[wi], w4 = w >> 4;
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    a[wi * 4 + i] = valid ? dequant_pair_nat(w, w4, i, s2, z2) : 0u;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty_bar(s));     // packed stage consumed
+            tmem_st_x32(tmem_a + lane_base + s * kACols, a);
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(afull_bar(s));
+        }
+        if (ok && mbar_wait(accum_bar, 0, wait_limit, abort_flag)) {
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < kTileM / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld_x32(tmem_acc + lane_base + c * 32, v);
+                if (valid) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int m = m0 + c * 32 + j;
+                        if (m < M)
+                            y[(int64_t)m * N + n] =
+                                (uint16_t)dev::f32_to_bf16_rne(__uint_as_float(v[j]));
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host: tensor maps through the driver entry point (no link-time libcuda).
+// ---------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner,
+                 uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                 CUtensorMapSwizzle swz) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t elem[2] = {1, 1};
+    return fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, elem,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+size_t gemm_workspace_bytes(int64_t, int64_t, int64_t) { return 0; }
+
+qz_status launch_w4a16_gemm(const void *a, const void *codes, const void *scales,
+                            const void *zeros, int64_t M, int64_t N, int64_t K,
+                            int64_t group_size, void *y, void *, cudaStream_t st) {
+    CUtensorMap act_map, pack_map;
+    if (!make_map_2d(&act_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a, (uint64_t)K, (uint64_t)M,
+                     (uint64_t)K * 2, kTileK, kTileM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&pack_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, (uint64_t)K / 2,
+                     (uint64_t)N, (uint64_t)K / 2, kTileK / 2, kTileN,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
+        return QZ_ERR_CUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return QZ_ERR_CUDA;
+    static std::once_flag attr_once[64];
+    if (dev >= 0 && dev < 64)
+        std::call_once(attr_once[dev], [] {
+            cudaFuncSetAttribute(w4a16_gemm_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kSmemBytes);
+        });
+    dim3 grid((unsigned)ceil_div(N, kTileN), (unsigned)ceil_div(M, kTileM));
+    w4a16_gemm_tcgen05<<<grid, kThreads, kSmemBytes, st>>>(
+        act_map, pack_map, static_cast<const uint16_t *>(scales),
+        static_cast<const uint8_t *>(zeros), (int)M, (int)N, (int)K, (int)group_size,
+        static_cast<uint16_t *>(y), device_wait_limit());
+    return launch_status();
+}
+
+}  // namespace qz
+
+extern "C" QZ_API qz_status qz_device_status(void) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return QZ_ERR_CUDA;
+    unsigned int word = 0;
+    if (cudaMemcpyFromSymbol(&word, qz::g_device_error_word, sizeof word) != cudaSuccess)
+        return QZ_ERR_CUDA;
+    if (word == 0) return QZ_OK;
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(qz::g_device_error_word, &zero, sizeof zero) != cudaSuccess)
+        return QZ_ERR_CUDA;
+    return QZ_ERR_DEVICE_TIMEOUT;
+}

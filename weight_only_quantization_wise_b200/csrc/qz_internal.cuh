@@ -1,0 +1,162 @@
+// qz_internal.cuh -- internal helpers shared by the libqz CUDA sources.
+// Not installed; the public interface is include/qz.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "qz.h"
+
+namespace qz {
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+
+// Number of SMs of the device the grids are sized for.  Sizing (and therefore
+// workspace sizes) uses this fixed B200 figure so that qz_workspace_bytes is
+// a pure function of the shapes.
+constexpr int kSmCount = 148;
+
+inline bool aligned(const void *p, size_t a) {
+    return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+inline qz_status launch_status() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? QZ_OK : QZ_ERR_CUDA;
+}
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Code range of a format (see qz.h).
+inline void code_range(int bits, int symmetric, int *qmin, int *qmax) {
+    if (symmetric) {
+        *qmax = (1 << (bits - 1)) - 1;
+        *qmin = -*qmax;
+    } else if (bits == 4) {
+        *qmin = 0;
+        *qmax = 15;
+    } else {
+        *qmin = -128;
+        *qmax = 127;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Launchers (defined in the .cu files; arguments already validated)
+// ---------------------------------------------------------------------------
+
+qz_status launch_quantize_pack(const void *w, int64_t N, int64_t K, int bits,
+                               int symmetric, int64_t group_size, void *codes,
+                               void *scales, void *zeros, void *workspace,
+                               cudaStream_t stream);
+size_t quantize_workspace_bytes(int64_t group_size);
+
+qz_status launch_dequantize(const void *codes, const void *scales, const void *zeros,
+                            int64_t N, int64_t K, int bits, int symmetric,
+                            int64_t group_size, void *w_hat, cudaStream_t stream);
+
+// GEMV split-K plan: number of K splits and workspace bytes.
+struct GemvPlan {
+    int splits;
+    int64_t tiles;        // 16-row tiles
+    size_t partial_bytes; // fp32 partials [splits][M][N]
+    size_t counter_bytes; // uint32 per tile
+    size_t total_bytes;
+};
+GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K);
+
+qz_status launch_w4a16_gemv(const void *a, const void *codes, const void *scales,
+                            const void *zeros, int64_t M, int64_t N, int64_t K,
+                            int64_t group_size, void *y, void *workspace,
+                            const GemvPlan &plan, cudaStream_t stream);
+qz_status launch_w8a16_gemv(const void *a, const void *codes, const void *scales,
+                            int64_t M, int64_t N, int64_t K, void *y, void *workspace,
+                            const GemvPlan &plan, cudaStream_t stream);
+
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+qz_status launch_w4a16_gemm(const void *a, const void *codes, const void *scales,
+                            const void *zeros, int64_t M, int64_t N, int64_t K,
+                            int64_t group_size, void *y, void *workspace,
+                            cudaStream_t stream);
+
+uint64_t device_wait_limit();
+
+}  // namespace qz
+
+// ---------------------------------------------------------------------------
+// Device side
+// ---------------------------------------------------------------------------
+#ifdef __CUDACC__
+namespace qz {
+namespace dev {
+
+// bf16 (as 16 raw bits) widened to fp32: exact.
+__device__ __forceinline__ float bf16_lo(uint32_t pair) { return __uint_as_float(pair << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t pair) { return __uint_as_float(pair & 0xFFFF0000u); }
+
+// fp32 -> bf16 bits, round to nearest even (hardware conversion).
+__device__ __forceinline__ uint32_t f32_to_bf16_rne(float x) {
+    uint16_t r;
+    asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(x));
+    return r;
+}
+
+// Two fp32 -> packed bf16x2 (lo in bits 0..15), round to nearest even.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// fp32 scale -> bf16 bits rounded toward +inf (S >= 0).
+__device__ __forceinline__ uint32_t bf16_round_up_bits(float s) {
+    uint32_t b = __float_as_uint(s);
+    uint32_t kept = b & 0xFFFF0000u;
+    if (b & 0x0000FFFFu) kept += 0x00010000u;
+    return kept >> 16;
+}
+
+// Packed bf16x2 arithmetic, one IEEE rounding to nearest even per lane.
+__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// Streaming 16-byte global load that does not allocate in L1.
+__device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// Warp-level tensor-core MMA: D(16x8 f32) += A(16x16 bf16, row) * B(16x8 bf16, col).
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Byte permute.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+}  // namespace dev
+}  // namespace qz
+#endif

@@ -1,0 +1,641 @@
+"""Benchmark of the weight-only quantization hot path on B200 GPUs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of every hot-path row over the 7B-class decode layer set
+(N, K) = (4096, 4096), (11008, 4096), (4096, 11008):
+  quantize_pack int4 asymmetric group-128   (3 launches)
+  quantize_pack int8 symmetric per-channel  (3 launches)
+  dequantize int4                           (3 launches)
+  W4A16 decode GEMV, M = 1                  (3 launches)
+  W8A16 decode GEMV, M = 1                  (3 launches)
+  W4A16 prefill GEMM, M = 2048 tokens       (3 launches)
+Every input is resident in HBM and rotates over ROT copies (ROT x the packed
+layer set is far larger than the 126 MB L2), so each part reads cold weights.
+Each part of each rotation is a captured CUDA graph; CUDA events on the
+launching stream bracket the parts.  `value` is the headline of the metric:
+W4A16 decode GEMV GB/s (algorithmic bytes / GEMV time), aggregated over all
+ranks.  The other parts, the roofline of every kernel, the configurations
+that are not part of the step (70B decode shapes, the 2048 x 8192 x 8192
+prefill GEMM, the 7.8e9-parameter bulk quantization), an end-to-end number
+through the public Python API with host buffers, and the CPU oracle baseline
+are reported in the same JSON line.
+
+With --impl reference the CPU oracle is the reference arm: it runs the same
+decode step (dequantize + fp64 matmul) on a row sample of the same layers.
+
+Multi-GPU: the path does not shard (one GPU per problem); N ranks run N
+independent replicas, launched by torchrun; times are the max over ranks.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+METRIC = "W4A16 decode GEMV GB/s (% of HBM peak); prefill GEMM TFLOP/s; quantize GB/s"
+LAYERS = synthetic.DECODE_7B
+PREFILL_M = synthetic.PREFILL["M"]
+ROT = 8
+GROUP = 128
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work per launch
+# ---------------------------------------------------------------------------
+
+def w4_gemv_bytes(M, N, K, g=GROUP):
+    return N * K // 2 + N * (K // g) * 3 + 2 * M * K + 2 * M * N
+
+
+def w8_gemv_bytes(M, N, K):
+    return N * K + 2 * N + 2 * M * K + 2 * M * N
+
+
+def quant_int4_bytes(N, K, g=GROUP):
+    return 2 * N * K + N * K // 2 + N * (K // g) * 3
+
+
+def quant_int8_bytes(N, K):
+    return 2 * N * K + N * K + 2 * N
+
+
+def dequant_int4_bytes(N, K, g=GROUP):
+    return quant_int4_bytes(N, K, g)
+
+
+def gemm_flops(M, N, K):
+    return 2 * M * N * K
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+            "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def ncu_traffic():
+    """Per-launch DRAM traffic from the committed ncu summary, keyed by kernel,
+    valid only while the kernel source is unchanged since the capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return {}
+    import hashlib
+    with open(path) as f:
+        data = json.load(f)
+    out = {}
+    for part, rec in data.get("kernels", {}).items():
+        src = os.path.join(ROOT, rec["source"])
+        if not os.path.exists(src):
+            continue
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if h == rec.get("source_sha256_16"):
+            out[part] = rec
+    return out
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    def __init__(self):
+        self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={CLOCK_QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self, device_index):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.tmp.flush()
+        self.tmp.seek(0)
+        rows = [r.split(",") for r in self.tmp.read().strip().splitlines() if r.strip()]
+        os.unlink(self.tmp.name)
+        rows = [[c.strip() for c in r] for r in rows if len(r) >= 9]
+        mine = [r for r in rows if r[0] == str(device_index)] or rows
+        if not mine:
+            return None
+        sm = [float(r[1]) for r in mine if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in mine if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in mine for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(mine)}
+
+
+# ---------------------------------------------------------------------------
+# workload
+# ---------------------------------------------------------------------------
+
+class LayerSet:
+    """Resident inputs/outputs of one step, ROT rotating copies of every input."""
+
+    def __init__(self, qz, dev):
+        self.qz, self.dev = qz, dev
+        self.w, self.c4, self.s4, self.z4, self.c8, self.s8 = ([] for _ in range(6))
+        for p in range(ROT):
+            w_p, c4_p, s4_p, z4_p, c8_p, s8_p = [], [], [], [], [], []
+            for li, (N, K) in enumerate(LAYERS):
+                if p == 0:
+                    w = synthetic.weights(N, K, sigma=0.02, seed=1 + li, device=dev)
+                else:
+                    w = self.w[0][li].clone()
+                c4, s4, z4 = qz.qz_quantize_pack(w, 4, False, GROUP)
+                c8, s8, _ = qz.qz_quantize_pack(w, 8, True, K)
+                w_p.append(w); c4_p.append(c4); s4_p.append(s4); z4_p.append(z4)
+                c8_p.append(c8); s8_p.append(s8)
+            self.w.append(w_p); self.c4.append(c4_p); self.s4.append(s4_p)
+            self.z4.append(z4_p); self.c8.append(c8_p); self.s8.append(s8_p)
+        # outputs (written every step) and activations
+        self.q4 = [qz.qz_quantize_pack(self.w[0][li], 4, False, GROUP) for li in range(len(LAYERS))]
+        self.q8 = [qz.qz_quantize_pack(self.w[0][li], 8, True, K)
+                   for li, (N, K) in enumerate(LAYERS)]
+        self.deq = [torch.empty((N, K), dtype=torch.bfloat16, device=dev) for N, K in LAYERS]
+        self.a1 = [synthetic.activations(1, K, seed=50 + li, device=dev)
+                   for li, (N, K) in enumerate(LAYERS)]
+        self.ap = [synthetic.activations(PREFILL_M, K, seed=60 + li, device=dev)
+                   for li, (N, K) in enumerate(LAYERS)]
+        self.y4 = [torch.empty((1, N), dtype=torch.bfloat16, device=dev) for N, K in LAYERS]
+        self.y8 = [torch.empty((1, N), dtype=torch.bfloat16, device=dev) for N, K in LAYERS]
+        self.yg = [torch.empty((PREFILL_M, N), dtype=torch.bfloat16, device=dev) for N, K in LAYERS]
+        ws = 256
+        for N, K in LAYERS:
+            ws = max(ws, qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMV, 1, N, K, GROUP),
+                     qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMV, 1, N, K, K),
+                     qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMM, PREFILL_M, N, K, GROUP))
+        self.ws = torch.zeros(ws, dtype=torch.uint8, device=dev)
+
+    # each part issues its launches for rotation p on the current stream
+    def quant4(self, p):
+        for li, (N, K) in enumerate(LAYERS):
+            c, s, z = self.q4[li]
+            self.qz.qz_quantize_pack(self.w[p][li], 4, False, GROUP, codes=c, scales=s, zeros=z)
+
+    def quant8(self, p):
+        for li, (N, K) in enumerate(LAYERS):
+            c, s, _ = self.q8[li]
+            self.qz.qz_quantize_pack(self.w[p][li], 8, True, K, codes=c, scales=s)
+
+    def dequant(self, p):
+        for li, (N, K) in enumerate(LAYERS):
+            self.qz.qz_dequantize(self.c4[p][li], self.s4[p][li], self.z4[p][li], N, K, 4, False,
+                                  GROUP, out=self.deq[li])
+
+    def gemv4(self, p):
+        for li, (N, K) in enumerate(LAYERS):
+            self.qz.qz_w4a16_gemv(self.a1[li], self.c4[p][li], self.s4[p][li], self.z4[p][li], N,
+                                  K, GROUP, y=self.y4[li], workspace=self.ws)
+
+    def gemv8(self, p):
+        for li, (N, K) in enumerate(LAYERS):
+            self.qz.qz_w8a16_gemv(self.a1[li], self.c8[p][li], self.s8[p][li], N, K,
+                                  y=self.y8[li], workspace=self.ws)
+
+    def gemm(self, p):
+        for li, (N, K) in enumerate(LAYERS):
+            self.qz.qz_w4a16_gemm(self.ap[li], self.c4[p][li], self.s4[p][li], self.z4[p][li], N,
+                                  K, GROUP, y=self.yg[li], workspace=self.ws)
+
+
+PARTS = [  # name, method, unit, work per step, bound
+    ("quantize_pack_int4_g128", "quant4", "GB/s",
+     sum(quant_int4_bytes(N, K) for N, K in LAYERS), "hbm"),
+    ("quantize_pack_int8_per_channel", "quant8", "GB/s",
+     sum(quant_int8_bytes(N, K) for N, K in LAYERS), "hbm"),
+    ("dequantize_int4", "dequant", "GB/s",
+     sum(dequant_int4_bytes(N, K) for N, K in LAYERS), "hbm"),
+    ("w4a16_gemv_m1", "gemv4", "GB/s", sum(w4_gemv_bytes(1, N, K) for N, K in LAYERS), "hbm"),
+    ("w8a16_gemv_m1", "gemv8", "GB/s", sum(w8_gemv_bytes(1, N, K) for N, K in LAYERS), "hbm"),
+    ("w4a16_gemm_prefill_m2048", "gemm", "TFLOP/s",
+     sum(gemm_flops(PREFILL_M, N, K) for N, K in LAYERS), "tensor"),
+]
+LAUNCHES_PER_STEP = 3 * len(PARTS)
+
+
+def capture(fn, stream):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    return g
+
+
+def rate(work, ms, unit):
+    if unit == "TFLOP/s":
+        return work / (ms * 1e-3) / 1e12
+    return work / (ms * 1e-3) / 1e9
+
+
+def roofline_obj(part, work, ms_per_launch_set, launches, bound, pk, traffic, sustained):
+    achieved = rate(work, ms_per_launch_set, "TFLOP/s" if bound == "tensor" else "GB/s")
+    if bound == "tensor":
+        peak = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
+        unit = "TFLOP/s"
+    else:
+        peak, unit = pk["hbm_gbs"], "GB/s"
+    t = traffic.get(part)
+    return {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+            "frac": round(achieved / peak, 4),
+            "peak_kind": ("sustained" if (bound == "tensor" and sustained) else "burst")
+            + (" of measured" if pk["source"] == "measured" else " of fallback"),
+            "traffic": (t["dram_bytes_per_launch_set"] if t else None),
+            "algorithmic": work, "launches": launches}
+
+
+def run_extras(qz, dev, pk, stream):
+    """Configurations outside the step, each timed with CUDA events on graphs."""
+    out = {}
+
+    def time_graph(g, reps=20, warm=3):
+        for _ in range(warm):
+            g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    with torch.cuda.stream(stream):
+        # prefill GEMM, M = 2048, N = K = 8192
+        cfg = synthetic.PREFILL
+        M, N, K = cfg["M"], cfg["N"], cfg["K"]
+        w = synthetic.weights(N, K, sigma=cfg["sigma"], seed=cfg["seed"], device=dev)
+        a = synthetic.activations(M, K, seed=cfg["seed"] + 1000, device=dev)
+        c, s, z = qz.qz_quantize_pack(w, 4, False, GROUP)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        qz.qz_w4a16_gemm(a, c, s, z, N, K, GROUP, y=y)
+        g = capture(lambda: qz.qz_w4a16_gemm(a, c, s, z, N, K, GROUP, y=y), stream)
+        ms = time_graph(g)
+        tf = gemm_flops(M, N, K) / (ms * 1e-3) / 1e12
+        out["prefill_gemm_2048x8192x8192"] = {
+            "ms": round(ms, 4), "TFLOP/s": round(tf, 1),
+            "frac_of_burst": round(tf / pk["bf16_tflops"], 4),
+            "frac_of_sustained": round(tf / pk["bf16_tflops_sustained"], 4)}
+        # cuBLAS bf16 GEMM of the same shape, as the practical ceiling
+        wb = qz.qz_dequantize(c, s, z, N, K, 4, False, GROUP)
+        yb = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        torch.matmul(a, wb.t(), out=yb)
+        gb = capture(lambda: torch.matmul(a, wb.t(), out=yb), stream)
+        msb = time_graph(gb)
+        out["prefill_gemm_2048x8192x8192"]["cublas_bf16_same_shape_TFLOP/s"] = round(
+            gemm_flops(M, N, K) / (msb * 1e-3) / 1e12, 1)
+        del w, a, c, s, z, y, wb, yb, g, gb
+
+        # 70B decode shapes, W4 and W8, M in {1, 4, 8, 16}
+        d70 = {}
+        for li, (N, K) in enumerate(synthetic.DECODE_70B):
+            w = synthetic.weights(N, K, sigma=0.015, seed=4 + li, device=dev)
+            packs4 = [qz.qz_quantize_pack(w if r == 0 else w.clone(), 4, False, GROUP) for r in range(2)]
+            packs8 = [qz.qz_quantize_pack(w if r == 0 else w.clone(), 8, True, K) for r in range(2)]
+            del w
+            for M in synthetic.DECODE_70B_M:
+                a = synthetic.activations(M, K, seed=M, device=dev)
+                y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+                ws = torch.zeros(max(256, qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMV, M, N, K, GROUP)),
+                                 dtype=torch.uint8, device=dev)
+
+                def f4():
+                    for c, s, z in packs4:
+                        qz.qz_w4a16_gemv(a, c, s, z, N, K, GROUP, y=y, workspace=ws)
+
+                def f8():
+                    for c, s, _ in packs8:
+                        qz.qz_w8a16_gemv(a, c, s, N, K, y=y, workspace=ws)
+
+                f4(); f8()
+                ms4 = time_graph(capture(f4, stream)) / 2
+                ms8 = time_graph(capture(f8, stream)) / 2
+                b4, b8 = w4_gemv_bytes(M, N, K), w8_gemv_bytes(M, N, K)
+                d70[f"N{N}_K{K}_M{M}"] = {
+                    "w4_us": round(ms4 * 1e3, 2), "w4_GB/s": round(b4 / ms4 / 1e6, 1),
+                    "w4_frac_hbm": round(b4 / ms4 / 1e6 / pk["hbm_gbs"], 4),
+                    "w8_us": round(ms8 * 1e3, 2), "w8_GB/s": round(b8 / ms8 / 1e6, 1),
+                    "w8_frac_hbm": round(b8 / ms8 / 1e6 / pk["hbm_gbs"], 4)}
+            del packs4, packs8
+        out["decode_70b"] = d70
+
+        # bulk quantization: 32 layer sets, 7.785e9 parameters
+        total_params, b4, b8 = 0, 0, 0
+        for N, K in synthetic.BULK_LAYER_SET:
+            total_params += N * K
+            b4 += quant_int4_bytes(N, K)
+            b8 += quant_int8_bytes(N, K)
+        sets = synthetic.BULK_SETS
+        layers = []
+        for si in range(sets):
+            for li, (N, K) in enumerate(synthetic.BULK_LAYER_SET):
+                layers.append((N, K, synthetic.weights(N, K, sigma=0.02, seed=100 + si * 16 + li,
+                                                       device=dev)))
+        outs4, outs8 = {}, {}
+        for N, K in set(synthetic.BULK_LAYER_SET):
+            outs4[(N, K)] = (torch.empty((N, K // 2), dtype=torch.uint8, device=dev),
+                             torch.empty((N, K // GROUP), dtype=torch.bfloat16, device=dev),
+                             torch.empty((N, K // GROUP), dtype=torch.uint8, device=dev))
+            outs8[(N, K)] = (torch.empty((N, K), dtype=torch.uint8, device=dev),
+                             torch.empty((N, 1), dtype=torch.bfloat16, device=dev), None)
+
+        def bulk4():
+            for N, K, w in layers:
+                c, s, z = outs4[(N, K)]
+                qz.qz_quantize_pack(w, 4, False, GROUP, codes=c, scales=s, zeros=z)
+
+        def bulk8():
+            for N, K, w in layers:
+                c, s, _ = outs8[(N, K)]
+                qz.qz_quantize_pack(w, 8, True, K, codes=c, scales=s)
+
+        bulk4(); bulk8()
+        ms4 = time_graph(capture(bulk4, stream), reps=3, warm=1)
+        ms8 = time_graph(capture(bulk8, stream), reps=3, warm=1)
+        out["bulk_quantize"] = {
+            "params": total_params * sets,
+            "int4_g128_ms": round(ms4, 3), "int4_g128_GB/s": round(b4 * sets / ms4 / 1e6, 1),
+            "int4_frac_hbm": round(b4 * sets / ms4 / 1e6 / pk["hbm_gbs"], 4),
+            "int8_pc_ms": round(ms8, 3), "int8_pc_GB/s": round(b8 * sets / ms8 / 1e6, 1),
+            "int8_frac_hbm": round(b8 * sets / ms8 / 1e6 / pk["hbm_gbs"], 4)}
+        del layers, outs4, outs8
+    torch.cuda.empty_cache()
+    return out
+
+
+def cpu_baseline(target_s=10.0):
+    """The oracle, as it stands, on this host's cores: the decode step
+    (dequantize + fp64 matmul, M = 1) over the 7B-class layer set."""
+    import oracle
+    threads = oracle.max_threads()
+    oracle.set_threads(threads)
+    prepared = []
+    for li, (N, K) in enumerate(LAYERS):
+        wb = synthetic.bf16_bits(synthetic.weights(N, K, sigma=0.02, seed=1 + li))
+        ab = synthetic.bf16_bits(synthetic.activations(1, K, seed=50 + li))
+        prepared.append((N, K, oracle.quantize_pack(wb, 4, False, GROUP), ab))
+    nbytes = sum(w4_gemv_bytes(1, N, K) for N, K in LAYERS)
+    passes, t0 = 0, time.perf_counter()
+    while True:
+        for N, K, (c, s, z), ab in prepared:
+            w_hat = oracle.dequantize(c, s, z, N, K, 4, False, GROUP)
+            oracle.matmul_f64(ab, w_hat)
+        passes += 1
+        el = time.perf_counter() - t0
+        if el >= target_s:
+            break
+    return {"value": round(nbytes * passes / el / 1e9, 4), "unit": "GB/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{passes} full decode passes (dequantize + fp64 matmul, M=1) over the three "
+                      f"7B-class layers, {el:.1f} s"}
+
+
+def run_reference(args):
+    """CPU oracle as the reference arm: each step is the oracle's decode pass
+    over a row sample (1/16 of the rows) of the three 7B-class layers."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    threads = oracle.max_threads()
+    oracle.set_threads(threads)
+    sample = []
+    nbytes = 0
+    for li, (N, K) in enumerate(LAYERS):
+        n = N // 16
+        wb = synthetic.bf16_bits(synthetic.weights(N, K, sigma=0.02, seed=1 + li))[:n]
+        ab = synthetic.bf16_bits(synthetic.activations(1, K, seed=50 + li))
+        sample.append((n, K, oracle.quantize_pack(wb, 4, False, GROUP), ab))
+        nbytes += w4_gemv_bytes(1, n, K)
+
+    def step():
+        for n, K, (c, s, z), ab in sample:
+            oracle.matmul_f64(ab, oracle.dequantize(c, s, z, n, K, 4, False, GROUP))
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    v = nbytes * args.steps / el / 1e9
+    line = {"metric": METRIC, "value": round(v, 4), "unit": "GB/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(el / args.steps * 1e3, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_obj(),
+            "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": threads,
+                             "kind": "oracle",
+                             "sample": "rows 0..N/16 of each of the three 7B-class layers per step"},
+            "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_obj():
+    return {"workload": "7B-class decode layer set (N,K)=(4096,4096),(11008,4096),(4096,11008): "
+                        "int4 asym group-128 + int8 sym per-channel quantize_pack, int4 dequantize, "
+                        "W4A16/W8A16 decode GEMV at M=1, W4A16 prefill GEMM at M=2048",
+            "weights": "bf16 ~N(0,0.02) + 0.1% x20 outliers, seeds 1..3",
+            "activations": "bf16 ~N(0,1)",
+            "l2": f"inputs rotate over {ROT} resident copies (packed W4 set {ROT} x 56 MB > L2)",
+            "value_is": "w4a16_gemv_m1 part (algorithmic bytes / event-timed GEMV time)",
+            "parallelism": "replicas"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    import weight_only_quantization_wise_b200 as qz
+    pk = peaks()
+    stream = torch.cuda.Stream(device=dev)
+    ls = LayerSet(qz, dev)
+    torch.cuda.synchronize()
+
+    # one graph per (part, rotation); run each part once eagerly first
+    graphs = {}
+    with torch.cuda.stream(stream):
+        for name, meth, *_ in PARTS:
+            fn = getattr(ls, meth)
+            fn(0)
+            for p in range(ROT):
+                graphs[(name, p)] = capture(lambda fn=fn, p=p: fn(p), stream)
+    torch.cuda.synchronize()
+    assert qz.qz_device_status() == 0
+
+    npart = len(PARTS)
+
+    def run_steps(k, events=None, start=0):
+        for i in range(k):
+            p = (start + i) % ROT
+            for j, (name, *_r) in enumerate(PARTS):
+                if events is not None:
+                    events[i][j][0].record(stream)
+                graphs[(name, p)].replay()
+                if events is not None:
+                    events[i][j][1].record(stream)
+
+    with torch.cuda.stream(stream):
+        run_steps(args.warmup)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(npart)] for _ in range(args.steps)]
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler()
+    sampler.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    with torch.cuda.stream(stream):
+        e_start.record(stream)
+        run_steps(args.steps, ev, start=args.warmup)
+        e_end.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop(local)
+    total_ms = e_start.elapsed_time(e_end)
+    part_ms = [sum(ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(args.steps)) / args.steps
+               for j in range(npart)]
+    assert qz.qz_device_status() == 0
+
+    # max over ranks
+    t = torch.tensor([total_ms] + part_ms, dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, part_ms = float(t[0]), [float(x) for x in t[1:]]
+
+    traffic = ncu_traffic()
+    parts, roofs = {}, {}
+    for (name, meth, unit, work, bound), ms in zip(PARTS, part_ms):
+        parts[name] = {"ms": round(ms, 5), "value": round(rate(work, ms, unit), 2), "unit": unit,
+                       "launches": 3}
+        roofs[name] = roofline_obj(name, work, ms, 3, bound, pk, traffic, sustained=True)
+    dominant = max(zip(PARTS, part_ms), key=lambda x: x[1])[0][0]
+    gemv_idx = [p[0] for p in PARTS].index("w4a16_gemv_m1")
+    gemv_bytes = PARTS[gemv_idx][3]
+    value = gemv_bytes * world / (part_ms[gemv_idx] * 1e-3) / 1e9
+
+    # end to end through the public API, host buffers, per decode step
+    e2e = None
+    host_a = [x.cpu().pin_memory() for x in ls.a1]
+    host_y = [torch.empty((1, N), dtype=torch.bfloat16).pin_memory() for N, K in LAYERS]
+    dev_a = [torch.empty_like(x) for x in ls.a1]
+    dev_y = [torch.empty((1, N), dtype=torch.bfloat16, device=dev) for N, K in LAYERS]
+    h2d = sum(x.numel() * 2 for x in host_a)
+    d2h = sum(x.numel() * 2 for x in host_y)
+
+    def e2e_step(p):
+        with torch.cuda.stream(stream):
+            for li, (N, K) in enumerate(LAYERS):
+                dev_a[li].copy_(host_a[li], non_blocking=True)
+                qz.qz_w4a16_gemv(dev_a[li], ls.c4[p][li], ls.s4[p][li], ls.z4[p][li], N, K, GROUP,
+                                 y=dev_y[li], workspace=ls.ws)
+                host_y[li].copy_(dev_y[li], non_blocking=True)
+        stream.synchronize()
+
+    for i in range(args.warmup):
+        e2e_step(i % ROT)
+    if dist:
+        dist.barrier()
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        e2e_step(i % ROT)
+    el = torch.tensor([time.perf_counter() - t0], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(el, op=dist.ReduceOp.MAX)
+    e2e = {"value": round(gemv_bytes * world * args.steps / float(el[0]) / 1e9, 3), "unit": "GB/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "note": "decode step through qz_w4a16_gemv with pinned host activations in and "
+                   "outputs out, one host sync per step; weights resident"}
+
+    extras = None
+    if rank == 0 and not args.no_extras:
+        del graphs
+        extras = run_extras(qz, dev, pk, stream)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline()
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total_ms / args.steps, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "weights_dtype": "int4 (int8 for the W8A16 part)", "data": "synthetic",
+            "config": config_obj(),
+            "roofline": roofs[dominant] | {"kernel": dominant},
+            "rooflines": roofs, "parts": parts,
+            "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "clocks": clocks, "peaks": pk, "extra": extras,
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

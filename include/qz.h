@@ -181,8 +181,8 @@ QZ_API qz_status qz_w8a16_gemv(const void *a, const void *codes, const void *sca
                         size_t workspace_bytes, void *stream);
 
 /*
- * Device-side wait bound used by kernels that wait on mbarriers (the GEMM).
- * `limit` counts polling iterations of one wait; 0 restores the default.
+ * Device-side wait bound used by kernels that wait on mbarriers (the GEMM),
+ * in nanoseconds of wall time per wait; 0 restores the default (2 s).
  * Not part of the method: a safety bound so that a broken pipeline returns an
  * error instead of hanging the GPU.  Host-only setter, applies to later calls.
  */

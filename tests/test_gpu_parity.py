@@ -335,3 +335,86 @@ def test_bulk_quantization_stack(dev):
             total += N * K
             del w
     assert total == 7_784_628_224
+
+
+# ---------------------------------------------------------------------------
+# Prefill GEMM (tcgen05)
+# ---------------------------------------------------------------------------
+
+GEMM_CASES = [  # (M, N, K, g)
+    (17, 128, 128, 128), (100, 200, 256, 64), (256, 128, 1024, 128),
+    (300, 1000, 1024, 128), (512, 384, 2048, 256), (257, 130, 640, 128),
+]
+
+
+@pytest.mark.parametrize("M,N,K,g", GEMM_CASES)
+def test_w4a16_gemm_tolerance(dev, M, N, K, g):
+    w = synthetic.weights(N, K, sigma=0.02, seed=M + N + K)
+    a = synthetic.activations(M, K, seed=M * 5)
+    c, s, z, w_hat = oracle_w4(u16(w), g)
+    y_ref, abs_ref = oracle.matmul_f64(u16(a), w_hat)
+    y = qz.qz_w4a16_gemm(a.to(dev), to_dev_u8(c, dev), to_dev_bf16(s, dev), to_dev_u8(z, dev),
+                         N, K, g)
+    torch.cuda.synchronize()
+    assert qz.qz_device_status() == 0
+    check_tolerance(u16(y), y_ref, abs_ref, f"gemm M={M} N={N} K={K} g={g}")
+
+
+def test_w4a16_gemm_onehot_is_exact(dev):
+    """One-hot token rows read back single dequantized weights exactly."""
+    M, N, K, g = 256, 256, 1024, 128
+    w = synthetic.weights(N, K, sigma=0.02, seed=77)
+    c, s, z, w_hat = oracle_w4(u16(w), g)
+    ks = np.arange(M) * (K // M) + (np.arange(M) % (K // M))
+    a = np.zeros((M, K), np.uint16)
+    a[np.arange(M), ks] = 0x3F80
+    y = qz.qz_w4a16_gemm(to_dev_bf16(a, dev), to_dev_u8(c, dev), to_dev_bf16(s, dev),
+                         to_dev_u8(z, dev), N, K, g)
+    torch.cuda.synchronize()
+    assert np.array_equal(u16(y), w_hat[:, ks].T)
+
+
+def test_prefill_config_sampled(dev):
+    """M = 2048 tokens, N = K = 8192, seed 6: sampled weight rows, all tokens."""
+    cfg = synthetic.PREFILL
+    M, N, K = cfg["M"], cfg["N"], cfg["K"]
+    w = synthetic.weights(N, K, sigma=cfg["sigma"], seed=cfg["seed"], device=dev)
+    a = synthetic.activations(M, K, seed=cfg["seed"] + 1000, device=dev)
+    c, s, z = qz.qz_quantize_pack(w, 4, False, 128)
+    y = qz.qz_w4a16_gemm(a, c, s, z, N, K, 128)
+    torch.cuda.synchronize()
+    assert qz.qz_device_status() == 0
+    idx = sample_rows(N, 24, 6)
+    ti = torch.from_numpy(idx).to(dev)
+    ref = oracle.quantize_pack(u16(w.index_select(0, ti)), 4, False, 128)
+    got = (u8(c.index_select(0, ti)), u16(s.index_select(0, ti)), u8(z.index_select(0, ti)))
+    assert_quant_equal(got, ref)
+    w_hat = oracle.dequantize(*ref, len(idx), K, 4, False, 128)
+    y_ref, abs_ref = oracle.matmul_f64(u16(a), w_hat)
+    check_tolerance(u16(y)[:, idx], y_ref, abs_ref, "prefill 2048x8192x8192")
+
+
+def test_gemm_bounded_wait_reports_timeout_and_recovers(dev):
+    """A 1 ns wait bound makes the first pipeline wait run out: the kernel
+    must return with the error word set (no hang, no fault), and the next call
+    with the default bound must be correct again."""
+    M, N, K, g = 256, 256, 2048, 128
+    w = synthetic.weights(N, K, seed=3, device=dev)
+    a = synthetic.activations(M, K, seed=3, device=dev)
+    c, s, z = qz.qz_quantize_pack(w, 4, False, g)
+    assert qz.qz_device_status() == 0
+    qz.qz_set_device_wait_limit(1)
+    try:
+        qz.qz_w4a16_gemm(a, c, s, z, N, K, g)
+        st = qz.qz_device_status()
+    finally:
+        qz.qz_set_device_wait_limit(0)
+    assert st == qz.QZ_ERR_DEVICE_TIMEOUT
+    assert qz.qz_device_status() == 0                      # cleared by the read
+    y = qz.qz_w4a16_gemm(a, c, s, z, N, K, g)
+    torch.cuda.synchronize()
+    assert qz.qz_device_status() == 0
+    wb = u16(w)
+    cref, sref, zref, w_hat = oracle_w4(wb, g)
+    y_ref, abs_ref = oracle.matmul_f64(u16(a), w_hat)
+    check_tolerance(u16(y), y_ref, abs_ref, "gemm after timeout")

@@ -9,7 +9,7 @@
 namespace qz {
 
 static std::atomic<uint64_t> g_wait_limit{0};
-constexpr uint64_t kDefaultWaitLimit = uint64_t(1) << 26;
+constexpr uint64_t kDefaultWaitLimit = 2000000000ull;   // 2 s in nanoseconds
 
 uint64_t device_wait_limit() {
     const uint64_t v = g_wait_limit.load(std::memory_order_relaxed);

@@ -25,7 +25,7 @@
 // accumulation in tensor memory (256 columns); B = activations from shared
 // memory.  Each weight tile is dequantized once per 256 tokens.
 //
-// Every mbarrier wait is bounded by a caller-set iteration limit; on expiry
+// Every mbarrier wait is bounded by a caller-set time limit; on expiry
 // the thread records the fault in g_device_error_word and in a CTA-local
 // abort flag, every role stops issuing work, in-flight copies and MMAs are
 // drained (with bounded waits), tensor memory is released and the CTA exits.
@@ -103,17 +103,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Bounded wait: true when the phase completed, false when the limit ran out
-// or another thread of the CTA aborted (then the caller unwinds).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit,
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait: true when the phase completed, false when `limit_ns` of wall
+// time ran out or another thread of the CTA aborted (then the caller unwinds).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns,
                                           volatile uint32_t *abort_flag) {
-    for (uint64_t i = 0; i < limit; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
+        if (global_ns() - t0 > limit_ns) break;
     }
     *abort_flag = 1u;
     atomicOr(&g_device_error_word, 1u);
     return false;
+}
+
+// Wait used while unwinding: copies and MMAs already issued complete on their
+// own, so this bound (2 s) is independent of the caller's limit.
+constexpr uint64_t kDrainLimitNs = 2000000000ull;
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+    volatile uint32_t never = 0;
+    mbar_wait(bar, parity, kDrainLimitNs, &never);
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
@@ -268,10 +285,7 @@ w4a16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
             }
             // drain: every issued copy must have landed before the CTA may exit
             for (int s = 0; s < kStages; ++s)
-                if (issued_round[s] >= 0) {
-                    volatile uint32_t never = 0;
-                    mbar_wait(full_bar(s), issued_round[s] & 1, wait_limit, &never);
-                }
+                if (issued_round[s] >= 0) mbar_drain(full_bar(s), issued_round[s] & 1);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -292,14 +306,11 @@ w4a16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
                 }
                 mma_commit(empty_bar(s));
             }
-            if (ok) {
-                mma_commit(accum_bar);
-            } else {
-                // let every issued MMA finish before tensor memory is released
-                mma_commit(drain_bar);
-                volatile uint32_t never = 0;
-                mbar_wait(drain_bar, 0, wait_limit, &never);
-            }
+            // Every issued MMA must finish before tensor memory is released,
+            // whether or not the epilogue warps are still waiting for it.
+            const uint32_t done_bar = ok ? accum_bar : drain_bar;
+            mma_commit(done_bar);
+            mbar_drain(done_bar, 0);
         }
         __syncwarp();
     } else {

@@ -476,6 +476,51 @@ def config_obj():
             "parallelism": "replicas"}
 
 
+PROFILE_CASES = {
+    # name: (kind, M, N, K)
+    "gemv_w4_70b": ("gemv4", 1, 28672, 8192),
+    "gemv_w4_70b_m16": ("gemv4", 16, 28672, 8192),
+    "gemv_w4_7b": ("gemv4", 1, 4096, 4096),
+    "gemv_w8_70b": ("gemv8", 1, 28672, 8192),
+    "gemm_prefill": ("gemm", 2048, 8192, 8192),
+    "quant_int4": ("quant4", 0, 28672, 8192),
+    "quant_int8": ("quant8", 0, 28672, 8192),
+    "dequant_int4": ("dequant", 0, 28672, 8192),
+}
+
+
+def run_kernel_case(name, reps):
+    """One kernel on one configuration, launched `reps` times after its
+    inputs are prepared (used for ncu captures: small, deterministic)."""
+    import weight_only_quantization_wise_b200 as qz
+    kind, M, N, K = PROFILE_CASES[name]
+    dev = torch.device("cuda", 0)
+    w = synthetic.weights(N, K, sigma=0.015, seed=4, device=dev)
+    ws = torch.zeros(1 << 24, dtype=torch.uint8, device=dev)
+    if kind in ("gemv4", "gemm", "dequant"):
+        c, s, z = qz.qz_quantize_pack(w, 4, False, GROUP)
+    if kind == "gemv8":
+        c, s, _ = qz.qz_quantize_pack(w, 8, True, K)
+    a = synthetic.activations(max(M, 1), K, seed=5, device=dev)
+    torch.cuda.synchronize()
+    for _ in range(reps):
+        if kind == "gemv4":
+            qz.qz_w4a16_gemv(a, c, s, z, N, K, GROUP, workspace=ws)
+        elif kind == "gemv8":
+            qz.qz_w8a16_gemv(a, c, s, N, K, workspace=ws)
+        elif kind == "gemm":
+            qz.qz_w4a16_gemm(a, c, s, z, N, K, GROUP, workspace=ws)
+        elif kind == "quant4":
+            qz.qz_quantize_pack(w, 4, False, GROUP)
+        elif kind == "quant8":
+            qz.qz_quantize_pack(w, 8, True, K)
+        elif kind == "dequant":
+            qz.qz_dequantize(c, s, z, N, K, 4, False, GROUP)
+    torch.cuda.synchronize()
+    assert qz.qz_device_status() == 0
+    print(f"{name}: {reps} launches ok")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -484,7 +529,13 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--kernel", choices=sorted(PROFILE_CASES),
+                    help="run one kernel case a few times (for profiling) and exit")
+    ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()
+    if args.kernel:
+        run_kernel_case(args.kernel, args.reps)
+        return
     if args.impl == "reference":
         run_reference(args)
         return
@@ -546,10 +597,12 @@ def main():
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
+    torch.cuda.nvtx.range_push("timed")
     with torch.cuda.stream(stream):
         e_start.record(stream)
         run_steps(args.steps, ev, start=args.warmup)
         e_end.record(stream)
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     if dist:
         dist.barrier()

@@ -1,6 +1,8 @@
 """Build libqz.so (the sm_100a CUDA library behind include/qz.h) in-tree.
 
-    python -m weight_only_quantization_wise_b200.build [--force] [--verbose]
+    python weight_only_quantization_wise_b200/build.py [--force] [--verbose]
+
+(run as a script: importing the package itself needs the built library)
 
 Each csrc/*.cu is compiled with nvcc for sm_100a only (no other arch, no
 fast-math, no flush-to-zero) into _build/, then linked into

@@ -181,6 +181,38 @@ QZ_API qz_status qz_w8a16_gemv(const void *a, const void *codes, const void *sca
                         size_t workspace_bytes, void *stream);
 
 /*
+ * Size of the scratch array built into the library for
+ * qz_w4a16_gemv_noalloc (4 MiB, held on every GPU that loads the library).
+ */
+#define QZ_GEMV_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/*
+ * W4A16 decode GEMV that allocates nothing and takes no workspace.  The
+ * quantization pages have no counterpart to this entry point: it exists for
+ * callers that cannot allocate device memory -- for example a plugin inside a
+ * host application that owns all device memory and offers no allocator, or
+ * latency-critical code that cannot afford cudaMalloc (which may synchronize
+ * the device).  Arguments, requirements and results are those of
+ * qz_w4a16_gemv; the split-K scratch lives in a fixed array of
+ * QZ_GEMV_NOALLOC_SCRATCH_BYTES inside the library.
+ *   - Sizes whose scratch need (qz_workspace_bytes(QZ_OP_W4A16_GEMV, ...))
+ *     exceeds that maximum are rejected with QZ_ERR_WORKSPACE before any
+ *     launch.
+ *   - The first call on a device looks up the array's device address on that
+ *     device (with it current); make that first call before any stream
+ *     capture.
+ *   - Each call clears the part of the array that must start at zero (with
+ *     cudaMemsetAsync on `stream`) and never calls cudaMalloc, cudaFree or
+ *     any allocating routine.
+ *   - All calls share the one array, which keeps the last call's contents:
+ *     calls that overlap on the GPU (different streams, or different host
+ *     threads on one device) race on it and give undefined results.
+ */
+QZ_API qz_status qz_w4a16_gemv_noalloc(const void *a, const void *codes, const void *scales,
+                                       const void *zeros, int64_t M, int64_t N, int64_t K,
+                                       int64_t group_size, void *y, void *stream);
+
+/*
  * Device-side wait bound used by kernels that wait on mbarriers (the GEMM),
  * in nanoseconds of wall time per wait; 0 restores the default (2 s).
  * Not part of the method: a safety bound so that a broken pipeline returns an

@@ -37,6 +37,7 @@ _SIGS = {
     "qz_w4a16_gemv": ([_p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p, _sz, _p], ctypes.c_int),
     "qz_w4a16_gemm": ([_p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p, _sz, _p], ctypes.c_int),
     "qz_w8a16_gemv": ([_p, _p, _p, _i64, _i64, _i64, _p, _p, _sz, _p], ctypes.c_int),
+    "qz_w4a16_gemv_noalloc": ([_p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p], ctypes.c_int),
     "qz_set_device_wait_limit": ([ctypes.c_uint64], None),
     "qz_device_status": ([], ctypes.c_int),
 }
@@ -44,7 +45,7 @@ EXPORTED_SYMBOLS = tuple(_SIGS)
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is not built; run `python -m weight_only_quantization_wise_b200.build` "
+        f"{LIB_PATH} is not built; run `python weight_only_quantization_wise_b200/build.py` "
         "(there is no fallback implementation)")
 
 lib = ctypes.CDLL(LIB_PATH)

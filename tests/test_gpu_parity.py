@@ -418,3 +418,40 @@ def test_gemm_bounded_wait_reports_timeout_and_recovers(dev):
     cref, sref, zref, w_hat = oracle_w4(wb, g)
     y_ref, abs_ref = oracle.matmul_f64(u16(a), w_hat)
     check_tolerance(u16(y), y_ref, abs_ref, "gemm after timeout")
+
+
+@pytest.mark.parametrize("bits,sym", FORMATS)
+@pytest.mark.parametrize("g", [128, 0, 4096])
+def test_quantize_dense_bit_exact(dev, bits, sym, g):
+    """2M values in one comparison.  About 0.3% of them land exactly on a
+    half-way point of their group's grid, so the tie handling of the
+    division-free path (round half to even) runs thousands of times."""
+    N, K = 512, 4096
+    w = synthetic.weights(N, K, sigma=0.02, seed=900 + bits + 2 * int(sym))
+    ref = oracle.quantize_pack(u16(w), bits, sym, g)
+    got = gpu_quantize(w.to(dev), bits, sym, g)
+    assert_quant_equal(got, ref)
+
+
+def _bf16_step(x, d):
+    """The bf16 value d representable steps away from bf16 x (x > 0)."""
+    b = np.array([x], np.float32).view(np.uint32)[0] >> 16
+    return float(np.array([(int(b) + d) << 16], np.uint32).view(np.float32)[0])
+
+
+def test_quantize_near_half_way_values(dev):
+    """Values placed exactly on, and one bf16 step either side of, every
+    half-way point of a group whose scale is exactly 1 (range [0, 15])."""
+    K = 128
+    vals = [0.0, 15.0]
+    for j in range(15):
+        h = j + 0.5
+        vals += [h, _bf16_step(h, 1), _bf16_step(h, -1)]
+    row = np.zeros(K, np.float32)
+    row[:len(vals)] = vals
+    w = torch.from_numpy(np.stack([row, -row[::-1].copy()])).to(torch.bfloat16)
+    for bits, sym in FORMATS:
+        for g in (128, 0):
+            ref = oracle.quantize_pack(u16(w), bits, sym, g)
+            got = gpu_quantize(w.to(dev), bits, sym, g)
+            assert_quant_equal(got, ref)

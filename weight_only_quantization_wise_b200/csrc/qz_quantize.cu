@@ -69,36 +69,122 @@ __device__ __forceinline__ void accumulate_stats(const float (&x)[8], float &vmi
     }
 }
 
-// Quantize the 8 values of one chunk and write their codes (int4: one 32-bit
-// word, int8: 8 bytes) at chunk index c.
+// Codes of one 8-value chunk (int4: one 32-bit word, value i in nibble i;
+// int8: two words, value i in byte i), computed with the IEEE division as the
+// definition states it.
 template <int BITS, bool SYM>
-__device__ __forceinline__ void quantize_chunk(const float (&x)[8], float s_f, int z,
-                                               uint8_t *__restrict__ codes, int64_t c) {
+__device__ __forceinline__ uint2 chunk_codes_exact(const float (&x)[8], float s_f, int z) {
     const float z_f = (float)z;
     if (BITS == 4) {
         uint32_t word = 0;
 #pragma unroll
         for (int i = 0; i < 8; ++i)
             word |= (uint32_t)(quantize_one<BITS, SYM>(x[i], s_f, z_f) & 0xF) << (4 * i);
-        reinterpret_cast<uint32_t *>(codes)[c] = word;
-    } else {
-        uint32_t lo = 0, hi = 0;
+        return make_uint2(word, 0u);
+    }
+    uint32_t lo = 0, hi = 0;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            lo |= (uint32_t)(quantize_one<BITS, SYM>(x[i], s_f, z_f) & 0xFF) << (8 * i);
-            hi |= (uint32_t)(quantize_one<BITS, SYM>(x[i + 4], s_f, z_f) & 0xFF) << (8 * i);
-        }
-        reinterpret_cast<uint2 *>(codes)[c] = make_uint2(lo, hi);
+    for (int i = 0; i < 4; ++i) {
+        lo |= (uint32_t)(quantize_one<BITS, SYM>(x[i], s_f, z_f) & 0xFF) << (8 * i);
+        hi |= (uint32_t)(quantize_one<BITS, SYM>(x[i + 4], s_f, z_f) & 0xFF) << (8 * i);
+    }
+    return make_uint2(lo, hi);
+}
+
+// Store the codes of chunk c.
+template <int BITS>
+__device__ __forceinline__ void store_codes(uint8_t *__restrict__ codes, int64_t c, uint2 v) {
+    if (BITS == 4) reinterpret_cast<uint32_t *>(codes)[c] = v.x;
+    else reinterpret_cast<uint2 *>(codes)[c] = v;
+}
+
+// Codes of one chunk without a division per value.
+//
+// The definition's fp32 steps, u = fl(fl(x/S) + Z) and round-half-even(u),
+// give the same integer as rounding the exact x/S + Z half-to-even: x and S
+// are bf16, so write x = m_x 2^a, S = m_s 2^b with integer significands below
+// 256.  Then x/S - (j + 1/2) = [2 m_x 2^(a-b) - (2j + 1) m_s] / (2 m_s).  For
+// a >= b the numerator is an integer; for a < b it is an integer multiple of
+// 2^(a-b+1), and |x/S| >= 0.49 (needed to be near a half-way point) forces
+// 2^(a-b) >= 0.49 m_s / 255.  Either way x/S + Z is exactly half-way between
+// two integers (a tie, which fp32 holds exactly) or at least 2^-10 from every
+// half-way point, far more than fp32 rounding moves u.
+//
+// Here C = 1.5 * 2^7 (int4) or 1.5 * 2^9 (int8) puts T = x/S + Z + C inside
+// one binade whose grid is 2^-16 (int4: T in [191.5, 207.5]) or 2^-14 (int8:
+// T in [639.5, 895.5]).  With r = 1/S rounded to nearest, x*r is within
+// |x/S| 2^-24 < 2^-16 (|x/S| <= 255) of x/S, which is under half a grid step,
+// so y = fma(x, r, Z + C) rounds to T itself when T is a tie, and otherwise
+// lands on T's side of its nearest half-way point (2^-10 away).  Adding
+// 1.5 * 2^23 - C then rounds y - C to an integer, half to even, in one fp32
+// add: the result is 1.5 * 2^23 + round_half_even(x/S + Z), with the code in
+// its low mantissa bits.  Only a tie at q_max + 1/2 leaves the code range
+// (x/S + Z stays within [q_min - 1/2, q_max + 1/2] and q_min is even), so the
+// asymmetric formats clamp at the top.  If 1/S overflows (tiny subnormal S)
+// the chunk falls back to the IEEE division.
+template <int BITS, bool SYM>
+__device__ __forceinline__ uint2 chunk_codes(const float (&x)[8], float s_f, float r, int z) {
+    using R = Range<BITS, SYM>;
+    constexpr float kC = BITS == 4 ? 192.0f : 768.0f;
+    constexpr float kRound = 12582912.0f - kC;         // 1.5 * 2^23 - C, exact
+    constexpr uint32_t kTop = 0x4B400000u + (uint32_t)R::qmax;   // bits of 1.5*2^23 + q_max
+    if (!(r < __int_as_float(0x7F800000))) return chunk_codes_exact<BITS, SYM>(x, s_f, z);
+    const float zc = __fadd_rn((float)z, kC);          // exact (small integers)
+    uint32_t b[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        b[i] = __float_as_uint(__fadd_rn(__fmaf_rn(x[i], r, zc), kRound));
+        if (!SYM) b[i] = min(b[i], kTop);
+    }
+    if (BITS == 4) {
+        uint32_t p[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)   // byte j: code 2j low nibble, code 2j+1 high nibble
+            p[j] = (b[2 * j] & 0x0Fu) | ((b[2 * j + 1] << 4) & 0xF0u);
+        const uint32_t lo = dev::prmt(p[0], p[1], 0x0040u);
+        const uint32_t hi = dev::prmt(p[2], p[3], 0x0040u);
+        return make_uint2(dev::prmt(lo, hi, 0x5410u), 0u);
+    }
+    const uint32_t w0 = dev::prmt(dev::prmt(b[0], b[1], 0x0040u), dev::prmt(b[2], b[3], 0x0040u), 0x5410u);
+    const uint32_t w1 = dev::prmt(dev::prmt(b[4], b[5], 0x0040u), dev::prmt(b[6], b[7], 0x0040u), 0x5410u);
+    return make_uint2(w0, w1);
+}
+
+// Three-input fp32 max/min (sm_100); exact, they select one of their inputs.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Fold the 8 values of a chunk into a running range (asymmetric: min and
+// max; symmetric: max |x| in vmax).
+template <bool SYM>
+__device__ __forceinline__ void fold_range(const float (&x)[8], float &vmin, float &vmax) {
+    if (SYM) {
+        const float a = fmax3(fabsf(x[0]), fabsf(x[1]), fabsf(x[2]));
+        const float b = fmax3(fabsf(x[3]), fabsf(x[4]), fabsf(x[5]));
+        vmax = fmax3(vmax, fmax3(a, b, fabsf(x[6])), fabsf(x[7]));
+    } else {
+        vmax = fmax3(vmax, fmax3(x[0], x[1], x[2]), fmax3(x[3], x[4], fmaxf(x[5], fmaxf(x[6], x[7]))));
+        vmin = fmin3(vmin, fmin3(x[0], x[1], x[2]), fmin3(x[3], x[4], fminf(x[5], fminf(x[6], x[7]))));
     }
 }
 
 // ---------------------------------------------------------------------------
-// Groups of 32..256 values: LPG = g/8 lanes own one group, one 16-byte chunk
-// each, and reduce its range with butterfly shuffles.  Every warp-wide load
-// instruction reads 512 contiguous bytes.
+// Groups of 32..256 values: each lane owns 4 consecutive 16-byte chunks (32
+// values) of one group, LPG = g/32 lanes share a group and combine their
+// ranges with butterfly shuffles.  The per-group work (range, S, Z, 1/S) is
+// done once per 32 values, and a lane writes its int4 codes with one 16-byte
+// store.  The four 16-byte loads of a lane are L1-cached so that they merge
+// into full sectors.
 // ---------------------------------------------------------------------------
 constexpr int kQuantThreads = 256;
-constexpr int kQuantUnroll = 4;
 
 template <int BITS, bool SYM, int LPG>
 __global__ void __launch_bounds__(kQuantThreads)
@@ -108,46 +194,105 @@ quantize_small_groups(const uint4 *__restrict__ w, int64_t total_chunks,
     const int lane = threadIdx.x & 31;
     const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    constexpr int64_t kSpan = 32 * kQuantUnroll;
-    for (int64_t base = warp * kSpan; base < total_chunks; base += nwarps * kSpan) {
-        uint4 v[kQuantUnroll];
+    for (int64_t base = warp * 128; base < total_chunks; base += nwarps * 128) {
+        const int64_t c0 = base + 4 * lane;       // total_chunks is a multiple of 4
+        const bool valid = c0 < total_chunks;
+        float x[4][8];
 #pragma unroll
-        for (int u = 0; u < kQuantUnroll; ++u) {
-            const int64_t c = base + u * 32 + lane;
-            v[u] = (c < total_chunks) ? dev::ld_stream_v4(w + c) : make_uint4(0, 0, 0, 0);
+        for (int u = 0; u < 4; ++u)
+            unpack8(valid ? __ldg(w + c0 + u) : make_uint4(0, 0, 0, 0), x[u]);
+        float vmin = 0.0f, vmax = 0.0f;           // the range always contains 0
+#pragma unroll
+        for (int u = 0; u < 4; ++u) fold_range<SYM>(x[u], vmin, vmax);
+#pragma unroll
+        for (int o = LPG / 2; o >= 1; o >>= 1) {
+            vmax = fmaxf(vmax, __shfl_xor_sync(0xFFFFFFFFu, vmax, o));
+            if (!SYM) vmin = fminf(vmin, __shfl_xor_sync(0xFFFFFFFFu, vmin, o));
         }
+        if (!valid) continue;                     // whole groups drop out together
+        uint32_t s_bits; float s_f; int z;
+        group_params<BITS, SYM>(vmin, vmax, vmax, s_bits, s_f, z);
+        const float r = __frcp_rn(s_f);
+        uint2 cw[4];
 #pragma unroll
-        for (int u = 0; u < kQuantUnroll; ++u) {
-            const int64_t c = base + u * 32 + lane;
-            float x[8];
-            unpack8(v[u], x);
-            float vmin = 0.0f, vmax = 0.0f, amax = 0.0f;
-            accumulate_stats<SYM>(x, vmin, vmax, amax);
-#pragma unroll
-            for (int o = LPG / 2; o >= 1; o >>= 1) {
-                if (SYM) {
-                    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-                } else {
-                    vmin = fminf(vmin, __shfl_xor_sync(0xFFFFFFFFu, vmin, o));
-                    vmax = fmaxf(vmax, __shfl_xor_sync(0xFFFFFFFFu, vmax, o));
-                }
-            }
-            if (c >= total_chunks) continue;   // whole groups drop out together
-            uint32_t s_bits; float s_f; int z;
-            group_params<BITS, SYM>(vmin, vmax, amax, s_bits, s_f, z);
-            quantize_chunk<BITS, SYM>(x, s_f, z, codes, c);
-            if ((lane % LPG) == 0) {
-                const int64_t gidx = c / LPG;
-                scales[gidx] = (uint16_t)s_bits;
-                if (!SYM) zeros[gidx] = (uint8_t)(int8_t)z;
-            }
+        for (int u = 0; u < 4; ++u) cw[u] = chunk_codes<BITS, SYM>(x[u], s_f, r, z);
+        if (BITS == 4) {
+            reinterpret_cast<uint4 *>(codes)[c0 >> 2] = make_uint4(cw[0].x, cw[1].x, cw[2].x, cw[3].x);
+        } else {
+            uint4 *dst = reinterpret_cast<uint4 *>(codes) + (c0 >> 1);
+            dst[0] = make_uint4(cw[0].x, cw[0].y, cw[1].x, cw[1].y);
+            dst[1] = make_uint4(cw[2].x, cw[2].y, cw[3].x, cw[3].y);
+        }
+        if ((lane % LPG) == 0) {
+            const int64_t gidx = c0 / (4 * LPG);
+            scales[gidx] = (uint16_t)s_bits;
+            if (!SYM) zeros[gidx] = (uint8_t)(int8_t)z;
         }
     }
 }
 
 // ---------------------------------------------------------------------------
-// Any other group size (including per-channel, g == K): one block per group,
-// two passes (the second re-reads the group from L2).
+// Groups of up to 65536 values (per-channel rows included): one block per
+// group holds the whole group in registers (at most 8 chunks per thread), so
+// the weights are read from HBM once; the range is combined with shuffles and
+// one shared-memory step.
+// ---------------------------------------------------------------------------
+constexpr int kRowChunksPerThread = 8;
+
+template <int BITS, bool SYM>
+__global__ void __launch_bounds__(1024)
+quantize_groups_block(const uint4 *__restrict__ w, int cpg, int64_t num_groups,
+                      uint8_t *__restrict__ codes, uint16_t *__restrict__ scales,
+                      uint8_t *__restrict__ zeros) {
+    __shared__ float red[64];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    for (int64_t gidx = blockIdx.x; gidx < num_groups; gidx += gridDim.x) {
+        const int64_t c0 = gidx * cpg;
+        uint4 v[kRowChunksPerThread];
+        float vmin = 0.0f, vmax = 0.0f;           // the range always contains 0
+#pragma unroll
+        for (int i = 0; i < kRowChunksPerThread; ++i) {
+            const int c = threadIdx.x + i * blockDim.x;
+            if (c < cpg) {
+                v[i] = __ldcs(w + c0 + c);
+                float x[8];
+                unpack8(v[i], x);
+                fold_range<SYM>(x, vmin, vmax);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            vmax = fmaxf(vmax, __shfl_xor_sync(0xFFFFFFFFu, vmax, o));
+            if (!SYM) vmin = fminf(vmin, __shfl_xor_sync(0xFFFFFFFFu, vmin, o));
+        }
+        if (lane == 0) { red[wid] = vmax; red[32 + wid] = vmin; }
+        __syncthreads();
+        vmax = red[0];
+        vmin = red[32];
+        for (int i = 1; i < nw; ++i) { vmax = fmaxf(vmax, red[i]); vmin = fminf(vmin, red[32 + i]); }
+        __syncthreads();                          // red[] is reused by the next group
+        uint32_t s_bits; float s_f; int z;
+        group_params<BITS, SYM>(vmin, vmax, vmax, s_bits, s_f, z);
+        const float r = __frcp_rn(s_f);
+#pragma unroll
+        for (int i = 0; i < kRowChunksPerThread; ++i) {
+            const int c = threadIdx.x + i * blockDim.x;
+            if (c < cpg) {
+                float x[8];
+                unpack8(v[i], x);
+                store_codes<BITS>(codes, c0 + c, chunk_codes<BITS, SYM>(x, s_f, r, z));
+            }
+        }
+        if (threadIdx.x == 0) {
+            scales[gidx] = (uint16_t)s_bits;
+            if (!SYM) zeros[gidx] = (uint8_t)(int8_t)z;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Groups of more than 65536 values: one block per group, two passes (the
+// second re-reads the group from L2).
 // ---------------------------------------------------------------------------
 template <bool SYM>
 __device__ __forceinline__ void block_reduce_stats(float &vmin, float &vmax, float &amax) {
@@ -178,19 +323,21 @@ quantize_large_groups(const uint4 *__restrict__ w, int64_t chunks_per_group,
                       uint16_t *__restrict__ scales, uint8_t *__restrict__ zeros) {
     for (int64_t gidx = blockIdx.x; gidx < num_groups; gidx += gridDim.x) {
         const int64_t c0 = gidx * chunks_per_group;
-        float vmin = 0.0f, vmax = 0.0f, amax = 0.0f;
+        float vmin = 0.0f, vmax = 0.0f;           // the range always contains 0
         for (int64_t i = threadIdx.x; i < chunks_per_group; i += blockDim.x) {
             float x[8];
             unpack8(__ldcg(w + c0 + i), x);
-            accumulate_stats<SYM>(x, vmin, vmax, amax);
+            fold_range<SYM>(x, vmin, vmax);
         }
+        float amax = vmax;
         block_reduce_stats<SYM>(vmin, vmax, amax);
         uint32_t s_bits; float s_f; int z;
         group_params<BITS, SYM>(vmin, vmax, amax, s_bits, s_f, z);
+        const float r = __frcp_rn(s_f);
         for (int64_t i = threadIdx.x; i < chunks_per_group; i += blockDim.x) {
             float x[8];
             unpack8(__ldcs(w + c0 + i), x);
-            quantize_chunk<BITS, SYM>(x, s_f, z, codes, c0 + i);
+            store_codes<BITS>(codes, c0 + i, chunk_codes<BITS, SYM>(x, s_f, r, z));
         }
         if (threadIdx.x == 0) {
             scales[gidx] = (uint16_t)s_bits;
@@ -249,11 +396,12 @@ tensor_quantize(const uint4 *__restrict__ w, int64_t total_chunks,
                 const uint32_t *__restrict__ ws, uint8_t *__restrict__ codes) {
     uint32_t s_bits; float s_f; int z;
     tensor_params<BITS, SYM>(ws, s_bits, s_f, z);
+    const float r = __frcp_rn(s_f);
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < total_chunks; c += stride) {
         float x[8];
         unpack8(dev::ld_stream_v4(w + c), x);
-        quantize_chunk<BITS, SYM>(x, s_f, z, codes, c);
+        store_codes<BITS>(codes, c, chunk_codes<BITS, SYM>(x, s_f, r, z));
     }
 }
 
@@ -292,43 +440,68 @@ qz_status quantize_typed(const void *w, int64_t N, int64_t K, int64_t g, void *c
         tensor_finish<BITS, SYM><<<1, 1, 0, st>>>(ws, s16, z8);
         return launch_status();
     }
-    const int grid = grid_for(total, kQuantThreads * kQuantUnroll);
+    const int grid = grid_for(total, kQuantThreads * 4);
     switch (g) {
     case 32:
-        quantize_small_groups<BITS, SYM, 4><<<grid, kQuantThreads, 0, st>>>(src, total, c8, s16, z8);
+        quantize_small_groups<BITS, SYM, 1><<<grid, kQuantThreads, 0, st>>>(src, total, c8, s16, z8);
         return launch_status();
     case 64:
-        quantize_small_groups<BITS, SYM, 8><<<grid, kQuantThreads, 0, st>>>(src, total, c8, s16, z8);
+        quantize_small_groups<BITS, SYM, 2><<<grid, kQuantThreads, 0, st>>>(src, total, c8, s16, z8);
         return launch_status();
     case 128:
-        quantize_small_groups<BITS, SYM, 16><<<grid, kQuantThreads, 0, st>>>(src, total, c8, s16, z8);
+        quantize_small_groups<BITS, SYM, 4><<<grid, kQuantThreads, 0, st>>>(src, total, c8, s16, z8);
         return launch_status();
     case 256:
-        quantize_small_groups<BITS, SYM, 32><<<grid, kQuantThreads, 0, st>>>(src, total, c8, s16, z8);
+        quantize_small_groups<BITS, SYM, 8><<<grid, kQuantThreads, 0, st>>>(src, total, c8, s16, z8);
         return launch_status();
-    default: {
-        const int64_t groups = N * (K / g);
-        const int blocks = (int)std::min<int64_t>(groups, (int64_t)kSmCount * 32);
-        quantize_large_groups<BITS, SYM><<<blocks, kQuantThreads, 0, st>>>(
-            src, g / 8, groups, c8, s16, z8);
+    default:
+        break;
+    }
+    const int64_t groups = N * (K / g);
+    const int64_t cpg = g / 8;
+    if (cpg <= (int64_t)kRowChunksPerThread * 1024) {
+        const int threads = (int)ceil_div(ceil_div(cpg, kRowChunksPerThread), 32) * 32;
+        const int per_sm = std::max(1, 2048 / threads);
+        const int blocks = (int)std::min<int64_t>(groups, (int64_t)kSmCount * per_sm * 4);
+        quantize_groups_block<BITS, SYM><<<blocks, threads, 0, st>>>(src, (int)cpg, groups, c8,
+                                                                      s16, z8);
         return launch_status();
     }
-    }
+    const int blocks = (int)std::min<int64_t>(groups, (int64_t)kSmCount * 32);
+    quantize_large_groups<BITS, SYM><<<blocks, kQuantThreads, 0, st>>>(src, cpg, groups, c8,
+                                                                        s16, z8);
+    return launch_status();
 }
 
 // ---------------------------------------------------------------------------
-// Dequantize: w_hat = bf16_rne(S * (q - Z)).  The fp32 product is exact (an
-// 8-bit-significand scale times an integer of at most 8 bits), so the only
-// rounding is the final conversion.  One 16-byte output chunk per thread.
+// Dequantize: w_hat = bf16_rne(S * (q - Z)).  The product of the bf16 scale
+// (8-bit significand) and q - Z (at most 9 bits) is exact in fp32, so the
+// only rounding is one round-to-nearest-even to bf16.  No integer-to-float
+// conversion is used:
+//   int4: byte i of the code word and of (word >> 4) hold codes 2i and 2i+1
+//         in their low nibbles; one PRMT + LOP3 builds bf16(128 + q) for the
+//         pair, sub.rn.bf16x2 removes (128 + Z) exactly and mul.rn.bf16x2 by
+//         the scale rounds the product once (symmetric codes are first made
+//         unsigned by XOR 8, with 8 added to Z).
+//   int8: the byte (XOR 0x80) is placed in the mantissa of 2^23; one packed
+//         fp32 add gives q - Z exactly, a packed fp32 multiply the exact
+//         product, cvt.rn.bf16x2 rounds it once.
+// One 16-byte output chunk (8 values) per thread per step.
 // ---------------------------------------------------------------------------
-template <int BITS, bool SYM>
-__device__ __forceinline__ int code_at(uint32_t lo, uint32_t hi, int i) {
-    if (BITS == 4) {
-        const uint32_t nib = (lo >> (4 * i)) & 0xF;
-        return SYM ? ((int)(nib << 28) >> 28) : (int)nib;
-    }
-    const uint32_t word = (i < 4) ? lo : hi;
-    return (int)(int8_t)((word >> (8 * (i & 3))) & 0xFF);
+__device__ __forceinline__ uint32_t dq_pair_u4(uint32_t w, uint32_t w4, int i, uint32_t s2,
+                                               uint32_t z2) {
+    const uint32_t t = dev::prmt(w, w4, (uint32_t)i | ((uint32_t)(4 + i) << 8));
+    const uint32_t x = (t & 0x000F000Fu) | 0x43004300u;            // bf16(128 + q)
+    return dev::bf16x2_mul(dev::bf16x2_sub(x, z2), s2);
+}
+
+__device__ __forceinline__ uint32_t dq_pair_i8(uint32_t word, int i, float off, float s) {
+    // bytes 2i and 2i+1 (i = 0, 1) of `word` (already XORed with 0x80808080)
+    const float f0 = __uint_as_float(dev::prmt(word, 0x4B000000u, (uint32_t)(2 * i) | 0x7540u));
+    const float f1 = __uint_as_float(dev::prmt(word, 0x4B000000u, (uint32_t)(2 * i + 1) | 0x7540u));
+    const float p0 = __fmul_rn(__fadd_rn(f0, off), s);             // q - Z exact, exact product
+    const float p1 = __fmul_rn(__fadd_rn(f1, off), s);
+    return dev::pack_bf16x2(p0, p1);
 }
 
 template <int BITS, bool SYM>
@@ -342,22 +515,27 @@ dequantize_kernel(const uint8_t *__restrict__ codes, const uint16_t *__restrict_
         if (chunks_per_group == 0) gidx = 0;
         else if (cpg_shift >= 0) gidx = c >> cpg_shift;
         else gidx = c / chunks_per_group;
-        const float s_f = __uint_as_float((uint32_t)__ldg(&scales[gidx]) << 16);
-        int z = 0;
-        if (!SYM) z = (BITS == 4) ? (int)__ldg(&zeros[gidx]) : (int)(int8_t)__ldg(&zeros[gidx]);
-        uint32_t lo, hi = 0;
+        const uint32_t s_bits = __ldg(&scales[gidx]);
+        uint32_t o[4];
         if (BITS == 4) {
-            lo = __ldcs(reinterpret_cast<const unsigned int *>(codes) + c);
+            uint32_t w = __ldcs(reinterpret_cast<const unsigned int *>(codes) + c);
+            uint32_t zb = SYM ? 8u : (uint32_t)__ldg(&zeros[gidx]);
+            if (SYM) w ^= 0x88888888u;                              // two's complement -> q + 8
+            const uint32_t s2 = s_bits * 0x00010001u;
+            const uint32_t z2 = (0x4300u + zb) * 0x00010001u;
+            const uint32_t w4 = w >> 4;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o[i] = dq_pair_u4(w, w4, i, s2, z2);
         } else {
             const uint2 p = __ldcs(reinterpret_cast<const uint2 *>(codes) + c);
-            lo = p.x; hi = p.y;
-        }
-        uint32_t o[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float p0 = __fmul_rn(s_f, (float)(code_at<BITS, SYM>(lo, hi, 2 * j) - z));
-            const float p1 = __fmul_rn(s_f, (float)(code_at<BITS, SYM>(lo, hi, 2 * j + 1) - z));
-            o[j] = dev::pack_bf16x2(p0, p1);
+            const int z = SYM ? 0 : (int)(int8_t)__ldg(&zeros[gidx]);
+            const float off = -(8388736.0f + (float)z);              // -(2^23 + 128 + Z), exact
+            const float s_f = __uint_as_float(s_bits << 16);
+            const uint32_t lo = p.x ^ 0x80808080u, hi = p.y ^ 0x80808080u;
+            o[0] = dq_pair_i8(lo, 0, off, s_f);
+            o[1] = dq_pair_i8(lo, 1, off, s_f);
+            o[2] = dq_pair_i8(hi, 0, off, s_f);
+            o[3] = dq_pair_i8(hi, 1, off, s_f);
         }
         __stcs(out + c, make_uint4(o[0], o[1], o[2], o[3]));
     }

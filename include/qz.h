@@ -182,9 +182,9 @@ QZ_API qz_status qz_w8a16_gemv(const void *a, const void *codes, const void *sca
 
 /*
  * Size of the scratch array built into the library for
- * qz_w4a16_gemv_noalloc (4 MiB, held on every GPU that loads the library).
+ * qz_w4a16_gemv_noalloc (8 MiB, held on every GPU that loads the library).
  */
-#define QZ_GEMV_NOALLOC_SCRATCH_BYTES (4u << 20)
+#define QZ_GEMV_NOALLOC_SCRATCH_BYTES (8u << 20)
 
 /*
  * W4A16 decode GEMV that allocates nothing and takes no workspace.  The

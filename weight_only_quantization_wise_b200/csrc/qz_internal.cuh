@@ -57,12 +57,16 @@ qz_status launch_dequantize(const void *codes, const void *scales, const void *z
                             int64_t N, int64_t K, int bits, int symmetric,
                             int64_t group_size, void *w_hat, cudaStream_t stream);
 
-// GEMV split-K plan: number of K splits and workspace bytes.
+// GEMV work plan (stream-K): the (32-row task x 128-wide K block) units are
+// split into equal contiguous ranges, one per launched warp; a task whose
+// units span several warps is reduced through per-task partial slots.
 struct GemvPlan {
-    int splits;
-    int64_t tiles;        // 16-row tiles
-    size_t partial_bytes; // fp32 partials [splits][M][N]
-    size_t counter_bytes; // uint32 per tile
+    int64_t tasks;        // 32-row tasks
+    int64_t kblocks;      // 128-wide K blocks per task
+    int64_t warps;        // launched warps (a multiple of the warps per CTA)
+    int64_t slots;        // partial slots per task (max contributors)
+    size_t partial_bytes; // fp32 partials [tasks][slots][M][32]
+    size_t counter_bytes; // uint32 arrival counter per task
     size_t total_bytes;
 };
 GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K);
@@ -122,6 +126,11 @@ __device__ __forceinline__ uint32_t bf16_round_up_bits(float s) {
 __device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
     uint32_t r;
     asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+__device__ __forceinline__ uint32_t bf16x2_add(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
     return r;
 }
 __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {

@@ -39,7 +39,7 @@
 
 #include <mutex>
 
-#include "qz_internal.cuh"
+#include "qz_sm100.cuh"
 
 namespace qz {
 
@@ -47,6 +47,8 @@ namespace qz {
 __device__ unsigned int g_device_error_word = 0;
 
 namespace {
+
+using namespace sm100;
 
 constexpr int kStages = 4;
 constexpr int kTileN = 128;               // weight rows per tile (MMA M)
@@ -65,10 +67,8 @@ constexpr int kThreads = 32 * (2 + kDequantWarps + kEpilogueWarps);
 constexpr int kSmemBytes =
     kStages * (kActStageBytes + kPackStageBytes) + kStagingBytes + 1024 + 256;
 
-// instruction descriptor, kind::f16: D f32, A bf16, B bf16, both K-major,
-// N = 256 (>>3), M = 128 (>>4)
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
-                            ((uint32_t)(kTileM >> 3) << 17) | ((uint32_t)(kTileN >> 4) << 24);
+// instruction descriptor: MMA M = 128 weight rows, N = 256 tokens
+constexpr uint32_t kIdesc = idesc_bf16(kTileN, kTileM);
 
 struct SmemLayout {
     // offsets from the 1024-aligned base
@@ -91,115 +91,13 @@ struct SmemLayout {
 static_assert(SmemLayout::end + 1024 <= kSmemBytes, "shared memory layout");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ uint64_t global_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    return t;
-}
-
-// Bounded wait: true when the phase completed, false when `limit_ns` of wall
-// time ran out or another thread of the CTA aborted (then the caller unwinds).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns,
+// Bounded waits that report through this file's device error word.
+__device__ __forceinline__ bool gemm_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns,
                                           volatile uint32_t *abort_flag) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_ns();
-    for (;;) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (global_ns() - t0 > limit_ns) break;
-    }
-    *abort_flag = 1u;
-    atomicOr(&g_device_error_word, 1u);
-    return false;
+    return mbar_wait(bar, parity, limit_ns, abort_flag, &g_device_error_word);
 }
-
-// Wait used while unwinding: copies and MMAs already issued complete on their
-// own, so this bound (2 s) is independent of the caller's limit.
-constexpr uint64_t kDrainLimitNs = 2000000000ull;
-__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
-    volatile uint32_t never = 0;
-    mbar_wait(bar, parity, kDrainLimitNs, &never);
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
-                                            uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-        : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() {
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
-// 1024 bytes apart (stride byte offset), leading byte offset unused (1),
-// descriptor version 1.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
-    uint64_t d = 0;
-    d |= (uint64_t)((addr >> 4) & 0x3FFFu);
-    d |= (uint64_t)1u << 16;                 // leading byte offset (16 B units)
-    d |= (uint64_t)(1024u >> 4) << 32;       // stride byte offset
-    d |= (uint64_t)1u << 46;                 // version
-    d |= (uint64_t)2u << 61;                 // 128-byte swizzle
-    return d;
-}
-
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                       uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(kIdesc), "r"(accumulate)
-        : "memory");
-}
-
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-        : "memory");
-}
-
-__device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {"
-        "%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-        "r"(r[15])
-        : "memory");
+__device__ __forceinline__ void gemm_drain(uint32_t bar, uint32_t parity) {
+    mbar_drain(bar, parity, &g_device_error_word);
 }
 
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int x, int y) {
@@ -210,36 +108,17 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t sr
         : "memory");
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
+
 __device__ __forceinline__ void tma_store_wait_read() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
+
 __device__ __forceinline__ void tma_store_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
+
 __device__ __forceinline__ void epilogue_bar_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpilogueWarps) : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {"
-        "%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr)
-        : "memory");
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// Natural-order bf16 pair (k = 2i, 2i+1) of a packed code word: byte i of
-// `w` holds q_{2i} in its low nibble, byte i of `w >> 4` holds q_{2i+1}.
-__device__ __forceinline__ uint32_t dequant_pair_nat(uint32_t w, uint32_t w4, int i,
-                                                     uint32_t s2, uint32_t z2) {
-    const uint32_t sel = (uint32_t)i | ((uint32_t)(4 + i) << 8);
-    const uint32_t t = dev::prmt(w, w4, sel);
-    const uint32_t x = (t & 0x000F000Fu) | 0x43004300u;          // bf16(128 + q)
-    return dev::bf16x2_mul(dev::bf16x2_sub(x, z2), s2);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -307,7 +186,7 @@ w4a16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
                 const int n0 = (tile % tiles_n) * kTileN, m0 = (tile / tiles_n) * kTileM;
                 for (int kt = 0; kt < KT; ++kt, ++it) {
                     const int s = it % kStages, r = it / kStages;
-                    if (r > 0 && !mbar_wait(empty_bar(s), (r - 1) & 1, wait_limit, abort_flag)) {
+                    if (r > 0 && !gemm_wait(empty_bar(s), (r - 1) & 1, wait_limit, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -321,7 +200,7 @@ w4a16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
             }
             // every issued copy must have landed before the CTA may exit
             for (int s = 0; s < kStages; ++s)
-                if (issued_round[s] >= 0) mbar_drain(full_bar(s), issued_round[s] & 1);
+                if (issued_round[s] >= 0) gemm_drain(full_bar(s), issued_round[s] & 1);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -330,29 +209,29 @@ w4a16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
             bool ok = true;
             int it = 0, tcount = 0;
             for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++tcount) {
-                if (tcount > 0 && !mbar_wait(dempty_bar, (tcount - 1) & 1, wait_limit, abort_flag)) {
+                if (tcount > 0 && !gemm_wait(dempty_bar, (tcount - 1) & 1, wait_limit, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 for (int kt = 0; kt < KT; ++kt, ++it) {
                     const int s = it % kStages, r = it / kStages;
-                    ok = mbar_wait(full_bar(s), r & 1, wait_limit, abort_flag) &&
-                         mbar_wait(afull_bar(s), r & 1, wait_limit, abort_flag);
+                    ok = gemm_wait(full_bar(s), r & 1, wait_limit, abort_flag) &&
+                         gemm_wait(afull_bar(s), r & 1, wait_limit, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t act_addr = sbase + SmemLayout::act + s * kActStageBytes;
 #pragma unroll
                     for (int j = 0; j < kTileK / 16; ++j)
                         mma_ts(tmem_acc, tmem_a + s * kACols + j * 8,
-                               smem_desc_sw128(act_addr + j * 32), (kt > 0 || j > 0) ? 1u : 0u);
+                               smem_desc_sw128(act_addr + j * 32), kIdesc, (kt > 0 || j > 0) ? 1u : 0u);
                     mma_commit(empty_bar(s));
                 }
                 if (ok) mma_commit(dfull_bar);
             }
             // every issued MMA must finish before tensor memory is released
             mma_commit(drain_bar);
-            mbar_drain(drain_bar, 0);
+            gemm_drain(drain_bar, 0);
         }
         __syncwarp();
     } else if (warp < kFirstEpilogueWarp) {
@@ -387,7 +266,7 @@ w4a16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
                     asm volatile("prefetch.global.L1 [%0];" ::"l"(&zrow[gp]));
                 }
                 // warp-uniform: the tcgen05.st below needs every lane
-                if (!__all_sync(0xFFFFFFFFu, mbar_wait(full_bar(s), r & 1, wait_limit, abort_flag))) {
+                if (!__all_sync(0xFFFFFFFFu, gemm_wait(full_bar(s), r & 1, wait_limit, abort_flag))) {
                     ok = false;
                     break;
                 }
@@ -430,7 +309,7 @@ w4a16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
             // One decision for the four epilogue warps (they meet at named
             // barriers below): the storer publishes the abort flag after every
             // warp has finished its bounded wait.
-            __all_sync(0xFFFFFFFFu, mbar_wait(dfull_bar, tcount & 1, wait_limit, abort_flag));
+            __all_sync(0xFFFFFFFFu, gemm_wait(dfull_bar, tcount & 1, wait_limit, abort_flag));
             epilogue_bar_sync();
             if (storer) {
                 // the previous tile's store must have finished reading the staging tile
@@ -483,46 +362,22 @@ w4a16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
     }
 }
 
-// ---------------------------------------------------------------------------
-// Host: tensor maps through the driver entry point (no link-time libcuda).
-// ---------------------------------------------------------------------------
-using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                   const cuuint32_t *, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion,
-                                   CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    });
-    return fn;
-}
-
-bool make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner,
-                 uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
-                 CUtensorMapSwizzle swz) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[2] = {inner, outer};
-    const cuuint64_t strides[1] = {row_bytes};
-    const cuuint32_t box[2] = {box_inner, box_outer};
-    const cuuint32_t elem[2] = {1, 1};
-    return fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, elem,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 size_t gemm_workspace_bytes(int64_t, int64_t, int64_t) { return 0; }
+
+unsigned int *device_error_word() {
+    static unsigned int *addr[64] = {};
+    static std::once_flag once[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::call_once(once[dev], [dev] {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error_word) == cudaSuccess)
+            addr[dev] = static_cast<unsigned int *>(p);
+    });
+    return addr[dev];
+}
 
 qz_status launch_w4a16_gemm(const void *a, const void *codes, const void *scales,
                             const void *zeros, int64_t M, int64_t N, int64_t K,

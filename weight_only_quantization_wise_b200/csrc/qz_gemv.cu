@@ -9,34 +9,41 @@
 // Design (one warp = 32 weight rows over a K range):
 //   * Lane (g = lane/4, t = lane%4) streams, per 128-wide K block, its 32
 //     consecutive k of rows g, g+8, g+16, g+24 (16 bytes of int4 codes or 32
-//     bytes of int8 codes per row) with cp.async into a ring of STAGES blocks
-//     in the warp's own slice of shared memory, so that STAGES-1 blocks are in
-//     flight while one is computed without holding them in registers.  Each
-//     lane reads back only what it copied, so the ring needs no barrier:
-//     cp.async.wait_group orders it.  Scales and zeros are prefetched one
-//     block ahead in registers; the activation vector, which every warp
-//     reads, is loaded from L1 when its block is computed.
+//     bytes of int8 codes per row) with cp.async into a ring of kStages
+//     blocks in the warp's own slice of shared memory, so that kStages-1
+//     blocks are in flight while one is computed, without holding them in
+//     registers.  The codes each lane copies are the ones it reads back.
+//   * int4 with groups of a multiple of 128: the scales and zeros of the
+//     block ride in the same ring slot.  Lane (g, t) copies the aligned
+//     32-bit words holding the scale and the zero of row g + 8t, so the 32
+//     rows of the warp take two 4-byte copies per lane; after
+//     cp.async.wait_group and a warp barrier every lane reads the words of
+//     its four rows with two 16-byte shared loads and builds (S, S) and
+//     bf16(-(128 + Z)) twice with one byte permute each.  Since the warp's
+//     first row is a multiple of 32 and its rows differ by multiples of 8,
+//     all four rows of a lane share the word offset of their entries.
+//     Other group sizes (32, 64) load the lane's scales and zeros directly.
 //   * Codes are dequantized in registers to bf16 exactly as qz_dequantize
 //     forms them.  int4: a LOP3 builds bf16(128 + q) for two nibbles,
-//     sub.rn.bf16x2 removes (128 + Z) exactly, mul.rn.bf16x2 by the bf16 scale
-//     rounds S*(q - Z) once.  int8: the byte (XOR 0x80) is placed in the
-//     mantissa of 2^23, one packed fp32 subtraction gives q exactly, a packed
-//     fp32 multiply gives the exact S*q, cvt.rn.bf16x2 rounds it once.
-//     The subtraction adds a precomputed -(128 + Z) so that no per-pair
-//     negation is needed.
+//     add.rn.bf16x2 of bf16(-(128 + Z)) leaves q - Z exactly, mul.rn.bf16x2
+//     by the bf16 scale rounds S*(q - Z) once.  int8: the byte (XOR 0x80) is
+//     placed in the mantissa of 2^23, one fp32 subtraction gives q exactly,
+//     an fp32 multiply gives the exact S*q, cvt.rn.bf16x2 rounds it once.
 //   * A byte of codes yields the pairs (q_j, q_{j+4}), so the K axis is
 //     permuted consistently for both MMA operands: the pairs are the A operand
 //     (16 rows x 16 k) of mma.sync m16n8k16 with fp32 accumulation and the
 //     activations (tokens as the 8 columns) are the B operand, permuted to
 //     match with PRMT once per k for both 16-row tiles of the warp.  For
-//     M > 8 a second MMA covers tokens 8..15.
+//     M > 8 a second MMA covers tokens 8..15.  Columns of tokens >= M read
+//     token M-1's activations; their outputs are dropped.
 //   * Stream-K: the (32-row task x 128-wide K block) units are divided into
 //     equal contiguous ranges, one per launched warp, and exactly a whole
 //     number of CTAs per SM is launched, so every SM gets the same work.  A
 //     task covered by one warp is written directly; otherwise each
 //     contributing warp writes its fp32 partial tile into the task's slot
 //     and bumps the task's counter, and the last one to arrive adds the
-//     slots in order (deterministic), writes bf16 y and resets the counter.
+//     slots in order (deterministic), one row per lane, writes bf16 y and
+//     resets the counter.
 #include <cuda_runtime.h>
 
 #include "qz_internal.cuh"
@@ -47,7 +54,6 @@ namespace {
 constexpr int kWarpsPerCta = 4;
 constexpr int kThreads = 32 * kWarpsPerCta;
 constexpr int kRowsPerWarp = 32;                       // two 16-row MMA tiles
-constexpr int kRowsPerCta = kRowsPerWarp * kWarpsPerCta;
 
 // bf16 pair (nibble j, nibble j+4) of a code word: bf16_rne(S * (q - Z)).
 // nz2 holds bf16(-(128 + Z)) twice.
@@ -85,9 +91,8 @@ struct RowWords {
     uint32_t w[4][kWordsPerRow];   // rows g, g+8, g+16, g+24
 };
 
-template <int BITS, int MB>
-struct Stage {
-    uint32_t s[4], z[4];           // int4: per-row scale bits and zero of this block
+struct RowParams {
+    uint32_t s2[4], z2[4];         // int4, rows g + 8j: (S, S) and bf16(-(128 + Z)) twice
 };
 
 template <int MB>
@@ -96,16 +101,22 @@ struct Act {
 };
 
 template <int BITS>
-constexpr int kGemvStages = BITS == 4 ? 8 : 4;           // a power of two
+constexpr int kStages = BITS == 4 ? 4 : 3;               // ring slots per warp
 template <int BITS>
 constexpr int kLaneRowBytes = BITS == 4 ? 16 : 32;     // codes of one row per lane per block
 template <int BITS>
-constexpr int kWarpStageBytes = 4 * 32 * kLaneRowBytes<BITS>;
+constexpr int kCodeBytes = 4 * 32 * kLaneRowBytes<BITS>;
+constexpr int kSzBytes = 256;                          // 32 scale words + 32 zero words
 template <int BITS>
-constexpr int kGemvSmemBytes = kWarpsPerCta * kGemvStages<BITS> * kWarpStageBytes<BITS>;
+constexpr int kSlotBytes = kCodeBytes<BITS> + (BITS == 4 ? kSzBytes : 0);
+template <int BITS>
+constexpr int kGemvSmemBytes = kWarpsPerCta * kStages<BITS> * kSlotBytes<BITS>;
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() {
     asm volatile("cp.async.commit_group;" ::: "memory");
@@ -115,7 +126,7 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Byte offset, inside a warp's stage, of 16-byte piece `half` of row j for
+// Byte offset, inside a warp's slot, of 16-byte piece `half` of row j for
 // `lane`: pieces of 32 lanes are contiguous, so each 8-lane phase of a
 // 16-byte shared load reads 128 consecutive bytes (no bank conflicts).
 template <int BITS>
@@ -124,37 +135,24 @@ __device__ __forceinline__ uint32_t piece_offset(int j, int half, int lane) {
 }
 
 template <int BITS>
-__device__ __forceinline__ void issue_block(uint32_t stage_base, const uint8_t *const (&rowp)[4],
-                                            const bool (&valid)[4], int kb, int lane) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        if (!valid[j]) continue;
-#pragma unroll
-        for (int h = 0; h < kLaneRowBytes<BITS> / 16; ++h)
-            cp_async16(stage_base + piece_offset<BITS>(j, h, lane),
-                       rowp[j] + kb * (BITS == 4 ? 64 : 128) + 16 * h);
-    }
-}
-
-template <int BITS>
-__device__ __forceinline__ void read_block(RowWords<BITS> &rw, const uint8_t *stage, int lane) {
+__device__ __forceinline__ void read_block(RowWords<BITS> &rw, const uint8_t *slot, int lane) {
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
         for (int h = 0; h < kLaneRowBytes<BITS> / 16; ++h) {
-            const uint4 v = *reinterpret_cast<const uint4 *>(stage + piece_offset<BITS>(j, h, lane));
+            const uint4 v = *reinterpret_cast<const uint4 *>(slot + piece_offset<BITS>(j, h, lane));
             rw.w[j][4 * h + 0] = v.x; rw.w[j][4 * h + 1] = v.y;
             rw.w[j][4 * h + 2] = v.z; rw.w[j][4 * h + 3] = v.w;
         }
 }
 
-template <int BITS, int MB>
 struct GemvArgs {
     const uint16_t *a;
     const uint8_t *codes;
     const uint16_t *scales;
     const uint8_t *zeros;
     int M, N, K, group_size, group_shift;
+    int blocks_per_group, bpg_shift;   // group_size / 128 and its log2 (-1: not a power of 2)
     uint16_t *y;
     float *partials;
     uint32_t *counters;
@@ -163,58 +161,51 @@ struct GemvArgs {
     int kblocks, slots;
 };
 
-template <int BITS, int MB>
-__device__ __forceinline__ void load_stage(Stage<BITS, MB> &st, const GemvArgs<BITS, MB> &p,
-                                           const bool (&valid)[4], const int (&rows)[4], int kb,
-                                           int g, int t) {
+// Group index of 128-wide block kb when the group size is a multiple of 128.
+__device__ __forceinline__ int group_of_block(const GemvArgs &p, int kb) {
+    return p.bpg_shift >= 0 ? (kb >> p.bpg_shift) : kb / p.blocks_per_group;
+}
+
+// Scales and zeros of the lane's four rows for block kb, loaded directly
+// (group sizes below 128, or scale/zero arrays the ring cannot copy).
+__device__ __forceinline__ void load_params_direct(RowParams &rp, const GemvArgs &p,
+                                                   const bool (&valid)[4], const int (&rows)[4],
+                                                   int kb, int t) {
     const int k0 = kb * 128 + t * 32;
-    if (BITS == 4) {
-        const int gpr = p.K / p.group_size;
-        const int gi = p.group_shift >= 0 ? (k0 >> p.group_shift) : (k0 / p.group_size);
+    const int64_t gpr = p.K / p.group_size;
+    const int gi = p.group_shift >= 0 ? (k0 >> p.group_shift) : (k0 / p.group_size);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            st.s[j] = valid[j] ? __ldg(&p.scales[(int64_t)rows[j] * gpr + gi]) : 0u;
-            st.z[j] = valid[j] ? __ldg(&p.zeros[(int64_t)rows[j] * gpr + gi]) : 0u;
-        }
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t s = valid[j] ? __ldg(&p.scales[(int64_t)rows[j] * gpr + gi]) : 0u;
+        const uint32_t z = valid[j] ? __ldg(&p.zeros[(int64_t)rows[j] * gpr + gi]) : 0u;
+        rp.s2[j] = s * 0x00010001u;                      // (S, S)
+        rp.z2[j] = (0xC300u + z) * 0x00010001u;          // bf16(-(128 + Z)) twice
     }
 }
 
-// Activations of one block for tokens g (and g + 8): read from L1/L2 (the
-// vector is shared by every warp) right before the block is computed.
-template <int BITS, int MB>
-__device__ __forceinline__ void load_act(Act<MB> &ac, const GemvArgs<BITS, MB> &p, int kb, int g,
-                                         int t) {
+// Activations of one block for tokens g (and g + 8), clamped to M - 1: read
+// from L1/L2 (the vector is shared by every warp) right before the block is
+// computed.
+template <int MB>
+__device__ __forceinline__ void load_act(Act<MB> &ac, const GemvArgs &p, int kb, int g, int t) {
     const int k0 = kb * 128 + t * 32;
 #pragma unroll
     for (int mb = 0; mb < MB; ++mb) {
-        const int tok = 8 * mb + g;
-        if (tok < p.M) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(p.a + (int64_t)tok * p.K + k0);
+        const int tok = min(8 * mb + g, p.M - 1);
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.a + (int64_t)tok * p.K + k0);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint4 v = __ldg(src + q);
-                ac.x[mb][4 * q + 0] = v.x; ac.x[mb][4 * q + 1] = v.y;
-                ac.x[mb][4 * q + 2] = v.z; ac.x[mb][4 * q + 3] = v.w;
-            }
-        } else {
-#pragma unroll
-            for (int q = 0; q < 16; ++q) ac.x[mb][q] = 0u;
+        for (int q = 0; q < 4; ++q) {
+            const uint4 v = __ldg(src + q);
+            ac.x[mb][4 * q + 0] = v.x; ac.x[mb][4 * q + 1] = v.y;
+            ac.x[mb][4 * q + 2] = v.z; ac.x[mb][4 * q + 3] = v.w;
         }
     }
 }
 
 template <int BITS, int MB>
-__device__ __forceinline__ void compute_stage(const Stage<BITS, MB> &st, const Act<MB> &ac,
+__device__ __forceinline__ void compute_block(const RowParams &rp, const Act<MB> &ac,
                                               const RowWords<BITS> &rw, const float (&sf)[4],
                                               float (&acc)[2][MB][4]) {
-    uint32_t s2[4], z2[4];
-    if (BITS == 4) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            s2[j] = st.s[j] * 0x00010001u;                  // (S, S)
-            z2[j] = (0xC300u + st.z[j]) * 0x00010001u;      // bf16(-(128 + Z)) twice
-        }
-    }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         uint32_t lo8[4], hi8[4];
@@ -235,10 +226,10 @@ __device__ __forceinline__ void compute_stage(const Stage<BITS, MB> &st, const A
                 const int ja = 2 * rt, jb = 2 * rt + 1;     // rows g(+16), g+8(+16)
                 uint32_t a0, a1, a2, a3;
                 if (BITS == 4) {
-                    a0 = dequant_pair_u4(rw.w[ja][i], 2 * h, s2[ja], z2[ja]);
-                    a1 = dequant_pair_u4(rw.w[jb][i], 2 * h, s2[jb], z2[jb]);
-                    a2 = dequant_pair_u4(rw.w[ja][i], 2 * h + 1, s2[ja], z2[ja]);
-                    a3 = dequant_pair_u4(rw.w[jb][i], 2 * h + 1, s2[jb], z2[jb]);
+                    a0 = dequant_pair_u4(rw.w[ja][i], 2 * h, rp.s2[ja], rp.z2[ja]);
+                    a1 = dequant_pair_u4(rw.w[jb][i], 2 * h, rp.s2[jb], rp.z2[jb]);
+                    a2 = dequant_pair_u4(rw.w[ja][i], 2 * h + 1, rp.s2[ja], rp.z2[ja]);
+                    a3 = dequant_pair_u4(rw.w[jb][i], 2 * h + 1, rp.s2[jb], rp.z2[jb]);
                 } else {
                     a0 = dequant_pair_i8(lo8[ja], hi8[ja], 2 * h, sf[ja]);
                     a1 = dequant_pair_i8(lo8[jb], hi8[jb], 2 * h, sf[jb]);
@@ -258,13 +249,61 @@ __device__ __forceinline__ int64_t warp_of_unit(int64_t u, int64_t U, int64_t W)
     return ((u + 1) * W - 1) / U;
 }
 
+// Deterministic split-K sum: y[t][row] = sum over slots c = 0, 1, ... of
+// base[c * slot_elems + t * ROWS + r], for the M <= MAXTOK tokens, added in
+// slot order.  The loads of two slots for every token (eight slots when
+// M = 1) are issued together.
+template <int MAXTOK, int ROWS>
+__device__ __forceinline__ void reduce_slots(const float *base, int64_t slot_elems,
+                                             int contributors, int M, int r, int64_t row,
+                                             int N, uint16_t *y) {
+    if (M == 1) {                      // one token: eight slots' loads per round trip
+        float sum = 0.0f;
+        for (int c0 = 0; c0 < contributors; c0 += 8) {
+            float v[8];
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc)
+                v[cc] = c0 + cc < contributors ? __ldcg(base + (int64_t)(c0 + cc) * slot_elems + r)
+                                               : 0.0f;
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc)
+                if (c0 + cc < contributors) sum += v[cc];
+        }
+        if (row < N) y[row] = (uint16_t)dev::f32_to_bf16_rne(sum);
+        return;
+    }
+    float sum[MAXTOK];
+#pragma unroll
+    for (int t = 0; t < MAXTOK; ++t) sum[t] = 0.0f;
+    for (int c = 0; c < contributors; c += 2) {
+        float x0[MAXTOK], x1[MAXTOK];
+        const float *s0 = base + (int64_t)c * slot_elems + r;
+        const bool two = c + 1 < contributors;
+#pragma unroll
+        for (int t = 0; t < MAXTOK; ++t) {
+            x0[t] = t < M ? __ldcg(s0 + t * ROWS) : 0.0f;
+            x1[t] = (t < M && two) ? __ldcg(s0 + slot_elems + t * ROWS) : 0.0f;
+        }
+#pragma unroll
+        for (int t = 0; t < MAXTOK; ++t) {
+            sum[t] += x0[t];
+            if (two) sum[t] += x1[t];
+        }
+    }
+    if (row < N) {
+#pragma unroll
+        for (int t = 0; t < MAXTOK; ++t)
+            if (t < M) y[(int64_t)t * N + row] = (uint16_t)dev::f32_to_bf16_rne(sum[t]);
+    }
+}
+
 // acc[rt][mb][j] holds y[tok = 8mb + 2t + (j&1)][row = n0 + 16rt + g + 8(j>>1)].
 // `whole`: this warp covered every K block of the task.  Otherwise the
 // partial goes to slot (this warp - the task's first warp) and the last of
-// the task's contributors adds the slots in order.
-template <int BITS, int MB>
-__device__ __forceinline__ void gemv_flush(float (&acc)[2][MB][4], const GemvArgs<BITS, MB> &p,
-                                           int task, bool whole, int64_t w, int lane) {
+// the task's contributors adds the slots in order, lane l summing row l.
+template <int MB>
+__device__ __forceinline__ void gemv_flush(float (&acc)[2][MB][4], const GemvArgs &p, int task,
+                                           bool whole, int64_t w, int lane) {
     const int g = lane >> 2, t = lane & 3;
     const int n0 = task * kRowsPerWarp;
     if (whole) {
@@ -304,68 +343,35 @@ __device__ __forceinline__ void gemv_flush(float (&acc)[2][MB][4], const GemvArg
     prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
     if (prev != (uint32_t)(contributors - 1)) return;
     __threadfence();
-    // Add the slots in order; four contributors' values are loaded at a time
-    // so that the L2 round trips overlap.
-    float sum[2][MB][4];
-#pragma unroll
-    for (int rt = 0; rt < 2; ++rt)
-#pragma unroll
-        for (int mb = 0; mb < MB; ++mb)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) sum[rt][mb][j] = 0.0f;
-    for (int c0 = 0; c0 < contributors; c0 += 4) {
-        float v[4][2][MB][4];
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
-#pragma unroll
-            for (int rt = 0; rt < 2; ++rt)
-#pragma unroll
-                for (int mb = 0; mb < MB; ++mb)
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int rl = 16 * rt + g + 8 * (j >> 1);
-                        const int tok = 8 * mb + 2 * t + (j & 1);
-                        v[cc][rt][mb][j] = (c0 + cc < contributors && tok < p.M)
-                            ? __ldcg(&base[(c0 + cc) * slot_elems + tok * kRowsPerWarp + rl])
-                            : 0.0f;
-                    }
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
-#pragma unroll
-            for (int rt = 0; rt < 2; ++rt)
-#pragma unroll
-                for (int mb = 0; mb < MB; ++mb)
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        if (c0 + cc < contributors) sum[rt][mb][j] += v[cc][rt][mb][j];
-    }
-#pragma unroll
-    for (int rt = 0; rt < 2; ++rt)
-#pragma unroll
-        for (int mb = 0; mb < MB; ++mb)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int row = n0 + 16 * rt + g + 8 * (j >> 1);
-                const int tok = 8 * mb + 2 * t + (j & 1);
-                if (row < p.N && tok < p.M)
-                    p.y[(int64_t)tok * p.N + row] = (uint16_t)dev::f32_to_bf16_rne(sum[rt][mb][j]);
-            }
+    // The last contributor: lane l adds row l of every slot in slot order,
+    // for all tokens at once (two slots' loads in flight per round trip).
+    reduce_slots<8 * MB, kRowsPerWarp>(base, slot_elems, contributors, p.M, lane, n0 + lane,
+                                       p.N, p.y);
     if (lane == 0) p.counters[task] = 0u;
 }
 
-template <int BITS, int MB>
-__global__ void __launch_bounds__(kThreads)
-gemv_kernel(const GemvArgs<BITS, MB> p) {
+// RING_SZ: int4 scales and zeros travel through the cp.async ring (group
+// size a multiple of 128, 4-byte aligned arrays whose 4-byte words stay
+// inside them).
+template <int BITS, int MB, bool RING_SZ>
+__global__ void __launch_bounds__(kThreads, MB == 1 ? 4 : 3)
+gemv_kernel(const GemvArgs p) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int64_t w = (int64_t)blockIdx.x * kWarpsPerCta + warp;
     int64_t u = w * p.units / p.warps;
     const int64_t u_end = (w + 1) * p.units / p.warps;
 
-    constexpr int S = kGemvStages<BITS>;
+    constexpr int S = kStages<BITS>;
+    constexpr int kSlot = kSlotBytes<BITS>;
     extern __shared__ __align__(16) uint8_t gemv_smem[];
-    uint8_t *ring = gemv_smem + warp * S * kWarpStageBytes<BITS>;
+    uint8_t *ring = gemv_smem + warp * S * kSlot;
     const uint32_t ring_u32 = (uint32_t)__cvta_generic_to_shared(ring);
+    const int64_t gpr = BITS == 4 ? p.K / p.group_size : 1;
+    const uint32_t *scale_words = reinterpret_cast<const uint32_t *>(p.scales);
+    const uint32_t *zero_words = reinterpret_cast<const uint32_t *>(p.zeros);
+    // (row * gpr) mod 4 is the same for rows g, g+8, g+16, g+24 of any task
+    const int word_phase = (int)(((int64_t)g * gpr) & 3);
 
     while (u < u_end) {
         const int task = (int)(u / p.kblocks);
@@ -389,6 +395,28 @@ gemv_kernel(const GemvArgs<BITS, MB> p) {
             if (BITS == 8 && valid[j])
                 sf[j] = __uint_as_float((uint32_t)__ldg(&p.scales[rows[j]]) << 16);
         }
+        // the row whose scale and zero words this lane copies
+        const int row_c = n0 + g + 8 * t;
+        const bool valid_c = RING_SZ && row_c < p.N;
+        const int64_t entry_c = (int64_t)(valid_c ? row_c : 0) * gpr;
+        const uint32_t sz_dst = kCodeBytes<BITS> + 4u * (uint32_t)(4 * g + t);
+
+        auto issue = [&](int kb, uint32_t slot) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (!valid[j]) continue;
+#pragma unroll
+                for (int h = 0; h < kLaneRowBytes<BITS> / 16; ++h)
+                    cp_async16(slot + piece_offset<BITS>(j, h, lane),
+                               rowp[j] + kb * (BITS == 4 ? 64 : 128) + 16 * h);
+            }
+            if (RING_SZ && valid_c) {
+                const int64_t e = entry_c + group_of_block(p, kb);
+                cp_async4(slot + sz_dst, scale_words + (e >> 1));
+                cp_async4(slot + sz_dst + 128u, zero_words + (e >> 2));
+            }
+        };
+
         float acc[2][MB][4];
 #pragma unroll
         for (int rt = 0; rt < 2; ++rt)
@@ -399,115 +427,143 @@ gemv_kernel(const GemvArgs<BITS, MB> p) {
 
 #pragma unroll
         for (int q = 0; q < S - 1; ++q) {
-            if (q < nkb) issue_block<BITS>(ring_u32 + q * kWarpStageBytes<BITS>, rowp, valid,
-                                           kb_begin + q, lane);
+            if (q < nkb) issue(kb_begin + q, ring_u32 + q * kSlot);
             cp_async_commit();
         }
-        Stage<BITS, MB> sa, sb;
-        load_stage(sa, p, valid, rows, kb_begin, g, t);
-        for (int i = 0; i < nkb; i += 2) {
+        int slot = 0;
+        for (int ii = 0; ii < nkb; ++ii) {
+            cp_async_wait<S - 2>();                  // block ii has landed in its slot
+            if (RING_SZ) __syncwarp();               // ... every lane's copies of it, too
+            const int refill = ii + S - 1;           // into the slot read one block ago
+            const int rslot = slot == 0 ? S - 1 : slot - 1;
+            if (refill < nkb) issue(kb_begin + refill, ring_u32 + rslot * kSlot);
+            cp_async_commit();
+            const int kb = kb_begin + ii;
+            const uint8_t *cur = ring + slot * kSlot;
+            Act<MB> ac;
+            load_act(ac, p, kb, g, t);
+            RowWords<BITS> rw;
+            read_block<BITS>(rw, cur, lane);
+            RowParams rp;
+            if (BITS == 4) {
+                if (RING_SZ) {
+                    const uint4 ws = *reinterpret_cast<const uint4 *>(cur + kCodeBytes<BITS> + 16 * g);
+                    const uint4 wz =
+                        *reinterpret_cast<const uint4 *>(cur + kCodeBytes<BITS> + 128 + 16 * g);
+                    const int phase = word_phase + group_of_block(p, kb);
+                    const uint32_t os = (uint32_t)(phase & 1) * 2u, oz = (uint32_t)(phase & 3);
+                    const uint32_t sel_s = os * 0x0101u + (os + 1u) * 0x1010u;   // (S, S)
+                    const uint32_t sel_z = oz * 0x0101u + 0x4040u;               // (0xC3, Z) x 2
+                    const uint32_t wsv[4] = {ws.x, ws.y, ws.z, ws.w};
+                    const uint32_t wzv[4] = {wz.x, wz.y, wz.z, wz.w};
 #pragma unroll
-            for (int v = 0; v < 2; ++v) {
-                const int ii = i + v;
-                if (ii >= nkb) break;
-                Stage<BITS, MB> &cur = v == 0 ? sa : sb;
-                Stage<BITS, MB> &nxt = v == 0 ? sb : sa;
-                cp_async_wait<S - 2>();               // block ii has landed in its slot
-                const int refill = ii + S - 1;       // into the slot read one block ago
-                if (refill < nkb)
-                    issue_block<BITS>(ring_u32 + (refill & (S - 1)) * kWarpStageBytes<BITS>, rowp,
-                                      valid, kb_begin + refill, lane);
-                cp_async_commit();
-                Act<MB> ac;
-                load_act(ac, p, kb_begin + ii, g, t);
-                RowWords<BITS> rw;
-                read_block<BITS>(rw, ring + (ii & (S - 1)) * kWarpStageBytes<BITS>, lane);
-                if (ii + 1 < nkb) load_stage(nxt, p, valid, rows, kb_begin + ii + 1, g, t);
-                compute_stage(cur, ac, rw, sf, acc);
+                    for (int j = 0; j < 4; ++j) {
+                        rp.s2[j] = dev::prmt(wsv[j], 0u, sel_s);
+                        rp.z2[j] = dev::prmt(wzv[j], 0xC3C3C3C3u, sel_z);
+                    }
+                } else {
+                    load_params_direct(rp, p, valid, rows, kb, t);
+                }
             }
+            compute_block<BITS, MB>(rp, ac, rw, sf, acc);
+            slot = slot == S - 1 ? 0 : slot + 1;
         }
         cp_async_wait<0>();
         __syncwarp();                                // the ring is reused by the next task
-        gemv_flush<BITS, MB>(acc, p, task, nkb == p.kblocks, w, lane);
+        gemv_flush<MB>(acc, p, task, nkb == p.kblocks, w, lane);
         u += nkb;
     }
 }
 
-int group_shift_of(int64_t g) {
-    if (g <= 0 || (g & (g - 1)) != 0) return -1;
+int log2_exact(int64_t v) {
+    if (v <= 0 || (v & (v - 1)) != 0) return -1;
     int s = 0;
-    while ((int64_t(1) << s) < g) ++s;
+    while ((int64_t(1) << s) < v) ++s;
     return s;
 }
 
-template <int BITS, int MB>
-void set_smem_once() {
-    static bool done[64] = {};
+template <typename Kernel>
+void set_smem_once(Kernel kernel, int bytes, bool (&done)[64]) {
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !done[dev]) {
-        cudaFuncSetAttribute(gemv_kernel<BITS, MB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kGemvSmemBytes<BITS>);
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
         done[dev] = true;
     }
+}
+
+template <int BITS, int MB, bool RING_SZ>
+void launch_variant(const GemvArgs &args, dim3 grid, cudaStream_t st) {
+    static bool done[64] = {};
+    constexpr int smem = kGemvSmemBytes<BITS>;
+    set_smem_once(gemv_kernel<BITS, MB, RING_SZ>, smem, done);
+    gemv_kernel<BITS, MB, RING_SZ><<<grid, kThreads, smem, st>>>(args);
 }
 
 template <int BITS>
 qz_status launch_gemv(const void *a, const void *codes, const void *scales, const void *zeros,
                       int64_t M, int64_t N, int64_t K, int64_t group_size, void *y,
                       void *workspace, const GemvPlan &plan, cudaStream_t st) {
-    float *partials = nullptr;
-    uint32_t *counters = nullptr;
+    GemvArgs args;
+    args.a = static_cast<const uint16_t *>(a);
+    args.codes = static_cast<const uint8_t *>(codes);
+    args.scales = static_cast<const uint16_t *>(scales);
+    args.zeros = static_cast<const uint8_t *>(zeros);
+    args.M = (int)M; args.N = (int)N; args.K = (int)K;
+    args.group_size = (int)group_size;
+    args.group_shift = log2_exact(group_size);
+    args.blocks_per_group = group_size % 128 == 0 ? (int)(group_size / 128) : 1;
+    args.bpg_shift = log2_exact(args.blocks_per_group);
+    args.y = static_cast<uint16_t *>(y);
+    args.partials = nullptr;
+    args.counters = nullptr;
     if (plan.total_bytes > 0) {
-        partials = static_cast<float *>(workspace);
-        counters = reinterpret_cast<uint32_t *>(static_cast<char *>(workspace) + plan.partial_bytes);
+        args.partials = static_cast<float *>(workspace);
+        args.counters =
+            reinterpret_cast<uint32_t *>(static_cast<char *>(workspace) + plan.partial_bytes);
     }
+    args.units = plan.tasks * plan.kblocks;
+    args.warps = plan.warps;
+    args.kblocks = (int)plan.kblocks;
+    args.slots = (int)plan.slots;
     const dim3 grid((unsigned)(plan.warps / kWarpsPerCta));
-    auto fill = [&](auto &args) {
-        args.a = static_cast<const uint16_t *>(a);
-        args.codes = static_cast<const uint8_t *>(codes);
-        args.scales = static_cast<const uint16_t *>(scales);
-        args.zeros = static_cast<const uint8_t *>(zeros);
-        args.M = (int)M; args.N = (int)N; args.K = (int)K;
-        args.group_size = (int)group_size;
-        args.group_shift = group_shift_of(group_size);
-        args.y = static_cast<uint16_t *>(y);
-        args.partials = partials;
-        args.counters = counters;
-        args.units = plan.tasks * plan.kblocks;
-        args.warps = plan.warps;
-        args.kblocks = (int)plan.kblocks;
-        args.slots = (int)plan.slots;
-    };
-    constexpr int smem = kGemvSmemBytes<BITS>;
-    if (M <= 8) {
-        GemvArgs<BITS, 1> args;
-        fill(args);
-        set_smem_once<BITS, 1>();
-        gemv_kernel<BITS, 1><<<grid, kThreads, smem, st>>>(args);
+
+    // The ring copies the aligned 4-byte words holding each scale and zero;
+    // they stay inside the arrays when N * K / g is a multiple of 4.
+    if constexpr (BITS == 4) {
+        const int64_t entries = N * (K / group_size);
+        const bool ring_sz = group_size % 128 == 0 && aligned(scales, 4) && aligned(zeros, 4) &&
+                             entries % 4 == 0;
+        if (M <= 8) {
+            if (ring_sz) launch_variant<4, 1, true>(args, grid, st);
+            else launch_variant<4, 1, false>(args, grid, st);
+        } else {
+            if (ring_sz) launch_variant<4, 2, true>(args, grid, st);
+            else launch_variant<4, 2, false>(args, grid, st);
+        }
     } else {
-        GemvArgs<BITS, 2> args;
-        fill(args);
-        set_smem_once<BITS, 2>();
-        gemv_kernel<BITS, 2><<<grid, kThreads, smem, st>>>(args);
+        if (M <= 8) launch_variant<8, 1, false>(args, grid, st);
+        else launch_variant<8, 2, false>(args, grid, st);
     }
     return launch_status();
 }
 
 }  // namespace
 
-// Stream-K plan.  Three 4-warp CTAs fit on an SM (64 KB of cp.async ring
-// each), so 1, 2 or 3 CTAs per SM are launched -- always the same number on
-// every SM -- with at least about four K blocks per warp.
-constexpr int kGemvCtasPerSm = 3;
+// Stream-K plan.  With at most 128 registers per thread four 4-warp CTAs fit
+// on an SM (three for M > 8), and the ring of a CTA takes 36 KB (int4) or
+// 48 KB (int8) of shared memory.  The same number of CTAs runs on every SM,
+// as many as give each warp at least two K blocks.
+constexpr int kGemvMinBlocksPerWarp = 2;
 
 GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K) {
     GemvPlan p{};
     p.tasks = ceil_div(N, kRowsPerWarp);
     p.kblocks = K / 128;
     const int64_t units = p.tasks * p.kblocks;
-    int64_t per_sm = units / ((int64_t)kSmCount * kWarpsPerCta * 4);
-    if (per_sm > kGemvCtasPerSm) per_sm = kGemvCtasPerSm;
+    const int64_t max_per_sm = M <= 8 ? 4 : 3;
+    int64_t per_sm = units / ((int64_t)kSmCount * kWarpsPerCta * kGemvMinBlocksPerWarp);
+    if (per_sm > max_per_sm) per_sm = max_per_sm;
     if (per_sm < 1) per_sm = 1;
     p.warps = (int64_t)kSmCount * per_sm * kWarpsPerCta;
     if (p.warps > units) p.warps = ceil_div(units, kWarpsPerCta) * kWarpsPerCta;
@@ -517,6 +573,8 @@ GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K) {
     if (p.slots > p.kblocks) p.slots = p.kblocks;
     p.partial_bytes = (size_t)p.tasks * p.slots * (size_t)M * kRowsPerWarp * sizeof(float);
     p.partial_bytes = (p.partial_bytes + 255) & ~(size_t)255;
+    const size_t tc_partials = tc_gemv_plan(M, N, K).partial_bytes;
+    if (tc_partials > p.partial_bytes) p.partial_bytes = tc_partials;
     p.counter_bytes = (size_t)ceil_div(p.tasks, 64) * 64 * sizeof(uint32_t);
     p.total_bytes = p.partial_bytes + p.counter_bytes;
     return p;
@@ -526,6 +584,10 @@ qz_status launch_w4a16_gemv(const void *a, const void *codes, const void *scales
                             const void *zeros, int64_t M, int64_t N, int64_t K,
                             int64_t group_size, void *y, void *workspace,
                             const GemvPlan &plan, cudaStream_t st) {
+    if (tc_gemv_eligible(a, codes, scales, zeros, M, N, K, group_size))
+        return launch_w4a16_gemv_tc(
+            a, codes, scales, zeros, M, N, K, group_size, y, static_cast<float *>(workspace),
+            reinterpret_cast<uint32_t *>(static_cast<char *>(workspace) + plan.partial_bytes), st);
     return launch_gemv<4>(a, codes, scales, zeros, M, N, K, group_size, y, workspace, plan, st);
 }
 

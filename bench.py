@@ -521,6 +521,24 @@ def run_kernel_case(name, reps):
     print(f"{name}: {reps} launches ok")
 
 
+def run_layer_sets():
+    """Every part of the step on the 7B layer set, one input copy, each part's
+    three launches issued twice in a row (for ncu: the second set of each part
+    is the measured one)."""
+    import weight_only_quantization_wise_b200 as qz
+    global ROT
+    ROT = 1
+    dev = torch.device("cuda", 0)
+    ls = LayerSet(qz, dev)
+    torch.cuda.synchronize()
+    for name, method, *_ in PARTS:
+        for _ in range(2):
+            getattr(ls, method)(0)
+    torch.cuda.synchronize()
+    assert qz.qz_device_status() == 0
+    print("layer sets: " + ", ".join(p[0] for p in PARTS) + " (x2 each) ok")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -529,10 +547,14 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--kernel", choices=sorted(PROFILE_CASES),
-                    help="run one kernel case a few times (for profiling) and exit")
+    ap.add_argument("--kernel", choices=sorted(PROFILE_CASES) + ["layer_sets"],
+                    help="run one kernel case a few times, or every part once on the 7B "
+                         "layer set (layer_sets), for profiling, and exit")
     ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()
+    if args.kernel == "layer_sets":
+        run_layer_sets()
+        return
     if args.kernel:
         run_kernel_case(args.kernel, args.reps)
         return

@@ -573,8 +573,6 @@ GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K) {
     if (p.slots > p.kblocks) p.slots = p.kblocks;
     p.partial_bytes = (size_t)p.tasks * p.slots * (size_t)M * kRowsPerWarp * sizeof(float);
     p.partial_bytes = (p.partial_bytes + 255) & ~(size_t)255;
-    const size_t tc_partials = tc_gemv_plan(M, N, K).partial_bytes;
-    if (tc_partials > p.partial_bytes) p.partial_bytes = tc_partials;
     p.counter_bytes = (size_t)ceil_div(p.tasks, 64) * 64 * sizeof(uint32_t);
     p.total_bytes = p.partial_bytes + p.counter_bytes;
     return p;
@@ -584,10 +582,6 @@ qz_status launch_w4a16_gemv(const void *a, const void *codes, const void *scales
                             const void *zeros, int64_t M, int64_t N, int64_t K,
                             int64_t group_size, void *y, void *workspace,
                             const GemvPlan &plan, cudaStream_t st) {
-    if (tc_gemv_eligible(a, codes, scales, zeros, M, N, K, group_size))
-        return launch_w4a16_gemv_tc(
-            a, codes, scales, zeros, M, N, K, group_size, y, static_cast<float *>(workspace),
-            reinterpret_cast<uint32_t *>(static_cast<char *>(workspace) + plan.partial_bytes), st);
     return launch_gemv<4>(a, codes, scales, zeros, M, N, K, group_size, y, workspace, plan, st);
 }
 

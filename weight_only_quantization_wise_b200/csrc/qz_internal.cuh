@@ -61,35 +61,16 @@ qz_status launch_dequantize(const void *codes, const void *scales, const void *z
 // split into equal contiguous ranges, one per launched warp; a task whose
 // units span several warps is reduced through per-task partial slots.
 struct GemvPlan {
-    int64_t tasks;        // 32-row tasks of the mma.sync kernel
+    int64_t tasks;        // 32-row tasks
     int64_t kblocks;      // 128-wide K blocks per task
     int64_t warps;        // launched warps (a multiple of the warps per CTA)
     int64_t slots;        // partial slots per task (max contributors)
-    size_t partial_bytes; // fp32 partials: max of [tasks][slots][M][32] and the tcgen05 layout
+    size_t partial_bytes; // fp32 partials [tasks][slots][M][32]
     size_t counter_bytes; // uint32 arrival counter per task
     size_t total_bytes;
 };
-// Workspace plan covering both GEMV kernels: partials (the larger of the two
-// layouts) at offset 0, then one uint32 counter per 32-row task (the tcgen05
-// kernel's 128-row tasks use the first ones).
+// Workspace: fp32 partials at offset 0, then one uint32 counter per task.
 GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K);
-
-// tcgen05 GEMV (int4, group size a multiple of 128): stream-K over
-// (128-row task x 128-wide K block) units, two CTAs per SM.
-struct TcGemvPlan {
-    int64_t tasks;        // 128-row tasks
-    int64_t kblocks;      // 128-wide K blocks per task
-    int64_t ctas;         // launched CTAs
-    int64_t slots;        // partial slots per task
-    size_t partial_bytes; // fp32 partials [tasks][slots][M][128]
-};
-TcGemvPlan tc_gemv_plan(int64_t M, int64_t N, int64_t K);
-bool tc_gemv_eligible(const void *a, const void *codes, const void *scales, const void *zeros,
-                      int64_t M, int64_t N, int64_t K, int64_t group_size);
-qz_status launch_w4a16_gemv_tc(const void *a, const void *codes, const void *scales,
-                               const void *zeros, int64_t M, int64_t N, int64_t K,
-                               int64_t group_size, void *y, float *partials, uint32_t *counters,
-                               cudaStream_t stream);
 
 qz_status launch_w4a16_gemv(const void *a, const void *codes, const void *scales,
                             const void *zeros, int64_t M, int64_t N, int64_t K,

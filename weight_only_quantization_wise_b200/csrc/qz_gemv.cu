@@ -13,7 +13,7 @@
 //     blocks in the warp's own slice of shared memory, so that kStages-1
 //     blocks are in flight while one is computed, without holding them in
 //     registers.  The codes each lane copies are the ones it reads back.
-//   * int4 with groups of a multiple of 128: the scales and zeros of the
+//   * int4 with groups of 128 * 2^i: the scales and zeros of the
 //     block ride in the same ring slot.  Lane (g, t) copies the aligned
 //     32-bit words holding the scale and the zero of row g + 8t, so the 32
 //     rows of the warp take two 4-byte copies per lane; after
@@ -22,7 +22,7 @@
 //     bf16(-(128 + Z)) twice with one byte permute each.  Since the warp's
 //     first row is a multiple of 32 and its rows differ by multiples of 8,
 //     all four rows of a lane share the word offset of their entries.
-//     Other group sizes (32, 64) load the lane's scales and zeros directly.
+//     Other group sizes load the lane's scales and zeros directly.
 //   * Codes are dequantized in registers to bf16 exactly as qz_dequantize
 //     forms them.  int4: a LOP3 builds bf16(128 + q) for two nibbles,
 //     add.rn.bf16x2 of bf16(-(128 + Z)) leaves q - Z exactly, mul.rn.bf16x2
@@ -59,7 +59,7 @@ constexpr int kRowsPerWarp = 32;                       // two 16-row MMA tiles
 // nz2 holds bf16(-(128 + Z)) twice.
 __device__ __forceinline__ uint32_t dequant_pair_u4(uint32_t word, int j, uint32_t s2,
                                                     uint32_t nz2) {
-    const uint32_t x = ((word >> (4 * j)) & 0x000F000Fu) | 0x43004300u;   // bf16(128+q)
+    const uint32_t x = dev::and_or<0x000F000Fu>(word >> (4 * j), 0x43004300u);   // bf16(128+q)
     return dev::bf16x2_mul(dev::bf16x2_add(x, nz2), s2);
 }
 
@@ -152,7 +152,7 @@ struct GemvArgs {
     const uint16_t *scales;
     const uint8_t *zeros;
     int M, N, K, group_size, group_shift;
-    int blocks_per_group, bpg_shift;   // group_size / 128 and its log2 (-1: not a power of 2)
+    int bpg_shift;                     // log2(group_size / 128) (ring path), else -1
     uint16_t *y;
     float *partials;
     uint32_t *counters;
@@ -161,9 +161,10 @@ struct GemvArgs {
     int kblocks, slots;
 };
 
-// Group index of 128-wide block kb when the group size is a multiple of 128.
+// Group index of 128-wide block kb when the group size is 128 * 2^bpg_shift
+// (the ring path's condition).
 __device__ __forceinline__ int group_of_block(const GemvArgs &p, int kb) {
-    return p.bpg_shift >= 0 ? (kb >> p.bpg_shift) : kb / p.blocks_per_group;
+    return kb >> p.bpg_shift;
 }
 
 // Scales and zeros of the lane's four rows for block kb, loaded directly
@@ -431,6 +432,7 @@ gemv_kernel(const GemvArgs p) {
             cp_async_commit();
         }
         int slot = 0;
+#pragma unroll 2
         for (int ii = 0; ii < nkb; ++ii) {
             cp_async_wait<S - 2>();                  // block ii has landed in its slot
             if (RING_SZ) __syncwarp();               // ... every lane's copies of it, too
@@ -512,8 +514,7 @@ qz_status launch_gemv(const void *a, const void *codes, const void *scales, cons
     args.M = (int)M; args.N = (int)N; args.K = (int)K;
     args.group_size = (int)group_size;
     args.group_shift = log2_exact(group_size);
-    args.blocks_per_group = group_size % 128 == 0 ? (int)(group_size / 128) : 1;
-    args.bpg_shift = log2_exact(args.blocks_per_group);
+    args.bpg_shift = group_size % 128 == 0 ? log2_exact(group_size / 128) : -1;
     args.y = static_cast<uint16_t *>(y);
     args.partials = nullptr;
     args.counters = nullptr;
@@ -532,7 +533,7 @@ qz_status launch_gemv(const void *a, const void *codes, const void *scales, cons
     // they stay inside the arrays when N * K / g is a multiple of 4.
     if constexpr (BITS == 4) {
         const int64_t entries = N * (K / group_size);
-        const bool ring_sz = group_size % 128 == 0 && aligned(scales, 4) && aligned(zeros, 4) &&
+        const bool ring_sz = args.bpg_shift >= 0 && aligned(scales, 4) && aligned(zeros, 4) &&
                              entries % 4 == 0;
         if (M <= 8) {
             if (ring_sz) launch_variant<4, 1, true>(args, grid, st);

@@ -140,7 +140,7 @@ __device__ __forceinline__ uint2 chunk_codes(const float (&x)[8], float s_f, flo
         uint32_t p[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j)   // byte j: code 2j low nibble, code 2j+1 high nibble
-            p[j] = (b[2 * j] & 0x0Fu) | ((b[2 * j + 1] << 4) & 0xF0u);
+            p[j] = dev::and_or<0x0Fu>(b[2 * j], b[2 * j + 1] << 4);   // only byte 0 is used
         const uint32_t lo = dev::prmt(p[0], p[1], 0x0040u);
         const uint32_t hi = dev::prmt(p[2], p[3], 0x0040u);
         return make_uint2(dev::prmt(lo, hi, 0x5410u), 0u);
@@ -491,7 +491,7 @@ qz_status quantize_typed(const void *w, int64_t N, int64_t K, int64_t g, void *c
 __device__ __forceinline__ uint32_t dq_pair_u4(uint32_t w, uint32_t w4, int i, uint32_t s2,
                                                uint32_t z2) {
     const uint32_t t = dev::prmt(w, w4, (uint32_t)i | ((uint32_t)(4 + i) << 8));
-    const uint32_t x = (t & 0x000F000Fu) | 0x43004300u;            // bf16(128 + q)
+    const uint32_t x = dev::and_or<0x000F000Fu>(t, 0x43004300u);  // bf16(128 + q)
     return dev::bf16x2_mul(dev::bf16x2_sub(x, z2), s2);
 }
 

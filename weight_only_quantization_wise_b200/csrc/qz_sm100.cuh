@@ -171,7 +171,7 @@ __device__ __forceinline__ uint32_t dequant_pair_nat(uint32_t w, uint32_t w4, in
                                                      uint32_t s2, uint32_t z2) {
     const uint32_t sel = (uint32_t)i | ((uint32_t)(4 + i) << 8);
     const uint32_t t = dev::prmt(w, w4, sel);
-    const uint32_t x = (t & 0x000F000Fu) | 0x43004300u;          // bf16(128 + q)
+    const uint32_t x = dev::and_or<0x000F000Fu>(t, 0x43004300u);  // bf16(128 + q)
     return dev::bf16x2_mul(dev::bf16x2_sub(x, z2), s2);
 }
 #endif  // __CUDACC__

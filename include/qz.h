@@ -221,6 +221,23 @@ QZ_API qz_status qz_w4a16_gemv_noalloc(const void *a, const void *codes, const v
 QZ_API void qz_set_device_wait_limit(uint64_t limit);
 
 /*
+ * How a decode GEMV launch (qz_w4a16_gemv, qz_w8a16_gemv, qz_w4a16_gemm with
+ * M <= 16) may overlap the kernel launched before it on the same stream.
+ * Not part of the method: a launch-latency optimisation for decode loops.
+ *   0  (default) plain stream order.
+ *   1  programmatic dependent launch: the GEMV may start while the previous
+ *      kernel finishes and fetches its first K blocks of packed codes, scales
+ *      and zeros at once; it reads activations and writes y and the
+ *      workspace only after that kernel has completed.  Only for callers
+ *      whose weights are not written by the kernel launched just before the
+ *      GEMV on the stream (weights quantized once and kept, as in a decode
+ *      loop); otherwise the GEMV may read stale weights.
+ * Host-only, process-wide, applies to later calls.  Returns
+ * QZ_ERR_INVALID_ARG for other values.  qz_w4a16_gemv_noalloc always uses 0.
+ */
+QZ_API qz_status qz_set_launch_overlap(int32_t mode);
+
+/*
  * Reads and clears the device error word of the current device (written by a
  * kernel whose bounded wait ran out).  Synchronizes the current device.
  * Returns QZ_OK or QZ_ERR_DEVICE_TIMEOUT (or QZ_ERR_CUDA).

@@ -132,3 +132,10 @@ def test_w8a16_gemv_rejects(args, expect):
 ])
 def test_w4a16_gemm_rejects(args, expect):
     assert L().qz_w4a16_gemm(*args) == expect
+
+
+def test_launch_overlap_setter():
+    assert qz.lib.qz_set_launch_overlap(2) == INVALID
+    assert qz.lib.qz_set_launch_overlap(-1) == INVALID
+    for mode in (1, 0):               # ends on the default
+        assert qz.lib.qz_set_launch_overlap(mode) == OK

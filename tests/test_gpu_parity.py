@@ -456,3 +456,30 @@ def test_quantize_near_half_way_values(dev):
             ref = oracle.quantize_pack(u16(w), bits, sym, g)
             got = gpu_quantize(w.to(dev), bits, sym, g)
             assert_quant_equal(got, ref)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_gemv_launch_overlap_modes_agree(dev, bits):
+    """Both launch-overlap modes give bit-identical results, also when GEMVs
+    follow each other on the stream (each reads the previous one's output)."""
+    N, K, M = 4096, 4096, 4
+    w = synthetic.weights(N, K, sigma=0.02, seed=71).to(dev)
+    if bits == 4:
+        c, s, z = qz.qz_quantize_pack(w, 4, False, 128)
+        run = lambda a: qz.qz_w4a16_gemv(a, c, s, z, N, K, 128)
+    else:
+        c, s, _ = qz.qz_quantize_pack(w, 8, True, K)
+        run = lambda a: qz.qz_w8a16_gemv(a, c, s, N, K)
+    a0 = synthetic.activations(M, K, seed=72, device=dev)
+    outs = {}
+    try:
+        for mode in (0, 1):
+            qz.qz_set_launch_overlap(mode)
+            a = a0
+            for _ in range(4):            # chained: each GEMV consumes the previous one's output
+                a = run(a)
+            torch.cuda.synchronize()
+            outs[mode] = u16(a)
+    finally:
+        qz.qz_set_launch_overlap(0)
+    assert np.array_equal(outs[0], outs[1])

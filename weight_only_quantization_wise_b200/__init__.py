@@ -14,7 +14,8 @@ import torch
 __all__ = [
     "QzError", "lib", "qz_version", "qz_status_string", "qz_packed_bytes",
     "qz_workspace_bytes", "qz_quantize_pack", "qz_dequantize", "qz_w4a16_gemv",
-    "qz_w4a16_gemm", "qz_w8a16_gemv", "qz_set_device_wait_limit", "qz_device_status",
+    "qz_w4a16_gemm", "qz_w8a16_gemv", "qz_set_device_wait_limit", "qz_set_launch_overlap",
+    "qz_device_status",
     "Workspace", "QZ_OP_QUANTIZE_PACK", "QZ_OP_DEQUANTIZE", "QZ_OP_W4A16_GEMV",
     "QZ_OP_W4A16_GEMM", "QZ_OP_W8A16_GEMV", "EXPORTED_SYMBOLS",
 ]
@@ -39,6 +40,7 @@ _SIGS = {
     "qz_w8a16_gemv": ([_p, _p, _p, _i64, _i64, _i64, _p, _p, _sz, _p], ctypes.c_int),
     "qz_w4a16_gemv_noalloc": ([_p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p], ctypes.c_int),
     "qz_set_device_wait_limit": ([ctypes.c_uint64], None),
+    "qz_set_launch_overlap": ([ctypes.c_int32], ctypes.c_int),
     "qz_device_status": ([], ctypes.c_int),
 }
 EXPORTED_SYMBOLS = tuple(_SIGS)
@@ -216,6 +218,11 @@ def qz_w8a16_gemv(a, codes, scales, N, K, y=None, workspace=None, stream=None):
 
 def qz_set_device_wait_limit(limit: int) -> None:
     lib.qz_set_device_wait_limit(int(limit))
+
+
+def qz_set_launch_overlap(mode: int) -> None:
+    """Launch overlap of the decode GEMV with the preceding kernel (see qz.h)."""
+    _check(lib.qz_set_launch_overlap(int(mode)), "qz_set_launch_overlap")
 
 
 def qz_device_status() -> int:

@@ -11,6 +11,10 @@ namespace qz {
 static std::atomic<uint64_t> g_wait_limit{0};
 constexpr uint64_t kDefaultWaitLimit = 2000000000ull;   // 2 s in nanoseconds
 
+static std::atomic<int32_t> g_launch_overlap{0};
+
+int32_t launch_overlap() { return g_launch_overlap.load(std::memory_order_relaxed); }
+
 uint64_t device_wait_limit() {
     const uint64_t v = g_wait_limit.load(std::memory_order_relaxed);
     return v ? v : kDefaultWaitLimit;
@@ -107,12 +111,12 @@ QZ_API qz_status qz_workspace_bytes(int32_t op, int64_t M, int64_t N, int64_t K,
     case QZ_OP_W8A16_GEMV: {
         const qz_status s = check_gemv_shape(M, N, K);
         if (s != QZ_OK) return s;
-        *bytes = gemv_plan(M, N, K).total_bytes;
+        *bytes = gemv_plan(M, N, K, op == QZ_OP_W4A16_GEMV ? 4 : 8).total_bytes;
         return QZ_OK;
     }
     case QZ_OP_W4A16_GEMM:
         if (M < 1 || N < 1 || K < 1) return QZ_ERR_INVALID_ARG;
-        *bytes = M <= 16 && K % 128 == 0 ? gemv_plan(M, N, K).total_bytes
+        *bytes = M <= 16 && K % 128 == 0 ? gemv_plan(M, N, K, 4).total_bytes
                                          : gemm_workspace_bytes(M, N, K);
         return QZ_OK;
     default:
@@ -158,11 +162,11 @@ QZ_API qz_status qz_w4a16_gemv(const void *a, const void *codes, const void *sca
     if (!a || !codes || !scales || !zeros || !y) return QZ_ERR_INVALID_ARG;
     if (!aligned(a, 16) || !aligned(codes, 16) || !aligned(scales, 2) || !aligned(y, 2))
         return QZ_ERR_ALIGNMENT;
-    const GemvPlan plan = gemv_plan(M, N, K);
+    const GemvPlan plan = gemv_plan(M, N, K, 4);
     s = check_workspace(plan.total_bytes, workspace, workspace_bytes);
     if (s != QZ_OK) return s;
     return launch_w4a16_gemv(a, codes, scales, zeros, M, N, K, group_size, y, workspace, plan,
-                             as_stream(stream));
+                             launch_overlap(), as_stream(stream));
 }
 
 QZ_API qz_status qz_w8a16_gemv(const void *a, const void *codes, const void *scales,
@@ -173,10 +177,11 @@ QZ_API qz_status qz_w8a16_gemv(const void *a, const void *codes, const void *sca
     if (!a || !codes || !scales || !y) return QZ_ERR_INVALID_ARG;
     if (!aligned(a, 16) || !aligned(codes, 16) || !aligned(scales, 2) || !aligned(y, 2))
         return QZ_ERR_ALIGNMENT;
-    const GemvPlan plan = gemv_plan(M, N, K);
+    const GemvPlan plan = gemv_plan(M, N, K, 8);
     s = check_workspace(plan.total_bytes, workspace, workspace_bytes);
     if (s != QZ_OK) return s;
-    return launch_w8a16_gemv(a, codes, scales, M, N, K, y, workspace, plan, as_stream(stream));
+    return launch_w8a16_gemv(a, codes, scales, M, N, K, y, workspace, plan, launch_overlap(),
+                             as_stream(stream));
 }
 
 QZ_API qz_status qz_w4a16_gemm(const void *a, const void *codes, const void *scales,
@@ -202,6 +207,12 @@ QZ_API qz_status qz_w4a16_gemm(const void *a, const void *codes, const void *sca
 
 QZ_API void qz_set_device_wait_limit(uint64_t limit) {
     g_wait_limit.store(limit, std::memory_order_relaxed);
+}
+
+QZ_API qz_status qz_set_launch_overlap(int32_t mode) {
+    if (mode < 0 || mode > 1) return QZ_ERR_INVALID_ARG;
+    g_launch_overlap.store(mode, std::memory_order_relaxed);
+    return QZ_OK;
 }
 
 }  // extern "C"

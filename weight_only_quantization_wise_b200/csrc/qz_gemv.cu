@@ -111,6 +111,10 @@ template <int BITS>
 constexpr int kSlotBytes = kCodeBytes<BITS> + (BITS == 4 ? kSzBytes : 0);
 template <int BITS>
 constexpr int kGemvSmemBytes = kWarpsPerCta * kStages<BITS> * kSlotBytes<BITS>;
+// Resident CTAs per SM: registers allow five (int4, M <= 8: at most 102 per
+// thread), four (int8, M <= 8: shared memory) or three (M > 8).
+template <int BITS, int MB>
+constexpr int kCtasPerSm = MB == 1 ? (BITS == 4 ? 5 : 4) : 3;
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -159,6 +163,7 @@ struct GemvArgs {
     int64_t units;        // tasks * kblocks
     int64_t warps;        // launched warps
     int kblocks, slots;
+    int prefetch_early;   // launch overlap: first blocks' weights before the grid wait
 };
 
 // Group index of 128-wide block kb when the group size is 128 * 2^bpg_shift
@@ -243,6 +248,16 @@ __device__ __forceinline__ void compute_block(const RowParams &rp, const Act<MB>
             }
         }
     }
+}
+
+// Programmatic dependent launch: let the next kernel on the stream be
+// scheduled; wait until the previous one has completed and its writes are
+// visible (a no-op when this grid was not launched as a dependent).
+__device__ __forceinline__ void allow_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void wait_for_previous_grid() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // First warp whose unit range contains unit u (ranges: [w*U/W, (w+1)*U/W)).
@@ -355,13 +370,18 @@ __device__ __forceinline__ void gemv_flush(float (&acc)[2][MB][4], const GemvArg
 // size a multiple of 128, 4-byte aligned arrays whose 4-byte words stay
 // inside them).
 template <int BITS, int MB, bool RING_SZ>
-__global__ void __launch_bounds__(kThreads, MB == 1 ? 4 : 3)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm<BITS, MB>)
 gemv_kernel(const GemvArgs p) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int64_t w = (int64_t)blockIdx.x * kWarpsPerCta + warp;
     int64_t u = w * p.units / p.warps;
     const int64_t u_end = (w + 1) * p.units / p.warps;
+    // With launch overlap, only the first ring fill of weights (which the
+    // caller guarantees the previous kernel does not write) precedes the
+    // wait for the previous grid; every other global access follows it.
+    allow_dependents();
+    bool waited = !p.prefetch_early;
 
     constexpr int S = kStages<BITS>;
     constexpr int kSlot = kSlotBytes<BITS>;
@@ -431,6 +451,10 @@ gemv_kernel(const GemvArgs p) {
             if (q < nkb) issue(kb_begin + q, ring_u32 + q * kSlot);
             cp_async_commit();
         }
+        if (!waited) {
+            wait_for_previous_grid();
+            waited = true;
+        }
         int slot = 0;
 #pragma unroll 2
         for (int ii = 0; ii < nkb; ++ii) {
@@ -495,17 +519,27 @@ void set_smem_once(Kernel kernel, int bytes, bool (&done)[64]) {
 }
 
 template <int BITS, int MB, bool RING_SZ>
-void launch_variant(const GemvArgs &args, dim3 grid, cudaStream_t st) {
+void launch_variant(const GemvArgs &args, dim3 grid, int overlap, cudaStream_t st) {
     static bool done[64] = {};
     constexpr int smem = kGemvSmemBytes<BITS>;
     set_smem_once(gemv_kernel<BITS, MB, RING_SZ>, smem, done);
-    gemv_kernel<BITS, MB, RING_SZ><<<grid, kThreads, smem, st>>>(args);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = overlap > 0 ? 1 : 0;
+    cudaLaunchKernelEx(&cfg, gemv_kernel<BITS, MB, RING_SZ>, args);
 }
 
 template <int BITS>
 qz_status launch_gemv(const void *a, const void *codes, const void *scales, const void *zeros,
                       int64_t M, int64_t N, int64_t K, int64_t group_size, void *y,
-                      void *workspace, const GemvPlan &plan, cudaStream_t st) {
+                      void *workspace, const GemvPlan &plan, int overlap, cudaStream_t st) {
     GemvArgs args;
     args.a = static_cast<const uint16_t *>(a);
     args.codes = static_cast<const uint8_t *>(codes);
@@ -527,6 +561,7 @@ qz_status launch_gemv(const void *a, const void *codes, const void *scales, cons
     args.warps = plan.warps;
     args.kblocks = (int)plan.kblocks;
     args.slots = (int)plan.slots;
+    args.prefetch_early = overlap;
     const dim3 grid((unsigned)(plan.warps / kWarpsPerCta));
 
     // The ring copies the aligned 4-byte words holding each scale and zero;
@@ -536,33 +571,34 @@ qz_status launch_gemv(const void *a, const void *codes, const void *scales, cons
         const bool ring_sz = args.bpg_shift >= 0 && aligned(scales, 4) && aligned(zeros, 4) &&
                              entries % 4 == 0;
         if (M <= 8) {
-            if (ring_sz) launch_variant<4, 1, true>(args, grid, st);
-            else launch_variant<4, 1, false>(args, grid, st);
+            if (ring_sz) launch_variant<4, 1, true>(args, grid, overlap, st);
+            else launch_variant<4, 1, false>(args, grid, overlap, st);
         } else {
-            if (ring_sz) launch_variant<4, 2, true>(args, grid, st);
-            else launch_variant<4, 2, false>(args, grid, st);
+            if (ring_sz) launch_variant<4, 2, true>(args, grid, overlap, st);
+            else launch_variant<4, 2, false>(args, grid, overlap, st);
         }
     } else {
-        if (M <= 8) launch_variant<8, 1, false>(args, grid, st);
-        else launch_variant<8, 2, false>(args, grid, st);
+        if (M <= 8) launch_variant<8, 1, false>(args, grid, overlap, st);
+        else launch_variant<8, 2, false>(args, grid, overlap, st);
     }
     return launch_status();
 }
 
 }  // namespace
 
-// Stream-K plan.  With at most 128 registers per thread four 4-warp CTAs fit
-// on an SM (three for M > 8), and the ring of a CTA takes 36 KB (int4) or
-// 48 KB (int8) of shared memory.  The same number of CTAs runs on every SM,
-// as many as give each warp at least two K blocks.
-constexpr int kGemvMinBlocksPerWarp = 2;
+// Stream-K plan.  Up to kCtasPerSm 4-warp CTAs are resident on an SM (the
+// ring of a CTA takes 36 KB (int4) or 48 KB (int8) of shared memory).  The
+// same number of CTAs runs on every SM, as many as give each warp at least
+// four K blocks (fewer contributors per task shorten the split-K tail).
+constexpr int kGemvMinBlocksPerWarp = 4;
 
-GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K) {
+GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K, int bits) {
     GemvPlan p{};
     p.tasks = ceil_div(N, kRowsPerWarp);
     p.kblocks = K / 128;
     const int64_t units = p.tasks * p.kblocks;
-    const int64_t max_per_sm = M <= 8 ? 4 : 3;
+    const int64_t max_per_sm = M <= 8 ? (bits == 4 ? kCtasPerSm<4, 1> : kCtasPerSm<8, 1>)
+                                      : kCtasPerSm<4, 2>;
     int64_t per_sm = units / ((int64_t)kSmCount * kWarpsPerCta * kGemvMinBlocksPerWarp);
     if (per_sm > max_per_sm) per_sm = max_per_sm;
     if (per_sm < 1) per_sm = 1;
@@ -582,14 +618,16 @@ GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K) {
 qz_status launch_w4a16_gemv(const void *a, const void *codes, const void *scales,
                             const void *zeros, int64_t M, int64_t N, int64_t K,
                             int64_t group_size, void *y, void *workspace,
-                            const GemvPlan &plan, cudaStream_t st) {
-    return launch_gemv<4>(a, codes, scales, zeros, M, N, K, group_size, y, workspace, plan, st);
+                            const GemvPlan &plan, int overlap, cudaStream_t st) {
+    return launch_gemv<4>(a, codes, scales, zeros, M, N, K, group_size, y, workspace, plan,
+                          overlap, st);
 }
 
 qz_status launch_w8a16_gemv(const void *a, const void *codes, const void *scales,
                             int64_t M, int64_t N, int64_t K, void *y, void *workspace,
-                            const GemvPlan &plan, cudaStream_t st) {
-    return launch_gemv<8>(a, codes, scales, nullptr, M, N, K, K, y, workspace, plan, st);
+                            const GemvPlan &plan, int overlap, cudaStream_t st) {
+    return launch_gemv<8>(a, codes, scales, nullptr, M, N, K, K, y, workspace, plan, overlap,
+                          st);
 }
 
 }  // namespace qz

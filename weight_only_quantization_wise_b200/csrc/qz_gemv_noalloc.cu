@@ -70,7 +70,7 @@ extern "C" QZ_API qz_status qz_w4a16_gemv_noalloc(const void *a, const void *cod
     if (!qz::is_aligned(a, 16) || !qz::is_aligned(codes, 16) || !qz::is_aligned(scales, 2) ||
         !qz::is_aligned(y, 2))
         return QZ_ERR_ALIGNMENT;
-    const qz::GemvPlan plan = qz::gemv_plan(M, N, K);
+    const qz::GemvPlan plan = qz::gemv_plan(M, N, K, 4);
     if (plan.total_bytes > qz::kScratchBytes) return QZ_ERR_WORKSPACE;   // beyond the built-in maximum
     void *scratch = nullptr;
     if (plan.total_bytes > 0) {
@@ -82,6 +82,8 @@ extern "C" QZ_API qz_status qz_w4a16_gemv_noalloc(const void *a, const void *cod
                             plan.counter_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
             return QZ_ERR_CUDA;
     }
+    // plain stream order: the counter reset above is not a kernel, so a
+    // programmatic dependency on it would not be ordered
     return qz::launch_w4a16_gemv(a, codes, scales, zeros, M, N, K, group_size, y, scratch, plan,
-                                 static_cast<cudaStream_t>(stream));
+                                 0, static_cast<cudaStream_t>(stream));
 }

@@ -70,15 +70,16 @@ struct GemvPlan {
     size_t total_bytes;
 };
 // Workspace: fp32 partials at offset 0, then one uint32 counter per task.
-GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K);
+GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K, int bits);
 
+// `overlap`: qz_set_launch_overlap mode for this launch.
 qz_status launch_w4a16_gemv(const void *a, const void *codes, const void *scales,
                             const void *zeros, int64_t M, int64_t N, int64_t K,
                             int64_t group_size, void *y, void *workspace,
-                            const GemvPlan &plan, cudaStream_t stream);
+                            const GemvPlan &plan, int overlap, cudaStream_t stream);
 qz_status launch_w8a16_gemv(const void *a, const void *codes, const void *scales,
                             int64_t M, int64_t N, int64_t K, void *y, void *workspace,
-                            const GemvPlan &plan, cudaStream_t stream);
+                            const GemvPlan &plan, int overlap, cudaStream_t stream);
 
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 qz_status launch_w4a16_gemm(const void *a, const void *codes, const void *scales,
@@ -87,6 +88,8 @@ qz_status launch_w4a16_gemm(const void *a, const void *codes, const void *scales
                             cudaStream_t stream);
 
 uint64_t device_wait_limit();
+// qz_set_launch_overlap mode (0 or 1) for the decode GEMV launches.
+int32_t launch_overlap();
 // Device address of the word that bounded device-side waits set on expiry
 // (read and cleared by qz_device_status); null if it cannot be resolved.
 unsigned int *device_error_word();

@@ -345,6 +345,7 @@ def test_bulk_quantization_stack(dev):
 GEMM_CASES = [  # (M, N, K, g)
     (17, 128, 128, 128), (100, 200, 256, 64), (256, 128, 1024, 128),
     (300, 1000, 1024, 128), (512, 384, 2048, 256), (257, 130, 640, 128),
+    (64, 256, 640, 640), (96, 192, 384, 192),      # groups of 10 and 3 stages
 ]
 
 

@@ -241,6 +241,7 @@ w4a16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
         const int row_local = quarter * 32 + lane;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         const int gpr = K / group_size;
+        const int spg = group_size / kTileK;          // stages per group
         int it = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
@@ -248,22 +249,29 @@ w4a16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
             const bool valid = n < N;
             const uint16_t *srow = scales + (int64_t)(valid ? n : 0) * gpr;
             const uint8_t *zrow = zeros + (int64_t)(valid ? n : 0) * gpr;
-            uint32_t s_next = valid ? __ldg(&srow[0]) : 0u;
-            uint32_t z_next = valid ? __ldg(&zrow[0]) : 0u;
+            // Scales and zeros of the next four groups wait in a register FIFO
+            // (a group spans spg stages), so their loads are issued up to four
+            // groups before use and no per-stage index arithmetic is needed.
+            uint32_t sq[4], zq[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                sq[q] = (valid && q < gpr) ? __ldg(&srow[q]) : 0u;
+                zq[q] = (valid && q < gpr) ? __ldg(&zrow[q]) : 0u;
+            }
+            int stage_in_group = 0, next_group = 4;
             for (int kt = 0; kt < KT; ++kt, ++it) {
                 const int s = it % kStages, r = it / kStages;
-                const uint32_t sb = s_next, zb = z_next;
-                if (kt + 1 < KT && valid) {
-                    const int gi = ((kt + 1) * kTileK) / group_size;
-                    s_next = __ldg(&srow[gi]);
-                    z_next = __ldg(&zrow[gi]);
-                }
-                if (kt + 5 < KT && valid) {
-                    // bring the metadata of a stage 5 ahead into L1, so that the
-                    // load above (one stage ahead) hits L1 instead of L2
-                    const int gp = ((kt + 5) * kTileK) / group_size;
-                    asm volatile("prefetch.global.L1 [%0];" ::"l"(&srow[gp]));
-                    asm volatile("prefetch.global.L1 [%0];" ::"l"(&zrow[gp]));
+                const uint32_t sb = sq[0], zb = zq[0];
+                if (++stage_in_group == spg) {               // the next stage starts a new group
+                    stage_in_group = 0;
+#pragma unroll
+                    for (int q = 0; q < 3; ++q) {
+                        sq[q] = sq[q + 1];
+                        zq[q] = zq[q + 1];
+                    }
+                    sq[3] = (valid && next_group < gpr) ? __ldg(&srow[next_group]) : 0u;
+                    zq[3] = (valid && next_group < gpr) ? __ldg(&zrow[next_group]) : 0u;
+                    ++next_group;
                 }
                 // warp-uniform: the tcgen05.st below needs every lane
                 if (!__all_sync(0xFFFFFFFFu, gemm_wait(full_bar(s), r & 1, wait_limit, abort_flag))) {

@@ -12,8 +12,9 @@ One step is one pass of every hot-path row over the 7B-class decode layer set
   W4A16 prefill GEMM, M = 2048 tokens       (3 launches)
 Every input is resident in HBM and rotates over ROT copies (ROT x the packed
 layer set is far larger than the 126 MB L2), so each part reads cold weights.
-Each part of each rotation is a captured CUDA graph; CUDA events on the
-launching stream bracket the parts.  `value` is the headline of the metric:
+Each step is one captured CUDA graph (all parts, one rotation) with external
+CUDA event nodes between the parts, so the GPU runs a step without host gaps
+and each part's time is the device time between its two event nodes.  `value` is the headline of the metric:
 W4A16 decode GEMV GB/s (algorithmic bytes / GEMV time), aggregated over all
 ranks.  The other parts, the roofline of every kernel, the configurations
 that are not part of the step (70B decode shapes, the 2048 x 8192 x 8192
@@ -593,37 +594,45 @@ def main():
     qz.qz_set_launch_overlap(GEMV_LAUNCH_OVERLAP)
     torch.cuda.synchronize()
 
-    # one graph per (part, rotation); run each part once eagerly first
-    graphs = {}
+    # Every part runs once eagerly, then each step (all parts, one rotation)
+    # becomes one CUDA graph with external timing events recorded between the
+    # parts inside it, so a step runs without host gaps and each part's time
+    # is the device time between its two event nodes.
     with torch.cuda.stream(stream):
         for name, meth, *_ in PARTS:
-            fn = getattr(ls, meth)
-            fn(0)
-            for p in range(ROT):
-                graphs[(name, p)] = capture(lambda fn=fn, p=p: fn(p), stream)
+            getattr(ls, meth)(0)
     torch.cuda.synchronize()
     assert qz.qz_device_status() == 0
 
     npart = len(PARTS)
 
-    def run_steps(k, events=None, start=0):
-        for i in range(k):
-            p = (start + i) % ROT
-            for j, (name, *_r) in enumerate(PARTS):
-                if events is not None:
-                    events[i][j][0].record(stream)
-                graphs[(name, p)].replay()
-                if events is not None:
-                    events[i][j][1].record(stream)
+    def new_events():
+        return [(torch.cuda.Event(enable_timing=True, external=True),
+                 torch.cuda.Event(enable_timing=True, external=True)) for _ in range(npart)]
+
+    def capture_step(p, evs):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for j, (name, meth, *_r) in enumerate(PARTS):
+                evs[j][0].record(stream)
+                getattr(ls, meth)(p)
+                evs[j][1].record(stream)
+        return g
+
+    # the events must outlive the graphs that record them
+    warm_ev = [new_events() for _ in range(args.warmup)]
+    warm = [capture_step(i % ROT, warm_ev[i]) for i in range(args.warmup)]
+    ev = [new_events() for _ in range(args.steps)]
+    timed = [capture_step((args.warmup + i) % ROT, ev[i]) for i in range(args.steps)]
+    torch.cuda.synchronize()
 
     with torch.cuda.stream(stream):
-        run_steps(args.warmup)
+        for g in warm:
+            g.replay()
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
 
-    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(npart)] for _ in range(args.steps)]
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler()
     sampler.start()
@@ -634,7 +643,8 @@ def main():
     torch.cuda.nvtx.range_push("timed")
     with torch.cuda.stream(stream):
         e_start.record(stream)
-        run_steps(args.steps, ev, start=args.warmup)
+        for g in timed:
+            g.replay()
         e_end.record(stream)
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
@@ -698,7 +708,8 @@ def main():
 
     extras = None
     if rank == 0 and not args.no_extras:
-        del graphs
+        del warm, timed                      # the graphs first, then their events
+        del warm_ev, ev
         extras = run_extras(qz, dev, pk, stream)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:

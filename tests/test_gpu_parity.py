@@ -484,3 +484,17 @@ def test_gemv_launch_overlap_modes_agree(dev, bits):
     finally:
         qz.qz_set_launch_overlap(0)
     assert np.array_equal(outs[0], outs[1])
+
+
+@pytest.mark.parametrize("bits,sym", FORMATS)
+def test_dequantize_leftover_chunks_bit_exact(dev, bits, sym):
+    """N * K / 8 = 15 chunks: three groups of four and three left over."""
+    N, K = 3, 40
+    w = synthetic.weights(N, K, sigma=0.02, seed=91)
+    for g in (8, 40, 0):
+        c, s, z = oracle.quantize_pack(u16(w), bits, sym, g)
+        ref = oracle.dequantize(c, s, z, N, K, bits, sym, g)
+        out = qz.qz_dequantize(to_dev_u8(c, dev), to_dev_bf16(s, dev),
+                               None if z is None else to_dev_u8(z, dev), N, K, bits, sym, g)
+        torch.cuda.synchronize()
+        assert np.array_equal(u16(out), ref), (bits, sym, g)

@@ -504,40 +504,75 @@ __device__ __forceinline__ uint32_t dq_pair_i8(uint32_t word, int i, float off, 
     return dev::pack_bf16x2(p0, p1);
 }
 
+// Output chunk c (8 values) of the dequantized matrix from its code word(s).
+template <int BITS, bool SYM>
+__device__ __forceinline__ uint4 dequant_chunk(uint32_t w_lo, uint32_t w_hi,
+                                               const uint16_t *__restrict__ scales,
+                                               const uint8_t *__restrict__ zeros, int64_t gidx) {
+    const uint32_t s_bits = __ldg(&scales[gidx]);
+    uint32_t o[4];
+    if (BITS == 4) {
+        uint32_t w = w_lo;
+        const uint32_t zb = SYM ? 8u : (uint32_t)__ldg(&zeros[gidx]);
+        if (SYM) w ^= 0x88888888u;                              // two's complement -> q + 8
+        const uint32_t s2 = s_bits * 0x00010001u;
+        const uint32_t z2 = (0x4300u + zb) * 0x00010001u;
+        const uint32_t w4 = w >> 4;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o[i] = dq_pair_u4(w, w4, i, s2, z2);
+    } else {
+        const int z = SYM ? 0 : (int)(int8_t)__ldg(&zeros[gidx]);
+        const float off = -(8388736.0f + (float)z);              // -(2^23 + 128 + Z), exact
+        const float s_f = __uint_as_float(s_bits << 16);
+        const uint32_t lo = w_lo ^ 0x80808080u, hi = w_hi ^ 0x80808080u;
+        o[0] = dq_pair_i8(lo, 0, off, s_f);
+        o[1] = dq_pair_i8(lo, 1, off, s_f);
+        o[2] = dq_pair_i8(hi, 0, off, s_f);
+        o[3] = dq_pair_i8(hi, 1, off, s_f);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ int64_t group_of_chunk(int64_t c, int64_t chunks_per_group,
+                                                  int cpg_shift) {
+    if (chunks_per_group == 0) return 0;
+    return cpg_shift >= 0 ? (c >> cpg_shift) : c / chunks_per_group;
+}
+
+// A warp dequantizes 128 consecutive chunks per iteration, lane l taking
+// chunks base + 32 i + l (i = 0..3): its four code loads are issued before any
+// arithmetic (four loads in flight per thread), and every load and store
+// instruction of the warp covers contiguous memory.
 template <int BITS, bool SYM>
 __global__ void __launch_bounds__(256)
 dequantize_kernel(const uint8_t *__restrict__ codes, const uint16_t *__restrict__ scales,
                   const uint8_t *__restrict__ zeros, int64_t total_chunks,
                   int64_t chunks_per_group, int cpg_shift, uint4 *__restrict__ out) {
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < total_chunks; c += stride) {
-        int64_t gidx;
-        if (chunks_per_group == 0) gidx = 0;
-        else if (cpg_shift >= 0) gidx = c >> cpg_shift;
-        else gidx = c / chunks_per_group;
-        const uint32_t s_bits = __ldg(&scales[gidx]);
-        uint32_t o[4];
-        if (BITS == 4) {
-            uint32_t w = __ldcs(reinterpret_cast<const unsigned int *>(codes) + c);
-            uint32_t zb = SYM ? 8u : (uint32_t)__ldg(&zeros[gidx]);
-            if (SYM) w ^= 0x88888888u;                              // two's complement -> q + 8
-            const uint32_t s2 = s_bits * 0x00010001u;
-            const uint32_t z2 = (0x4300u + zb) * 0x00010001u;
-            const uint32_t w4 = w >> 4;
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+    const int64_t warp = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    for (int64_t base = warp * 128; base < total_chunks; base += warps * 128) {
+        uint32_t wl[4], wh[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) o[i] = dq_pair_u4(w, w4, i, s2, z2);
-        } else {
-            const uint2 p = __ldcs(reinterpret_cast<const uint2 *>(codes) + c);
-            const int z = SYM ? 0 : (int)(int8_t)__ldg(&zeros[gidx]);
-            const float off = -(8388736.0f + (float)z);              // -(2^23 + 128 + Z), exact
-            const float s_f = __uint_as_float(s_bits << 16);
-            const uint32_t lo = p.x ^ 0x80808080u, hi = p.y ^ 0x80808080u;
-            o[0] = dq_pair_i8(lo, 0, off, s_f);
-            o[1] = dq_pair_i8(lo, 1, off, s_f);
-            o[2] = dq_pair_i8(hi, 0, off, s_f);
-            o[3] = dq_pair_i8(hi, 1, off, s_f);
+        for (int i = 0; i < 4; ++i) {
+            const int64_t c = base + 32 * i + lane;
+            wl[i] = wh[i] = 0u;
+            if (c < total_chunks) {
+                if (BITS == 4) {
+                    wl[i] = __ldcs(reinterpret_cast<const unsigned int *>(codes) + c);
+                } else {
+                    const uint2 v = __ldcs(reinterpret_cast<const uint2 *>(codes) + c);
+                    wl[i] = v.x; wh[i] = v.y;
+                }
+            }
         }
-        __stcs(out + c, make_uint4(o[0], o[1], o[2], o[3]));
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int64_t c = base + 32 * i + lane;
+            if (c < total_chunks)
+                __stcs(out + c, dequant_chunk<BITS, SYM>(wl[i], wh[i], scales, zeros,
+                                                         group_of_chunk(c, chunks_per_group, cpg_shift)));
+        }
     }
 }
 
@@ -551,7 +586,7 @@ qz_status dequantize_typed(const void *codes, const void *scales, const void *ze
         shift = 0;
         while ((int64_t(1) << shift) < cpg) ++shift;
     }
-    dequantize_kernel<BITS, SYM><<<grid_for(total, 256), 256, 0, st>>>(
+    dequantize_kernel<BITS, SYM><<<grid_for(ceil_div(total, 4), 256), 256, 0, st>>>(
         static_cast<const uint8_t *>(codes), static_cast<const uint16_t *>(scales),
         static_cast<const uint8_t *>(zeros), total, cpg, shift, static_cast<uint4 *>(w_hat));
     return launch_status();

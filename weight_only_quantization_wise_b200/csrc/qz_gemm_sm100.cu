@@ -61,6 +61,7 @@ constexpr int kAccCols = kTileM;                         // fp32 accumulator col
 constexpr int kACols = kTileK / 2;                       // A columns per stage (bf16 pairs)
 constexpr int kTmemCols = 512;
 constexpr int kDequantWarps = 8;
+constexpr int kMetaFifo = 2;              // groups of scales/zeros loaded ahead
 constexpr int kEpilogueWarps = 4;
 constexpr int kFirstEpilogueWarp = 2 + kDequantWarps;
 constexpr int kThreads = 32 * (2 + kDequantWarps + kEpilogueWarps);
@@ -249,28 +250,29 @@ w4a16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
             const bool valid = n < N;
             const uint16_t *srow = scales + (int64_t)(valid ? n : 0) * gpr;
             const uint8_t *zrow = zeros + (int64_t)(valid ? n : 0) * gpr;
-            // Scales and zeros of the next four groups wait in a register FIFO
-            // (a group spans spg stages), so their loads are issued up to four
-            // groups before use and no per-stage index arithmetic is needed.
-            uint32_t sq[4], zq[4];
+            // Scales and zeros of the next kMetaFifo groups wait in a register
+            // FIFO (a group spans spg stages), so their loads are issued up to
+            // kMetaFifo groups before use and no per-stage index arithmetic is
+            // needed.
+            uint32_t sq[kMetaFifo], zq[kMetaFifo];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < kMetaFifo; ++q) {
                 sq[q] = (valid && q < gpr) ? __ldg(&srow[q]) : 0u;
                 zq[q] = (valid && q < gpr) ? __ldg(&zrow[q]) : 0u;
             }
-            int stage_in_group = 0, next_group = 4;
+            int stage_in_group = 0, next_group = kMetaFifo;
             for (int kt = 0; kt < KT; ++kt, ++it) {
                 const int s = it % kStages, r = it / kStages;
                 const uint32_t sb = sq[0], zb = zq[0];
                 if (++stage_in_group == spg) {               // the next stage starts a new group
                     stage_in_group = 0;
 #pragma unroll
-                    for (int q = 0; q < 3; ++q) {
+                    for (int q = 0; q < kMetaFifo - 1; ++q) {
                         sq[q] = sq[q + 1];
                         zq[q] = zq[q + 1];
                     }
-                    sq[3] = (valid && next_group < gpr) ? __ldg(&srow[next_group]) : 0u;
-                    zq[3] = (valid && next_group < gpr) ? __ldg(&zrow[next_group]) : 0u;
+                    sq[kMetaFifo - 1] = (valid && next_group < gpr) ? __ldg(&srow[next_group]) : 0u;
+                    zq[kMetaFifo - 1] = (valid && next_group < gpr) ? __ldg(&zrow[next_group]) : 0u;
                     ++next_group;
                 }
                 // warp-uniform: the tcgen05.st below needs every lane

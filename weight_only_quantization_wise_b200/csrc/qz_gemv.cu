@@ -28,7 +28,7 @@
 //     add.rn.bf16x2 of bf16(-(128 + Z)) leaves q - Z exactly, mul.rn.bf16x2
 //     by the bf16 scale rounds S*(q - Z) once.  int8: the byte (XOR 0x80) is
 //     placed in the mantissa of 2^23, one fp32 subtraction gives q exactly,
-//     an fp32 multiply gives the exact S*q, cvt.rn.bf16x2 rounds it once.
+//     the pair is packed to bf16 exactly and mul.rn.bf16x2 rounds S*q once.
 //   * A byte of codes yields the pairs (q_j, q_{j+4}), so the K axis is
 //     permuted consistently for both MMA operands: the pairs are the A operand
 //     (16 rows x 16 k) of mma.sync m16n8k16 with fp32 accumulation and the
@@ -65,14 +65,16 @@ __device__ __forceinline__ uint32_t dequant_pair_u4(uint32_t word, int j, uint32
 
 // bf16 pair (code c_j, code c_{j+4}) of 8 consecutive int8 codes held in
 // words lo (c0..c3) and hi (c4..c7), already XORed with 0x80808080:
-// bits 0x4B000000 | byte is the fp32 2^23 + q + 128.
-__device__ __forceinline__ uint32_t dequant_pair_i8(uint32_t lo, uint32_t hi, int j, float s) {
+// bits 0x4B000000 | byte is the fp32 2^23 + q + 128.  One subtraction leaves
+// q exactly, the pair is packed to bf16 exactly (|q| <= 127), and
+// mul.rn.bf16x2 by (S, S) rounds the exact product S*q once, as
+// qz_dequantize does.
+__device__ __forceinline__ uint32_t dequant_pair_i8(uint32_t lo, uint32_t hi, int j, uint32_t s2) {
     const uint32_t sel = (uint32_t)j | 0x7540u;
     const float f0 = __uint_as_float(dev::prmt(lo, 0x4B000000u, sel));
     const float f1 = __uint_as_float(dev::prmt(hi, 0x4B000000u, sel));
-    const float p0 = __fmul_rn(__fsub_rn(f0, 8388736.0f), s);     // - (2^23 + 128): exact
-    const float p1 = __fmul_rn(__fsub_rn(f1, 8388736.0f), s);     // then the exact product
-    return dev::pack_bf16x2(p0, p1);
+    const uint32_t q2 = dev::pack_bf16x2(__fsub_rn(f0, 8388736.0f), __fsub_rn(f1, 8388736.0f));
+    return dev::bf16x2_mul(q2, s2);
 }
 
 // Activation operand for code word i (k = 8i..8i+7 of the lane's 32) and
@@ -210,7 +212,7 @@ __device__ __forceinline__ void load_act(Act<MB> &ac, const GemvArgs &p, int kb,
 
 template <int BITS, int MB>
 __device__ __forceinline__ void compute_block(const RowParams &rp, const Act<MB> &ac,
-                                              const RowWords<BITS> &rw, const float (&sf)[4],
+                                              const RowWords<BITS> &rw, const uint32_t (&s8)[4],
                                               float (&acc)[2][MB][4]) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -237,10 +239,10 @@ __device__ __forceinline__ void compute_block(const RowParams &rp, const Act<MB>
                     a2 = dequant_pair_u4(rw.w[ja][i], 2 * h + 1, rp.s2[ja], rp.z2[ja]);
                     a3 = dequant_pair_u4(rw.w[jb][i], 2 * h + 1, rp.s2[jb], rp.z2[jb]);
                 } else {
-                    a0 = dequant_pair_i8(lo8[ja], hi8[ja], 2 * h, sf[ja]);
-                    a1 = dequant_pair_i8(lo8[jb], hi8[jb], 2 * h, sf[jb]);
-                    a2 = dequant_pair_i8(lo8[ja], hi8[ja], 2 * h + 1, sf[ja]);
-                    a3 = dequant_pair_i8(lo8[jb], hi8[jb], 2 * h + 1, sf[jb]);
+                    a0 = dequant_pair_i8(lo8[ja], hi8[ja], 2 * h, s8[ja]);
+                    a1 = dequant_pair_i8(lo8[jb], hi8[jb], 2 * h, s8[jb]);
+                    a2 = dequant_pair_i8(lo8[ja], hi8[ja], 2 * h + 1, s8[ja]);
+                    a3 = dequant_pair_i8(lo8[jb], hi8[jb], 2 * h + 1, s8[jb]);
                 }
 #pragma unroll
                 for (int mb = 0; mb < MB; ++mb)
@@ -405,16 +407,14 @@ gemv_kernel(const GemvArgs p) {
         int rows[4];
         bool valid[4];
         const uint8_t *rowp[4];
-        float sf[4];
+        uint32_t s8[4];                              // int8: (S, S) of rows g + 8j
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             rows[j] = n0 + g + 8 * j;
             valid[j] = rows[j] < p.N;
             rowp[j] = p.codes + (int64_t)(valid[j] ? rows[j] : 0) * (BITS == 4 ? p.K / 2 : p.K) +
                       t * (BITS == 4 ? 16 : 32);
-            sf[j] = 0.0f;
-            if (BITS == 8 && valid[j])
-                sf[j] = __uint_as_float((uint32_t)__ldg(&p.scales[rows[j]]) << 16);
+            s8[j] = (BITS == 8 && valid[j]) ? (uint32_t)__ldg(&p.scales[rows[j]]) * 0x00010001u : 0u;
         }
         // the row whose scale and zero words this lane copies
         const int row_c = n0 + g + 8 * t;
@@ -491,7 +491,7 @@ gemv_kernel(const GemvArgs p) {
                     load_params_direct(rp, p, valid, rows, kb, t);
                 }
             }
-            compute_block<BITS, MB>(rp, ac, rw, sf, acc);
+            compute_block<BITS, MB>(rp, ac, rw, s8, acc);
             slot = slot == S - 1 ? 0 : slot + 1;
         }
         cp_async_wait<0>();

@@ -254,6 +254,21 @@ PARTS = [  # name, method, unit, work per step, bound
 LAUNCHES_PER_STEP = 3 * len(PARTS)
 
 
+def max_over_ranks(values, dist=None, device="cpu"):
+    """Element-wise max over ranks of per-rank times (the replicas' timing
+    rule: a multi-GPU number is as slow as its slowest rank)."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def replica_rate(work_per_rank, seconds, world):
+    """Whole-job throughput of `world` independent replicas that each did
+    `work_per_rank` in at most `seconds` (max over ranks)."""
+    return work_per_rank * world / seconds
+
+
 def capture(fn, stream):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
@@ -657,10 +672,8 @@ def main():
     assert qz.qz_device_status() == 0
 
     # max over ranks
-    t = torch.tensor([total_ms] + part_ms, dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, part_ms = float(t[0]), [float(x) for x in t[1:]]
+    agg = max_over_ranks([total_ms] + part_ms, dist, dev)
+    total_ms, part_ms = agg[0], agg[1:]
 
     traffic = ncu_traffic()
     parts, roofs = {}, {}
@@ -671,7 +684,7 @@ def main():
     dominant = max(zip(PARTS, part_ms), key=lambda x: x[1])[0][0]
     gemv_idx = [p[0] for p in PARTS].index("w4a16_gemv_m1")
     gemv_bytes = PARTS[gemv_idx][3]
-    value = gemv_bytes * world / (part_ms[gemv_idx] * 1e-3) / 1e9
+    value = replica_rate(gemv_bytes, part_ms[gemv_idx] * 1e-3, world) / 1e9
 
     # end to end through the public API, host buffers, per decode step
     e2e = None
@@ -698,10 +711,8 @@ def main():
     t0 = time.perf_counter()
     for i in range(args.steps):
         e2e_step(i % ROT)
-    el = torch.tensor([time.perf_counter() - t0], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(el, op=dist.ReduceOp.MAX)
-    e2e = {"value": round(gemv_bytes * world * args.steps / float(el[0]) / 1e9, 3), "unit": "GB/s",
+    el = max_over_ranks([time.perf_counter() - t0], dist, dev)[0]
+    e2e = {"value": round(replica_rate(gemv_bytes * args.steps, el, world) / 1e9, 3), "unit": "GB/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
            "note": "decode step through qz_w4a16_gemv with pinned host activations in and "
                    "outputs out, one host sync per step; weights resident"}

@@ -122,7 +122,7 @@ __device__ __forceinline__ void store_codes(uint8_t *__restrict__ codes, int64_t
 // (x/S + Z stays within [q_min - 1/2, q_max + 1/2] and q_min is even), so the
 // asymmetric formats clamp at the top.  If 1/S overflows (tiny subnormal S)
 // the chunk falls back to the IEEE division.
-template <int BITS, bool SYM>
+template <int BITS, bool SYM, bool CLAMP = true>
 __device__ __forceinline__ uint2 chunk_codes(const float (&x)[8], float s_f, float r, int z) {
     using R = Range<BITS, SYM>;
     constexpr float kC = BITS == 4 ? 192.0f : 768.0f;
@@ -134,7 +134,7 @@ __device__ __forceinline__ uint2 chunk_codes(const float (&x)[8], float s_f, flo
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         b[i] = __float_as_uint(__fadd_rn(__fmaf_rn(x[i], r, zc), kRound));
-        if (!SYM) b[i] = min(b[i], kTop);
+        if (!SYM && CLAMP) b[i] = min(b[i], kTop);
     }
     if (BITS == 4) {
         uint32_t p[4];
@@ -148,6 +148,29 @@ __device__ __forceinline__ uint2 chunk_codes(const float (&x)[8], float s_f, flo
     const uint32_t w0 = dev::prmt(dev::prmt(b[0], b[1], 0x0040u), dev::prmt(b[2], b[3], 0x0040u), 0x5410u);
     const uint32_t w1 = dev::prmt(dev::prmt(b[4], b[5], 0x0040u), dev::prmt(b[6], b[7], 0x0040u), 0x5410u);
     return make_uint2(w0, w1);
+}
+
+// Whether any code of a group can exceed q_max: only a value at the group's
+// maximum can land on the tie q_max + 1/2 (x/S + Z is monotone in x and at
+// most q_max + 1/2), so the maximum's code, computed as chunk_codes computes
+// it, decides.  Groups for which this is false skip the clamp.
+template <int BITS, bool SYM>
+__device__ __forceinline__ bool needs_clamp(float vmax, float r, int z) {
+    if (SYM) return false;                             // |x/S| <= q_max
+    using R = Range<BITS, SYM>;
+    constexpr float kC = BITS == 4 ? 192.0f : 768.0f;
+    constexpr float kRound = 12582912.0f - kC;
+    constexpr uint32_t kTop = 0x4B400000u + (uint32_t)R::qmax;
+    const float zc = __fadd_rn((float)z, kC);
+    // a non-finite r (the IEEE fallback) compares greater as well
+    return __float_as_uint(__fadd_rn(__fmaf_rn(vmax, r, zc), kRound)) > kTop;
+}
+
+template <int BITS, bool SYM>
+__device__ __forceinline__ uint2 group_chunk_codes(const float (&x)[8], float s_f, float r, int z,
+                                                   bool clamp) {
+    return clamp ? chunk_codes<BITS, SYM, true>(x, s_f, r, z)
+                 : chunk_codes<BITS, SYM, false>(x, s_f, r, z);
 }
 
 // Three-input fp32 max/min (sm_100); exact, they select one of their inputs.
@@ -215,7 +238,8 @@ quantize_small_groups(const uint4 *__restrict__ w, int64_t total_chunks,
         const float r = __frcp_rn(s_f);
         uint2 cw[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) cw[u] = chunk_codes<BITS, SYM>(x[u], s_f, r, z);
+        const bool clamp = needs_clamp<BITS, SYM>(vmax, r, z);
+        for (int u = 0; u < 4; ++u) cw[u] = group_chunk_codes<BITS, SYM>(x[u], s_f, r, z, clamp);
         if (BITS == 4) {
             reinterpret_cast<uint4 *>(codes)[c0 >> 2] = make_uint4(cw[0].x, cw[1].x, cw[2].x, cw[3].x);
         } else {
@@ -274,13 +298,14 @@ quantize_groups_block(const uint4 *__restrict__ w, int cpg, int64_t num_groups,
         uint32_t s_bits; float s_f; int z;
         group_params<BITS, SYM>(vmin, vmax, vmax, s_bits, s_f, z);
         const float r = __frcp_rn(s_f);
+        const bool clamp = needs_clamp<BITS, SYM>(vmax, r, z);
 #pragma unroll
         for (int i = 0; i < kRowChunksPerThread; ++i) {
             const int c = threadIdx.x + i * blockDim.x;
             if (c < cpg) {
                 float x[8];
                 unpack8(v[i], x);
-                store_codes<BITS>(codes, c0 + c, chunk_codes<BITS, SYM>(x, s_f, r, z));
+                store_codes<BITS>(codes, c0 + c, group_chunk_codes<BITS, SYM>(x, s_f, r, z, clamp));
             }
         }
         if (threadIdx.x == 0) {
@@ -334,10 +359,11 @@ quantize_large_groups(const uint4 *__restrict__ w, int64_t chunks_per_group,
         uint32_t s_bits; float s_f; int z;
         group_params<BITS, SYM>(vmin, vmax, amax, s_bits, s_f, z);
         const float r = __frcp_rn(s_f);
+        const bool clamp = needs_clamp<BITS, SYM>(vmax, r, z);
         for (int64_t i = threadIdx.x; i < chunks_per_group; i += blockDim.x) {
             float x[8];
             unpack8(__ldcs(w + c0 + i), x);
-            store_codes<BITS>(codes, c0 + i, chunk_codes<BITS, SYM>(x, s_f, r, z));
+            store_codes<BITS>(codes, c0 + i, group_chunk_codes<BITS, SYM>(x, s_f, r, z, clamp));
         }
         if (threadIdx.x == 0) {
             scales[gidx] = (uint16_t)s_bits;

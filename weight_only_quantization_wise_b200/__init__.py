@@ -83,10 +83,18 @@ def qz_packed_bytes(N, K, bits=4, symmetric=False, group_size=128):
     return c.value, s.value, z.value
 
 
+_WS_SIZES = {}
+
+
 def qz_workspace_bytes(op, M, N, K, group_size=128) -> int:
-    b = _sz()
-    _check(lib.qz_workspace_bytes(op, M, N, K, group_size, ctypes.byref(b)), "qz_workspace_bytes")
-    return b.value
+    """Workspace bytes of a call (a pure function of the arguments; cached)."""
+    key = (int(op), int(M), int(N), int(K), int(group_size))
+    v = _WS_SIZES.get(key)
+    if v is None:
+        b = _sz()
+        _check(lib.qz_workspace_bytes(*key, ctypes.byref(b)), "qz_workspace_bytes")
+        v = _WS_SIZES[key] = b.value
+    return v
 
 
 def _ptr(t):

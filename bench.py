@@ -338,7 +338,52 @@ def run_extras(qz, dev, pk, stream):
         msb = time_graph(gb)
         out["prefill_gemm_2048x8192x8192"]["cublas_bf16_same_shape_TFLOP/s"] = round(
             gemm_flops(M, N, K) / (msb * 1e-3) / 1e12, 1)
-        del w, a, c, s, z, y, wb, yb, g, gb
+        del wb, yb, g, gb, c, s, z
+        # W8A16 prefill GEMM, same shape, int8 symmetric per-channel
+        c8, s8, _ = qz.qz_quantize_pack(w, 8, True, K)
+        qz.qz_w8a16_gemm(a, c8, s8, N, K, y=y)
+        ms = time_graph(capture(lambda: qz.qz_w8a16_gemm(a, c8, s8, N, K, y=y), stream))
+        tf = gemm_flops(M, N, K) / (ms * 1e-3) / 1e12
+        out["prefill_w8a16_gemm_2048x8192x8192"] = {
+            "ms": round(ms, 4), "TFLOP/s": round(tf, 1),
+            "frac_of_burst": round(tf / pk["bf16_tflops"], 4),
+            "frac_of_sustained": round(tf / pk["bf16_tflops_sustained"], 4)}
+        del c8, s8, a, y
+
+        # Small-M crossover on the same layer: M <= 16 runs the decode kernel,
+        # larger M the tcgen05 GEMM.  Weights rotate over copies larger than L2.
+        packs4 = [qz.qz_quantize_pack(w if r == 0 else w.clone(), 4, False, GROUP) for r in range(4)]
+        packs8 = [qz.qz_quantize_pack(w if r == 0 else w.clone(), 8, True, K) for r in range(2)]
+        sweep = {}
+        for Ms in (16, 32, 64, 128, 256, 512):
+            a = synthetic.activations(Ms, K, seed=Ms, device=dev)
+            y = torch.empty((Ms, N), dtype=torch.bfloat16, device=dev)
+            ws = torch.zeros(max(256, qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMM, Ms, N, K, GROUP),
+                                 qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMM, Ms, N, K, K)),
+                             dtype=torch.uint8, device=dev)
+
+            def f4():
+                for c, s, z in packs4:
+                    qz.qz_w4a16_gemm(a, c, s, z, N, K, GROUP, y=y, workspace=ws)
+
+            def f8():
+                for c, s, _ in packs8:
+                    qz.qz_w8a16_gemm(a, c, s, N, K, y=y, workspace=ws)
+
+            f4(); f8()
+            ms4 = time_graph(capture(f4, stream)) / len(packs4)
+            ms8 = time_graph(capture(f8, stream)) / len(packs8)
+            b4, b8 = w4_gemv_bytes(Ms, N, K), w8_gemv_bytes(Ms, N, K)
+            sweep[f"M{Ms}"] = {
+                "kernel": "decode GEMV" if Ms <= 16 else "tcgen05 GEMM",
+                "w4_us": round(ms4 * 1e3, 2), "w4_GB/s": round(b4 / ms4 / 1e6, 1),
+                "w4_frac_hbm": round(b4 / ms4 / 1e6 / pk["hbm_gbs"], 4),
+                "w4_TFLOP/s": round(gemm_flops(Ms, N, K) / (ms4 * 1e-3) / 1e12, 1),
+                "w8_us": round(ms8 * 1e3, 2), "w8_GB/s": round(b8 / ms8 / 1e6, 1),
+                "w8_frac_hbm": round(b8 / ms8 / 1e6 / pk["hbm_gbs"], 4),
+                "w8_TFLOP/s": round(gemm_flops(Ms, N, K) / (ms8 * 1e-3) / 1e12, 1)}
+        out["small_m_crossover_8192x8192"] = sweep
+        del w, a, y, ws, packs4, packs8
 
         # 70B decode shapes, W4 and W8, M in {1, 4, 8, 16}
         d70 = {}
@@ -508,6 +553,8 @@ PROFILE_CASES = {
     "gemv_w4_7b": ("gemv4", 1, 4096, 4096),
     "gemv_w8_70b": ("gemv8", 1, 28672, 8192),
     "gemm_prefill": ("gemm", 2048, 8192, 8192),
+    "gemm8_prefill": ("gemm8", 2048, 8192, 8192),
+    "gemm_m32": ("gemm", 32, 8192, 8192),
     "quant_int4": ("quant4", 0, 28672, 8192),
     "quant_int8": ("quant8", 0, 28672, 8192),
     "dequant_int4": ("dequant", 0, 28672, 8192),
@@ -524,7 +571,7 @@ def run_kernel_case(name, reps):
     ws = torch.zeros(1 << 24, dtype=torch.uint8, device=dev)
     if kind in ("gemv4", "gemm", "dequant"):
         c, s, z = qz.qz_quantize_pack(w, 4, False, GROUP)
-    if kind == "gemv8":
+    if kind in ("gemv8", "gemm8"):
         c, s, _ = qz.qz_quantize_pack(w, 8, True, K)
     a = synthetic.activations(max(M, 1), K, seed=5, device=dev)
     torch.cuda.synchronize()
@@ -535,6 +582,8 @@ def run_kernel_case(name, reps):
             qz.qz_w8a16_gemv(a, c, s, N, K, workspace=ws)
         elif kind == "gemm":
             qz.qz_w4a16_gemm(a, c, s, z, N, K, GROUP, workspace=ws)
+        elif kind == "gemm8":
+            qz.qz_w8a16_gemm(a, c, s, N, K, workspace=ws)
         elif kind == "quant4":
             qz.qz_quantize_pack(w, 4, False, GROUP)
         elif kind == "quant8":

@@ -82,7 +82,8 @@ enum {
     QZ_OP_DEQUANTIZE = 1,
     QZ_OP_W4A16_GEMV = 2,
     QZ_OP_W4A16_GEMM = 3,
-    QZ_OP_W8A16_GEMV = 4
+    QZ_OP_W8A16_GEMV = 4,
+    QZ_OP_W8A16_GEMM = 5
 };
 
 /* Static description of a status code (never NULL). */
@@ -156,13 +157,21 @@ QZ_API qz_status qz_w4a16_gemv(const void *a, const void *codes, const void *sca
 
 /*
  * W4A16 prefill GEMM: the same product as qz_w4a16_gemv for any M >= 1,
- * dequantizing weight tiles into shared memory for the tcgen05 tensor cores
+ * dequantizing weight tiles into tensor memory for the tcgen05 tensor cores
  * (guide, "Quantize weights or activations": prefill and large batches are
- * compute-bound).  Requirements: M >= 1; N >= 1; K % 128 == 0; group_size a
- * multiple of 64 dividing K.  Workspace as reported by qz_workspace_bytes
- * (currently 0).  A device-side wait that runs out (see
- * qz_set_device_wait_limit) makes the kernel return early; the next
- * qz_device_status call reports QZ_ERR_DEVICE_TIMEOUT.
+ * compute-bound).  M <= 16 runs the decode kernel of qz_w4a16_gemv.  Each
+ * output tile is 128 weight rows x up to 256 tokens, and the MMAs cover only
+ * the tile's tokens (rounded up to 16).  When the tiles are fewer than the
+ * SMs, the K range of each tile is split over up to 4 CTAs whose fp32
+ * partials meet in the workspace and are added in a fixed order (results do
+ * not depend on timing).  Requirements: M >= 1; N >= 1; K % 128 == 0;
+ * group_size a multiple of 64 dividing K (32 suffices for M <= 16).
+ * Workspace: qz_workspace_bytes(QZ_OP_W4A16_GEMM, M, N, K, group_size)
+ * bytes, zero-filled before first use, left zero-filled by each call that
+ * completes.  A device-side wait that runs out (see qz_set_device_wait_limit)
+ * makes the kernel return early and the next qz_device_status call reports
+ * QZ_ERR_DEVICE_TIMEOUT; the workspace of that call must then be zero-filled
+ * again before reuse.
  */
 QZ_API qz_status qz_w4a16_gemm(const void *a, const void *codes, const void *scales,
                         const void *zeros, int64_t M, int64_t N, int64_t K,
@@ -177,6 +186,27 @@ QZ_API qz_status qz_w4a16_gemm(const void *a, const void *codes, const void *sca
  * Workspace as for qz_w4a16_gemv with QZ_OP_W8A16_GEMV.
  */
 QZ_API qz_status qz_w8a16_gemv(const void *a, const void *codes, const void *scales,
+                        int64_t M, int64_t N, int64_t K, void *y, void *workspace,
+                        size_t workspace_bytes, void *stream);
+
+/*
+ * W8A16 prefill GEMM: the same product as qz_w8a16_gemv for any M >= 1.
+ * Weight tiles are dequantized (w_hat = bf16_rne(S * q), exactly as
+ * qz_dequantize forms it) into tensor memory as the A operand of tcgen05
+ * BF16 MMAs with fp32 accumulation; y is rounded to bf16.  M <= 16 runs the
+ * decode kernel of qz_w8a16_gemv.  Tiles and split-K as for qz_w4a16_gemm.
+ * Arguments: a (M x K bf16, row-major), codes (N x K int8, row-major),
+ * scales (N bf16), y (M x N bf16, row-major), all device pointers owned by
+ * the caller; a, codes and y 16-byte aligned, scales 2-byte aligned.
+ * Requirements: M >= 1; N >= 1; K % 128 == 0.  Workspace:
+ * qz_workspace_bytes(QZ_OP_W8A16_GEMM, M, N, K, K) bytes, zero-filled before
+ * first use, left zero-filled by each call that completes.  Errors: argument
+ * errors return before any launch; QZ_ERR_CUDA if the launch fails; a
+ * device-side wait that runs out makes the kernel return early, the next
+ * qz_device_status call reports QZ_ERR_DEVICE_TIMEOUT, and the workspace of
+ * that call must be zero-filled again before reuse.
+ */
+QZ_API qz_status qz_w8a16_gemm(const void *a, const void *codes, const void *scales,
                         int64_t M, int64_t N, int64_t K, void *y, void *workspace,
                         size_t workspace_bytes, void *stream);
 

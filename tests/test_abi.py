@@ -134,6 +134,30 @@ def test_w4a16_gemm_rejects(args, expect):
     assert L().qz_w4a16_gemm(*args) == expect
 
 
+@pytest.mark.parametrize("args,expect", [
+    ((A, B, C, 0, 64, 128, Y, None, 0, None), INVALID),                # M = 0
+    ((A, B, C, 64, 64, 192, Y, None, 0, None), UNSUP),                 # K % 128
+    ((A, B, None, 64, 64, 256, Y, None, 0, None), INVALID),            # null scales
+    ((A, B, C, 64, 64, 256, None, None, 0, None), INVALID),            # null y
+    ((MIS, B, C, 64, 64, 256, Y, None, 0, None), ALIGN),
+    ((A, B, C, 64, 64, 256, MIS, None, 0, None), ALIGN),               # y for the TMA store
+    ((A, B, C, 16, 4096, 4096, Y, None, 0, None), WS),                 # M <= 16: GEMV split-K
+])
+def test_w8a16_gemm_rejects(args, expect):
+    assert L().qz_w8a16_gemm(*args) == expect
+
+
+def test_w8a16_gemm_workspace_follows_the_route():
+    assert qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMM, 2048, 8192, 8192, 8192) == 0
+    # 64 tiles on 148 SMs: two K splits, fp32 partials [2][M][N] + counters
+    assert qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMM, 64, 8192, 8192, 8192) == \
+        2 * 64 * 8192 * 4 + 64 * 4
+    assert qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMM, 64, 8192, 8192, 128) == \
+        qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMM, 64, 8192, 8192, 8192)
+    assert (qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMM, 16, 4096, 4096, 4096) ==
+            qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMV, 16, 4096, 4096, 4096))
+
+
 def test_launch_overlap_setter():
     assert qz.lib.qz_set_launch_overlap(2) == INVALID
     assert qz.lib.qz_set_launch_overlap(-1) == INVALID

@@ -342,10 +342,11 @@ def test_bulk_quantization_stack(dev):
 # Prefill GEMM (tcgen05)
 # ---------------------------------------------------------------------------
 
-GEMM_CASES = [  # (M, N, K, g)
+GEMM_CASES = [  # (M, N, K, g); most have fewer tiles than SMs and run split-K
     (17, 128, 128, 128), (100, 200, 256, 64), (256, 128, 1024, 128),
     (300, 1000, 1024, 128), (512, 384, 2048, 256), (257, 130, 640, 128),
     (64, 256, 640, 640), (96, 192, 384, 192),      # groups of 10 and 3 stages
+    (32, 1024, 4096, 128), (200, 512, 2048, 128),  # 2 and 4 splits, partial token tiles
 ]
 
 
@@ -360,6 +361,31 @@ def test_w4a16_gemm_tolerance(dev, M, N, K, g):
     torch.cuda.synchronize()
     assert qz.qz_device_status() == 0
     check_tolerance(u16(y), y_ref, abs_ref, f"gemm M={M} N={N} K={K} g={g}")
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_gemm_split_k_repeats_and_leaves_workspace_zeroed(dev, bits):
+    """Split-K partials are added in split order: the same inputs give the
+    same bits on every call, and each call leaves the workspace zero-filled."""
+    M, N, K, g = 48, 1024, 2048, 128
+    assert qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMM, M, N, K, g) > 0
+    w = synthetic.weights(N, K, sigma=0.02, seed=41, device=dev)
+    a = synthetic.activations(M, K, seed=42, device=dev)
+    ws = torch.zeros(qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMM, M, N, K, g), dtype=torch.uint8,
+                     device=dev)
+    if bits == 4:
+        c, s, z = qz.qz_quantize_pack(w, 4, False, g)
+        run = lambda: qz.qz_w4a16_gemm(a, c, s, z, N, K, g, workspace=ws)
+    else:
+        c, s, _ = qz.qz_quantize_pack(w, 8, True, K)
+        run = lambda: qz.qz_w8a16_gemm(a, c, s, N, K, workspace=ws)
+    ys = [run() for _ in range(3)]
+    torch.cuda.synchronize()
+    assert qz.qz_device_status() == 0
+    assert all(torch.equal(ys[0], yi) for yi in ys[1:])
+    # the counters after the partials are back to zero
+    counters = ws[qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMM, M, N, K, g) - 64 * 4:]
+    assert int(counters.count_nonzero()) == 0
 
 
 def test_w4a16_gemm_onehot_is_exact(dev):
@@ -394,6 +420,81 @@ def test_prefill_config_sampled(dev):
     w_hat = oracle.dequantize(*ref, len(idx), K, 4, False, 128)
     y_ref, abs_ref = oracle.matmul_f64(u16(a), w_hat)
     check_tolerance(u16(y)[:, idx], y_ref, abs_ref, "prefill 2048x8192x8192")
+
+
+W8_GEMM_CASES = [  # (M, N, K): ragged token and row tiles, N % 8 != 0 (direct stores)
+    (17, 128, 128), (100, 200, 256), (256, 128, 1024), (300, 1000, 1024),
+    (257, 130, 640), (512, 384, 2048), (64, 36, 384),
+]
+
+
+@pytest.mark.parametrize("M,N,K", W8_GEMM_CASES)
+def test_w8a16_gemm_tolerance(dev, M, N, K):
+    w = synthetic.weights(N, K, sigma=0.015, seed=M + 2 * N + K)
+    a = synthetic.activations(M, K, seed=M * 7)
+    c, s, _ = oracle.quantize_pack(u16(w), 8, True, K)
+    w_hat = oracle.dequantize(c, s, None, N, K, 8, True, K)
+    y_ref, abs_ref = oracle.matmul_f64(u16(a), w_hat)
+    y = qz.qz_w8a16_gemm(a.to(dev), to_dev_u8(c, dev), to_dev_bf16(s, dev), N, K)
+    torch.cuda.synchronize()
+    assert qz.qz_device_status() == 0
+    check_tolerance(u16(y), y_ref, abs_ref, f"w8 gemm M={M} N={N} K={K}")
+
+
+def test_w8a16_gemm_onehot_is_exact(dev):
+    """One-hot token rows read back single dequantized int8 weights exactly,
+    including the extreme codes +-127 of every row."""
+    M, N, K = 256, 256, 1024
+    w = synthetic.weights(N, K, sigma=0.015, seed=78)
+    c, s, _ = oracle.quantize_pack(u16(w), 8, True, K)
+    w_hat = oracle.dequantize(c, s, None, N, K, 8, True, K)
+    ks = np.arange(M) * (K // M) + (np.arange(M) % (K // M))
+    a = np.zeros((M, K), np.uint16)
+    a[np.arange(M), ks] = 0x3F80
+    y = qz.qz_w8a16_gemm(to_dev_bf16(a, dev), to_dev_u8(c, dev), to_dev_bf16(s, dev), N, K)
+    torch.cuda.synchronize()
+    assert np.array_equal(u16(y), w_hat[:, ks].T)
+    # the column of each row's extreme code
+    kx = np.abs(c.view(np.int8).astype(np.int32)).argmax(axis=1)[:M]
+    a2 = np.zeros((M, K), np.uint16)
+    a2[np.arange(M), kx] = 0x3F80
+    y2 = qz.qz_w8a16_gemm(to_dev_bf16(a2, dev), to_dev_u8(c, dev), to_dev_bf16(s, dev), N, K)
+    torch.cuda.synchronize()
+    assert np.array_equal(u16(y2), w_hat[:, kx].T)
+
+
+def test_w8a16_gemm_small_m_matches_the_gemv(dev):
+    """M <= 16 takes the decode kernel: the same bits as qz_w8a16_gemv."""
+    N, K = 1000, 1024
+    w = synthetic.weights(N, K, sigma=0.015, seed=5)
+    c, s, _ = oracle.quantize_pack(u16(w), 8, True, K)
+    cd, sd = to_dev_u8(c, dev), to_dev_bf16(s, dev)
+    for M in (1, 16):
+        a = synthetic.activations(M, K, seed=M).to(dev)
+        y1 = qz.qz_w8a16_gemm(a, cd, sd, N, K)
+        y2 = qz.qz_w8a16_gemv(a, cd, sd, N, K)
+        torch.cuda.synchronize()
+        assert torch.equal(y1, y2)
+
+
+def test_w8a16_prefill_sampled(dev):
+    """M = 2048 tokens, N = K = 8192 int8 per-channel: sampled rows, all tokens."""
+    cfg = synthetic.PREFILL
+    M, N, K = cfg["M"], cfg["N"], cfg["K"]
+    w = synthetic.weights(N, K, sigma=cfg["sigma"], seed=cfg["seed"], device=dev)
+    a = synthetic.activations(M, K, seed=cfg["seed"] + 1000, device=dev)
+    c, s, _ = qz.qz_quantize_pack(w, 8, True, K)
+    y = qz.qz_w8a16_gemm(a, c, s, N, K)
+    torch.cuda.synchronize()
+    assert qz.qz_device_status() == 0
+    idx = sample_rows(N, 24, 8)
+    ti = torch.from_numpy(idx).to(dev)
+    ref = oracle.quantize_pack(u16(w.index_select(0, ti)), 8, True, K)
+    got = (u8(c.index_select(0, ti)), u16(s.index_select(0, ti)), None)
+    assert_quant_equal(got, ref)
+    w_hat = oracle.dequantize(*ref, len(idx), K, 8, True, K)
+    y_ref, abs_ref = oracle.matmul_f64(u16(a), w_hat)
+    check_tolerance(u16(y)[:, idx], y_ref, abs_ref, "w8 prefill 2048x8192x8192")
 
 
 def test_gemm_bounded_wait_reports_timeout_and_recovers(dev):

@@ -14,17 +14,18 @@ import torch
 __all__ = [
     "QzError", "lib", "qz_version", "qz_status_string", "qz_packed_bytes",
     "qz_workspace_bytes", "qz_quantize_pack", "qz_dequantize", "qz_w4a16_gemv",
-    "qz_w4a16_gemm", "qz_w8a16_gemv", "qz_set_device_wait_limit", "qz_set_launch_overlap",
-    "qz_device_status",
+    "qz_w4a16_gemm", "qz_w8a16_gemv", "qz_w8a16_gemm", "qz_set_device_wait_limit",
+    "qz_set_launch_overlap", "qz_device_status",
     "Workspace", "QZ_OP_QUANTIZE_PACK", "QZ_OP_DEQUANTIZE", "QZ_OP_W4A16_GEMV",
-    "QZ_OP_W4A16_GEMM", "QZ_OP_W8A16_GEMV", "EXPORTED_SYMBOLS",
+    "QZ_OP_W4A16_GEMM", "QZ_OP_W8A16_GEMV", "QZ_OP_W8A16_GEMM", "EXPORTED_SYMBOLS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqz.so")
 
 QZ_OK = 0
 QZ_ERR_DEVICE_TIMEOUT = 6
-QZ_OP_QUANTIZE_PACK, QZ_OP_DEQUANTIZE, QZ_OP_W4A16_GEMV, QZ_OP_W4A16_GEMM, QZ_OP_W8A16_GEMV = range(5)
+(QZ_OP_QUANTIZE_PACK, QZ_OP_DEQUANTIZE, QZ_OP_W4A16_GEMV, QZ_OP_W4A16_GEMM, QZ_OP_W8A16_GEMV,
+ QZ_OP_W8A16_GEMM) = range(6)
 
 _i32, _i64, _sz, _p = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p
 _SIGS = {
@@ -38,6 +39,7 @@ _SIGS = {
     "qz_w4a16_gemv": ([_p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p, _sz, _p], ctypes.c_int),
     "qz_w4a16_gemm": ([_p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p, _sz, _p], ctypes.c_int),
     "qz_w8a16_gemv": ([_p, _p, _p, _i64, _i64, _i64, _p, _p, _sz, _p], ctypes.c_int),
+    "qz_w8a16_gemm": ([_p, _p, _p, _i64, _i64, _i64, _p, _p, _sz, _p], ctypes.c_int),
     "qz_w4a16_gemv_noalloc": ([_p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p], ctypes.c_int),
     "qz_set_device_wait_limit": ([ctypes.c_uint64], None),
     "qz_set_launch_overlap": ([ctypes.c_int32], ctypes.c_int),
@@ -221,6 +223,17 @@ def qz_w8a16_gemv(a, codes, scales, N, K, y=None, workspace=None, stream=None):
                                 a.device)
     _check(lib.qz_w8a16_gemv(_ptr(a), _ptr(codes), _ptr(scales), M, N, K, _ptr(y), ws_ptr,
                              ws_bytes, _stream(stream, a.device)), "qz_w8a16_gemv")
+    return y
+
+
+def qz_w8a16_gemm(a, codes, scales, N, K, y=None, workspace=None, stream=None):
+    """y = a * w_hat^T for int8 symmetric per-channel weights, any M."""
+    y = _matmul_out(a, N, y)
+    M = a.shape[0]
+    ws_ptr, ws_bytes = _ws_args(workspace, qz_workspace_bytes(QZ_OP_W8A16_GEMM, M, N, K, K),
+                                a.device)
+    _check(lib.qz_w8a16_gemm(_ptr(a), _ptr(codes), _ptr(scales), M, N, K, _ptr(y), ws_ptr,
+                             ws_bytes, _stream(stream, a.device)), "qz_w8a16_gemm")
     return y
 
 

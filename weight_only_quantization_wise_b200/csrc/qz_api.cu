@@ -79,7 +79,7 @@ QZ_API const char *qz_status_string(int status) {
     }
 }
 
-QZ_API int qz_version(void) { return 100; }
+QZ_API int qz_version(void) { return 101; }
 
 QZ_API qz_status qz_packed_bytes(int64_t N, int64_t K, int32_t bits, int32_t symmetric,
                                  int64_t group_size, size_t *codes_bytes,
@@ -115,9 +115,11 @@ QZ_API qz_status qz_workspace_bytes(int32_t op, int64_t M, int64_t N, int64_t K,
         return QZ_OK;
     }
     case QZ_OP_W4A16_GEMM:
+    case QZ_OP_W8A16_GEMM:
         if (M < 1 || N < 1 || K < 1) return QZ_ERR_INVALID_ARG;
-        *bytes = M <= 16 && K % 128 == 0 ? gemv_plan(M, N, K, 4).total_bytes
-                                         : gemm_workspace_bytes(M, N, K);
+        *bytes = M <= 16 && K % 128 == 0
+                     ? gemv_plan(M, N, K, op == QZ_OP_W4A16_GEMM ? 4 : 8).total_bytes
+                     : gemm_workspace_bytes(M, N, K);
         return QZ_OK;
     default:
         return QZ_ERR_INVALID_ARG;
@@ -203,6 +205,22 @@ QZ_API qz_status qz_w4a16_gemm(const void *a, const void *codes, const void *sca
     if (s != QZ_OK) return s;
     return launch_w4a16_gemm(a, codes, scales, zeros, M, N, K, group_size, y, workspace,
                              as_stream(stream));
+}
+
+QZ_API qz_status qz_w8a16_gemm(const void *a, const void *codes, const void *scales,
+                               int64_t M, int64_t N, int64_t K, void *y, void *workspace,
+                               size_t workspace_bytes, void *stream) {
+    if (M < 1 || N < 1 || K < 1 || M > kMaxDim || N > kMaxDim || K > kMaxDim)
+        return QZ_ERR_INVALID_ARG;
+    if (K % 128 != 0) return QZ_ERR_UNSUPPORTED;
+    if (!a || !codes || !scales || !y) return QZ_ERR_INVALID_ARG;
+    if (M <= 16)   // the decode kernel covers small M with the same arithmetic
+        return qz_w8a16_gemv(a, codes, scales, M, N, K, y, workspace, workspace_bytes, stream);
+    if (!aligned(a, 16) || !aligned(codes, 16) || !aligned(scales, 2) || !aligned(y, 16))
+        return QZ_ERR_ALIGNMENT;
+    const qz_status s = check_workspace(gemm_workspace_bytes(M, N, K), workspace, workspace_bytes);
+    if (s != QZ_OK) return s;
+    return launch_w8a16_gemm(a, codes, scales, M, N, K, y, workspace, as_stream(stream));
 }
 
 QZ_API void qz_set_device_wait_limit(uint64_t limit) {

@@ -1,5 +1,5 @@
-// qz_gemm_sm100.cu -- W4A16 prefill GEMM on the sm_100a (tcgen05) tensor cores,
-// and the device error word used by bounded device-side waits.
+// qz_gemm_sm100.cu -- W4A16 and W8A16 prefill GEMMs on the sm_100a (tcgen05)
+// tensor cores, and the device error word used by bounded device-side waits.
 //
 // Quantization concepts guide, "Quantize weights or activations": weight-only
 // methods dequantize the weights to the compute dtype before each matmul;
@@ -7,13 +7,16 @@
 // tensor cores busy.  The GPTQ explainer: the dequantization happens inside
 // the matmul kernel, with no separate conversion pass.
 //
-// y (M x N) = a (M x K) * w_hat^T with w_hat = bf16_rne(S * (q - Z)).
+// y (M x N) = a (M x K) * w_hat^T with w_hat = bf16_rne(S * (q - Z)) (int4,
+// group-wise scales and zeros) or w_hat = bf16_rne(S * q) (int8, symmetric,
+// one scale per weight row).
 //
 // Persistent kernel: each CTA loops over tiles of 128 weight rows x 256
 // tokens (tile t = blockIdx.x + i * gridDim.x).  The roles:
 //   warp 0       TMA producer: per 64-wide K step, the activation tile
-//                (256 tokens x 64 bf16, 128-byte swizzle) and the packed codes
-//                (128 rows x 32 bytes) into a STAGES-deep shared-memory ring.
+//                (256 tokens x 64 bf16, 128-byte swizzle) and the codes
+//                (128 rows x 32 bytes of int4, or x 64 bytes of int8) into a
+//                STAGES-deep shared-memory ring.
 //   warp 1       allocates tensor memory; one lane issues tcgen05.mma.
 //   warps 2..9   dequantize: warp w owns weight rows 32*(w%4) .. +31 (the
 //                tensor-memory lane quarter that warp may access) and half of
@@ -50,47 +53,71 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kStages = 4;
 constexpr int kTileN = 128;               // weight rows per tile (MMA M)
 constexpr int kTileM = 256;               // tokens per tile (MMA N)
 constexpr int kTileK = 64;                // K per stage
-constexpr int kActStageBytes = kTileM * kTileK * 2;      // 32 KB
-constexpr int kPackStageBytes = kTileN * kTileK / 2;     // 4 KB
-constexpr int kStagingBytes = kTileM * kTileN * 2;       // 64 KB bf16 output tile
-constexpr int kAccCols = kTileM;                         // fp32 accumulator columns
+template <int BITS>
+constexpr int kPackStageBytes = kTileN * kTileK * BITS / 8;   // 4 KB (int4), 8 KB (int8)
 constexpr int kACols = kTileK / 2;                       // A columns per stage (bf16 pairs)
 constexpr int kTmemCols = 512;
 constexpr int kDequantWarps = 8;
 constexpr int kMetaFifo = 2;              // groups of scales/zeros loaded ahead
+constexpr int kMaxSplits = 4;             // split-K ranges per tile at most
+constexpr int kMaxStages = 16;            // ring depth at most
 constexpr int kEpilogueWarps = 4;
 constexpr int kFirstEpilogueWarp = 2 + kDequantWarps;
 constexpr int kThreads = 32 * (2 + kDequantWarps + kEpilogueWarps);
-constexpr int kSmemBytes =
-    kStages * (kActStageBytes + kPackStageBytes) + kStagingBytes + 1024 + 256;
+constexpr int kSmemLimit = 227 * 1024;    // dynamic shared memory of one CTA
 
-// instruction descriptor: MMA M = 128 weight rows, N = 256 tokens
-constexpr uint32_t kIdesc = idesc_bf16(kTileN, kTileM);
-
-struct SmemLayout {
-    // offsets from the 1024-aligned base
-    static constexpr uint32_t act = 0;
-    static constexpr uint32_t pack = act + kStages * kActStageBytes;
-    static constexpr uint32_t staging = pack + kStages * kPackStageBytes;
-    static constexpr uint32_t bars = staging + kStagingBytes;
-    // barriers: full[S], empty[S], afull[S], dfull, dempty, drain
-    static constexpr uint32_t full = bars;
-    static constexpr uint32_t empty = full + 8 * kStages;
-    static constexpr uint32_t afull = empty + 8 * kStages;
-    static constexpr uint32_t dfull = afull + 8 * kStages;
-    static constexpr uint32_t dempty = dfull + 8;
-    static constexpr uint32_t drain = dempty + 8;
-    static constexpr uint32_t tmem_slot = drain + 8;
-    static constexpr uint32_t abort_flag = tmem_slot + 4;
-    static constexpr uint32_t epi_decision = abort_flag + 4;
-    static constexpr uint32_t end = epi_decision + 4;
+// Shared- and tensor-memory layout of one launch.  The activation box holds
+// act_rows tokens (a multiple of 16, at most 256), so a stage takes
+// act_rows x 128 bytes of activations plus the codes of 128 rows, and the
+// ring is as deep as shared memory (and the A slots in tensor memory) allow:
+// short token tiles get more stages in flight to cover the memory latency.
+struct GemmLayout {
+    int stages;
+    uint32_t act_stage, pack_stage;
+    // byte offsets from the 1024-aligned base
+    uint32_t act, pack, staging, full, empty, afull, dfull, dempty, drain, tmem_slot,
+        abort_flag, epi_decision, epi_last, end;
+    uint32_t a_col0;   // first tensor-memory column of the A slots (accumulator at 0)
 };
-static_assert(SmemLayout::end + 1024 <= kSmemBytes, "shared memory layout");
-static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+
+__host__ __device__ constexpr GemmLayout gemm_layout(int bits, int act_rows, int stages) {
+    GemmLayout L{};
+    L.stages = stages;
+    L.act_stage = (uint32_t)act_rows * kTileK * 2;
+    L.pack_stage = (uint32_t)(kTileN * kTileK * bits / 8);
+    L.act = 0;
+    L.pack = L.act + stages * L.act_stage;
+    L.staging = L.pack + stages * L.pack_stage;
+    L.full = L.staging + (uint32_t)act_rows * kTileN * 2;
+    L.empty = L.full + 8 * stages;
+    L.afull = L.empty + 8 * stages;
+    L.dfull = L.afull + 8 * stages;
+    L.dempty = L.dfull + 8;
+    L.drain = L.dempty + 8;
+    L.tmem_slot = L.drain + 8;
+    L.abort_flag = L.tmem_slot + 4;
+    L.epi_decision = L.abort_flag + 4;
+    L.epi_last = L.epi_decision + 4;
+    L.end = L.epi_last + 4;
+    L.a_col0 = (uint32_t)((act_rows + 31) & ~31);
+    return L;
+}
+
+// Deepest ring that fits for this activation box.
+constexpr int gemm_stages(int bits, int act_rows) {
+    int s = kMaxStages;
+    while (s > 2 && gemm_layout(bits, act_rows, s).end + 1024 > (uint32_t)kSmemLimit) --s;
+    const int by_tmem = (kTmemCols - (int)gemm_layout(bits, act_rows, 1).a_col0) / kACols;
+    return s < by_tmem ? s : by_tmem;
+}
+constexpr int kFullTileStages = 4;
+static_assert(gemm_stages(4, kTileM) == kFullTileStages && gemm_stages(8, kTileM) == kFullTileStages,
+              "a full token tile keeps four stages");
+static_assert(gemm_stages(4, 16) == kMaxStages - 1 || gemm_stages(4, 16) == kMaxStages,
+              "short token tiles get a deep ring");
 
 // Bounded waits that report through this file's device error word.
 __device__ __forceinline__ bool gemm_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns,
@@ -122,34 +149,89 @@ __device__ __forceinline__ void epilogue_bar_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpilogueWarps) : "memory");
 }
 
+// int8 codes: bf16 pair (byte 2i, byte 2i+1) of word wx (the code word XOR
+// 0x80808080).  Bits 0x4B000000 | byte form the fp32 2^23 + q + 128; one
+// subtraction leaves q exactly, the pair packs to bf16 exactly (|q| <= 127)
+// and mul.rn.bf16x2 by (S, S) rounds S*q once, as qz_dequantize does.
+__device__ __forceinline__ uint32_t dequant_pair_i8_nat(uint32_t wx, int i, uint32_t s2) {
+    const float f0 = __uint_as_float(dev::prmt(wx, 0x4B000000u, (uint32_t)(2 * i) | 0x7540u));
+    const float f1 = __uint_as_float(dev::prmt(wx, 0x4B000000u, (uint32_t)(2 * i + 1) | 0x7540u));
+    return dev::bf16x2_mul(dev::pack_bf16x2(__fsub_rn(f0, 8388736.0f), __fsub_rn(f1, 8388736.0f)),
+                           s2);
+}
+
+// Work item: one 128-row x 256-token output tile and, when the tiles are
+// fewer than the SMs, one of `splits` equal K ranges of it (split-K).
+struct WorkItem {
+    int tile, split, n0, m0, kt0, kt1;
+};
+__device__ __forceinline__ WorkItem work_item(int item, int splits, int tiles_n, int KT) {
+    WorkItem w;
+    w.tile = item / splits;
+    w.split = item - w.tile * splits;
+    w.n0 = (w.tile % tiles_n) * kTileN;
+    w.m0 = (w.tile / tiles_n) * kTileM;
+    w.kt0 = (int)((int64_t)w.split * KT / splits);
+    w.kt1 = (int)((int64_t)(w.split + 1) * KT / splits);
+    return w;
+}
+
+// MMA N for a tile: its tokens rounded up to 16 (the kind::f16 granularity).
+__device__ __forceinline__ int mma_n(int M, int m0) {
+    const int mt = M - m0 < kTileM ? M - m0 : kTileM;
+    return (mt + 15) & ~15;
+}
+
+// FIXED_STAGES > 0: full 256-token tiles with a ring of that depth, the
+// layout known at compile time (the large-M path); 0: layout from the
+// launch's activation box and ring depth.
+template <int BITS, int FIXED_STAGES>
+__device__ __forceinline__ GemmLayout kernel_layout(int act_rows, int stages) {
+    if constexpr (FIXED_STAGES > 0) {
+        constexpr GemmLayout L = gemm_layout(BITS, kTileM, FIXED_STAGES);
+        return L;
+    } else {
+        return gemm_layout(BITS, act_rows, stages);
+    }
+}
+
+template <int BITS, int FIXED_STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
-w4a16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
+wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
                    const __grid_constant__ CUtensorMap pack_map,
                    const __grid_constant__ CUtensorMap y_map,
                    const uint16_t *__restrict__ scales, const uint8_t *__restrict__ zeros,
                    int M, int N, int K, int group_size, uint16_t *__restrict__ y,
-                   int use_tma_store, uint64_t wait_limit) {
+                   int use_tma_store, int act_rows, int stages_rt, int splits,
+                   float *__restrict__ partials, uint32_t *__restrict__ counters,
+                   uint64_t wait_limit) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
-    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + SmemLayout::abort_flag);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SmemLayout::tmem_slot);
+    const int stages = FIXED_STAGES > 0 ? FIXED_STAGES : stages_rt;
+    const GemmLayout SmemLayout = kernel_layout<BITS, FIXED_STAGES>(act_rows, stages_rt);
+    constexpr int kPackBytes = kPackStageBytes<BITS>;
+    const uint32_t kActStageBytes = SmemLayout.act_stage;
+    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + SmemLayout.abort_flag);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SmemLayout.tmem_slot);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KT = K / kTileK;
     const int tiles_n = (N + kTileN - 1) / kTileN;
     const int tiles = tiles_n * ((M + kTileM - 1) / kTileM);
+    const int items = tiles * splits;
+    const uint32_t act_bytes = kActStageBytes;                    // one activation box
 
-    auto full_bar = [&](int s) { return sbase + SmemLayout::full + 8 * s; };
-    auto empty_bar = [&](int s) { return sbase + SmemLayout::empty + 8 * s; };
-    auto afull_bar = [&](int s) { return sbase + SmemLayout::afull + 8 * s; };
-    const uint32_t dfull_bar = sbase + SmemLayout::dfull;
-    const uint32_t dempty_bar = sbase + SmemLayout::dempty;
-    const uint32_t drain_bar = sbase + SmemLayout::drain;
+    auto full_bar = [&](int s) { return sbase + SmemLayout.full + 8 * s; };
+    auto empty_bar = [&](int s) { return sbase + SmemLayout.empty + 8 * s; };
+    auto afull_bar = [&](int s) { return sbase + SmemLayout.afull + 8 * s; };
+    const uint32_t dfull_bar = sbase + SmemLayout.dfull;
+    const uint32_t dempty_bar = sbase + SmemLayout.dempty;
+    const uint32_t drain_bar = sbase + SmemLayout.drain;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < stages; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1 + kDequantWarps);   // MMA commit + dequant warps
             mbar_init(afull_bar(s), kDequantWarps);
@@ -173,59 +255,62 @@ w4a16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const uint32_t tmem_acc = tmem_base;                // columns [0, 256)
-    const uint32_t tmem_a = tmem_base + kAccCols;       // A slots: kStages x 32 columns
+    const uint32_t tmem_acc = tmem_base;                     // columns [0, act_rows)
+    const uint32_t tmem_a = tmem_base + SmemLayout.a_col0;   // A slots: stages x 32 columns
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
         if (lane == 0) {
-            int issued_round[kStages];
-            for (int s = 0; s < kStages; ++s) issued_round[s] = -1;
-            int it = 0;
+            int issued_round[kMaxStages];
+            for (int s = 0; s < kMaxStages; ++s) issued_round[s] = -1;
+            int s = 0, r = 0;                         // ring slot and its round
             bool ok = true;
-            for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-                const int n0 = (tile % tiles_n) * kTileN, m0 = (tile / tiles_n) * kTileM;
-                for (int kt = 0; kt < KT; ++kt, ++it) {
-                    const int s = it % kStages, r = it / kStages;
+            for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
+                const WorkItem wk = work_item(item, splits, tiles_n, KT);
+                for (int kt = wk.kt0; kt < wk.kt1; ++kt, s = (s + 1 == stages ? 0 : s + 1),
+                         r += (s == 0)) {
                     if (r > 0 && !gemm_wait(empty_bar(s), (r - 1) & 1, wait_limit, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(full_bar(s), kActStageBytes + kPackStageBytes);
-                    tma_load_2d(sbase + SmemLayout::act + s * kActStageBytes, &act_map,
-                                kt * kTileK, m0, full_bar(s));
-                    tma_load_2d(sbase + SmemLayout::pack + s * kPackStageBytes, &pack_map,
-                                kt * (kTileK / 2), n0, full_bar(s));
+                    mbar_arrive_expect_tx(full_bar(s), act_bytes + kPackBytes);
+                    tma_load_2d(sbase + SmemLayout.act + s * kActStageBytes, &act_map,
+                                kt * kTileK, wk.m0, full_bar(s));
+                    tma_load_2d(sbase + SmemLayout.pack + s * kPackBytes, &pack_map,
+                                kt * (kTileK * BITS / 8), wk.n0, full_bar(s));
                     issued_round[s] = r;
                 }
             }
             // every issued copy must have landed before the CTA may exit
-            for (int s = 0; s < kStages; ++s)
-                if (issued_round[s] >= 0) gemm_drain(full_bar(s), issued_round[s] & 1);
+            for (int q = 0; q < stages; ++q)
+                if (issued_round[q] >= 0) gemm_drain(full_bar(q), issued_round[q] & 1);
         }
         __syncwarp();
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
             bool ok = true;
-            int it = 0, tcount = 0;
-            for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++tcount) {
+            int s = 0, r = 0, tcount = 0;
+            for (int item = blockIdx.x; item < items && ok; item += gridDim.x, ++tcount) {
+                const WorkItem wk = work_item(item, splits, tiles_n, KT);
+                const uint32_t idesc = idesc_bf16(kTileN, mma_n(M, wk.m0));
                 if (tcount > 0 && !gemm_wait(dempty_bar, (tcount - 1) & 1, wait_limit, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                for (int kt = 0; kt < KT; ++kt, ++it) {
-                    const int s = it % kStages, r = it / kStages;
+                for (int kt = wk.kt0; kt < wk.kt1;
+                     ++kt, s = (s + 1 == stages ? 0 : s + 1), r += (s == 0)) {
                     ok = gemm_wait(full_bar(s), r & 1, wait_limit, abort_flag) &&
                          gemm_wait(afull_bar(s), r & 1, wait_limit, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
-                    const uint32_t act_addr = sbase + SmemLayout::act + s * kActStageBytes;
+                    const uint32_t act_addr = sbase + SmemLayout.act + s * kActStageBytes;
 #pragma unroll
                     for (int j = 0; j < kTileK / 16; ++j)
                         mma_ts(tmem_acc, tmem_a + s * kACols + j * 8,
-                               smem_desc_sw128(act_addr + j * 32), kIdesc, (kt > 0 || j > 0) ? 1u : 0u);
+                               smem_desc_sw128(act_addr + j * 32), idesc,
+                               (kt > wk.kt0 || j > 0) ? 1u : 0u);
                     mma_commit(empty_bar(s));
                 }
                 if (ok) mma_commit(dfull_bar);
@@ -241,66 +326,104 @@ w4a16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
         const int khalf = (warp - 2) / 4;             // which 32 of the 64 k of a stage
         const int row_local = quarter * 32 + lane;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-        const int gpr = K / group_size;
-        const int spg = group_size / kTileK;          // stages per group
-        int it = 0;
+        int s = 0, r = 0;                             // ring slot and its round
         bool ok = true;
-        for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-            const int n = (tile % tiles_n) * kTileN + row_local;
+        for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
+            const WorkItem wk = work_item(item, splits, tiles_n, KT);
+            const int n = wk.n0 + row_local;
             const bool valid = n < N;
-            const uint16_t *srow = scales + (int64_t)(valid ? n : 0) * gpr;
-            const uint8_t *zrow = zeros + (int64_t)(valid ? n : 0) * gpr;
-            // Scales and zeros of the next kMetaFifo groups wait in a register
-            // FIFO (a group spans spg stages), so their loads are issued up to
-            // kMetaFifo groups before use and no per-stage index arithmetic is
-            // needed.
-            uint32_t sq[kMetaFifo], zq[kMetaFifo];
+            if constexpr (BITS == 4) {
+                const int gpr = K / group_size;
+                const int spg = group_size / kTileK;      // stages per group
+                const uint16_t *srow = scales + (int64_t)(valid ? n : 0) * gpr;
+                const uint8_t *zrow = zeros + (int64_t)(valid ? n : 0) * gpr;
+                // Scales and zeros of the next kMetaFifo groups wait in a
+                // register FIFO (a group spans spg stages), so their loads are
+                // issued up to kMetaFifo groups before use and no per-stage
+                // index arithmetic is needed.
+                const int g0 = wk.kt0 / spg;              // group of the first stage
+                uint32_t sq[kMetaFifo], zq[kMetaFifo];
 #pragma unroll
-            for (int q = 0; q < kMetaFifo; ++q) {
-                sq[q] = (valid && q < gpr) ? __ldg(&srow[q]) : 0u;
-                zq[q] = (valid && q < gpr) ? __ldg(&zrow[q]) : 0u;
-            }
-            int stage_in_group = 0, next_group = kMetaFifo;
-            for (int kt = 0; kt < KT; ++kt, ++it) {
-                const int s = it % kStages, r = it / kStages;
-                const uint32_t sb = sq[0], zb = zq[0];
-                if (++stage_in_group == spg) {               // the next stage starts a new group
-                    stage_in_group = 0;
+                for (int q = 0; q < kMetaFifo; ++q) {
+                    sq[q] = (valid && g0 + q < gpr) ? __ldg(&srow[g0 + q]) : 0u;
+                    zq[q] = (valid && g0 + q < gpr) ? __ldg(&zrow[g0 + q]) : 0u;
+                }
+                int stage_in_group = wk.kt0 - g0 * spg, next_group = g0 + kMetaFifo;
+                for (int kt = wk.kt0; kt < wk.kt1;
+                     ++kt, s = (s + 1 == stages ? 0 : s + 1), r += (s == 0)) {
+                    const uint32_t sb = sq[0], zb = zq[0];
+                    if (++stage_in_group == spg) {           // the next stage starts a new group
+                        stage_in_group = 0;
 #pragma unroll
-                    for (int q = 0; q < kMetaFifo - 1; ++q) {
-                        sq[q] = sq[q + 1];
-                        zq[q] = zq[q + 1];
+                        for (int q = 0; q < kMetaFifo - 1; ++q) {
+                            sq[q] = sq[q + 1];
+                            zq[q] = zq[q + 1];
+                        }
+                        sq[kMetaFifo - 1] =
+                            (valid && next_group < gpr) ? __ldg(&srow[next_group]) : 0u;
+                        zq[kMetaFifo - 1] =
+                            (valid && next_group < gpr) ? __ldg(&zrow[next_group]) : 0u;
+                        ++next_group;
                     }
-                    sq[kMetaFifo - 1] = (valid && next_group < gpr) ? __ldg(&srow[next_group]) : 0u;
-                    zq[kMetaFifo - 1] = (valid && next_group < gpr) ? __ldg(&zrow[next_group]) : 0u;
-                    ++next_group;
-                }
-                // warp-uniform: the tcgen05.st below needs every lane
-                if (!__all_sync(0xFFFFFFFFu, gemm_wait(full_bar(s), r & 1, wait_limit, abort_flag))) {
-                    ok = false;
-                    break;
-                }
-                const uint4 p = *reinterpret_cast<const uint4 *>(
-                    smem + SmemLayout::pack + s * kPackStageBytes + row_local * (kTileK / 2) +
-                    khalf * 16);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty_bar(s));     // packed stage consumed
-                const uint32_t s2 = sb * 0x00010001u;
-                const uint32_t z2 = (0x4300u + zb) * 0x00010001u;
-                const uint32_t words[4] = {p.x, p.y, p.z, p.w};
-                uint32_t a[16];
+                    // warp-uniform: the tcgen05.st below needs every lane
+                    if (!__all_sync(0xFFFFFFFFu,
+                                    gemm_wait(full_bar(s), r & 1, wait_limit, abort_flag))) {
+                        ok = false;
+                        break;
+                    }
+                    const uint4 p = *reinterpret_cast<const uint4 *>(
+                        smem + SmemLayout.pack + s * kPackBytes + row_local * (kTileK / 2) +
+                        khalf * 16);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(empty_bar(s));   // code stage consumed
+                    const uint32_t s2 = sb * 0x00010001u;
+                    const uint32_t z2 = (0x4300u + zb) * 0x00010001u;
+                    const uint32_t words[4] = {p.x, p.y, p.z, p.w};
+                    uint32_t a[16];
 #pragma unroll
-                for (int wi = 0; wi < 4; ++wi) {
-                    const uint32_t w = words[wi], w4 = w >> 4;
+                    for (int wi = 0; wi < 4; ++wi) {
+                        const uint32_t w = words[wi], w4 = w >> 4;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        a[wi * 4 + i] = valid ? dequant_pair_nat(w, w4, i, s2, z2) : 0u;
+                        for (int i = 0; i < 4; ++i)
+                            a[wi * 4 + i] = valid ? dequant_pair_nat(w, w4, i, s2, z2) : 0u;
+                    }
+                    tmem_st_x16(tmem_a + lane_base + s * kACols + khalf * 16, a);
+                    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(afull_bar(s));
                 }
-                tmem_st_x16(tmem_a + lane_base + s * kACols + khalf * 16, a);
-                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(afull_bar(s));
+            } else {
+                // one scale per weight row for the whole K
+                const uint32_t s2 = valid ? (uint32_t)__ldg(&scales[n]) * 0x00010001u : 0u;
+                for (int kt = wk.kt0; kt < wk.kt1;
+                     ++kt, s = (s + 1 == stages ? 0 : s + 1), r += (s == 0)) {
+                    if (!__all_sync(0xFFFFFFFFu,
+                                    gemm_wait(full_bar(s), r & 1, wait_limit, abort_flag))) {
+                        ok = false;
+                        break;
+                    }
+                    const uint8_t *src =
+                        smem + SmemLayout.pack + s * kPackBytes + row_local * kTileK + khalf * 32;
+                    const uint4 p0 = *reinterpret_cast<const uint4 *>(src);
+                    const uint4 p1 = *reinterpret_cast<const uint4 *>(src + 16);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(empty_bar(s));   // code stage consumed
+                    const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+                    uint32_t a[16];
+#pragma unroll
+                    for (int wi = 0; wi < 8; ++wi) {
+                        const uint32_t wx = words[wi] ^ 0x80808080u;
+#pragma unroll
+                        for (int i = 0; i < 2; ++i)
+                            a[wi * 2 + i] = valid ? dequant_pair_i8_nat(wx, i, s2) : 0u;
+                    }
+                    tmem_st_x16(tmem_a + lane_base + s * kACols + khalf * 16, a);
+                    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(afull_bar(s));
+                }
             }
         }
         __syncwarp();
@@ -310,12 +433,15 @@ w4a16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
         const int row_local = quarter * 32 + lane;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         const bool storer = warp == kFirstEpilogueWarp && lane == 0;
-        uint16_t *staging = reinterpret_cast<uint16_t *>(smem + SmemLayout::staging);
+        uint16_t *staging = reinterpret_cast<uint16_t *>(smem + SmemLayout.staging);
         volatile uint32_t *epi_decision =
-            reinterpret_cast<volatile uint32_t *>(smem + SmemLayout::epi_decision);
+            reinterpret_cast<volatile uint32_t *>(smem + SmemLayout.epi_decision);
+        volatile uint32_t *epi_last = reinterpret_cast<volatile uint32_t *>(smem + SmemLayout.epi_last);
         int tcount = 0;
-        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tcount) {
-            const int n0 = (tile % tiles_n) * kTileN, m0 = (tile / tiles_n) * kTileM;
+        for (int item = blockIdx.x; item < items; item += gridDim.x, ++tcount) {
+            const WorkItem wk = work_item(item, splits, tiles_n, KT);
+            const int n0 = wk.n0, m0 = wk.m0;
+            const int chunks = mma_n(M, m0) / 16;     // accumulator columns the MMAs wrote
             // One decision for the four epilogue warps (they meet at named
             // barriers below): the storer publishes the abort flag after every
             // warp has finished its bounded wait.
@@ -330,8 +456,99 @@ w4a16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
             if (*epi_decision) break;
             tc_fence_after();
             const int n = n0 + row_local;
+            if (splits > 1) {
+                // split-K: this split's fp32 partial goes to partials[split][m][n]
+                float *part = partials + (int64_t)wk.split * M * N;
 #pragma unroll 1
-            for (int c = 0; c < kTileM / 16; ++c) {
+                for (int c = 0; c < chunks; ++c) {
+                    uint32_t v[16];
+                    tmem_ld_x16(tmem_acc + lane_base + c * 16, v);
+                    if (n < N) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int m = m0 + c * 16 + j;
+                            if (m < M) part[(int64_t)m * N + n] = __uint_as_float(v[j]);
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(dempty_bar);
+                __threadfence();
+                epilogue_bar_sync();
+                if (storer) *epi_last = atomicAdd(&counters[wk.tile], 1u) == (uint32_t)(splits - 1);
+                epilogue_bar_sync();
+                if (*epi_last) {
+                    // The last split of the tile adds the partials in split
+                    // order.  With N % 4 == 0 thread t takes rows n0 + 4(t%32)
+                    // .. +3 (float4) and tokens m0 + t/32, +4, ...; otherwise
+                    // one row per thread.
+                    __threadfence();
+                    const int m_end = M < m0 + kTileM ? M : m0 + kTileM;
+                    const int t = (int)threadIdx.x - 32 * kFirstEpilogueWarp;
+                    if ((N & 3) == 0) {
+                        const int nq = n0 + 4 * (t & 31);
+                        if (nq < N) {
+                            for (int mb = m0 + (t >> 5); mb < m_end; mb += 16) {
+                                float4 v[kMaxSplits][4];
+#pragma unroll
+                                for (int sp = 0; sp < kMaxSplits; ++sp)
+#pragma unroll
+                                    for (int j = 0; j < 4; ++j) {
+                                        const int m = mb + 4 * j;
+                                        v[sp][j] = (sp < splits && m < m_end)
+                                                       ? __ldcg(reinterpret_cast<const float4 *>(
+                                                             &partials[((int64_t)sp * M + m) * N + nq]))
+                                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+                                    }
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    const int m = mb + 4 * j;
+                                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                                    for (int sp = 0; sp < kMaxSplits; ++sp)
+                                        if (sp < splits) {
+                                            acc.x += v[sp][j].x;
+                                            acc.y += v[sp][j].y;
+                                            acc.z += v[sp][j].z;
+                                            acc.w += v[sp][j].w;
+                                        }
+                                    if (m < m_end) {
+                                        uint2 o;
+                                        o.x = dev::f32_to_bf16_rne(acc.x) | (dev::f32_to_bf16_rne(acc.y) << 16);
+                                        o.y = dev::f32_to_bf16_rne(acc.z) | (dev::f32_to_bf16_rne(acc.w) << 16);
+                                        *reinterpret_cast<uint2 *>(&y[(int64_t)m * N + nq]) = o;
+                                    }
+                                }
+                            }
+                        }
+                    } else if (n < N) {
+                        for (int mb = m0; mb < m_end; mb += 8) {
+                            float acc[8], v[kMaxSplits][8];
+#pragma unroll
+                            for (int sp = 0; sp < kMaxSplits; ++sp)
+#pragma unroll
+                                for (int j = 0; j < 8; ++j)
+                                    v[sp][j] = (sp < splits && mb + j < m_end)
+                                                   ? __ldcg(&partials[((int64_t)sp * M + mb + j) * N + n])
+                                                   : 0.0f;
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                acc[j] = 0.0f;
+#pragma unroll
+                                for (int sp = 0; sp < kMaxSplits; ++sp)
+                                    if (sp < splits) acc[j] += v[sp][j];
+                                if (mb + j < m_end)
+                                    y[(int64_t)(mb + j) * N + n] = (uint16_t)dev::f32_to_bf16_rne(acc[j]);
+                            }
+                        }
+                    }
+                    if (storer) counters[wk.tile] = 0u;
+                }
+                continue;
+            }
+#pragma unroll 1
+            for (int c = 0; c < chunks; ++c) {
                 uint32_t v[16];
                 tmem_ld_x16(tmem_acc + lane_base + c * 16, v);
                 if (use_tma_store) {
@@ -356,7 +573,7 @@ w4a16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
             if (use_tma_store) {
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 epilogue_bar_sync();
-                if (storer) tma_store_2d(&y_map, sbase + SmemLayout::staging, n0, m0);
+                if (storer) tma_store_2d(&y_map, sbase + SmemLayout.staging, n0, m0);
             }
         }
         if (storer) tma_store_wait_all();
@@ -374,7 +591,30 @@ w4a16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
 
 }  // namespace
 
-size_t gemm_workspace_bytes(int64_t, int64_t, int64_t) { return 0; }
+// Split-K: when the 128 x 256 output tiles are fewer than the SMs, each
+// tile's K range is divided among up to kMaxSplits CTAs (at least 4 stages
+// each); their fp32 partials meet in the workspace.
+int gemm_splits(int64_t M, int64_t N, int64_t K) {
+    const int64_t tiles = ceil_div(N, kTileN) * ceil_div(M, kTileM);
+    if (tiles >= kSmCount) return 1;
+    int64_t s = kSmCount / tiles;
+    if (s > kMaxSplits) s = kMaxSplits;
+    if (s > K / kTileK / 4) s = K / kTileK / 4;
+    return s < 1 ? 1 : (int)s;
+}
+
+// fp32 partials [splits][M][N], then one uint32 arrival counter per tile
+size_t gemm_partial_bytes(int64_t M, int64_t N, int64_t K) {
+    const int s = gemm_splits(M, N, K);
+    if (s == 1) return 0;
+    return (((size_t)s * M * N * sizeof(float)) + 255) & ~(size_t)255;
+}
+
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    if (gemm_splits(M, N, K) == 1) return 0;
+    const int64_t tiles = ceil_div(N, kTileN) * ceil_div(M, kTileM);
+    return gemm_partial_bytes(M, N, K) + (size_t)ceil_div(tiles, 64) * 64 * sizeof(uint32_t);
+}
 
 unsigned int *device_error_word() {
     static unsigned int *addr[64] = {};
@@ -389,21 +629,36 @@ unsigned int *device_error_word() {
     return addr[dev];
 }
 
-qz_status launch_w4a16_gemm(const void *a, const void *codes, const void *scales,
-                            const void *zeros, int64_t M, int64_t N, int64_t K,
-                            int64_t group_size, void *y, void *, cudaStream_t st) {
+namespace {
+
+template <int BITS>
+qz_status launch_gemm(const void *a, const void *codes, const void *scales, const void *zeros,
+                      int64_t M, int64_t N, int64_t K, int64_t group_size, void *y,
+                      void *workspace, cudaStream_t st) {
+    constexpr int kRowBytesPerK = BITS;   // code bytes of a row per 8 k
+    // tokens per activation box: a whole tile, or all of M rounded to 16
+    const int act_rows = M >= kTileM ? kTileM : (int)((M + 15) & ~int64_t(15));
+    const int splits = gemm_splits(M, N, K);
+    float *partials = nullptr;
+    uint32_t *counters = nullptr;
+    if (splits > 1) {
+        partials = static_cast<float *>(workspace);
+        counters = reinterpret_cast<uint32_t *>(static_cast<char *>(workspace) +
+                                                gemm_partial_bytes(M, N, K));
+    }
     CUtensorMap act_map, pack_map, y_map;
     if (!make_map_2d(&act_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a, (uint64_t)K, (uint64_t)M,
-                     (uint64_t)K * 2, kTileK, kTileM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_2d(&pack_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, (uint64_t)K / 2,
-                     (uint64_t)N, (uint64_t)K / 2, kTileK / 2, kTileN,
+                     (uint64_t)K * 2, kTileK, act_rows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&pack_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes,
+                     (uint64_t)K * kRowBytesPerK / 8, (uint64_t)N,
+                     (uint64_t)K * kRowBytesPerK / 8, kTileK * kRowBytesPerK / 8, kTileN,
                      CU_TENSOR_MAP_SWIZZLE_NONE))
         return QZ_ERR_CUDA;
     // bf16 output rows must be 16-byte multiples for a TMA store
     const int use_tma_store = (N % 8 == 0) ? 1 : 0;
     if (use_tma_store) {
         if (!make_map_2d(&y_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M,
-                         (uint64_t)N * 2, kTileN, kTileM, CU_TENSOR_MAP_SWIZZLE_NONE))
+                         (uint64_t)N * 2, kTileN, act_rows, CU_TENSOR_MAP_SWIZZLE_NONE))
             return QZ_ERR_CUDA;
     } else {
         y_map = act_map;   // unused
@@ -413,16 +668,36 @@ qz_status launch_w4a16_gemm(const void *a, const void *codes, const void *scales
     static std::once_flag attr_once[64];
     if (dev >= 0 && dev < 64)
         std::call_once(attr_once[dev], [] {
-            cudaFuncSetAttribute(w4a16_gemm_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kSmemBytes);
+            cudaFuncSetAttribute(wa16_gemm_tcgen05<BITS, kFullTileStages>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+            cudaFuncSetAttribute(wa16_gemm_tcgen05<BITS, 0>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
         });
-    const int64_t tiles = ceil_div(N, kTileN) * ceil_div(M, kTileM);
-    const int grid = (int)std::min<int64_t>(tiles, kSmCount);
-    w4a16_gemm_tcgen05<<<grid, kThreads, kSmemBytes, st>>>(
+    const int stages = gemm_stages(BITS, act_rows);
+    const uint32_t smem_bytes = gemm_layout(BITS, act_rows, stages).end + 1024;
+    const int64_t items = ceil_div(N, kTileN) * ceil_div(M, kTileM) * splits;
+    const int grid = (int)std::min<int64_t>(items, kSmCount);
+    auto kernel = act_rows == kTileM ? wa16_gemm_tcgen05<BITS, kFullTileStages>
+                                     : wa16_gemm_tcgen05<BITS, 0>;
+    kernel<<<grid, kThreads, smem_bytes, st>>>(
         act_map, pack_map, y_map, static_cast<const uint16_t *>(scales),
         static_cast<const uint8_t *>(zeros), (int)M, (int)N, (int)K, (int)group_size,
-        static_cast<uint16_t *>(y), use_tma_store, device_wait_limit());
+        static_cast<uint16_t *>(y), use_tma_store, act_rows, stages, splits, partials, counters,
+        device_wait_limit());
     return launch_status();
+}
+
+}  // namespace
+
+qz_status launch_w4a16_gemm(const void *a, const void *codes, const void *scales,
+                            const void *zeros, int64_t M, int64_t N, int64_t K,
+                            int64_t group_size, void *y, void *workspace, cudaStream_t st) {
+    return launch_gemm<4>(a, codes, scales, zeros, M, N, K, group_size, y, workspace, st);
+}
+
+qz_status launch_w8a16_gemm(const void *a, const void *codes, const void *scales, int64_t M,
+                            int64_t N, int64_t K, void *y, void *workspace, cudaStream_t st) {
+    return launch_gemm<8>(a, codes, scales, nullptr, M, N, K, K, y, workspace, st);
 }
 
 }  // namespace qz

@@ -86,6 +86,8 @@ qz_status launch_w4a16_gemm(const void *a, const void *codes, const void *scales
                             const void *zeros, int64_t M, int64_t N, int64_t K,
                             int64_t group_size, void *y, void *workspace,
                             cudaStream_t stream);
+qz_status launch_w8a16_gemm(const void *a, const void *codes, const void *scales, int64_t M,
+                            int64_t N, int64_t K, void *y, void *workspace, cudaStream_t stream);
 
 uint64_t device_wait_limit();
 // qz_set_launch_overlap mode (0 or 1) for the decode GEMV launches.

@@ -182,9 +182,9 @@ __device__ __forceinline__ int mma_n(int M, int m0) {
     return (mt + 15) & ~15;
 }
 
-// FIXED_STAGES > 0: full 256-token tiles with a ring of that depth, the
-// layout known at compile time (the large-M path); 0: layout from the
-// launch's activation box and ring depth.
+// FIXED_STAGES > 0: full 256-token tiles, no split-K, a ring of that depth,
+// the layout known at compile time (the large-M path); 0: layout from the
+// launch's activation box and ring depth, split-K allowed.
 template <int BITS, int FIXED_STAGES>
 __device__ __forceinline__ GemmLayout kernel_layout(int act_rows, int stages) {
     if constexpr (FIXED_STAGES > 0) {
@@ -210,6 +210,7 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
     const int stages = FIXED_STAGES > 0 ? FIXED_STAGES : stages_rt;
+    if (FIXED_STAGES > 0) splits = 1;             // the host launches it only unsplit
     const GemmLayout SmemLayout = kernel_layout<BITS, FIXED_STAGES>(act_rows, stages_rt);
     constexpr int kPackBytes = kPackStageBytes<BITS>;
     const uint32_t kActStageBytes = SmemLayout.act_stage;
@@ -331,6 +332,9 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
         for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
             const WorkItem wk = work_item(item, splits, tiles_n, KT);
             const int n = wk.n0 + row_local;
+            // Rows beyond N: the codes are TMA fill (zero) and the scale is
+            // taken as 0, so their A entries are +-0 and their outputs are
+            // never stored.
             const bool valid = n < N;
             if constexpr (BITS == 4) {
                 const int gpr = K / group_size;
@@ -385,7 +389,7 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
                         const uint32_t w = words[wi], w4 = w >> 4;
 #pragma unroll
                         for (int i = 0; i < 4; ++i)
-                            a[wi * 4 + i] = valid ? dequant_pair_nat(w, w4, i, s2, z2) : 0u;
+                            a[wi * 4 + i] = dequant_pair_nat(w, w4, i, s2, z2);
                     }
                     tmem_st_x16(tmem_a + lane_base + s * kACols + khalf * 16, a);
                     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
@@ -416,7 +420,7 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
                         const uint32_t wx = words[wi] ^ 0x80808080u;
 #pragma unroll
                         for (int i = 0; i < 2; ++i)
-                            a[wi * 2 + i] = valid ? dequant_pair_i8_nat(wx, i, s2) : 0u;
+                            a[wi * 2 + i] = dequant_pair_i8_nat(wx, i, s2);
                     }
                     tmem_st_x16(tmem_a + lane_base + s * kACols + khalf * 16, a);
                     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
@@ -456,7 +460,7 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
             if (*epi_decision) break;
             tc_fence_after();
             const int n = n0 + row_local;
-            if (splits > 1) {
+            if (FIXED_STAGES == 0 && splits > 1) {
                 // split-K: this split's fp32 partial goes to partials[split][m][n]
                 float *part = partials + (int64_t)wk.split * M * N;
 #pragma unroll 1
@@ -677,8 +681,8 @@ qz_status launch_gemm(const void *a, const void *codes, const void *scales, cons
     const uint32_t smem_bytes = gemm_layout(BITS, act_rows, stages).end + 1024;
     const int64_t items = ceil_div(N, kTileN) * ceil_div(M, kTileM) * splits;
     const int grid = (int)std::min<int64_t>(items, kSmCount);
-    auto kernel = act_rows == kTileM ? wa16_gemm_tcgen05<BITS, kFullTileStages>
-                                     : wa16_gemm_tcgen05<BITS, 0>;
+    auto kernel = act_rows == kTileM && splits == 1 ? wa16_gemm_tcgen05<BITS, kFullTileStages>
+                                                    : wa16_gemm_tcgen05<BITS, 0>;
     kernel<<<grid, kThreads, smem_bytes, st>>>(
         act_map, pack_map, y_map, static_cast<const uint16_t *>(scales),
         static_cast<const uint8_t *>(zeros), (int)M, (int)N, (int)K, (int)group_size,

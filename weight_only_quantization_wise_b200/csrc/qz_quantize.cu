@@ -237,8 +237,8 @@ quantize_small_groups(const uint4 *__restrict__ w, int64_t total_chunks,
         group_params<BITS, SYM>(vmin, vmax, vmax, s_bits, s_f, z);
         const float r = __frcp_rn(s_f);
         uint2 cw[4];
-#pragma unroll
         const bool clamp = needs_clamp<BITS, SYM>(vmax, r, z);
+#pragma unroll
         for (int u = 0; u < 4; ++u) cw[u] = group_chunk_codes<BITS, SYM>(x[u], s_f, r, z, clamp);
         if (BITS == 4) {
             reinterpret_cast<uint4 *>(codes)[c0 >> 2] = make_uint4(cw[0].x, cw[1].x, cw[2].x, cw[3].x);

@@ -149,9 +149,13 @@ def test_w8a16_gemm_rejects(args, expect):
 
 def test_w8a16_gemm_workspace_follows_the_route():
     assert qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMM, 2048, 8192, 8192, 8192) == 0
-    # 64 tiles on 148 SMs: two K splits, fp32 partials [2][M][N] + counters
+    # 64 tiles, two CTAs per SM for 64-token tiles: four K splits, fp32
+    # partials [4][M][N] + counters
     assert qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMM, 64, 8192, 8192, 8192) == \
-        2 * 64 * 8192 * 4 + 64 * 4
+        4 * 64 * 8192 * 4 + 64 * 4
+    # 128-token tiles run one CTA per SM: two splits
+    assert qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMM, 128, 8192, 8192, 8192) == \
+        2 * 128 * 8192 * 4 + 64 * 4
     assert qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMM, 64, 8192, 8192, 128) == \
         qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMM, 64, 8192, 8192, 8192)
     assert (qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMM, 16, 4096, 4096, 4096) ==

@@ -68,6 +68,10 @@ constexpr int kEpilogueWarps = 4;
 constexpr int kFirstEpilogueWarp = 2 + kDequantWarps;
 constexpr int kThreads = 32 * (2 + kDequantWarps + kEpilogueWarps);
 constexpr int kSmemLimit = 227 * 1024;    // dynamic shared memory of one CTA
+constexpr int kSmemPerSm = 228 * 1024;    // shared memory of an SM (1 KB of it reserved per CTA)
+// Short token tiles (at most kPairMaxRows tokens) run two CTAs per SM, each
+// with half of the tensor memory, so that twice as many warps dequantize.
+constexpr int kPairMaxRows = 64;
 
 // Shared- and tensor-memory layout of one launch.  The activation box holds
 // act_rows tokens (a multiple of 16, at most 256), so a stage takes
@@ -106,13 +110,19 @@ __host__ __device__ constexpr GemmLayout gemm_layout(int bits, int act_rows, int
     return L;
 }
 
-// Deepest ring that fits for this activation box.
-constexpr int gemm_stages(int bits, int act_rows) {
+constexpr int gemm_ctas_per_sm(int act_rows) { return act_rows <= kPairMaxRows ? 2 : 1; }
+
+// Deepest ring that fits for this activation box, with `ctas` CTAs per SM
+// sharing its shared and tensor memory.
+constexpr int gemm_stages(int bits, int act_rows, int ctas = 1) {
+    const int smem = ctas == 1 ? kSmemLimit : kSmemPerSm / ctas - 1024;
     int s = kMaxStages;
-    while (s > 2 && gemm_layout(bits, act_rows, s).end + 1024 > (uint32_t)kSmemLimit) --s;
-    const int by_tmem = (kTmemCols - (int)gemm_layout(bits, act_rows, 1).a_col0) / kACols;
+    while (s > 2 && gemm_layout(bits, act_rows, s).end + 1024 > (uint32_t)smem) --s;
+    const int by_tmem = (kTmemCols / ctas - (int)gemm_layout(bits, act_rows, 1).a_col0) / kACols;
     return s < by_tmem ? s : by_tmem;
 }
+static_assert(gemm_stages(4, kPairMaxRows, 2) >= 4 && gemm_stages(8, kPairMaxRows, 2) >= 4,
+              "paired CTAs keep at least four stages");
 constexpr int kFullTileStages = 4;
 static_assert(gemm_stages(4, kTileM) == kFullTileStages && gemm_stages(8, kTileM) == kFullTileStages,
               "a full token tile keeps four stages");
@@ -195,8 +205,8 @@ __device__ __forceinline__ GemmLayout kernel_layout(int act_rows, int stages) {
     }
 }
 
-template <int BITS, int FIXED_STAGES>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int BITS, int FIXED_STAGES, int CTAS>
+__global__ void __launch_bounds__(kThreads, CTAS)
 wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
                    const __grid_constant__ CUtensorMap pack_map,
                    const __grid_constant__ CUtensorMap y_map,
@@ -248,7 +258,7 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(tmem_slot)),
-                     "r"(kTmemCols)
+                     "r"(kTmemCols / CTAS)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -494,33 +504,34 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
                         const int nq = n0 + 4 * (t & 31);
                         if (nq < N) {
                             for (int mb = m0 + (t >> 5); mb < m_end; mb += 16) {
-                                float4 v[kMaxSplits][4];
+                                float4 acc[4];
 #pragma unroll
-                                for (int sp = 0; sp < kMaxSplits; ++sp)
+                                for (int j = 0; j < 4; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+                                for (int sp = 0; sp < splits; ++sp) {
+                                    float4 v[4];
 #pragma unroll
                                     for (int j = 0; j < 4; ++j) {
                                         const int m = mb + 4 * j;
-                                        v[sp][j] = (sp < splits && m < m_end)
-                                                       ? __ldcg(reinterpret_cast<const float4 *>(
-                                                             &partials[((int64_t)sp * M + m) * N + nq]))
-                                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+                                        v[j] = m < m_end ? __ldcg(reinterpret_cast<const float4 *>(
+                                                               &partials[((int64_t)sp * M + m) * N + nq]))
+                                                         : make_float4(0.f, 0.f, 0.f, 0.f);
                                     }
+#pragma unroll
+                                    for (int j = 0; j < 4; ++j) {
+                                        acc[j].x += v[j].x;
+                                        acc[j].y += v[j].y;
+                                        acc[j].z += v[j].z;
+                                        acc[j].w += v[j].w;
+                                    }
+                                }
 #pragma unroll
                                 for (int j = 0; j < 4; ++j) {
                                     const int m = mb + 4 * j;
-                                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                                    for (int sp = 0; sp < kMaxSplits; ++sp)
-                                        if (sp < splits) {
-                                            acc.x += v[sp][j].x;
-                                            acc.y += v[sp][j].y;
-                                            acc.z += v[sp][j].z;
-                                            acc.w += v[sp][j].w;
-                                        }
                                     if (m < m_end) {
                                         uint2 o;
-                                        o.x = dev::f32_to_bf16_rne(acc.x) | (dev::f32_to_bf16_rne(acc.y) << 16);
-                                        o.y = dev::f32_to_bf16_rne(acc.z) | (dev::f32_to_bf16_rne(acc.w) << 16);
+                                        o.x = dev::f32_to_bf16_rne(acc[j].x) | (dev::f32_to_bf16_rne(acc[j].y) << 16);
+                                        o.y = dev::f32_to_bf16_rne(acc[j].z) | (dev::f32_to_bf16_rne(acc[j].w) << 16);
                                         *reinterpret_cast<uint2 *>(&y[(int64_t)m * N + nq]) = o;
                                     }
                                 }
@@ -528,23 +539,24 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
                         }
                     } else if (n < N) {
                         for (int mb = m0; mb < m_end; mb += 8) {
-                            float acc[8], v[kMaxSplits][8];
+                            float acc[8];
 #pragma unroll
-                            for (int sp = 0; sp < kMaxSplits; ++sp)
+                            for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+#pragma unroll 2
+                            for (int sp = 0; sp < splits; ++sp) {
+                                float v[8];
 #pragma unroll
                                 for (int j = 0; j < 8; ++j)
-                                    v[sp][j] = (sp < splits && mb + j < m_end)
-                                                   ? __ldcg(&partials[((int64_t)sp * M + mb + j) * N + n])
-                                                   : 0.0f;
+                                    v[j] = mb + j < m_end
+                                               ? __ldcg(&partials[((int64_t)sp * M + mb + j) * N + n])
+                                               : 0.0f;
 #pragma unroll
-                            for (int j = 0; j < 8; ++j) {
-                                acc[j] = 0.0f;
+                                for (int j = 0; j < 8; ++j) acc[j] += v[j];
+                            }
 #pragma unroll
-                                for (int sp = 0; sp < kMaxSplits; ++sp)
-                                    if (sp < splits) acc[j] += v[sp][j];
+                            for (int j = 0; j < 8; ++j)
                                 if (mb + j < m_end)
                                     y[(int64_t)(mb + j) * N + n] = (uint16_t)dev::f32_to_bf16_rne(acc[j]);
-                            }
                         }
                     }
                     if (storer) counters[wk.tile] = 0u;
@@ -588,7 +600,7 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
     if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                     "r"(kTmemCols)
+                     "r"(kTmemCols / CTAS)
                      : "memory");
     }
 }
@@ -598,10 +610,14 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
 // Split-K: when the 128 x 256 output tiles are fewer than the SMs, each
 // tile's K range is divided among up to kMaxSplits CTAs (at least 4 stages
 // each); their fp32 partials meet in the workspace.
+// Tokens per activation box: a whole tile, or all of M rounded up to 16.
+int gemm_act_rows(int64_t M) { return M >= kTileM ? kTileM : (int)((M + 15) & ~int64_t(15)); }
+
 int gemm_splits(int64_t M, int64_t N, int64_t K) {
     const int64_t tiles = ceil_div(N, kTileN) * ceil_div(M, kTileM);
-    if (tiles >= kSmCount) return 1;
-    int64_t s = kSmCount / tiles;
+    const int64_t slots = (int64_t)kSmCount * gemm_ctas_per_sm(gemm_act_rows(M));
+    if (tiles >= slots) return 1;
+    int64_t s = slots / tiles;
     if (s > kMaxSplits) s = kMaxSplits;
     if (s > K / kTileK / 4) s = K / kTileK / 4;
     return s < 1 ? 1 : (int)s;
@@ -640,8 +656,8 @@ qz_status launch_gemm(const void *a, const void *codes, const void *scales, cons
                       int64_t M, int64_t N, int64_t K, int64_t group_size, void *y,
                       void *workspace, cudaStream_t st) {
     constexpr int kRowBytesPerK = BITS;   // code bytes of a row per 8 k
-    // tokens per activation box: a whole tile, or all of M rounded to 16
-    const int act_rows = M >= kTileM ? kTileM : (int)((M + 15) & ~int64_t(15));
+    const int act_rows = gemm_act_rows(M);
+    const int ctas = gemm_ctas_per_sm(act_rows);
     const int splits = gemm_splits(M, N, K);
     float *partials = nullptr;
     uint32_t *counters = nullptr;
@@ -672,17 +688,23 @@ qz_status launch_gemm(const void *a, const void *codes, const void *scales, cons
     static std::once_flag attr_once[64];
     if (dev >= 0 && dev < 64)
         std::call_once(attr_once[dev], [] {
-            cudaFuncSetAttribute(wa16_gemm_tcgen05<BITS, kFullTileStages>,
+            cudaFuncSetAttribute(wa16_gemm_tcgen05<BITS, kFullTileStages, 1>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
-            cudaFuncSetAttribute(wa16_gemm_tcgen05<BITS, 0>,
+            cudaFuncSetAttribute(wa16_gemm_tcgen05<BITS, 0, 1>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+            cudaFuncSetAttribute(wa16_gemm_tcgen05<BITS, 0, 2>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+            // two CTAs per SM need the whole unified memory as shared memory
+            cudaFuncSetAttribute(wa16_gemm_tcgen05<BITS, 0, 2>,
+                                 cudaFuncAttributePreferredSharedMemoryCarveout, 100);
         });
-    const int stages = gemm_stages(BITS, act_rows);
+    const int stages = gemm_stages(BITS, act_rows, ctas);
     const uint32_t smem_bytes = gemm_layout(BITS, act_rows, stages).end + 1024;
     const int64_t items = ceil_div(N, kTileN) * ceil_div(M, kTileM) * splits;
-    const int grid = (int)std::min<int64_t>(items, kSmCount);
-    auto kernel = act_rows == kTileM && splits == 1 ? wa16_gemm_tcgen05<BITS, kFullTileStages>
-                                                    : wa16_gemm_tcgen05<BITS, 0>;
+    const int grid = (int)std::min<int64_t>(items, (int64_t)kSmCount * ctas);
+    auto kernel = act_rows == kTileM && splits == 1 ? wa16_gemm_tcgen05<BITS, kFullTileStages, 1>
+                  : ctas == 2                      ? wa16_gemm_tcgen05<BITS, 0, 2>
+                                                   : wa16_gemm_tcgen05<BITS, 0, 1>;
     kernel<<<grid, kThreads, smem_bytes, st>>>(
         act_map, pack_map, y_map, static_cast<const uint16_t *>(scales),
         static_cast<const uint8_t *>(zeros), (int)M, (int)N, (int)K, (int)group_size,

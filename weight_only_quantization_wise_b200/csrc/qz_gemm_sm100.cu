@@ -351,40 +351,14 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
                 const int spg = group_size / kTileK;      // stages per group
                 const uint16_t *srow = scales + (int64_t)(valid ? n : 0) * gpr;
                 const uint8_t *zrow = zeros + (int64_t)(valid ? n : 0) * gpr;
-                // Scales and zeros of the next kMetaFifo groups wait in a
-                // register FIFO (a group spans spg stages), so their loads are
-                // issued up to kMetaFifo groups before use and no per-stage
-                // index arithmetic is needed.
                 const int g0 = wk.kt0 / spg;              // group of the first stage
-                uint32_t sq[kMetaFifo], zq[kMetaFifo];
-#pragma unroll
-                for (int q = 0; q < kMetaFifo; ++q) {
-                    sq[q] = (valid && g0 + q < gpr) ? __ldg(&srow[g0 + q]) : 0u;
-                    zq[q] = (valid && g0 + q < gpr) ? __ldg(&zrow[g0 + q]) : 0u;
-                }
-                int stage_in_group = wk.kt0 - g0 * spg, next_group = g0 + kMetaFifo;
-                for (int kt = wk.kt0; kt < wk.kt1;
-                     ++kt, s = (s + 1 == stages ? 0 : s + 1), r += (s == 0)) {
-                    const uint32_t sb = sq[0], zb = zq[0];
-                    if (++stage_in_group == spg) {           // the next stage starts a new group
-                        stage_in_group = 0;
-#pragma unroll
-                        for (int q = 0; q < kMetaFifo - 1; ++q) {
-                            sq[q] = sq[q + 1];
-                            zq[q] = zq[q + 1];
-                        }
-                        sq[kMetaFifo - 1] =
-                            (valid && next_group < gpr) ? __ldg(&srow[next_group]) : 0u;
-                        zq[kMetaFifo - 1] =
-                            (valid && next_group < gpr) ? __ldg(&zrow[next_group]) : 0u;
-                        ++next_group;
-                    }
+                int kt = wk.kt0;
+                // One stage: convert the codes of slot s with scale bits sb and zero zb.
+                auto stage = [&](uint32_t sb, uint32_t zb) -> bool {
                     // warp-uniform: the tcgen05.st below needs every lane
                     if (!__all_sync(0xFFFFFFFFu,
-                                    gemm_wait(full_bar(s), r & 1, wait_limit, abort_flag))) {
-                        ok = false;
-                        break;
-                    }
+                                    gemm_wait(full_bar(s), r & 1, wait_limit, abort_flag)))
+                        return false;
                     const uint4 p = *reinterpret_cast<const uint4 *>(
                         smem + SmemLayout.pack + s * kPackBytes + row_local * (kTileK / 2) +
                         khalf * 16);
@@ -406,6 +380,84 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(afull_bar(s));
+                    ++kt;
+                    s = s + 1 == stages ? 0 : s + 1;
+                    r += (s == 0);
+                    return true;
+                };
+                const bool quads = (gpr & 3) == 0 && (reinterpret_cast<uintptr_t>(scales) & 7) == 0 &&
+                                   (reinterpret_cast<uintptr_t>(zeros) & 3) == 0;
+                if (quads) {
+                    // Scales and zeros of four consecutive groups come in one 8-byte
+                    // and one 4-byte load.  Two register sets alternate over the
+                    // quads, and a set is reloaded only after its quad is done, so a
+                    // load is issued four groups before its first use and no
+                    // register holding a load in flight is ever copied.
+                    const uint2 *squad = reinterpret_cast<const uint2 *>(srow);
+                    const uint32_t *zquad = reinterpret_cast<const uint32_t *>(zrow);
+                    const int nq = gpr >> 2;
+                    int qa = g0 >> 2, gi = g0 & 3, st = wk.kt0 - g0 * spg;
+                    int qb = qa + 1;
+                    uint2 sA = (valid && qa < nq) ? __ldg(&squad[qa]) : make_uint2(0u, 0u);
+                    uint32_t zA = (valid && qa < nq) ? __ldg(&zquad[qa]) : 0u;
+                    uint2 sB = (valid && qb < nq) ? __ldg(&squad[qb]) : make_uint2(0u, 0u);
+                    uint32_t zB = (valid && qb < nq) ? __ldg(&zquad[qb]) : 0u;
+                    // the stages of groups gi..3 of one quad
+                    auto run_quad = [&](uint2 sw, uint32_t zw) {
+                        for (; gi < 4 && kt < wk.kt1 && ok; ++gi, st = 0) {
+                            const uint32_t sb = ((gi < 2 ? sw.x : sw.y) >> (16 * (gi & 1))) & 0xFFFFu;
+                            const uint32_t zb = (zw >> (8 * gi)) & 0xFFu;
+                            for (; st < spg && kt < wk.kt1; ++st)
+                                if (!stage(sb, zb)) {
+                                    ok = false;
+                                    break;
+                                }
+                        }
+                        gi = 0;
+                    };
+                    while (true) {
+                        run_quad(sA, zA);
+                        if (kt >= wk.kt1 || !ok) break;
+                        qa += 2;
+                        sA = (valid && qa < nq) ? __ldg(&squad[qa]) : make_uint2(0u, 0u);
+                        zA = (valid && qa < nq) ? __ldg(&zquad[qa]) : 0u;
+                        run_quad(sB, zB);
+                        if (kt >= wk.kt1 || !ok) break;
+                        qb += 2;
+                        sB = (valid && qb < nq) ? __ldg(&squad[qb]) : make_uint2(0u, 0u);
+                        zB = (valid && qb < nq) ? __ldg(&zquad[qb]) : 0u;
+                    }
+                } else {
+                    // Scales and zeros of the next kMetaFifo groups wait in a
+                    // register FIFO (a group spans spg stages); no per-stage
+                    // index arithmetic is needed.
+                    uint32_t sq[kMetaFifo], zq[kMetaFifo];
+#pragma unroll
+                    for (int q = 0; q < kMetaFifo; ++q) {
+                        sq[q] = (valid && g0 + q < gpr) ? __ldg(&srow[g0 + q]) : 0u;
+                        zq[q] = (valid && g0 + q < gpr) ? __ldg(&zrow[g0 + q]) : 0u;
+                    }
+                    int stage_in_group = wk.kt0 - g0 * spg, next_group = g0 + kMetaFifo;
+                    while (kt < wk.kt1) {
+                        const uint32_t sb = sq[0], zb = zq[0];
+                        if (++stage_in_group == spg) {       // the next stage starts a new group
+                            stage_in_group = 0;
+#pragma unroll
+                            for (int q = 0; q < kMetaFifo - 1; ++q) {
+                                sq[q] = sq[q + 1];
+                                zq[q] = zq[q + 1];
+                            }
+                            sq[kMetaFifo - 1] =
+                                (valid && next_group < gpr) ? __ldg(&srow[next_group]) : 0u;
+                            zq[kMetaFifo - 1] =
+                                (valid && next_group < gpr) ? __ldg(&zrow[next_group]) : 0u;
+                            ++next_group;
+                        }
+                        if (!stage(sb, zb)) {
+                            ok = false;
+                            break;
+                        }
+                    }
                 }
             } else {
                 // one scale per weight row for the whole K

@@ -18,6 +18,8 @@
 // [n][k/g] layout gives.
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "qz_internal.cuh"
 
 namespace qz {
@@ -205,11 +207,14 @@ __device__ __forceinline__ void fold_range(const float (&x)[8], float &vmin, flo
 // ranges with butterfly shuffles.  The per-group work (range, S, Z, 1/S) is
 // done once per 32 values, and a lane writes its int4 codes with one 16-byte
 // store.  The four 16-byte loads of a lane are L1-cached so that they merge
-// into full sectors.
+// into full sectors.  PREFETCH (chosen when a warp makes at least
+// kPrefetchIters passes): the next pass's loads are issued before this pass
+// is converted, at the cost of 16 registers per thread.
 // ---------------------------------------------------------------------------
 constexpr int kQuantThreads = 256;
+constexpr int kPrefetchIters = 4;
 
-template <int BITS, bool SYM, int LPG>
+template <int BITS, bool SYM, int LPG, bool PREFETCH>
 __global__ void __launch_bounds__(kQuantThreads)
 quantize_small_groups(const uint4 *__restrict__ w, int64_t total_chunks,
                       uint8_t *__restrict__ codes, uint16_t *__restrict__ scales,
@@ -217,13 +222,29 @@ quantize_small_groups(const uint4 *__restrict__ w, int64_t total_chunks,
     const int lane = threadIdx.x & 31;
     const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    uint4 nxt[4];
+    if (PREFETCH) {
+        const int64_t c0 = warp * 128 + 4 * lane;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            nxt[u] = c0 < total_chunks ? __ldg(w + c0 + u) : make_uint4(0, 0, 0, 0);
+    }
     for (int64_t base = warp * 128; base < total_chunks; base += nwarps * 128) {
         const int64_t c0 = base + 4 * lane;       // total_chunks is a multiple of 4
         const bool valid = c0 < total_chunks;
         float x[4][8];
+        if (PREFETCH) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-            unpack8(valid ? __ldg(w + c0 + u) : make_uint4(0, 0, 0, 0), x[u]);
+            for (int u = 0; u < 4; ++u) unpack8(nxt[u], x[u]);
+            const int64_t cn = c0 + nwarps * 128;
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                nxt[u] = cn < total_chunks ? __ldg(w + cn + u) : make_uint4(0, 0, 0, 0);
+        } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                unpack8(valid ? __ldg(w + c0 + u) : make_uint4(0, 0, 0, 0), x[u]);
+        }
         float vmin = 0.0f, vmax = 0.0f;           // the range always contains 0
 #pragma unroll
         for (int u = 0; u < 4; ++u) fold_range<SYM>(x[u], vmin, vmax);
@@ -467,19 +488,23 @@ qz_status quantize_typed(const void *w, int64_t N, int64_t K, int64_t g, void *c
         return launch_status();
     }
     const int grid = grid_for(total, kQuantThreads * 4);
+    // passes per warp: each pass of a warp covers 128 chunks
+    const bool prefetch = total >= (int64_t)grid * (kQuantThreads / 32) * 128 * kPrefetchIters;
+    auto small = [&](auto lpg) {
+        constexpr int LPG = decltype(lpg)::value;
+        if (prefetch)
+            quantize_small_groups<BITS, SYM, LPG, true><<<grid, kQuantThreads, 0, st>>>(
+                src, total, c8, s16, z8);
+        else
+            quantize_small_groups<BITS, SYM, LPG, false><<<grid, kQuantThreads, 0, st>>>(
+                src, total, c8, s16, z8);
+        return launch_status();
+    };
     switch (g) {
-    case 32:
-        quantize_small_groups<BITS, SYM, 1><<<grid, kQuantThreads, 0, st>>>(src, total, c8, s16, z8);
-        return launch_status();
-    case 64:
-        quantize_small_groups<BITS, SYM, 2><<<grid, kQuantThreads, 0, st>>>(src, total, c8, s16, z8);
-        return launch_status();
-    case 128:
-        quantize_small_groups<BITS, SYM, 4><<<grid, kQuantThreads, 0, st>>>(src, total, c8, s16, z8);
-        return launch_status();
-    case 256:
-        quantize_small_groups<BITS, SYM, 8><<<grid, kQuantThreads, 0, st>>>(src, total, c8, s16, z8);
-        return launch_status();
+    case 32: return small(std::integral_constant<int, 1>{});
+    case 64: return small(std::integral_constant<int, 2>{});
+    case 128: return small(std::integral_constant<int, 4>{});
+    case 256: return small(std::integral_constant<int, 8>{});
     default:
         break;
     }

@@ -587,9 +587,15 @@ qz_status launch_gemv(const void *a, const void *codes, const void *scales, cons
 }  // namespace
 
 // Stream-K plan.  Up to kCtasPerSm 4-warp CTAs are resident on an SM (the
-// ring of a CTA takes 36 KB (int4) or 48 KB (int8) of shared memory).  The
-// same number of CTAs runs on every SM, as many as give each warp at least
-// four K blocks (fewer contributors per task shorten the split-K tail).
+// ring of a CTA takes 36 KB (int4) or 48 KB (int8) of shared memory), and
+// the same number k runs on every SM.
+//   M = 1: a warp streams its ceil(U / W) K blocks one after another, and a
+//   block takes longer the more warps share an SM sub-partition: about
+//   (0.40 + 0.33 k) us with k CTAs per SM, fitted to the decode layers.  k
+//   minimises ceil(U / W) * (40 + 33 k); ties go to the smaller k.
+//   M > 1: the split-K partials grow with M, so k is the largest that gives
+//   each warp at least kGemvMinBlocksPerWarp blocks (fewer contributors).
+constexpr int kBlockCostBase = 40, kBlockCostPerCta = 33;
 constexpr int kGemvMinBlocksPerWarp = 4;
 
 GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K, int bits) {
@@ -599,9 +605,22 @@ GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K, int bits) {
     const int64_t units = p.tasks * p.kblocks;
     const int64_t max_per_sm = M <= 8 ? (bits == 4 ? kCtasPerSm<4, 1> : kCtasPerSm<8, 1>)
                                       : kCtasPerSm<4, 2>;
-    int64_t per_sm = units / ((int64_t)kSmCount * kWarpsPerCta * kGemvMinBlocksPerWarp);
-    if (per_sm > max_per_sm) per_sm = max_per_sm;
-    if (per_sm < 1) per_sm = 1;
+    int64_t per_sm = 1;
+    if (M == 1) {
+        int64_t best_cost = -1;
+        for (int64_t k = 1; k <= max_per_sm; ++k) {
+            const int64_t cost = ceil_div(units, (int64_t)kSmCount * kWarpsPerCta * k) *
+                                 (kBlockCostBase + kBlockCostPerCta * k);
+            if (best_cost < 0 || cost < best_cost) {
+                best_cost = cost;
+                per_sm = k;
+            }
+        }
+    } else {
+        per_sm = units / ((int64_t)kSmCount * kWarpsPerCta * kGemvMinBlocksPerWarp);
+        if (per_sm > max_per_sm) per_sm = max_per_sm;
+        if (per_sm < 1) per_sm = 1;
+    }
     p.warps = (int64_t)kSmCount * per_sm * kWarpsPerCta;
     if (p.warps > units) p.warps = ceil_div(units, kWarpsPerCta) * kWarpsPerCta;
     // contributors of one task: at most ceil(KB / floor(U/W)) + 1

@@ -162,6 +162,23 @@ def test_w8a16_gemm_workspace_follows_the_route():
             qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMV, 16, 4096, 4096, 4096))
 
 
+@pytest.mark.parametrize("op,M,N,K,g,expect", [
+    # M = 1: CTAs per SM from the per-block cost model (4096 x 4096: four,
+    # 1.73 blocks per warp, every task split over up to 32 slots)
+    ("W4A16_GEMV", 1, 4096, 4096, 128, 128 * 32 * 1 * 32 * 4 + 2 * 64 * 4),
+    # 70B layer: five CTAs per SM, 19 blocks per warp, 5 slots per task
+    ("W4A16_GEMV", 1, 28672, 8192, 128, 896 * 5 * 1 * 32 * 4 + 14 * 64 * 4),
+    ("W8A16_GEMV", 1, 4096, 4096, 4096, 128 * 32 * 1 * 32 * 4 + 2 * 64 * 4),
+    # M > 1: the largest CTA count giving each warp at least four blocks
+    ("W4A16_GEMV", 8, 11008, 4096, 128, 344 * 9 * 8 * 32 * 4 + 6 * 64 * 4),
+    ("W4A16_GEMV", 16, 28672, 8192, 128, 896 * 3 * 16 * 32 * 4 + 14 * 64 * 4),
+])
+def test_gemv_plan_workspace(op, M, N, K, g, expect):
+    """The stream-K plan (host logic) through the workspace it asks for:
+    fp32 partial slots [task][slot][M][32] plus one counter per task."""
+    assert qz.qz_workspace_bytes(getattr(qz, "QZ_OP_" + op), M, N, K, g) == expect
+
+
 def test_launch_overlap_setter():
     assert qz.lib.qz_set_launch_overlap(2) == INVALID
     assert qz.lib.qz_set_launch_overlap(-1) == INVALID

@@ -158,6 +158,14 @@ def matmul_f64(a_bits, w_hat_bits):
     return y, ya
 
 
+# Half the spacing of the bf16 subnormals (2^-133).  Below 2^-126 a bf16
+# output cannot come closer than this to an arbitrary real value, while the
+# relative term 8e-3 |y| assumes bf16's normal relative precision (2^-8).
+BF16_SUBNORMAL_HALF_SPACING = 2.0 ** -134
+
+
 def tolerance(y_ref: np.ndarray, abs_ref: np.ndarray) -> np.ndarray:
-    """Per-element bound |y - y_ref| <= 8e-3 |y_ref| + 1e-4 sum_k |a_k w_k|."""
-    return 8e-3 * np.abs(y_ref) + 1e-4 * abs_ref
+    """Per-element bound |y - y_ref| <= 8e-3 |y_ref| + 1e-4 sum_k |a_k w_k|,
+    plus half the bf16 subnormal spacing so that outputs below the smallest
+    normal bf16 can meet it (negligible for every normal output)."""
+    return 8e-3 * np.abs(y_ref) + 1e-4 * abs_ref + BF16_SUBNORMAL_HALF_SPACING

@@ -19,6 +19,7 @@ import os
 from fractions import Fraction
 
 import numpy as np
+import pytest
 import torch
 
 import oracle
@@ -383,6 +384,22 @@ def pin_matmul_f64():
     assert np.array_equal(y1[0], wf[:, 7])
     y0, _ = oracle.matmul_f64(a, np.zeros((N, K), np.uint16))
     assert (y0 == 0).all()
+
+
+def pin_tolerance_reaches_bf16_outputs():
+    """The bound admits the correctly rounded bf16 of the exact product at
+    every magnitude: at least half a bf16 spacing, 2^-9 |y| for normal
+    outputs (inside 8e-3 |y|) and 2^-134 for subnormal ones."""
+    rng = np.random.default_rng(11)
+    for scale in (1e3, 1.0, 1e-30, 1e-38, 1e-39, 1e-40):
+        y = rng.normal(0, scale, 4000)
+        ya = np.abs(y)                       # the smallest sum_k |a_k w_k| a product can have
+        yb = oracle.bf16_bits_to_f32(_bf16_round(y.astype(np.float32))).astype(np.float64)
+        finite = np.isfinite(yb)
+        assert (np.abs(yb - y)[finite] <= oracle.tolerance(y, ya)[finite]).all(), scale
+    # the subnormal term is negligible against normal outputs
+    assert oracle.BF16_SUBNORMAL_HALF_SPACING == 2.0 ** -134
+    assert oracle.tolerance(np.array([1e-30]), np.array([1e-30]))[0] == pytest.approx(8.1e-33)
 
 
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -142,6 +142,37 @@ def test_edge_groups_bit_exact(dev, bits, sym):
         assert np.array_equal(u16(out), wref)
 
 
+@pytest.mark.parametrize("M", [1, 16, 17, 64])
+def test_matmuls_on_edge_rows(dev, M):
+    """The edge rows (all zero, constant, ties, top clamp, tiny and huge
+    ranges, one outlier, one-signed, -0) through every matmul: the all-zero
+    row gives exactly 0 and every output is within the tolerance of the fp64
+    product over the oracle's dequantized weights."""
+    w = edge_matrix()
+    N, K = w.shape
+    a = synthetic.activations(M, K, seed=90 + M)
+    for bits, sym, g in ((4, False, 128), (8, True, K)):
+        c, s, z = oracle.quantize_pack(u16(w), bits, sym, g)
+        w_hat = oracle.dequantize(c, s, z, N, K, bits, sym, g)
+        y_ref, abs_ref = oracle.matmul_f64(u16(a), w_hat)
+        ad, cd, sd = a.to(dev), to_dev_u8(c, dev), to_dev_bf16(s, dev)
+        if bits == 4:
+            zd = to_dev_u8(z, dev)
+            outs = [("gemm", qz.qz_w4a16_gemm(ad, cd, sd, zd, N, K, g))]
+            if M <= 16:
+                outs.append(("gemv", qz.qz_w4a16_gemv(ad, cd, sd, zd, N, K, g)))
+        else:
+            outs = [("gemm", qz.qz_w8a16_gemm(ad, cd, sd, N, K))]
+            if M <= 16:
+                outs.append(("gemv", qz.qz_w8a16_gemv(ad, cd, sd, N, K)))
+        torch.cuda.synchronize()
+        assert qz.qz_device_status() == 0
+        for what, y in outs:
+            yb = u16(y).reshape(M, N)
+            assert (oracle.bf16_bits_to_f32(yb[:, 0]) == 0).all(), (bits, what)   # all-zero row
+            check_tolerance(yb, y_ref, abs_ref, f"edge rows bits={bits} {what} M={M}")
+
+
 # ---------------------------------------------------------------------------
 # GEMV
 # ---------------------------------------------------------------------------

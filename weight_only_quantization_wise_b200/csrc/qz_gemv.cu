@@ -377,6 +377,7 @@ gemv_kernel(const GemvArgs p) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int64_t w = (int64_t)blockIdx.x * kWarpsPerCta + warp;
+    if (w >= p.warps) return;                      // the last CTA of a short grid
     int64_t u = w * p.units / p.warps;
     const int64_t u_end = (w + 1) * p.units / p.warps;
     // With launch overlap, only the first ring fill of weights (which the
@@ -562,7 +563,7 @@ qz_status launch_gemv(const void *a, const void *codes, const void *scales, cons
     args.kblocks = (int)plan.kblocks;
     args.slots = (int)plan.slots;
     args.prefetch_early = overlap;
-    const dim3 grid((unsigned)(plan.warps / kWarpsPerCta));
+    const dim3 grid((unsigned)ceil_div(plan.warps, (int64_t)kWarpsPerCta));
 
     // The ring copies the aligned 4-byte words holding each scale and zero;
     // they stay inside the arrays when N * K / g is a multiple of 4.
@@ -622,7 +623,10 @@ GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K, int bits) {
         if (per_sm < 1) per_sm = 1;
     }
     p.warps = (int64_t)kSmCount * per_sm * kWarpsPerCta;
-    if (p.warps > units) p.warps = ceil_div(units, kWarpsPerCta) * kWarpsPerCta;
+    // Fewer units than warps: one unit per warp.  Every warp must own at
+    // least one unit, or a split task would count a contributor that never
+    // arrives.
+    if (p.warps > units) p.warps = units;
     // contributors of one task: at most ceil(KB / floor(U/W)) + 1
     const int64_t per_warp = units / p.warps;
     p.slots = per_warp >= 1 ? ceil_div(p.kblocks, per_warp) + 1 : p.kblocks + 1;

@@ -63,7 +63,7 @@ qz_status launch_dequantize(const void *codes, const void *scales, const void *z
 struct GemvPlan {
     int64_t tasks;        // 32-row tasks
     int64_t kblocks;      // 128-wide K blocks per task
-    int64_t warps;        // launched warps (a multiple of the warps per CTA)
+    int64_t warps;        // launched warps (each owns at least one unit)
     int64_t slots;        // partial slots per task (max contributors)
     size_t partial_bytes; // fp32 partials [tasks][slots][M][32]
     size_t counter_bytes; // uint32 arrival counter per task

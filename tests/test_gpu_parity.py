@@ -4,7 +4,9 @@ Bars (fixed before any kernel was written):
   * codes, scales, zeros: bit-exact;
   * dequantized bf16 weights: bit-exact;
   * matmul outputs: |y - y_ref| <= 8e-3 |y_ref| + 1e-4 sum_k |a_k w_k| against
-    the oracle's fp64 product over its own bf16 dequantized weights.
+    the oracle's fp64 product over its own bf16 dequantized weights, plus half
+    the bf16 subnormal spacing (2^-134) so that outputs below 2^-126 can meet
+    it at all (oracle.tolerance).
 Large configurations are checked on sampled rows that the oracle computes on
 its own; everything else is compared element by element.
 """

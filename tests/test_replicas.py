@@ -39,7 +39,7 @@ def _rank_main(rank, world, port, out):
 def test_two_replicas_take_the_slowest_rank():
     world = 2
     port = _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:   # no fork of a threaded process
         out = mgr.dict()
         mp.start_processes(_rank_main, args=(world, port, out), nprocs=world, join=True,
                            start_method="spawn")

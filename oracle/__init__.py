@@ -34,8 +34,6 @@ def load(path: str):
     L.qzo_f32_to_bf16_up.restype = ctypes.c_uint16
     L.qzo_code_range.argtypes = [_int, _int, ctypes.POINTER(_int), ctypes.POINTER(_int)]
     L.qzo_code_range.restype = _int
-    L.qzo_num_groups.argtypes = [_i64, _i64, _i64]
-    L.qzo_num_groups.restype = _i64
     L.qzo_quantize_pack.argtypes = [_p, _i64, _i64, _int, _int, _i64, _p, _p, _p]
     L.qzo_quantize_pack.restype = _int
     L.qzo_dequantize.argtypes = [_p, _p, _p, _i64, _i64, _int, _int, _i64, _p]
@@ -88,10 +86,6 @@ def code_range(bits: int, symmetric: bool):
     if lib().qzo_code_range(bits, int(symmetric), ctypes.byref(lo), ctypes.byref(hi)):
         raise ValueError("unsupported format")
     return lo.value, hi.value
-
-
-def num_groups(N: int, K: int, group_size: int) -> int:
-    return int(lib().qzo_num_groups(N, K, group_size))
 
 
 def packed_shapes(N: int, K: int, bits: int, symmetric: bool, group_size: int):

@@ -163,12 +163,6 @@ static void quantize_group(const float *x, int64_t n, int bits, int symmetric,
 /*            two's complement for int8.                                  */
 /* ------------------------------------------------------------------ */
 
-int64_t qzo_num_groups(int64_t N, int64_t K, int64_t g)
-{
-    if (g == 0) return 1;
-    return N * (K / g);
-}
-
 static int check_shape(int64_t N, int64_t K, int bits, int64_t g)
 {
     if (N < 1 || K < 1) return -1;

@@ -10,6 +10,9 @@ One step is one pass of every hot-path row over the 7B-class decode layer set
   W4A16 decode GEMV, M = 1                  (3 launches)
   W8A16 decode GEMV, M = 1                  (3 launches)
   W4A16 prefill GEMM, M = 2048 tokens       (3 launches)
+plus the 70B-class decode layers (N, K) = (28672, 8192), (8192, 28672):
+  W4A16 decode GEMV, M = 1                  (2 launches)
+  W8A16 decode GEMV, M = 1                  (2 launches)
 Every input is resident in HBM and rotates over ROT copies (ROT x the packed
 layer set is far larger than the 126 MB L2), so each part reads cold weights.
 Each step is one captured CUDA graph (all parts, one rotation) with external
@@ -17,8 +20,8 @@ CUDA event nodes between the parts, so the GPU runs a step without host gaps
 and each part's time is the device time between its two event nodes.  `value` is the headline of the metric:
 W4A16 decode GEMV GB/s (algorithmic bytes / GEMV time), aggregated over all
 ranks.  The other parts, the roofline of every kernel, the configurations
-that are not part of the step (70B decode shapes, the 2048 x 8192 x 8192
-prefill GEMM, the 7.8e9-parameter bulk quantization), an end-to-end number
+that are not part of the step (70B decode shapes at M = 4, 8, 16, the
+2048 x 8192 x 8192 prefill GEMM, the 7.8e9-parameter bulk quantization), an end-to-end number
 through the public Python API with host buffers, and the CPU oracle baseline
 are reported in the same JSON line.
 
@@ -46,6 +49,7 @@ import synthetic  # noqa: E402
 
 METRIC = "W4A16 decode GEMV GB/s (% of HBM peak); prefill GEMM TFLOP/s; quantize GB/s"
 LAYERS = synthetic.DECODE_7B
+LAYERS_70B = synthetic.DECODE_70B
 PREFILL_M = synthetic.PREFILL["M"]
 ROT = 8
 GEMV_LAUNCH_OVERLAP = 1      # static weights: see qz_set_launch_overlap in qz.h
@@ -197,6 +201,23 @@ class LayerSet:
                    for li, (N, K) in enumerate(LAYERS)]
         self.ap = [synthetic.activations(PREFILL_M, K, seed=60 + li, device=dev)
                    for li, (N, K) in enumerate(LAYERS)]
+        # 70B-class decode layers (W4A16 and W8A16 at M = 1): packed weights
+        # only, ROT copies each (ROT x 246 MB int4, ROT x 470 MB int8)
+        self.c4_70, self.s4_70, self.z4_70, self.c8_70, self.s8_70 = ([] for _ in range(5))
+        for li, (N, K) in enumerate(LAYERS_70B):
+            w = synthetic.weights(N, K, sigma=0.015, seed=4 + li, device=dev)
+            c4, s4, z4 = qz.qz_quantize_pack(w, 4, False, GROUP)
+            c8, s8, _ = qz.qz_quantize_pack(w, 8, True, K)
+            del w
+            self.c4_70.append([c4] + [c4.clone() for _ in range(ROT - 1)])
+            self.s4_70.append([s4] + [s4.clone() for _ in range(ROT - 1)])
+            self.z4_70.append([z4] + [z4.clone() for _ in range(ROT - 1)])
+            self.c8_70.append([c8] + [c8.clone() for _ in range(ROT - 1)])
+            self.s8_70.append([s8] + [s8.clone() for _ in range(ROT - 1)])
+        self.a1_70 = [synthetic.activations(1, K, seed=70 + li, device=dev)
+                      for li, (N, K) in enumerate(LAYERS_70B)]
+        self.y4_70 = [torch.empty((1, N), dtype=torch.bfloat16, device=dev) for N, K in LAYERS_70B]
+        self.y8_70 = [torch.empty((1, N), dtype=torch.bfloat16, device=dev) for N, K in LAYERS_70B]
         self.y4 = [torch.empty((1, N), dtype=torch.bfloat16, device=dev) for N, K in LAYERS]
         self.y8 = [torch.empty((1, N), dtype=torch.bfloat16, device=dev) for N, K in LAYERS]
         self.yg = [torch.empty((PREFILL_M, N), dtype=torch.bfloat16, device=dev) for N, K in LAYERS]
@@ -205,6 +226,9 @@ class LayerSet:
             ws = max(ws, qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMV, 1, N, K, GROUP),
                      qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMV, 1, N, K, K),
                      qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMM, PREFILL_M, N, K, GROUP))
+        for N, K in LAYERS_70B:
+            ws = max(ws, qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMV, 1, N, K, GROUP),
+                     qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMV, 1, N, K, K))
         self.ws = torch.zeros(ws, dtype=torch.uint8, device=dev)
 
     # each part issues its launches for rotation p on the current stream
@@ -233,25 +257,42 @@ class LayerSet:
             self.qz.qz_w8a16_gemv(self.a1[li], self.c8[p][li], self.s8[p][li], N, K,
                                   y=self.y8[li], workspace=self.ws)
 
+    def gemv4_70b(self, p):
+        for li, (N, K) in enumerate(LAYERS_70B):
+            self.qz.qz_w4a16_gemv(self.a1_70[li], self.c4_70[li][p], self.s4_70[li][p],
+                                  self.z4_70[li][p], N, K, GROUP, y=self.y4_70[li],
+                                  workspace=self.ws)
+
+    def gemv8_70b(self, p):
+        for li, (N, K) in enumerate(LAYERS_70B):
+            self.qz.qz_w8a16_gemv(self.a1_70[li], self.c8_70[li][p], self.s8_70[li][p], N, K,
+                                  y=self.y8_70[li], workspace=self.ws)
+
     def gemm(self, p):
         for li, (N, K) in enumerate(LAYERS):
             self.qz.qz_w4a16_gemm(self.ap[li], self.c4[p][li], self.s4[p][li], self.z4[p][li], N,
                                   K, GROUP, y=self.yg[li], workspace=self.ws)
 
 
-PARTS = [  # name, method, unit, work per step, bound
+PARTS = [  # name, method, unit, work per step, bound, launches per step
     ("quantize_pack_int4_g128", "quant4", "GB/s",
-     sum(quant_int4_bytes(N, K) for N, K in LAYERS), "hbm"),
+     sum(quant_int4_bytes(N, K) for N, K in LAYERS), "hbm", len(LAYERS)),
     ("quantize_pack_int8_per_channel", "quant8", "GB/s",
-     sum(quant_int8_bytes(N, K) for N, K in LAYERS), "hbm"),
+     sum(quant_int8_bytes(N, K) for N, K in LAYERS), "hbm", len(LAYERS)),
     ("dequantize_int4", "dequant", "GB/s",
-     sum(dequant_int4_bytes(N, K) for N, K in LAYERS), "hbm"),
-    ("w4a16_gemv_m1", "gemv4", "GB/s", sum(w4_gemv_bytes(1, N, K) for N, K in LAYERS), "hbm"),
-    ("w8a16_gemv_m1", "gemv8", "GB/s", sum(w8_gemv_bytes(1, N, K) for N, K in LAYERS), "hbm"),
+     sum(dequant_int4_bytes(N, K) for N, K in LAYERS), "hbm", len(LAYERS)),
+    ("w4a16_gemv_m1", "gemv4", "GB/s", sum(w4_gemv_bytes(1, N, K) for N, K in LAYERS), "hbm",
+     len(LAYERS)),
+    ("w8a16_gemv_m1", "gemv8", "GB/s", sum(w8_gemv_bytes(1, N, K) for N, K in LAYERS), "hbm",
+     len(LAYERS)),
+    ("w4a16_gemv_70b_m1", "gemv4_70b", "GB/s",
+     sum(w4_gemv_bytes(1, N, K) for N, K in LAYERS_70B), "hbm", len(LAYERS_70B)),
+    ("w8a16_gemv_70b_m1", "gemv8_70b", "GB/s",
+     sum(w8_gemv_bytes(1, N, K) for N, K in LAYERS_70B), "hbm", len(LAYERS_70B)),
     ("w4a16_gemm_prefill_m2048", "gemm", "TFLOP/s",
-     sum(gemm_flops(PREFILL_M, N, K) for N, K in LAYERS), "tensor"),
+     sum(gemm_flops(PREFILL_M, N, K) for N, K in LAYERS), "tensor", len(LAYERS)),
 ]
-LAUNCHES_PER_STEP = 3 * len(PARTS)
+LAUNCHES_PER_STEP = sum(p[5] for p in PARTS)
 
 
 def max_over_ranks(values, dist=None, device="cpu"):
@@ -462,31 +503,70 @@ def run_extras(qz, dev, pk, stream):
     return out
 
 
-def cpu_baseline(target_s=10.0):
-    """The oracle, as it stands, on this host's cores: the decode step
-    (dequantize + fp64 matmul, M = 1) over the 7B-class layer set."""
+def cpu_model():
+    """The host CPU's model name (from /proc/cpuinfo), or the platform's."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or platform.machine()
+
+
+def _timed_passes(fn, target_s):
+    passes, t0 = 0, time.perf_counter()
+    while True:
+        fn()
+        passes += 1
+        el = time.perf_counter() - t0
+        if el >= target_s:
+            return passes, el
+
+
+def cpu_baseline(decode_s=6.0, quant_s=3.0):
+    """The oracle, as it stands, on this host's cores, with all threads and
+    with one: the decode step (dequantize + fp64 matmul, M = 1) over the
+    7B-class layer set, and quantize_pack int4 group-128 of the same layers.
+    Bounded: about 2 x (decode_s + quant_s) seconds of CPU work."""
     import oracle
     threads = oracle.max_threads()
-    oracle.set_threads(threads)
     prepared = []
     for li, (N, K) in enumerate(LAYERS):
         wb = synthetic.bf16_bits(synthetic.weights(N, K, sigma=0.02, seed=1 + li))
         ab = synthetic.bf16_bits(synthetic.activations(1, K, seed=50 + li))
-        prepared.append((N, K, oracle.quantize_pack(wb, 4, False, GROUP), ab))
-    nbytes = sum(w4_gemv_bytes(1, N, K) for N, K in LAYERS)
-    passes, t0 = 0, time.perf_counter()
-    while True:
-        for N, K, (c, s, z), ab in prepared:
-            w_hat = oracle.dequantize(c, s, z, N, K, 4, False, GROUP)
-            oracle.matmul_f64(ab, w_hat)
-        passes += 1
-        el = time.perf_counter() - t0
-        if el >= target_s:
-            break
-    return {"value": round(nbytes * passes / el / 1e9, 4), "unit": "GB/s", "cores": threads,
-            "kind": "oracle",
-            "sample": f"{passes} full decode passes (dequantize + fp64 matmul, M=1) over the three "
-                      f"7B-class layers, {el:.1f} s"}
+        prepared.append((N, K, wb, oracle.quantize_pack(wb, 4, False, GROUP), ab))
+    dec_bytes = sum(w4_gemv_bytes(1, N, K) for N, K in LAYERS)
+    q_bytes = sum(quant_int4_bytes(N, K) for N, K in LAYERS)
+
+    def decode():
+        for N, K, _, (c, s, z), ab in prepared:
+            oracle.matmul_f64(ab, oracle.dequantize(c, s, z, N, K, 4, False, GROUP))
+
+    def quantize():
+        for N, K, wb, _, _ in prepared:
+            oracle.quantize_pack(wb, 4, False, GROUP)
+
+    out = {}
+    for label, n in (("all", threads), ("1thread", 1)):
+        oracle.set_threads(n)
+        dp, de = _timed_passes(decode, decode_s)
+        qp, qe = _timed_passes(quantize, quant_s)
+        out[label] = (dec_bytes * dp / de / 1e9, dp, de, q_bytes * qp / qe / 1e9, qp, qe)
+    oracle.set_threads(threads)
+    d_all, dp, de, q_all, qp, qe = out["all"]
+    d_one, dp1, de1, q_one, qp1, qe1 = out["1thread"]
+    return {"value": round(d_all, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "cpu_model": cpu_model(),
+            "value_1thread": round(d_one, 4),
+            "quantize_pack_int4_g128_GB/s": round(q_all, 4),
+            "quantize_pack_int4_g128_GB/s_1thread": round(q_one, 4),
+            "sample": f"decode (dequantize + fp64 matmul, M=1) over the three 7B-class layers: "
+                      f"{dp} passes in {de:.1f} s on {threads} threads, {dp1} in {de1:.1f} s on "
+                      f"1; quantize_pack int4 g128 of the same layers: {qp} passes in "
+                      f"{qe:.1f} s on {threads} threads, {qp1} in {qe1:.1f} s on 1"}
 
 
 def run_reference(args):
@@ -524,7 +604,7 @@ def run_reference(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_obj(),
             "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": threads,
-                             "kind": "oracle",
+                             "kind": "oracle", "cpu_model": cpu_model(),
                              "sample": "rows 0..N/16 of each of the three 7B-class layers per step"},
             "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -534,10 +614,13 @@ def run_reference(args):
 def config_obj():
     return {"workload": "7B-class decode layer set (N,K)=(4096,4096),(11008,4096),(4096,11008): "
                         "int4 asym group-128 + int8 sym per-channel quantize_pack, int4 dequantize, "
-                        "W4A16/W8A16 decode GEMV at M=1, W4A16 prefill GEMM at M=2048",
+                        "W4A16/W8A16 decode GEMV at M=1, W4A16 prefill GEMM at M=2048; plus "
+                        "the 70B-class decode layers' W4A16/W8A16 GEMV at M=1",
             "weights": "bf16 ~N(0,0.02) + 0.1% x20 outliers, seeds 1..3",
             "activations": "bf16 ~N(0,1)",
             "l2": f"inputs rotate over {ROT} resident copies (packed W4 set {ROT} x 56 MB > L2)",
+            "decode_70b": "W4A16 and W8A16 GEMV at M=1 on (28672,8192),(8192,28672), weights "
+                          "bf16 ~N(0,0.015) + 0.1% x20, rotating over the same number of copies",
             "value_is": "w4a16_gemv_m1 part (algorithmic bytes / event-timed GEMV time)",
             "gemv_launch_overlap": (
                 f"qz_set_launch_overlap({GEMV_LAUNCH_OVERLAP}): each decode GEMV may start while "
@@ -726,10 +809,12 @@ def main():
 
     traffic = ncu_traffic()
     parts, roofs = {}, {}
-    for (name, meth, unit, work, bound), ms in zip(PARTS, part_ms):
+    # every kernel is timed inside a step of about a millisecond, far short
+    # of the seconds it takes to reach the power cap: burst peaks apply
+    for (name, meth, unit, work, bound, nl), ms in zip(PARTS, part_ms):
         parts[name] = {"ms": round(ms, 5), "value": round(rate(work, ms, unit), 2), "unit": unit,
-                       "launches": 3}
-        roofs[name] = roofline_obj(name, work, ms, 3, bound, pk, traffic, sustained=True)
+                       "launches": nl}
+        roofs[name] = roofline_obj(name, work, ms, nl, bound, pk, traffic, sustained=False)
     dominant = max(zip(PARTS, part_ms), key=lambda x: x[1])[0][0]
     gemv_idx = [p[0] for p in PARTS].index("w4a16_gemv_m1")
     gemv_bytes = PARTS[gemv_idx][3]

@@ -106,10 +106,23 @@ QZ_API qz_status qz_packed_bytes(int64_t N, int64_t K, int32_t bits, int32_t sym
  * Device workspace needed by `op` for the given sizes (0 when none).  The
  * workspace of QZ_OP_QUANTIZE_PACK (per-tensor only) and of the GEMV/GEMM
  * split-K paths must be zero-filled once before its first use; every call
- * leaves it zero-filled again when it completes.  Host-only.
+ * leaves it zero-filled again when it completes.  Host-only.  The kernels
+ * size their grids for the device's SM count (a B200 has 148; a device with
+ * more is treated as 148); the size returned here serves every SM count up
+ * to 148, so it does not depend on the device.
  */
 QZ_API qz_status qz_workspace_bytes(int32_t op, int64_t M, int64_t N, int64_t K,
                              int64_t group_size, size_t *bytes);
+
+/*
+ * The workspace a call uses when its grid is sized for `sms` SMs
+ * (1 <= sms <= 148; a device's own count, capped at 148, is what the
+ * kernels use).  qz_workspace_bytes returns the largest of these over every
+ * `sms`, so a buffer of that size serves any device.  Host-only; a planning
+ * query, not part of the method.
+ */
+QZ_API qz_status qz_workspace_bytes_for_sms(int32_t op, int64_t M, int64_t N, int64_t K,
+                                            int64_t group_size, int32_t sms, size_t *bytes);
 
 /*
  * quantize_pack: w (N x K bf16) -> codes, scales (bf16), zeros.
@@ -190,8 +203,11 @@ QZ_API qz_status qz_w8a16_gemv(const void *a, const void *codes, const void *sca
                         size_t workspace_bytes, void *stream);
 
 /*
- * W8A16 prefill GEMM: the same product as qz_w8a16_gemv for any M >= 1.
- * Weight tiles are dequantized (w_hat = bf16_rne(S * q), exactly as
+ * W8A16 prefill GEMM: the same product as qz_w8a16_gemv for any M >= 1
+ * (taqaniya.com "What is quantization", IBM absmax example, for the int8
+ * symmetric weight; Quantization concepts guide, "Quantize weights or
+ * activations": weight-only methods dequantize to the compute dtype before
+ * each matmul, and prefill is compute-bound).  Weight tiles are dequantized (w_hat = bf16_rne(S * q), exactly as
  * qz_dequantize forms it) into tensor memory as the A operand of tcgen05
  * BF16 MMAs with fp32 accumulation; y is rounded to bf16.  M <= 16 runs the
  * decode kernel of qz_w8a16_gemv.  Tiles and split-K as for qz_w4a16_gemm.
@@ -230,7 +246,8 @@ QZ_API qz_status qz_w8a16_gemm(const void *a, const void *codes, const void *sca
  *     launch.
  *   - The first call on a device looks up the array's device address on that
  *     device (with it current); make that first call before any stream
- *     capture.
+ *     capture.  A look-up that fails returns QZ_ERR_CUDA and is not
+ *     remembered: the next call on that device tries again.
  *   - Each call clears the part of the array that must start at zero (with
  *     cudaMemsetAsync on `stream`) and never calls cudaMalloc, cudaFree or
  *     any allocating routine.

@@ -184,3 +184,27 @@ def test_launch_overlap_setter():
     assert qz.lib.qz_set_launch_overlap(-1) == INVALID
     for mode in (1, 0):               # ends on the default
         assert qz.lib.qz_set_launch_overlap(mode) == OK
+
+
+WS_SHAPES = [  # (op, M, N, K, g): decode GEMV shapes, short and long layers, small-M GEMMs
+    (qz.QZ_OP_W4A16_GEMV, 1, 4096, 4096, 128), (qz.QZ_OP_W4A16_GEMV, 1, 28672, 8192, 128),
+    (qz.QZ_OP_W4A16_GEMV, 16, 8192, 28672, 128), (qz.QZ_OP_W4A16_GEMV, 4, 11008, 4096, 128),
+    (qz.QZ_OP_W4A16_GEMV, 3, 17, 128, 32), (qz.QZ_OP_W8A16_GEMV, 1, 28672, 8192, 8192),
+    (qz.QZ_OP_W8A16_GEMV, 8, 4096, 11008, 11008), (qz.QZ_OP_W4A16_GEMM, 48, 1024, 2048, 128),
+    (qz.QZ_OP_W4A16_GEMM, 32, 8192, 8192, 128), (qz.QZ_OP_W8A16_GEMM, 200, 512, 2048, 2048),
+    (qz.QZ_OP_W4A16_GEMM, 2048, 8192, 8192, 128), (qz.QZ_OP_W4A16_GEMM, 12, 4096, 4096, 128),
+]
+
+
+@pytest.mark.parametrize("op,M,N,K,g", WS_SHAPES)
+def test_workspace_bound_serves_every_sm_count(op, M, N, K, g):
+    """Grids are sized for the device's own SM count (at most 148), while
+    qz_workspace_bytes does not depend on the device: it must be at least the
+    workspace of the plan for every count, and equal to the largest."""
+    bound = qz.qz_workspace_bytes(op, M, N, K, g)
+    per_sms = [qz.qz_workspace_bytes_for_sms(op, M, N, K, g, sms) for sms in range(1, 149)]
+    assert max(per_sms) == bound
+    assert per_sms[-1] == qz.qz_workspace_bytes_for_sms(op, M, N, K, g, 148)
+    for bad in (0, 149):
+        with pytest.raises(qz.QzError):
+            qz.qz_workspace_bytes_for_sms(op, M, N, K, g, bad)

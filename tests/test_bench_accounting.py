@@ -63,12 +63,18 @@ def test_step_parts_cover_the_hot_path():
     names = [p[0] for p in bench.PARTS]
     assert names == ["quantize_pack_int4_g128", "quantize_pack_int8_per_channel",
                      "dequantize_int4", "w4a16_gemv_m1", "w8a16_gemv_m1",
-                     "w4a16_gemm_prefill_m2048"]
+                     "w4a16_gemv_70b_m1", "w8a16_gemv_70b_m1", "w4a16_gemm_prefill_m2048"]
     work = {p[0]: p[3] for p in bench.PARTS}
     assert work["w4a16_gemv_m1"] == sum(bench.w4_gemv_bytes(1, N, K) for N, K in synthetic.DECODE_7B)
+    assert work["w4a16_gemv_70b_m1"] == sum(
+        bench.w4_gemv_bytes(1, N, K) for N, K in synthetic.DECODE_70B)
+    assert abs(work["w4a16_gemv_70b_m1"] / MB - 246.0) <= 0.1
+    assert abs(work["w8a16_gemv_70b_m1"] / MB - 470.0) <= 0.1
     assert work["w4a16_gemm_prefill_m2048"] == sum(
         bench.gemm_flops(2048, N, K) for N, K in synthetic.DECODE_7B)
-    assert bench.LAUNCHES_PER_STEP == 3 * len(bench.PARTS)
+    launches = {p[0]: p[5] for p in bench.PARTS}
+    assert launches["w4a16_gemv_70b_m1"] == 2 and launches["w4a16_gemv_m1"] == 3
+    assert bench.LAUNCHES_PER_STEP == 3 * 6 + 2 * 2
 
 
 PK = {"hbm_gbs": 6500.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0,

@@ -3,9 +3,12 @@
 Argument marshalling only: every function below validates Python-side types,
 allocates outputs with PyTorch when the caller did not pass them, and calls
 the C entry point of the same name (declared in ``include/qz.h``) on the
-current CUDA stream.  All arithmetic runs in the library's CUDA kernels; there
-is no CPU or PyTorch fallback.  If ``libqz.so`` is missing the import fails.
+``stream`` argument, else the current CUDA stream; outputs and temporary
+workspaces are allocated on that same stream.  All arithmetic runs in the
+library's CUDA kernels; there is no CPU or PyTorch fallback.  If ``libqz.so``
+is missing the import fails.
 """
+import contextlib
 import ctypes
 import os
 
@@ -13,7 +16,8 @@ import torch
 
 __all__ = [
     "QzError", "lib", "qz_version", "qz_status_string", "qz_packed_bytes",
-    "qz_workspace_bytes", "qz_quantize_pack", "qz_dequantize", "qz_w4a16_gemv",
+    "qz_workspace_bytes", "qz_workspace_bytes_for_sms", "qz_quantize_pack", "qz_dequantize",
+    "qz_w4a16_gemv",
     "qz_w4a16_gemm", "qz_w8a16_gemv", "qz_w8a16_gemm", "qz_set_device_wait_limit",
     "qz_set_launch_overlap", "qz_device_status",
     "Workspace", "QZ_OP_QUANTIZE_PACK", "QZ_OP_DEQUANTIZE", "QZ_OP_W4A16_GEMV",
@@ -34,6 +38,8 @@ _SIGS = {
     "qz_packed_bytes": ([_i64, _i64, _i32, _i32, _i64, ctypes.POINTER(_sz),
                          ctypes.POINTER(_sz), ctypes.POINTER(_sz)], ctypes.c_int),
     "qz_workspace_bytes": ([_i32, _i64, _i64, _i64, _i64, ctypes.POINTER(_sz)], ctypes.c_int),
+    "qz_workspace_bytes_for_sms": ([_i32, _i64, _i64, _i64, _i64, _i32, ctypes.POINTER(_sz)],
+                                   ctypes.c_int),
     "qz_quantize_pack": ([_p, _i64, _i64, _i32, _i32, _i64, _p, _p, _p, _p, _sz, _p], ctypes.c_int),
     "qz_dequantize": ([_p, _p, _p, _i64, _i64, _i32, _i32, _i64, _p, _p], ctypes.c_int),
     "qz_w4a16_gemv": ([_p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p, _sz, _p], ctypes.c_int),
@@ -99,6 +105,14 @@ def qz_workspace_bytes(op, M, N, K, group_size=128) -> int:
     return v
 
 
+def qz_workspace_bytes_for_sms(op, M, N, K, group_size, sms) -> int:
+    """Workspace bytes of a call whose grid is sized for `sms` SMs."""
+    b = _sz()
+    _check(lib.qz_workspace_bytes_for_sms(int(op), int(M), int(N), int(K), int(group_size),
+                                          int(sms), ctypes.byref(b)), "qz_workspace_bytes_for_sms")
+    return b.value
+
+
 def _ptr(t):
     if t is None:
         return None
@@ -109,9 +123,18 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream, device):
-    if stream is None:
-        stream = torch.cuda.current_stream(device)
+def _launch_stream(stream, device):
+    """The torch stream a call runs on: `stream`, else the current stream."""
+    return torch.cuda.current_stream(device) if stream is None else stream
+
+
+def _on(stream):
+    """Context that makes an explicitly passed stream current for the call's
+    allocations (nothing to do when the call runs on the current stream)."""
+    return contextlib.nullcontext() if stream is None else torch.cuda.stream(stream)
+
+
+def _handle(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
@@ -136,6 +159,11 @@ class Workspace:
 
 
 def _ws_args(workspace, nbytes, device):
+    """Pointer and size of the call's workspace.  Called inside
+    ``torch.cuda.stream(launch stream)``: a temporary workspace is then
+    allocated and zero-filled on the stream the kernel runs on, so the fill
+    is ordered before the kernel and the caching allocator hands the memory
+    out again only to work queued after it on that stream."""
     if nbytes == 0:
         return None, 0
     if workspace is None:
@@ -151,21 +179,25 @@ def qz_quantize_pack(w, bits=4, symmetric=False, group_size=128, codes=None, sca
     if w.dtype != torch.bfloat16 or w.dim() != 2:
         raise ValueError("w must be a 2-D bf16 tensor")
     N, K = w.shape
-    cb, sb, zb = qz_packed_bytes(N, K, bits, symmetric, group_size)
+    qz_packed_bytes(N, K, bits, symmetric, group_size)      # validates the format
     dev = w.device
-    if codes is None:
-        codes = torch.empty((N, K // 2) if bits == 4 else (N, K), dtype=torch.uint8, device=dev)
-    if scales is None:
-        shape = (1,) if group_size == 0 else (N, K // group_size)
-        scales = torch.empty(shape, dtype=torch.bfloat16, device=dev)
-    if zeros is None and not symmetric:
-        shape = (1,) if group_size == 0 else (N, K // group_size)
-        zeros = torch.empty(shape, dtype=torch.uint8, device=dev)
-    ws_ptr, ws_bytes = _ws_args(workspace, qz_workspace_bytes(QZ_OP_QUANTIZE_PACK, 1, N, K,
-                                                              group_size), dev)
-    _check(lib.qz_quantize_pack(_ptr(w), N, K, bits, int(symmetric), group_size, _ptr(codes),
-                                _ptr(scales), _ptr(zeros) if not symmetric else None, ws_ptr,
-                                ws_bytes, _stream(stream, dev)), "qz_quantize_pack")
+    st = _launch_stream(stream, dev)
+    with _on(stream):
+        if codes is None:
+            codes = torch.empty((N, K // 2) if bits == 4 else (N, K), dtype=torch.uint8,
+                                device=dev)
+        if scales is None:
+            shape = (1,) if group_size == 0 else (N, K // group_size)
+            scales = torch.empty(shape, dtype=torch.bfloat16, device=dev)
+        if zeros is None and not symmetric:
+            shape = (1,) if group_size == 0 else (N, K // group_size)
+            zeros = torch.empty(shape, dtype=torch.uint8, device=dev)
+        ws_ptr, ws_bytes = _ws_args(workspace, qz_workspace_bytes(QZ_OP_QUANTIZE_PACK, 1, N, K,
+                                                                  group_size), dev)
+        _check(lib.qz_quantize_pack(_ptr(w), N, K, bits, int(symmetric), group_size,
+                                    _ptr(codes), _ptr(scales),
+                                    _ptr(zeros) if not symmetric else None, ws_ptr, ws_bytes,
+                                    _handle(st)), "qz_quantize_pack")
     return codes, scales, (None if symmetric else zeros)
 
 
@@ -173,11 +205,13 @@ def qz_dequantize(codes, scales, zeros, N, K, bits=4, symmetric=False, group_siz
                   out=None, stream=None):
     """w_hat = bf16(S * (q - Z)) as an N x K bf16 tensor."""
     dev = codes.device
-    if out is None:
-        out = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
-    _check(lib.qz_dequantize(_ptr(codes), _ptr(scales), _ptr(zeros), N, K, bits,
-                             int(symmetric), group_size, _ptr(out), _stream(stream, dev)),
-           "qz_dequantize")
+    st = _launch_stream(stream, dev)
+    with _on(stream):
+        if out is None:
+            out = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+        _check(lib.qz_dequantize(_ptr(codes), _ptr(scales), _ptr(zeros), N, K, bits,
+                                 int(symmetric), group_size, _ptr(out), _handle(st)),
+               "qz_dequantize")
     return out
 
 
@@ -192,48 +226,56 @@ def _matmul_out(a, N, y):
 def qz_w4a16_gemv(a, codes, scales, zeros, N, K, group_size=128, y=None, workspace=None,
                   stream=None):
     """y = a * w_hat^T for int4 asymmetric group-wise weights, M <= 16."""
-    y = _matmul_out(a, N, y)
+    st = _launch_stream(stream, a.device)
     M = a.shape[0]
-    ws_ptr, ws_bytes = _ws_args(workspace, qz_workspace_bytes(QZ_OP_W4A16_GEMV, M, N, K,
-                                                              group_size), a.device)
-    _check(lib.qz_w4a16_gemv(_ptr(a), _ptr(codes), _ptr(scales), _ptr(zeros), M, N, K,
-                             group_size, _ptr(y), ws_ptr, ws_bytes, _stream(stream, a.device)),
-           "qz_w4a16_gemv")
+    with _on(stream):
+        y = _matmul_out(a, N, y)
+        nbytes = qz_workspace_bytes(QZ_OP_W4A16_GEMV, M, N, K, group_size)
+        ws_ptr, ws_bytes = _ws_args(workspace, nbytes, a.device)
+        _check(lib.qz_w4a16_gemv(_ptr(a), _ptr(codes), _ptr(scales), _ptr(zeros), M, N, K,
+                                 group_size, _ptr(y), ws_ptr, ws_bytes, _handle(st)),
+               "qz_w4a16_gemv")
     return y
 
 
 def qz_w4a16_gemm(a, codes, scales, zeros, N, K, group_size=128, y=None, workspace=None,
                   stream=None):
     """y = a * w_hat^T for int4 asymmetric group-wise weights, any M."""
-    y = _matmul_out(a, N, y)
+    st = _launch_stream(stream, a.device)
     M = a.shape[0]
-    ws_ptr, ws_bytes = _ws_args(workspace, qz_workspace_bytes(QZ_OP_W4A16_GEMM, M, N, K,
-                                                              group_size), a.device)
-    _check(lib.qz_w4a16_gemm(_ptr(a), _ptr(codes), _ptr(scales), _ptr(zeros), M, N, K,
-                             group_size, _ptr(y), ws_ptr, ws_bytes, _stream(stream, a.device)),
-           "qz_w4a16_gemm")
+    with _on(stream):
+        y = _matmul_out(a, N, y)
+        nbytes = qz_workspace_bytes(QZ_OP_W4A16_GEMM, M, N, K, group_size)
+        ws_ptr, ws_bytes = _ws_args(workspace, nbytes, a.device)
+        _check(lib.qz_w4a16_gemm(_ptr(a), _ptr(codes), _ptr(scales), _ptr(zeros), M, N, K,
+                                 group_size, _ptr(y), ws_ptr, ws_bytes, _handle(st)),
+               "qz_w4a16_gemm")
     return y
 
 
 def qz_w8a16_gemv(a, codes, scales, N, K, y=None, workspace=None, stream=None):
     """y = a * w_hat^T for int8 symmetric per-channel weights, M <= 16."""
-    y = _matmul_out(a, N, y)
+    st = _launch_stream(stream, a.device)
     M = a.shape[0]
-    ws_ptr, ws_bytes = _ws_args(workspace, qz_workspace_bytes(QZ_OP_W8A16_GEMV, M, N, K, K),
-                                a.device)
-    _check(lib.qz_w8a16_gemv(_ptr(a), _ptr(codes), _ptr(scales), M, N, K, _ptr(y), ws_ptr,
-                             ws_bytes, _stream(stream, a.device)), "qz_w8a16_gemv")
+    with _on(stream):
+        y = _matmul_out(a, N, y)
+        nbytes = qz_workspace_bytes(QZ_OP_W8A16_GEMV, M, N, K, K)
+        ws_ptr, ws_bytes = _ws_args(workspace, nbytes, a.device)
+        _check(lib.qz_w8a16_gemv(_ptr(a), _ptr(codes), _ptr(scales), M, N, K, _ptr(y),
+                                 ws_ptr, ws_bytes, _handle(st)), "qz_w8a16_gemv")
     return y
 
 
 def qz_w8a16_gemm(a, codes, scales, N, K, y=None, workspace=None, stream=None):
     """y = a * w_hat^T for int8 symmetric per-channel weights, any M."""
-    y = _matmul_out(a, N, y)
+    st = _launch_stream(stream, a.device)
     M = a.shape[0]
-    ws_ptr, ws_bytes = _ws_args(workspace, qz_workspace_bytes(QZ_OP_W8A16_GEMM, M, N, K, K),
-                                a.device)
-    _check(lib.qz_w8a16_gemm(_ptr(a), _ptr(codes), _ptr(scales), M, N, K, _ptr(y), ws_ptr,
-                             ws_bytes, _stream(stream, a.device)), "qz_w8a16_gemm")
+    with _on(stream):
+        y = _matmul_out(a, N, y)
+        nbytes = qz_workspace_bytes(QZ_OP_W8A16_GEMM, M, N, K, K)
+        ws_ptr, ws_bytes = _ws_args(workspace, nbytes, a.device)
+        _check(lib.qz_w8a16_gemm(_ptr(a), _ptr(codes), _ptr(scales), M, N, K, _ptr(y),
+                                 ws_ptr, ws_bytes, _handle(st)), "qz_w8a16_gemm")
     return y
 
 

@@ -20,6 +20,23 @@ uint64_t device_wait_limit() {
     return v ? v : kDefaultWaitLimit;
 }
 
+int device_sm_count() {
+    static DeviceOnce once;
+    static int count[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return kSmCount;
+    }
+    const cudaError_t e = once.run(dev, [dev] {
+        int n = 0;
+        const cudaError_t r = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (r == cudaSuccess) count[dev] = n < 1 ? 1 : (n > kSmCount ? kSmCount : n);
+        return r;
+    });
+    return e == cudaSuccess ? count[dev] : kSmCount;
+}
+
 namespace {
 
 constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
@@ -111,18 +128,41 @@ QZ_API qz_status qz_workspace_bytes(int32_t op, int64_t M, int64_t N, int64_t K,
     case QZ_OP_W8A16_GEMV: {
         const qz_status s = check_gemv_shape(M, N, K);
         if (s != QZ_OK) return s;
-        *bytes = gemv_plan(M, N, K, op == QZ_OP_W4A16_GEMV ? 4 : 8).total_bytes;
+        *bytes = gemv_workspace_bound(M, N, K, op == QZ_OP_W4A16_GEMV ? 4 : 8);
         return QZ_OK;
     }
     case QZ_OP_W4A16_GEMM:
     case QZ_OP_W8A16_GEMM:
         if (M < 1 || N < 1 || K < 1) return QZ_ERR_INVALID_ARG;
         *bytes = M <= 16 && K % 128 == 0
-                     ? gemv_plan(M, N, K, op == QZ_OP_W4A16_GEMM ? 4 : 8).total_bytes
+                     ? gemv_workspace_bound(M, N, K, op == QZ_OP_W4A16_GEMM ? 4 : 8)
                      : gemm_workspace_bytes(M, N, K);
         return QZ_OK;
     default:
         return QZ_ERR_INVALID_ARG;
+    }
+}
+
+QZ_API qz_status qz_workspace_bytes_for_sms(int32_t op, int64_t M, int64_t N, int64_t K,
+                                            int64_t group_size, int32_t sms, size_t *bytes) {
+    if (!bytes || sms < 1 || sms > kSmCount) return QZ_ERR_INVALID_ARG;
+    switch (op) {
+    case QZ_OP_W4A16_GEMV:
+    case QZ_OP_W8A16_GEMV: {
+        const qz_status s = check_gemv_shape(M, N, K);
+        if (s != QZ_OK) return s;
+        *bytes = gemv_plan(M, N, K, op == QZ_OP_W4A16_GEMV ? 4 : 8, sms).total_bytes;
+        return QZ_OK;
+    }
+    case QZ_OP_W4A16_GEMM:
+    case QZ_OP_W8A16_GEMM:
+        if (M < 1 || N < 1 || K < 1) return QZ_ERR_INVALID_ARG;
+        *bytes = M <= 16 && K % 128 == 0
+                     ? gemv_plan(M, N, K, op == QZ_OP_W4A16_GEMM ? 4 : 8, sms).total_bytes
+                     : gemm_workspace_bytes_for(M, N, K, sms);
+        return QZ_OK;
+    default:
+        return qz_workspace_bytes(op, M, N, K, group_size, bytes);
     }
 }
 
@@ -164,7 +204,7 @@ QZ_API qz_status qz_w4a16_gemv(const void *a, const void *codes, const void *sca
     if (!a || !codes || !scales || !zeros || !y) return QZ_ERR_INVALID_ARG;
     if (!aligned(a, 16) || !aligned(codes, 16) || !aligned(scales, 2) || !aligned(y, 2))
         return QZ_ERR_ALIGNMENT;
-    const GemvPlan plan = gemv_plan(M, N, K, 4);
+    const GemvPlan plan = gemv_plan(M, N, K, 4, device_sm_count());
     s = check_workspace(plan.total_bytes, workspace, workspace_bytes);
     if (s != QZ_OK) return s;
     return launch_w4a16_gemv(a, codes, scales, zeros, M, N, K, group_size, y, workspace, plan,
@@ -179,7 +219,7 @@ QZ_API qz_status qz_w8a16_gemv(const void *a, const void *codes, const void *sca
     if (!a || !codes || !scales || !y) return QZ_ERR_INVALID_ARG;
     if (!aligned(a, 16) || !aligned(codes, 16) || !aligned(scales, 2) || !aligned(y, 2))
         return QZ_ERR_ALIGNMENT;
-    const GemvPlan plan = gemv_plan(M, N, K, 8);
+    const GemvPlan plan = gemv_plan(M, N, K, 8, device_sm_count());
     s = check_workspace(plan.total_bytes, workspace, workspace_bytes);
     if (s != QZ_OK) return s;
     return launch_w8a16_gemv(a, codes, scales, M, N, K, y, workspace, plan, launch_overlap(),

@@ -665,9 +665,11 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
 // Tokens per activation box: a whole tile, or all of M rounded up to 16.
 int gemm_act_rows(int64_t M) { return M >= kTileM ? kTileM : (int)((M + 15) & ~int64_t(15)); }
 
-int gemm_splits(int64_t M, int64_t N, int64_t K) {
+// `sms`: the SMs the grid is sized for (fewer SMs give fewer or equal splits,
+// so a workspace sized for kSmCount serves every device).
+int gemm_splits(int64_t M, int64_t N, int64_t K, int sms) {
     const int64_t tiles = ceil_div(N, kTileN) * ceil_div(M, kTileM);
-    const int64_t slots = (int64_t)kSmCount * gemm_ctas_per_sm(gemm_act_rows(M));
+    const int64_t slots = (int64_t)sms * gemm_ctas_per_sm(gemm_act_rows(M));
     if (tiles >= slots) return 1;
     int64_t s = slots / tiles;
     if (s > kMaxSplits) s = kMaxSplits;
@@ -676,29 +678,35 @@ int gemm_splits(int64_t M, int64_t N, int64_t K) {
 }
 
 // fp32 partials [splits][M][N], then one uint32 arrival counter per tile
-size_t gemm_partial_bytes(int64_t M, int64_t N, int64_t K) {
-    const int s = gemm_splits(M, N, K);
+size_t gemm_partial_bytes(int64_t M, int64_t N, int64_t K, int sms) {
+    const int s = gemm_splits(M, N, K, sms);
     if (s == 1) return 0;
     return (((size_t)s * M * N * sizeof(float)) + 255) & ~(size_t)255;
 }
 
-size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-    if (gemm_splits(M, N, K) == 1) return 0;
+size_t gemm_workspace_bytes_for(int64_t M, int64_t N, int64_t K, int sms) {
+    if (gemm_splits(M, N, K, sms) == 1) return 0;
     const int64_t tiles = ceil_div(N, kTileN) * ceil_div(M, kTileM);
-    return gemm_partial_bytes(M, N, K) + (size_t)ceil_div(tiles, 64) * 64 * sizeof(uint32_t);
+    return gemm_partial_bytes(M, N, K, sms) +
+           (size_t)ceil_div(tiles, 64) * 64 * sizeof(uint32_t);
+}
+
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    return gemm_workspace_bytes_for(M, N, K, kSmCount);
 }
 
 unsigned int *device_error_word() {
-    static unsigned int *addr[64] = {};
-    static std::once_flag once[64];
+    static void *addr[kMaxDevices] = {};
+    static DeviceOnce once;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    std::call_once(once[dev], [dev] {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_device_error_word) == cudaSuccess)
-            addr[dev] = static_cast<unsigned int *>(p);
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    const cudaError_t e = once.run(dev, [dev] {
+        return cudaGetSymbolAddress(&addr[dev], g_device_error_word);
     });
-    return addr[dev];
+    return e == cudaSuccess ? static_cast<unsigned int *>(addr[dev]) : nullptr;
 }
 
 namespace {
@@ -710,13 +718,14 @@ qz_status launch_gemm(const void *a, const void *codes, const void *scales, cons
     constexpr int kRowBytesPerK = BITS;   // code bytes of a row per 8 k
     const int act_rows = gemm_act_rows(M);
     const int ctas = gemm_ctas_per_sm(act_rows);
-    const int splits = gemm_splits(M, N, K);
+    const int sms = device_sm_count();
+    const int splits = gemm_splits(M, N, K, sms);
     float *partials = nullptr;
     uint32_t *counters = nullptr;
     if (splits > 1) {
         partials = static_cast<float *>(workspace);
         counters = reinterpret_cast<uint32_t *>(static_cast<char *>(workspace) +
-                                                gemm_partial_bytes(M, N, K));
+                                                gemm_partial_bytes(M, N, K, sms));
     }
     CUtensorMap act_map, pack_map, y_map;
     if (!make_map_2d(&act_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a, (uint64_t)K, (uint64_t)M,
@@ -736,24 +745,32 @@ qz_status launch_gemm(const void *a, const void *codes, const void *scales, cons
         y_map = act_map;   // unused
     }
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return QZ_ERR_CUDA;
-    static std::once_flag attr_once[64];
-    if (dev >= 0 && dev < 64)
-        std::call_once(attr_once[dev], [] {
-            cudaFuncSetAttribute(wa16_gemm_tcgen05<BITS, kFullTileStages, 1>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
-            cudaFuncSetAttribute(wa16_gemm_tcgen05<BITS, 0, 1>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
-            cudaFuncSetAttribute(wa16_gemm_tcgen05<BITS, 0, 2>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
-            // two CTAs per SM need the whole unified memory as shared memory
-            cudaFuncSetAttribute(wa16_gemm_tcgen05<BITS, 0, 2>,
-                                 cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-        });
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return QZ_ERR_CUDA;
+    }
+    static DeviceOnce attr_once;
+    const cudaError_t attr_err = attr_once.run(dev, [] {
+        cudaError_t e = cudaFuncSetAttribute(wa16_gemm_tcgen05<BITS, kFullTileStages, 1>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kSmemLimit);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(wa16_gemm_tcgen05<BITS, 0, 1>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(wa16_gemm_tcgen05<BITS, 0, 2>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+        // two CTAs per SM need the whole unified memory as shared memory
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(wa16_gemm_tcgen05<BITS, 0, 2>,
+                                     cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        return e;
+    });
+    if (attr_err != cudaSuccess) return QZ_ERR_CUDA;
     const int stages = gemm_stages(BITS, act_rows, ctas);
     const uint32_t smem_bytes = gemm_layout(BITS, act_rows, stages).end + 1024;
     const int64_t items = ceil_div(N, kTileN) * ceil_div(M, kTileM) * splits;
-    const int grid = (int)std::min<int64_t>(items, (int64_t)kSmCount * ctas);
+    const int grid = (int)std::min<int64_t>(items, (int64_t)sms * ctas);
     auto kernel = act_rows == kTileM && splits == 1 ? wa16_gemm_tcgen05<BITS, kFullTileStages, 1>
                   : ctas == 2                      ? wa16_gemm_tcgen05<BITS, 0, 2>
                                                    : wa16_gemm_tcgen05<BITS, 0, 1>;

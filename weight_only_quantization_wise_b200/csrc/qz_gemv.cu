@@ -509,21 +509,20 @@ int log2_exact(int64_t v) {
     return s;
 }
 
-template <typename Kernel>
-void set_smem_once(Kernel kernel, int bytes, bool (&done)[64]) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !done[dev]) {
-        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-        done[dev] = true;
-    }
-}
-
 template <int BITS, int MB, bool RING_SZ>
-void launch_variant(const GemvArgs &args, dim3 grid, int overlap, cudaStream_t st) {
-    static bool done[64] = {};
+qz_status launch_variant(const GemvArgs &args, dim3 grid, int overlap, cudaStream_t st) {
     constexpr int smem = kGemvSmemBytes<BITS>;
-    set_smem_once(gemv_kernel<BITS, MB, RING_SZ>, smem, done);
+    static DeviceOnce attr_once;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return QZ_ERR_CUDA;
+    }
+    if (attr_once.run(dev, [] {
+            return cudaFuncSetAttribute(gemv_kernel<BITS, MB, RING_SZ>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        }) != cudaSuccess)
+        return QZ_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = dim3(kThreads);
@@ -535,6 +534,7 @@ void launch_variant(const GemvArgs &args, dim3 grid, int overlap, cudaStream_t s
     cfg.attrs = attr;
     cfg.numAttrs = overlap > 0 ? 1 : 0;
     cudaLaunchKernelEx(&cfg, gemv_kernel<BITS, MB, RING_SZ>, args);
+    return launch_status();
 }
 
 template <int BITS>
@@ -571,18 +571,15 @@ qz_status launch_gemv(const void *a, const void *codes, const void *scales, cons
         const int64_t entries = N * (K / group_size);
         const bool ring_sz = args.bpg_shift >= 0 && aligned(scales, 4) && aligned(zeros, 4) &&
                              entries % 4 == 0;
-        if (M <= 8) {
-            if (ring_sz) launch_variant<4, 1, true>(args, grid, overlap, st);
-            else launch_variant<4, 1, false>(args, grid, overlap, st);
-        } else {
-            if (ring_sz) launch_variant<4, 2, true>(args, grid, overlap, st);
-            else launch_variant<4, 2, false>(args, grid, overlap, st);
-        }
+        if (M <= 8)
+            return ring_sz ? launch_variant<4, 1, true>(args, grid, overlap, st)
+                           : launch_variant<4, 1, false>(args, grid, overlap, st);
+        return ring_sz ? launch_variant<4, 2, true>(args, grid, overlap, st)
+                       : launch_variant<4, 2, false>(args, grid, overlap, st);
     } else {
-        if (M <= 8) launch_variant<8, 1, false>(args, grid, overlap, st);
-        else launch_variant<8, 2, false>(args, grid, overlap, st);
+        return M <= 8 ? launch_variant<8, 1, false>(args, grid, overlap, st)
+                      : launch_variant<8, 2, false>(args, grid, overlap, st);
     }
-    return launch_status();
 }
 
 }  // namespace
@@ -599,7 +596,7 @@ qz_status launch_gemv(const void *a, const void *codes, const void *scales, cons
 constexpr int kBlockCostBase = 40, kBlockCostPerCta = 33;
 constexpr int kGemvMinBlocksPerWarp = 4;
 
-GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K, int bits) {
+GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K, int bits, int sms) {
     GemvPlan p{};
     p.tasks = ceil_div(N, kRowsPerWarp);
     p.kblocks = K / 128;
@@ -610,7 +607,7 @@ GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K, int bits) {
     if (M == 1) {
         int64_t best_cost = -1;
         for (int64_t k = 1; k <= max_per_sm; ++k) {
-            const int64_t cost = ceil_div(units, (int64_t)kSmCount * kWarpsPerCta * k) *
+            const int64_t cost = ceil_div(units, (int64_t)sms * kWarpsPerCta * k) *
                                  (kBlockCostBase + kBlockCostPerCta * k);
             if (best_cost < 0 || cost < best_cost) {
                 best_cost = cost;
@@ -618,11 +615,11 @@ GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K, int bits) {
             }
         }
     } else {
-        per_sm = units / ((int64_t)kSmCount * kWarpsPerCta * kGemvMinBlocksPerWarp);
+        per_sm = units / ((int64_t)sms * kWarpsPerCta * kGemvMinBlocksPerWarp);
         if (per_sm > max_per_sm) per_sm = max_per_sm;
         if (per_sm < 1) per_sm = 1;
     }
-    p.warps = (int64_t)kSmCount * per_sm * kWarpsPerCta;
+    p.warps = (int64_t)sms * per_sm * kWarpsPerCta;
     // Fewer units than warps: one unit per warp.  Every warp must own at
     // least one unit, or a split task would count a contributor that never
     // arrives.
@@ -636,6 +633,18 @@ GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K, int bits) {
     p.counter_bytes = (size_t)ceil_div(p.tasks, 64) * 64 * sizeof(uint32_t);
     p.total_bytes = p.partial_bytes + p.counter_bytes;
     return p;
+}
+
+// The plan's workspace is not monotone in the SM count (fewer SMs can pick
+// more CTAs per SM), so the size callers allocate is the largest over every
+// count up to kSmCount.
+size_t gemv_workspace_bound(int64_t M, int64_t N, int64_t K, int bits) {
+    size_t most = 0;
+    for (int sms = 1; sms <= kSmCount; ++sms) {
+        const size_t b = gemv_plan(M, N, K, bits, sms).total_bytes;
+        if (b > most) most = b;
+    }
+    return most;
 }
 
 qz_status launch_w4a16_gemv(const void *a, const void *codes, const void *scales,

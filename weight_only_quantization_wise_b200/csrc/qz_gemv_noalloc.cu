@@ -17,37 +17,33 @@
 // GPU race on it and must not be issued concurrently.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "qz_internal.cuh"
 
 namespace qz {
 namespace {
 
 constexpr size_t kScratchBytes = QZ_GEMV_NOALLOC_SCRATCH_BYTES;
-constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_gemv_scratch[kScratchBytes];
 
-struct ScratchSlot {
-    std::once_flag once;
-    void *ptr = nullptr;
-    cudaError_t err = cudaSuccess;
-};
-ScratchSlot g_slots[kMaxDevices];
+DeviceOnce g_scratch_once;
+void *g_scratch_ptr[kMaxDevices];
 
-// Device address of the scratch array on the current device (looked up on
-// the first call for that device).
+// Device address of the scratch array on the current device, looked up with
+// that device current on the first call that succeeds for it (a failed
+// look-up is retried by the next call).
 qz_status scratch_address(void **out) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return QZ_ERR_CUDA;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return QZ_ERR_CUDA;
+    }
     if (dev < 0 || dev >= kMaxDevices) return QZ_ERR_UNSUPPORTED;
-    ScratchSlot &s = g_slots[dev];
-    std::call_once(s.once, [&s] {
-        s.err = cudaGetSymbolAddress(&s.ptr, g_gemv_scratch);
+    const cudaError_t e = g_scratch_once.run(dev, [dev] {
+        return cudaGetSymbolAddress(&g_scratch_ptr[dev], g_gemv_scratch);
     });
-    if (s.err != cudaSuccess || s.ptr == nullptr) return QZ_ERR_CUDA;
-    *out = s.ptr;
+    if (e != cudaSuccess || g_scratch_ptr[dev] == nullptr) return QZ_ERR_CUDA;
+    *out = g_scratch_ptr[dev];
     return QZ_OK;
 }
 
@@ -70,7 +66,7 @@ extern "C" QZ_API qz_status qz_w4a16_gemv_noalloc(const void *a, const void *cod
     if (!qz::is_aligned(a, 16) || !qz::is_aligned(codes, 16) || !qz::is_aligned(scales, 2) ||
         !qz::is_aligned(y, 2))
         return QZ_ERR_ALIGNMENT;
-    const qz::GemvPlan plan = qz::gemv_plan(M, N, K, 4);
+    const qz::GemvPlan plan = qz::gemv_plan(M, N, K, 4, qz::device_sm_count());
     if (plan.total_bytes > qz::kScratchBytes) return QZ_ERR_WORKSPACE;   // beyond the built-in maximum
     void *scratch = nullptr;
     if (plan.total_bytes > 0) {

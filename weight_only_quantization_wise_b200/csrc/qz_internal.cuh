@@ -5,6 +5,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "qz.h"
 
 namespace qz {
@@ -13,10 +16,41 @@ namespace qz {
 // Host side
 // ---------------------------------------------------------------------------
 
-// Number of SMs of the device the grids are sized for.  Sizing (and therefore
-// workspace sizes) uses this fixed B200 figure so that qz_workspace_bytes is
-// a pure function of the shapes.
+// SMs of a B200.  Workspace sizes (qz_workspace_bytes, a pure function of
+// the shapes) are computed for this count; grids are sized for the device's
+// own count capped at it (device_sm_count), and every split-K plan made for
+// fewer SMs needs no more workspace than the plan for kSmCount.
 constexpr int kSmCount = 148;
+constexpr int kMaxDevices = 64;
+
+// A set-up step that must succeed once per device (a symbol address, a
+// kernel attribute).  run() calls `setup` (which returns a cudaError_t) until
+// it has succeeded once for the device; a failure is not remembered, so the
+// next call retries (and the failed call's CUDA error is cleared, so it does
+// not surface in a later launch check).  Thread-safe.
+class DeviceOnce {
+  public:
+    template <typename F>
+    cudaError_t run(int dev, F &&setup) {
+        if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+        if (done_[dev].load(std::memory_order_acquire)) return cudaSuccess;
+        std::lock_guard<std::mutex> lock(mu_);
+        if (done_[dev].load(std::memory_order_relaxed)) return cudaSuccess;
+        const cudaError_t e = setup();
+        if (e == cudaSuccess) done_[dev].store(true, std::memory_order_release);
+        else cudaGetLastError();
+        return e;
+    }
+
+  private:
+    std::mutex mu_;
+    std::atomic<bool> done_[kMaxDevices] = {};
+};
+
+// SMs the grids of the current device are sized for: its multiprocessor
+// count, capped at kSmCount (read once per device; kSmCount if the query
+// fails).
+int device_sm_count();
 
 inline bool aligned(const void *p, size_t a) {
     return (reinterpret_cast<uintptr_t>(p) % a) == 0;
@@ -70,7 +104,10 @@ struct GemvPlan {
     size_t total_bytes;
 };
 // Workspace: fp32 partials at offset 0, then one uint32 counter per task.
-GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K, int bits);
+// `sms`: the SMs the grid is sized for (device_sm_count() at launch).
+GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K, int bits, int sms);
+// Workspace bytes that serve the plan of every SM count up to kSmCount.
+size_t gemv_workspace_bound(int64_t M, int64_t N, int64_t K, int bits);
 
 // `overlap`: qz_set_launch_overlap mode for this launch.
 qz_status launch_w4a16_gemv(const void *a, const void *codes, const void *scales,
@@ -81,6 +118,9 @@ qz_status launch_w8a16_gemv(const void *a, const void *codes, const void *scales
                             int64_t M, int64_t N, int64_t K, void *y, void *workspace,
                             const GemvPlan &plan, int overlap, cudaStream_t stream);
 
+// Split-K workspace of the GEMM whose grid is sized for `sms` SMs; the
+// kSmCount figure (gemm_workspace_bytes) bounds every smaller count.
+size_t gemm_workspace_bytes_for(int64_t M, int64_t N, int64_t K, int sms);
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 qz_status launch_w4a16_gemm(const void *a, const void *codes, const void *scales,
                             const void *zeros, int64_t M, int64_t N, int64_t K,

@@ -465,7 +465,7 @@ __global__ void tensor_finish(uint32_t *__restrict__ ws, uint16_t *__restrict__ 
 
 int grid_for(int64_t work_items, int per_block) {
     int64_t b = ceil_div(work_items, per_block);
-    const int64_t cap = (int64_t)kSmCount * 16;
+    const int64_t cap = (int64_t)device_sm_count() * 16;
     if (b > cap) b = cap;
     if (b < 1) b = 1;
     return (int)b;
@@ -513,12 +513,12 @@ qz_status quantize_typed(const void *w, int64_t N, int64_t K, int64_t g, void *c
     if (cpg <= (int64_t)kRowChunksPerThread * 1024) {
         const int threads = (int)ceil_div(ceil_div(cpg, kRowChunksPerThread), 32) * 32;
         const int per_sm = std::max(1, 2048 / threads);
-        const int blocks = (int)std::min<int64_t>(groups, (int64_t)kSmCount * per_sm * 4);
+        const int blocks = (int)std::min<int64_t>(groups, (int64_t)device_sm_count() * per_sm * 4);
         quantize_groups_block<BITS, SYM><<<blocks, threads, 0, st>>>(src, (int)cpg, groups, c8,
                                                                       s16, z8);
         return launch_status();
     }
-    const int blocks = (int)std::min<int64_t>(groups, (int64_t)kSmCount * 32);
+    const int blocks = (int)std::min<int64_t>(groups, (int64_t)device_sm_count() * 32);
     quantize_large_groups<BITS, SYM><<<blocks, kQuantThreads, 0, st>>>(src, cpg, groups, c8,
                                                                         s16, z8);
     return launch_status();

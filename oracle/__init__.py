@@ -40,6 +40,14 @@ def load(path: str):
     L.qzo_dequantize.restype = _int
     L.qzo_matmul_f64.argtypes = [_p, _p, _i64, _i64, _i64, _p, _p]
     L.qzo_matmul_f64.restype = _int
+    L.qzo_gptq_hessian_factor.argtypes = [_p, _i64, _i64, ctypes.c_double, _p, _p]
+    L.qzo_gptq_hessian_factor.restype = _int
+    L.qzo_gptq_quantize_with_factor.argtypes = [_p, _p, _i64, _i64, _i64, _int, _int, _i64,
+                                                _p, _p, _p, _p]
+    L.qzo_gptq_quantize_with_factor.restype = _int
+    L.qzo_gptq_quantize.argtypes = [_p, _p, _i64, _i64, _i64, ctypes.c_double, _i64, _int,
+                                    _int, _i64, _p, _p, _p]
+    L.qzo_gptq_quantize.restype = _int
     L.qzo_set_threads.argtypes = [_int]
     L.qzo_set_threads.restype = None
     L.qzo_max_threads.argtypes = []
@@ -136,6 +144,74 @@ def dequantize(codes, scales, zeros, N: int, K: int, bits: int = 4,
     if rc != 0:
         raise ValueError("qzo_dequantize rejected the arguments")
     return out
+
+
+GPTQ_BLOCK = 128      # the GPTQ explainer's lazy-batch width
+GPTQ_DAMP = 0.01      # lambda = GPTQ_DAMP * mean(diag H) (a reading: the page gives no value)
+
+
+def _weights_f32(w):
+    w = np.asarray(w)
+    if w.dtype == np.uint16:
+        return bf16_bits_to_f32(w)
+    return np.ascontiguousarray(w, dtype=np.float32)
+
+
+def gptq_hessian_factor(x_bits, damp: float = GPTQ_DAMP):
+    """H = 2 X X^T + lambda I from calibration samples (``x_bits``: bf16 bits,
+    one sample per row, n x K) and U, the upper Cholesky factor of H^-1."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    n, K = x.shape
+    H = np.zeros((K, K), dtype=np.float64)
+    U = np.zeros((K, K), dtype=np.float64)
+    if lib().qzo_gptq_hessian_factor(_ptr(x), K, n, float(damp), _ptr(H), _ptr(U)) != 0:
+        raise ValueError("the damped Hessian is not positive definite")
+    return H, U
+
+
+def gptq_quantize_with_factor(w, U, bits: int = 4, symmetric: bool = False,
+                              group_size: int = 128, block: int = GPTQ_BLOCK):
+    """GPTQ's column loop over the weights ``w`` (bf16 bits or fp32 values)
+    with the factor ``U``; returns (codes, scales, zeros | None, compensated
+    weights fp64)."""
+    wf = _weights_f32(w)
+    N, K = wf.shape
+    Uc = np.ascontiguousarray(U, dtype=np.float64)
+    if Uc.shape != (K, K):
+        raise ValueError("U must be K x K")
+    cs, ss, zs = packed_shapes(N, K, bits, symmetric, group_size)
+    codes = np.zeros(cs, dtype=np.uint8)
+    scales = np.zeros(ss, dtype=np.uint16)
+    zeros = None if zs is None else np.zeros(zs, dtype=np.uint8)
+    w_out = np.zeros((N, K), dtype=np.float64)
+    rc = lib().qzo_gptq_quantize_with_factor(_ptr(wf), _ptr(Uc), N, K, block, bits,
+                                             int(symmetric), group_size, _ptr(codes),
+                                             _ptr(scales), _ptr(zeros), _ptr(w_out))
+    if rc != 0:
+        raise ValueError("qzo_gptq_quantize_with_factor rejected the arguments")
+    return codes, scales, zeros, w_out
+
+
+def gptq_quantize(w, x_bits, bits: int = 4, symmetric: bool = False, group_size: int = 128,
+                  damp: float = GPTQ_DAMP, block: int = GPTQ_BLOCK):
+    """GPTQ of one layer: weights ``w`` (N x K), calibration samples
+    ``x_bits`` (n x K bf16 bits); returns (codes, scales, zeros | None) in
+    the packed format of :func:`quantize_pack`."""
+    wf = _weights_f32(w)
+    N, K = wf.shape
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    if x.shape[1] != K:
+        raise ValueError("calibration samples must have K features")
+    cs, ss, zs = packed_shapes(N, K, bits, symmetric, group_size)
+    codes = np.zeros(cs, dtype=np.uint8)
+    scales = np.zeros(ss, dtype=np.uint16)
+    zeros = None if zs is None else np.zeros(zs, dtype=np.uint8)
+    rc = lib().qzo_gptq_quantize(_ptr(wf), _ptr(x), N, K, x.shape[0], float(damp), block, bits,
+                                 int(symmetric), group_size, _ptr(codes), _ptr(scales),
+                                 _ptr(zeros))
+    if rc != 0:
+        raise ValueError("qzo_gptq_quantize rejected the arguments")
+    return codes, scales, zeros
 
 
 def matmul_f64(a_bits, w_hat_bits):

@@ -192,6 +192,17 @@ def _check_format_invariants(w_bits, bits, symmetric, group_size, exact_rounding
     up = np.where(near_v >= s32, near, near + 1).astype(np.uint16)
     assert np.array_equal(up.reshape(np.asarray(scales).shape), np.asarray(scales)), \
         "stored scale is not the smallest bf16 >= S"
+    # range figure of the guide's "Mapping values to fewer bits": the low end
+    # of the range lands on q_min (the range is widened to contain 0.0, so a
+    # group with no negative value has Z == q_min)
+    if not symmetric:
+        qg = q.reshape(-1) if group_size == 0 else q.reshape(N, K // gs, gs)
+        Zg = Z.reshape(-1)[:1] if group_size == 0 else Z.reshape(N, K // gs, gs)[..., 0]
+        lo = xs.min(axis=-1)
+        at_lo = np.take_along_axis(qg, xs.argmin(axis=-1)[..., None], axis=-1)[..., 0]
+        neg = lo < 0
+        assert (at_lo[neg] == qmin).all(), "the range minimum does not map to q_min"
+        assert (Zg[~neg] == qmin).all(), "a group without negatives needs Z == q_min"
     # round trip: every element within half a step of its reconstruction
     err = np.abs(x - S * (q - Z))
     assert (err <= S / 2 * (1 + 1e-12)).all(), float((err / S).max())
@@ -400,6 +411,116 @@ def pin_tolerance_reaches_bf16_outputs():
     # the subnormal term is negligible against normal outputs
     assert oracle.BF16_SUBNORMAL_HALF_SPACING == 2.0 ** -134
     assert oracle.tolerance(np.array([1e-30]), np.array([1e-30]))[0] == pytest.approx(8.1e-33)
+
+
+
+
+# --------------------------------------------------------------------------
+# GPTQ (GPTQ explainer, azimuth.plus/paper/gptq)
+# --------------------------------------------------------------------------
+
+def _gptq_inputs(N, K, n, seed):
+    w = _random_bf16((N, K), 0.02, seed)
+    x = _random_bf16((n, K), 1.0, seed + 1, outliers=False)
+    return w, x
+
+
+def pin_gptq_identity_hessian_is_rtn():
+    """H = 2 X X^T proportional to the identity (one calibration sample per
+    input feature, x_t = e_t): the inverse Hessian is diagonal, no weight is
+    ever adjusted, and GPTQ reduces to the round-to-nearest quantizer."""
+    N, K = 8, 256
+    w = _random_bf16((N, K), 0.02, 311)
+    x = np.zeros((K, K), np.uint16)
+    x[np.arange(K), np.arange(K)] = 0x3F80                    # bf16 1.0
+    for bits, symmetric in FORMATS:
+        for g in (32, 128, K):
+            got = oracle.gptq_quantize(w, x, bits, symmetric, g)
+            ref = oracle.quantize_pack(w, bits, symmetric, g)
+            for a, b in zip(got, ref):
+                if b is None:
+                    assert a is None
+                else:
+                    assert np.array_equal(a, b), (bits, symmetric, g)
+
+
+def _obq_fixed_order(w_bits, x_bits, bits, symmetric, g, damp=oracle.GPTQ_DAMP):
+    """OBQ as the page first describes it, with GPTQ's fixed column order:
+    quantize column q of every row, move every later weight by
+    -err / [Hinv]_qq * Hinv[q, k], then eliminate q from the inverse Hessian
+    (Gaussian elimination).  No Cholesky, no batching.  The round-to-nearest
+    quantizer of a value is restated here from the guide's formulas (scale
+    and zero-point of the group, taken when its first column is reached)."""
+    W = oracle.bf16_bits_to_f32(w_bits).astype(np.float64)
+    X = oracle.bf16_bits_to_f32(x_bits).astype(np.float64).T       # K x n
+    N, K = W.shape
+    H = 2.0 * X @ X.T
+    H += np.eye(K) * damp * np.mean(np.diag(H))
+    Hinv = np.linalg.inv(H)
+    qmin, qmax = oracle.code_range(bits, symmetric)
+    codes = np.zeros((N, K), np.int64)
+    S = np.zeros((N, K // g))
+    Z = np.zeros((N, K // g), np.int64)
+    for q in range(K):
+        if q % g == 0:
+            grp = W[:, q:q + g].astype(np.float32)
+            _, sc, zz = oracle.quantize_pack(grp, bits, symmetric, g)     # group scale / zero
+            S[:, q // g] = oracle.bf16_bits_to_f32(sc[:, 0])
+            Z[:, q // g] = 0 if zz is None else _zeros_int(zz, bits, symmetric, zz.shape)[:, 0]
+        s32 = S[:, q // g].astype(np.float32)
+        u = (W[:, q].astype(np.float32) / s32 + Z[:, q // g].astype(np.float32)).astype(np.float32)
+        c = np.clip(np.rint(u), qmin, qmax).astype(np.int64)
+        codes[:, q] = c
+        w_hat = S[:, q // g] * (c - Z[:, q // g])
+        err = (W[:, q] - w_hat) / Hinv[q, q]
+        W[:, q + 1:] -= np.outer(err, Hinv[q, q + 1:])
+        W[:, q] = w_hat
+        Hinv = Hinv - np.outer(Hinv[:, q], Hinv[q, :]) / Hinv[q, q]
+    return codes, W
+
+
+def pin_gptq_matches_sequential_obq():
+    """The Cholesky form with lazy batches equals OBQ's sequential form with
+    the fixed column order (the page's three innovations change the cost,
+    not the result): same codes, same compensated weights."""
+    for (bits, symmetric, N, K, g, block) in ((4, False, 6, 48, 16, 8), (4, False, 5, 40, 8, 128),
+                                             (8, True, 4, 32, 32, 8), (4, True, 3, 64, 32, 16)):
+        w, x = _gptq_inputs(N, K, 24, 400 + K)
+        H, U = oracle.gptq_hessian_factor(x)
+        codes, scales, zeros, w_out = oracle.gptq_quantize_with_factor(w, U, bits, symmetric, g,
+                                                                       block)
+        q = _as_int_codes(codes, N, K, bits, symmetric)
+        ref_q, ref_w = _obq_fixed_order(w, x, bits, symmetric, g)
+        assert np.array_equal(q, ref_q), (bits, symmetric, K, g, block)
+        assert np.allclose(w_out, ref_w, rtol=0, atol=1e-9), float(np.abs(w_out - ref_w).max())
+
+
+def pin_gptq_lazy_batch_is_a_reordering():
+    """Blocks of 8 columns and one block of all columns give the same codes:
+    the lazy update only postpones additions."""
+    w, x = _gptq_inputs(16, 256, 64, 520)
+    for bits, symmetric, g in ((4, False, 128), (4, False, 32), (8, True, 256)):
+        a = oracle.gptq_quantize(w, x, bits, symmetric, g, block=8)
+        b = oracle.gptq_quantize(w, x, bits, symmetric, g, block=256)
+        for u, v in zip(a, b):
+            assert (u is None and v is None) or np.array_equal(u, v), (bits, symmetric, g)
+
+
+def pin_gptq_lowers_the_layer_error():
+    """GPTQ's purpose: the layer output (W - W_hat) X^T is much smaller than
+    with round-to-nearest on the same calibration data."""
+    N, K = 64, 256
+    w, x = _gptq_inputs(N, K, 128, 600)
+    W = oracle.bf16_bits_to_f32(w).astype(np.float64)
+    X = oracle.bf16_bits_to_f32(x).astype(np.float64)
+    for bits, symmetric, g in ((4, False, 128), (4, True, 64)):
+        errs = []
+        for codes, scales, zeros in (oracle.gptq_quantize(w, x, bits, symmetric, g),
+                                     oracle.quantize_pack(w, bits, symmetric, g)):
+            w_hat = oracle.bf16_bits_to_f32(
+                oracle.dequantize(codes, scales, zeros, N, K, bits, symmetric, g))
+            errs.append(float((((W - w_hat) @ X.T) ** 2).sum()))
+        assert errs[0] < 0.5 * errs[1], errs
 
 
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

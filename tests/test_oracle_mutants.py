@@ -6,7 +6,8 @@ quotient) and round-half-even of q_min - 1/2 is q_min, so removing it changes
 no result.
 
 Every mutant below is a plausible slip in the oracle (a dropped term, a wrong
-sign, rounding or index, a transposed operand).  The copy is compiled on the
+sign, rounding or index, a transposed operand), in the round-to-nearest
+quantizer, the dequantization, the reference matmul and the GPTQ column loop.  The copy is compiled on the
 CPU into a temporary directory; the real oracle is never modified.
 """
 import os
@@ -31,10 +32,10 @@ MUTANTS = {
                                  "uint16_t Sb = qzo_f32_to_bf16_rne(S);"),
     "range_without_zero": ("float vmin = 0.0f, vmax = 0.0f;",
                            "float vmin = x[0], vmax = x[0];"),
-    "divide_by_unrounded_scale": ("float u = x[i] / Sf + (float)Z;",
-                                  "float u = x[i] / S + (float)Z;"),
-    "shift_before_divide": ("float u = x[i] / Sf + (float)Z;",
-                            "float u = (x[i] + (float)Z) / Sf;"),
+    "zero_point_from_unrounded_scale": ("Z = qmin - (int32_t)rintf(vmin / Sf);",
+                                        "Z = qmin - (int32_t)rintf(vmin / S);"),
+    "shift_before_divide": ("float u = x / Sf + (float)Z;",
+                            "float u = (x + (float)Z) / Sf;"),
     "code_span_off_by_one": ("S = (vmax - vmin) / (float)(qmax - qmin);",
                              "S = (vmax - vmin) / (float)(qmax - qmin + 1);"),
     "symmetric_qmax_128": ("*qmax = (1 << (bits - 1)) - 1;", "*qmax = (1 << (bits - 1));"),
@@ -47,6 +48,16 @@ MUTANTS = {
     "matmul_transposed_operand": ("(double)qzo_bf16_to_f32(w_hat[n * K + k]);",
                                   "(double)qzo_bf16_to_f32(w_hat[k * N + n % K]);"),
     "matmul_abs_sum_signed": ("sa += fabs(p);", "sa += p;"),
+    # GPTQ
+    "gptq_error_not_scaled": ("double e = (W[j] - w_hat) / U[j * K + j];",
+                              "double e = (W[j] - w_hat);"),
+    "gptq_lazy_update_dropped": ("                W[k] -= v;\n", "\n"),
+    "gptq_factor_transposed": ("for (int64_t k = j + 1; k < end; ++k) W[k] -= e * U[j * K + k];",
+                               "for (int64_t k = j + 1; k < end; ++k) W[k] -= e * U[k * K + j];"),
+    "gptq_group_scale_from_original_weights": ("for (int64_t k = 0; k < g; ++k) grp[k] = (float)W[j + k];",
+                                               "for (int64_t k = 0; k < g; ++k) grp[k] = w[n * K + j + k];"),
+    "gptq_no_damping": ("double lambda = mean > 0.0 ? damp * mean : 1.0;",
+                        "double lambda = mean > 0.0 ? 0.0 : 1.0;"),
 }
 
 

@@ -163,20 +163,27 @@ def test_w8a16_gemm_workspace_follows_the_route():
 
 
 @pytest.mark.parametrize("op,M,N,K,g,expect", [
-    # M = 1: CTAs per SM from the per-block cost model (4096 x 4096: four,
-    # 1.73 blocks per warp, every task split over up to 32 slots)
-    ("W4A16_GEMV", 1, 4096, 4096, 128, 128 * 32 * 1 * 32 * 4 + 2 * 64 * 4),
-    # 70B layer: five CTAs per SM, 19 blocks per warp, 5 slots per task
-    ("W4A16_GEMV", 1, 28672, 8192, 128, 896 * 5 * 1 * 32 * 4 + 14 * 64 * 4),
-    ("W8A16_GEMV", 1, 4096, 4096, 4096, 128 * 32 * 1 * 32 * 4 + 2 * 64 * 4),
-    # M > 1: the largest CTA count giving each warp at least four blocks
-    ("W4A16_GEMV", 8, 11008, 4096, 128, 344 * 9 * 8 * 32 * 4 + 6 * 64 * 4),
+    # Units are 128 rows x 128 k; CTAs per SM: the most (up to 3) that give
+    # each CTA at least 4 units.  4096 x 4096: 1024 units -> 1 CTA per SM,
+    # 6 units per CTA, ceil(32/6) + 1 = 7 slots per 32-row subtask, 128
+    # subtasks.
+    ("W4A16_GEMV", 1, 4096, 4096, 128, 128 * 7 * 1 * 32 * 4 + 2 * 64 * 4),
+    # 70B layer: 14336 units -> 3 CTAs per SM (444), 32 units per CTA,
+    # ceil(64/32) + 1 = 3 slots, 896 subtasks
+    ("W4A16_GEMV", 1, 28672, 8192, 128, 896 * 3 * 1 * 32 * 4 + 14 * 64 * 4),
+    ("W8A16_GEMV", 1, 4096, 4096, 4096, 128 * 7 * 1 * 32 * 4 + 2 * 64 * 4),
+    # 11008 x 4096: 86 tasks x 32 blocks = 2752 units -> 444 CTAs, 6 units
+    # each, 7 slots, 344 subtasks
+    ("W4A16_GEMV", 8, 11008, 4096, 128, 344 * 7 * 8 * 32 * 4 + 6 * 64 * 4),
     ("W4A16_GEMV", 16, 28672, 8192, 128, 896 * 3 * 16 * 32 * 4 + 14 * 64 * 4),
 ])
 def test_gemv_plan_workspace(op, M, N, K, g, expect):
-    """The stream-K plan (host logic) through the workspace it asks for:
-    fp32 partial slots [task][slot][M][32] plus one counter per task."""
-    assert qz.qz_workspace_bytes(getattr(qz, "QZ_OP_" + op), M, N, K, g) == expect
+    """The stream-K plan (host logic) on a 148-SM device through the
+    workspace it asks for: fp32 partial slots [subtask][slot][M][32] plus one
+    counter per 32-row subtask; qz_workspace_bytes is at least that."""
+    code = getattr(qz, "QZ_OP_" + op)
+    assert qz.qz_workspace_bytes_for_sms(code, M, N, K, g, 148) == expect
+    assert qz.qz_workspace_bytes(code, M, N, K, g) >= expect
 
 
 def test_launch_overlap_setter():
@@ -208,3 +215,35 @@ def test_workspace_bound_serves_every_sm_count(op, M, N, K, g):
     for bad in (0, 149):
         with pytest.raises(qz.QzError):
             qz.qz_workspace_bytes_for_sms(op, M, N, K, g, bad)
+
+
+def _gptq(w=A, x=B, N=64, K=256, n=128, bits=4, sym=0, g=128, damp=0.01, codes=C, scales=D,
+          zeros=Y, ws=None, ws_bytes=0):
+    return L().qz_gptq_quantize(w, x, N, K, n, bits, sym, g, damp, codes, scales, zeros, ws,
+                                ws_bytes, None)
+
+
+@pytest.mark.parametrize("kwargs,expect", [
+    (dict(), WS),                                    # no workspace
+    (dict(bits=3), UNSUP),
+    (dict(N=0), INVALID), (dict(n=0), INVALID), (dict(K=0), INVALID),
+    (dict(g=100), INVALID),                          # does not divide K
+    (dict(g=16, K=256), UNSUP),                      # below 32
+    (dict(g=96, K=384), UNSUP),                      # neither nests with the 128-wide blocks
+    (dict(K=260, g=4), UNSUP),                       # K % 8 != 0 (and g too small)
+    (dict(damp=-1.0), INVALID), (dict(damp=float("nan")), INVALID),
+    (dict(zeros=None), INVALID),                     # asymmetric needs zeros
+    (dict(sym=1), INVALID),                          # symmetric takes none
+    (dict(x=None), INVALID),
+    (dict(w=ctypes.c_void_p(0x10001)), ALIGN),
+])
+def test_gptq_rejects(kwargs, expect):
+    assert _gptq(**kwargs) == expect
+
+
+def test_gptq_workspace_bytes():
+    # fp64: two K x K matrices, N x K working weights, N x 128 block errors
+    N, K = 4096, 4096
+    assert qz.qz_workspace_bytes(qz.QZ_OP_GPTQ, 1, N, K, 128) == \
+        2 * K * K * 8 + N * K * 8 + N * 128 * 8
+    assert qz.qz_workspace_bytes(qz.QZ_OP_GPTQ, 1, 37, 384, 128) >= 2 * 384 * 384 * 8 + 37 * 384 * 8

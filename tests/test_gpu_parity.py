@@ -253,8 +253,8 @@ def test_gemv_workspace_is_left_zeroed_and_results_repeat(dev):
     torch.cuda.synchronize()
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
     # the counter region (after the partials) must be zero again
-    tasks = (N + 31) // 32                       # one counter per 32-row warp task
-    plan_partials = nbytes - (-(-tasks // 64)) * 64 * 4
+    subtasks = (N + 31) // 32                    # one counter per 32-row subtask
+    plan_partials = nbytes - (-(-subtasks // 64)) * 64 * 4
     assert int(ws[plan_partials:].count_nonzero()) == 0
 
 

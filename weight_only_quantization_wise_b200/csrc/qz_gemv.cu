@@ -6,54 +6,88 @@
 // the step reading weights, so 4-bit weights move a quarter of the bytes.
 // GPTQ explainer: the gain needs kernels that dequantize inside the matmul.
 //
-// Design (one warp = 32 weight rows over a K range):
-//   * Lane (g = lane/4, t = lane%4) streams, per 128-wide K block, its 32
-//     consecutive k of rows g, g+8, g+16, g+24 (16 bytes of int4 codes or 32
-//     bytes of int8 codes per row) with cp.async into a ring of kStages
-//     blocks in the warp's own slice of shared memory, so that kStages-1
-//     blocks are in flight while one is computed, without holding them in
-//     registers.  The codes each lane copies are the ones it reads back.
-//   * int4 with groups of 128 * 2^i: the scales and zeros of the
-//     block ride in the same ring slot.  Lane (g, t) copies the aligned
-//     32-bit words holding the scale and the zero of row g + 8t, so the 32
-//     rows of the warp take two 4-byte copies per lane; after
-//     cp.async.wait_group and a warp barrier every lane reads the words of
-//     its four rows with two 16-byte shared loads and builds (S, S) and
-//     bf16(-(128 + Z)) twice with one byte permute each.  Since the warp's
-//     first row is a multiple of 32 and its rows differ by multiples of 8,
-//     all four rows of a lane share the word offset of their entries.
-//     Other group sizes load the lane's scales and zeros directly.
-//   * Codes are dequantized in registers to bf16 exactly as qz_dequantize
-//     forms them.  int4: a LOP3 builds bf16(128 + q) for two nibbles,
-//     add.rn.bf16x2 of bf16(-(128 + Z)) leaves q - Z exactly, mul.rn.bf16x2
-//     by the bf16 scale rounds S*(q - Z) once.  int8: the byte (XOR 0x80) is
-//     placed in the mantissa of 2^23, one fp32 subtraction gives q exactly,
-//     the pair is packed to bf16 exactly and mul.rn.bf16x2 rounds S*q once.
+// Design: each CTA is one producer warp and four consumer warps around a
+// ring of shared-memory stages; a stage is one unit of work, 128 weight rows
+// x 128 k (8 KB of int4 codes, 16 KB of int8).
+//   * Producer (warp 0).  One lane issues a TMA 2D copy of the unit's codes
+//     into the stage (completing on the stage's "full" mbarrier with a
+//     transaction count).  For int4 with groups of 128 * 2^i the 32 lanes
+//     also gather, with 4-byte cp.async copies, the aligned words that hold
+//     the scale and the zero of each of the 128 rows and signal the same
+//     barrier when they land (cp.async.mbarrier.arrive.noinc), so codes,
+//     scales and zeros of a unit arrive together.  The producer waits on a
+//     stage's "empty" barrier before refilling it; it never touches
+//     activations, outputs or the workspace.
+//   * Consumers (warps 1..4).  Warp w owns rows 32w..32w+31 of each unit.
+//     Lane (g = lane/4, t = lane%4) reads the 16 (int4) or 32 (int8) code
+//     bytes of k = 32t..32t+31 of rows g, g+8, g+16, g+24 from the stage with
+//     16-byte shared loads (int8 rows are 128 B, loaded with the 128-byte
+//     swizzle so that those loads are free of bank conflicts), reads the
+//     four rows' scale and zero words with one 16-byte load each, releases
+//     the stage, and dequantizes in registers to bf16 exactly as
+//     qz_dequantize forms each weight.  int4: a LOP3 builds bf16(128 + q) for
+//     two nibbles, add.rn.bf16x2 of bf16(-(128 + Z)) leaves q - Z exactly,
+//     mul.rn.bf16x2 by the bf16 scale rounds S*(q - Z) once.  int8: the byte
+//     (XOR 0x80) is placed in the mantissa of 2^23, one fp32 subtraction
+//     gives q exactly, the pair is packed to bf16 exactly and mul.rn.bf16x2
+//     rounds S*q once.
 //   * A byte of codes yields the pairs (q_j, q_{j+4}), so the K axis is
-//     permuted consistently for both MMA operands: the pairs are the A operand
-//     (16 rows x 16 k) of mma.sync m16n8k16 with fp32 accumulation and the
-//     activations (tokens as the 8 columns) are the B operand, permuted to
-//     match with PRMT once per k for both 16-row tiles of the warp.  For
-//     M > 8 a second MMA covers tokens 8..15.  Columns of tokens >= M read
-//     token M-1's activations; their outputs are dropped.
-//   * Stream-K: the (32-row task x 128-wide K block) units are divided into
-//     equal contiguous ranges, one per launched warp, and exactly a whole
-//     number of CTAs per SM is launched, so every SM gets the same work.  A
-//     task covered by one warp is written directly; otherwise each
-//     contributing warp writes its fp32 partial tile into the task's slot
-//     and bumps the task's counter, and the last one to arrive adds the
-//     slots in order (deterministic), one row per lane, writes bf16 y and
-//     resets the counter.
+//     permuted consistently for both MMA operands: the pairs are the A
+//     operand (16 rows x 16 k) of mma.sync m16n8k16 with fp32 accumulation
+//     and the activations (tokens as the 8 columns, read through L1) are the
+//     B operand, permuted to match with PRMT once per k for both 16-row tiles
+//     of the warp.  For M > 8 a second MMA covers tokens 8..15.  Columns of
+//     tokens >= M read token M-1's activations; their outputs are dropped.
+//   * Stream-K: the units, in (row task, k block) order, are divided into
+//     equal contiguous ranges, one per CTA, with the same number of CTAs on
+//     every SM, so every SM streams the same number of bytes.  A 32-row
+//     subtask covered by one CTA is written directly; otherwise each
+//     contributing CTA's warp writes its fp32 partial tile into the
+//     subtask's slot and bumps the subtask's counter, and the last one to
+//     arrive adds the slots in order (deterministic), one row per lane,
+//     writes bf16 y and resets the counter.
+//   * Every mbarrier wait is bounded (wall time, qz_set_device_wait_limit):
+//     on expiry the waiting warp records the fault in the device error word
+//     and a CTA-local abort flag, the producer stops issuing, waits (again
+//     bounded) for every copy it issued to land, and the CTA exits.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
-#include "qz_internal.cuh"
+#include "qz_sm100.cuh"
 
 namespace qz {
 namespace {
 
-constexpr int kWarpsPerCta = 4;
-constexpr int kThreads = 32 * kWarpsPerCta;
-constexpr int kRowsPerWarp = 32;                       // two 16-row MMA tiles
+using namespace sm100;
+
+constexpr int kConsumerWarps = 4;
+constexpr int kRowsPerWarp = 32;                               // two 16-row MMA tiles
+constexpr int kTileRows = kConsumerWarps * kRowsPerWarp;       // rows of a unit
+constexpr int kThreads = 32 * (1 + kConsumerWarps);
+constexpr int kBlockK = 128;                                   // k of a unit
+template <int BITS>
+constexpr int kRowBytes = kBlockK * BITS / 8;                  // code bytes of a row in a unit
+template <int BITS>
+constexpr int kCodeStage = kTileRows * kRowBytes<BITS>;        // 8 KB (int4), 16 KB (int8)
+constexpr int kSzStage = kTileRows * 8;                        // 128 scale words + 128 zero words
+template <int BITS>
+constexpr int kStages = BITS == 4 ? 8 : 4;
+constexpr int kMaxCtasPerSm = 3;
+
+// Shared-memory layout (offsets from the 1024-byte aligned base).
+template <int BITS>
+struct Layout {
+    static constexpr int S = kStages<BITS>;
+    static constexpr uint32_t codes = 0;
+    static constexpr uint32_t sz = codes + S * kCodeStage<BITS>;
+    static constexpr uint32_t full = sz + (BITS == 4 ? S * kSzStage : 0);
+    static constexpr uint32_t empty = full + 8 * S;
+    static constexpr uint32_t abort_flag = empty + 8 * S;
+    static constexpr uint32_t end = abort_flag + 16;
+    static constexpr uint32_t bytes = end + 1024;                // + alignment slack
+};
+static_assert(kMaxCtasPerSm * (Layout<4>::bytes + 1024) <= 228 * 1024, "int4 ring fits 3 CTAs");
+static_assert(kMaxCtasPerSm * (Layout<8>::bytes + 1024) <= 228 * 1024, "int8 ring fits 3 CTAs");
 
 // bf16 pair (nibble j, nibble j+4) of a code word: bf16_rne(S * (q - Z)).
 // nz2 holds bf16(-(128 + Z)) twice.
@@ -102,84 +136,72 @@ struct Act {
     uint32_t x[MB][16];            // tokens g (+8): 32 bf16 each
 };
 
-template <int BITS>
-constexpr int kStages = BITS == 4 ? 4 : 3;               // ring slots per warp
-template <int BITS>
-constexpr int kLaneRowBytes = BITS == 4 ? 16 : 32;     // codes of one row per lane per block
-template <int BITS>
-constexpr int kCodeBytes = 4 * 32 * kLaneRowBytes<BITS>;
-constexpr int kSzBytes = 256;                          // 32 scale words + 32 zero words
-template <int BITS>
-constexpr int kSlotBytes = kCodeBytes<BITS> + (BITS == 4 ? kSzBytes : 0);
-template <int BITS>
-constexpr int kGemvSmemBytes = kWarpsPerCta * kStages<BITS> * kSlotBytes<BITS>;
-// Resident CTAs per SM: registers allow five (int4, M <= 8: at most 102 per
-// thread), four (int8, M <= 8: shared memory) or three (M > 8).
-template <int BITS, int MB>
-constexpr int kCtasPerSm = MB == 1 ? (BITS == 4 ? 5 : 4) : 3;
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
 __device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() {
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+// Arrive on `bar` once every cp.async this thread issued so far has landed
+// (the arrival is counted in the barrier's expected count: no increment).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
-// Byte offset, inside a warp's slot, of 16-byte piece `half` of row j for
-// `lane`: pieces of 32 lanes are contiguous, so each 8-lane phase of a
-// 16-byte shared load reads 128 consecutive bytes (no bank conflicts).
-template <int BITS>
-__device__ __forceinline__ uint32_t piece_offset(int j, int half, int lane) {
-    return (uint32_t)(((j * (kLaneRowBytes<BITS> / 16) + half) * 32 + lane) * 16);
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
 }
 
+// Codes of the lane's four rows from a stage.  int4: row r at 64 r, lane t
+// reads bytes 16t..16t+15 (rows g and g+1 of an 8-lane phase are adjacent:
+// 128 consecutive bytes).  int8: row r at 128 r with the 128-byte swizzle
+// (16-byte chunk c stored at chunk c ^ (r & 7)); lane t reads chunks 2t and
+// 2t+1, and r & 7 == g for every row of the lane.
 template <int BITS>
-__device__ __forceinline__ void read_block(RowWords<BITS> &rw, const uint8_t *slot, int lane) {
+__device__ __forceinline__ void read_codes(RowWords<BITS> &rw, uint32_t stage, int row0, int g,
+                                           int t) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t row = stage + (uint32_t)(row0 + 8 * j) * kRowBytes<BITS>;
+        if (BITS == 4) {
+            const uint4 v = lds128(row + 16u * t);
+            rw.w[j][0] = v.x; rw.w[j][1] = v.y; rw.w[j][2] = v.z; rw.w[j][3] = v.w;
+        } else {
 #pragma unroll
-        for (int h = 0; h < kLaneRowBytes<BITS> / 16; ++h) {
-            const uint4 v = *reinterpret_cast<const uint4 *>(slot + piece_offset<BITS>(j, h, lane));
-            rw.w[j][4 * h + 0] = v.x; rw.w[j][4 * h + 1] = v.y;
-            rw.w[j][4 * h + 2] = v.z; rw.w[j][4 * h + 3] = v.w;
+            for (int h = 0; h < 2; ++h) {
+                const uint4 v = lds128(row + 16u * ((2 * t + h) ^ g));
+                rw.w[j][4 * h + 0] = v.x; rw.w[j][4 * h + 1] = v.y;
+                rw.w[j][4 * h + 2] = v.z; rw.w[j][4 * h + 3] = v.w;
+            }
         }
+    }
 }
 
 struct GemvArgs {
     const uint16_t *a;
-    const uint8_t *codes;
     const uint16_t *scales;
     const uint8_t *zeros;
     int M, N, K, group_size, group_shift;
-    int bpg_shift;                     // log2(group_size / 128) (ring path), else -1
+    int bpg_shift;             // log2(group_size / 128) (ring path), else -1
+    int kblocks;               // K / 128
     uint16_t *y;
     float *partials;
     uint32_t *counters;
-    int64_t units;        // tasks * kblocks
-    int64_t warps;        // launched warps
-    int kblocks, slots;
-    int prefetch_early;   // launch overlap: first blocks' weights before the grid wait
+    int64_t units;             // tasks * kblocks
+    int64_t ctas;              // launched CTAs (each owns at least one unit)
+    int slots;
+    int prefetch_early;        // launch overlap: weights may be read before the grid wait
+    uint64_t wait_limit;
+    unsigned int *err_word;    // device error word (set when a bounded wait runs out)
 };
 
-// Group index of 128-wide block kb when the group size is 128 * 2^bpg_shift
-// (the ring path's condition).
-__device__ __forceinline__ int group_of_block(const GemvArgs &p, int kb) {
-    return kb >> p.bpg_shift;
-}
-
 // Scales and zeros of the lane's four rows for block kb, loaded directly
-// (group sizes below 128, or scale/zero arrays the ring cannot copy).
+// (group sizes below 128, or scale/zero arrays the ring cannot gather).
 __device__ __forceinline__ void load_params_direct(RowParams &rp, const GemvArgs &p,
                                                    const bool (&valid)[4], const int (&rows)[4],
                                                    int kb, int t) {
-    const int k0 = kb * 128 + t * 32;
+    const int k0 = kb * kBlockK + t * 32;
     const int64_t gpr = p.K / p.group_size;
     const int gi = p.group_shift >= 0 ? (k0 >> p.group_shift) : (k0 / p.group_size);
 #pragma unroll
@@ -192,11 +214,10 @@ __device__ __forceinline__ void load_params_direct(RowParams &rp, const GemvArgs
 }
 
 // Activations of one block for tokens g (and g + 8), clamped to M - 1: read
-// from L1/L2 (the vector is shared by every warp) right before the block is
-// computed.
+// through L1 (the vector is shared by every warp of the SM).
 template <int MB>
 __device__ __forceinline__ void load_act(Act<MB> &ac, const GemvArgs &p, int kb, int g, int t) {
-    const int k0 = kb * 128 + t * 32;
+    const int k0 = kb * kBlockK + t * 32;
 #pragma unroll
     for (int mb = 0; mb < MB; ++mb) {
         const int tok = min(8 * mb + g, p.M - 1);
@@ -262,9 +283,9 @@ __device__ __forceinline__ void wait_for_previous_grid() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-// First warp whose unit range contains unit u (ranges: [w*U/W, (w+1)*U/W)).
-__device__ __forceinline__ int64_t warp_of_unit(int64_t u, int64_t U, int64_t W) {
-    return ((u + 1) * W - 1) / U;
+// First CTA whose unit range contains unit u (ranges: [c*U/C, (c+1)*U/C)).
+__device__ __forceinline__ int64_t cta_of_unit(int64_t u, int64_t U, int64_t C) {
+    return ((u + 1) * C - 1) / U;
 }
 
 // Deterministic split-K sum: y[t][row] = sum over slots c = 0, 1, ... of
@@ -315,15 +336,16 @@ __device__ __forceinline__ void reduce_slots(const float *base, int64_t slot_ele
     }
 }
 
-// acc[rt][mb][j] holds y[tok = 8mb + 2t + (j&1)][row = n0 + 16rt + g + 8(j>>1)].
-// `whole`: this warp covered every K block of the task.  Otherwise the
-// partial goes to slot (this warp - the task's first warp) and the last of
-// the task's contributors adds the slots in order, lane l summing row l.
+// acc[rt][mb][j] holds y[tok = 8mb + 2t + (j&1)][row = n0 + 16rt + g + 8(j>>1)]
+// for the warp's 32 rows n0.. of task `task`.  `whole`: this CTA covered
+// every K block of the task.  Otherwise the partial goes to slot (this CTA -
+// the task's first CTA) of the warp's subtask and the last of the
+// subtask's contributors adds the slots in order, lane l summing row l.
 template <int MB>
 __device__ __forceinline__ void gemv_flush(float (&acc)[2][MB][4], const GemvArgs &p, int task,
-                                           bool whole, int64_t w, int lane) {
+                                           int w, bool whole, int64_t cta, int lane) {
     const int g = lane >> 2, t = lane & 3;
-    const int n0 = task * kRowsPerWarp;
+    const int n0 = task * kTileRows + w * kRowsPerWarp;
     if (whole) {
 #pragma unroll
         for (int rt = 0; rt < 2; ++rt)
@@ -334,16 +356,18 @@ __device__ __forceinline__ void gemv_flush(float (&acc)[2][MB][4], const GemvArg
                     const int row = n0 + 16 * rt + g + 8 * (j >> 1);
                     const int tok = 8 * mb + 2 * t + (j & 1);
                     if (row < p.N && tok < p.M)
-                        p.y[(int64_t)tok * p.N + row] = (uint16_t)dev::f32_to_bf16_rne(acc[rt][mb][j]);
+                        p.y[(int64_t)tok * p.N + row] =
+                            (uint16_t)dev::f32_to_bf16_rne(acc[rt][mb][j]);
                 }
         return;
     }
-    const int64_t first = warp_of_unit((int64_t)task * p.kblocks, p.units, p.warps);
-    const int64_t last = warp_of_unit((int64_t)(task + 1) * p.kblocks - 1, p.units, p.warps);
+    const int64_t first = cta_of_unit((int64_t)task * p.kblocks, p.units, p.ctas);
+    const int64_t last = cta_of_unit((int64_t)(task + 1) * p.kblocks - 1, p.units, p.ctas);
     const int contributors = (int)(last - first + 1);
     const int64_t slot_elems = (int64_t)p.M * kRowsPerWarp;
-    float *base = p.partials + ((int64_t)task * p.slots) * slot_elems;
-    float *mine = base + (w - first) * slot_elems;
+    const int64_t sub = (int64_t)task * kConsumerWarps + w;
+    float *base = p.partials + (sub * p.slots) * slot_elems;
+    float *mine = base + (cta - first) * slot_elems;
 #pragma unroll
     for (int rt = 0; rt < 2; ++rt)
 #pragma unroll
@@ -357,88 +381,134 @@ __device__ __forceinline__ void gemv_flush(float (&acc)[2][MB][4], const GemvArg
     __threadfence();
     __syncwarp();
     uint32_t prev = 0;
-    if (lane == 0) prev = atomicAdd(&p.counters[task], 1u);
+    if (lane == 0) prev = atomicAdd(&p.counters[sub], 1u);
     prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
     if (prev != (uint32_t)(contributors - 1)) return;
     __threadfence();
     // The last contributor: lane l adds row l of every slot in slot order,
-    // for all tokens at once (two slots' loads in flight per round trip).
+    // for all tokens at once.
     reduce_slots<8 * MB, kRowsPerWarp>(base, slot_elems, contributors, p.M, lane, n0 + lane,
                                        p.N, p.y);
-    if (lane == 0) p.counters[task] = 0u;
+    if (lane == 0) p.counters[sub] = 0u;
 }
 
-// RING_SZ: int4 scales and zeros travel through the cp.async ring (group
-// size a multiple of 128, 4-byte aligned arrays whose 4-byte words stay
-// inside them).
+// RING_SZ: int4 scales and zeros travel with the codes (group size a
+// multiple of 128, 4-byte aligned arrays whose 4-byte words stay inside
+// them).
 template <int BITS, int MB, bool RING_SZ>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm<BITS, MB>)
-gemv_kernel(const GemvArgs p) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int g = lane >> 2, t = lane & 3;
-    const int64_t w = (int64_t)blockIdx.x * kWarpsPerCta + warp;
-    if (w >= p.warps) return;                      // the last CTA of a short grid
-    int64_t u = w * p.units / p.warps;
-    const int64_t u_end = (w + 1) * p.units / p.warps;
-    // With launch overlap, only the first ring fill of weights (which the
-    // caller guarantees the previous kernel does not write) precedes the
-    // wait for the previous grid; every other global access follows it.
+__global__ void __launch_bounds__(kThreads, kMaxCtasPerSm)
+gemv_kernel(const __grid_constant__ CUtensorMap code_map, const GemvArgs p) {
+    using L = Layout<BITS>;
+    constexpr int S = L::S;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + L::abort_flag);
+    auto full_bar = [&](int s) { return sbase + L::full + 8u * s; };
+    auto empty_bar = [&](int s) { return sbase + L::empty + 8u * s; };
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t cta = blockIdx.x;
+    const int64_t u_begin = cta * p.units / p.ctas;
+    const int64_t u_end = (cta + 1) * p.units / p.ctas;
+    const int KB = p.kblocks;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full_bar(s), RING_SZ ? 1 + 32 : 1);   // TMA arrive + 32 gather arrivals
+            mbar_init(empty_bar(s), kConsumerWarps);
+        }
+        *abort_flag = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&code_map))
+                     : "memory");
+    }
+    __syncthreads();
     allow_dependents();
-    bool waited = !p.prefetch_early;
 
-    constexpr int S = kStages<BITS>;
-    constexpr int kSlot = kSlotBytes<BITS>;
-    extern __shared__ __align__(16) uint8_t gemv_smem[];
-    uint8_t *ring = gemv_smem + warp * S * kSlot;
-    const uint32_t ring_u32 = (uint32_t)__cvta_generic_to_shared(ring);
-    const int64_t gpr = BITS == 4 ? p.K / p.group_size : 1;
-    const uint32_t *scale_words = reinterpret_cast<const uint32_t *>(p.scales);
-    const uint32_t *zero_words = reinterpret_cast<const uint32_t *>(p.zeros);
-    // (row * gpr) mod 4 is the same for rows g, g+8, g+16, g+24 of any task
-    const int word_phase = (int)(((int64_t)g * gpr) & 3);
+    if (warp == 0) {
+        // ---------------- producer ----------------
+        // Weights only: with launch overlap this may run before the previous
+        // grid completes (the caller guarantees it does not write them).
+        const int64_t gpr = p.K / p.group_size;
+        const uint32_t *scale_words = reinterpret_cast<const uint32_t *>(p.scales);
+        const uint32_t *zero_words = reinterpret_cast<const uint32_t *>(p.zeros);
+        // the rows whose scale and zero words this lane gathers: rows
+        // 32 (lane / 8) + (lane % 8) + 8j of the unit, into words 4 lane + j
+        // of the stage's scale area (and of its zero area, 512 bytes on)
+        const int prow = 32 * (lane >> 3) + (lane & 7);
+        int task = (int)(u_begin / KB);
+        int kb = (int)(u_begin - (int64_t)task * KB);
+        int s = 0, r = 0;
+        int64_t issued = 0;
+        for (int64_t u = u_begin; u < u_end; ++u) {
+            if (r > 0 && !mbar_wait(empty_bar(s), (r - 1) & 1, p.wait_limit, abort_flag,
+                                    p.err_word))
+                break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(full_bar(s), kCodeStage<BITS>);
+                tma_load_2d(sbase + L::codes + s * kCodeStage<BITS>, &code_map,
+                            kb * kRowBytes<BITS>, task * kTileRows, full_bar(s));
+            }
+            if (RING_SZ) {
+                const uint32_t dst = sbase + L::sz + s * kSzStage + 16u * lane;
+                const int gi = kb >> p.bpg_shift;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int row = task * kTileRows + prow + 8 * j;
+                    if (row < p.N) {
+                        const int64_t e = (int64_t)row * gpr + gi;
+                        cp_async4(dst + 4u * j, scale_words + (e >> 1));
+                        cp_async4(dst + 512u + 4u * j, zero_words + (e >> 2));
+                    }
+                }
+                cp_async_arrive_noinc(full_bar(s));
+            }
+            ++issued;
+            if (++kb == KB) {
+                kb = 0;
+                ++task;
+            }
+            if (++s == S) {
+                s = 0;
+                ++r;
+            }
+        }
+        // every issued copy must have landed before the CTA may exit: the
+        // last unit issued into stage q < issued is unit q + S * rq
+#pragma unroll
+        for (int q = 0; q < S; ++q)
+            if (q < issued) {
+                const int64_t rq = (issued - 1 - q) / S;
+                mbar_drain(full_bar(q), (uint32_t)(rq & 1), p.err_word);
+            }
+        return;
+    }
 
-    while (u < u_end) {
-        const int task = (int)(u / p.kblocks);
-        const int kb_begin = (int)(u - (int64_t)task * p.kblocks);
-        const int64_t kb_lim = kb_begin + (u_end - u);
-        const int kb_end = (int)(kb_lim < p.kblocks ? kb_lim : (int64_t)p.kblocks);
-        const int nkb = kb_end - kb_begin;
-        const int n0 = task * kRowsPerWarp;
-
+    // ---------------- consumers ----------------
+    const int w = warp - 1;
+    const int g = lane >> 2, t = lane & 3;
+    if (p.prefetch_early) wait_for_previous_grid();   // before activations, y and workspace
+    int task = (int)(u_begin / KB);
+    int kb0 = (int)(u_begin - (int64_t)task * KB);
+    int s = 0, r = 0;
+    const int word_phase = (int)(((int64_t)g * (p.K / p.group_size)) & 3);
+    for (int64_t u = u_begin; u < u_end;) {
+        const int64_t kb_lim = kb0 + (u_end - u);
+        const int kb_end = (int)(kb_lim < KB ? kb_lim : (int64_t)KB);
+        const int nkb = kb_end - kb0;
+        const int n0 = task * kTileRows + w * kRowsPerWarp;
         int rows[4];
         bool valid[4];
-        const uint8_t *rowp[4];
         uint32_t s8[4];                              // int8: (S, S) of rows g + 8j
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             rows[j] = n0 + g + 8 * j;
             valid[j] = rows[j] < p.N;
-            rowp[j] = p.codes + (int64_t)(valid[j] ? rows[j] : 0) * (BITS == 4 ? p.K / 2 : p.K) +
-                      t * (BITS == 4 ? 16 : 32);
-            s8[j] = (BITS == 8 && valid[j]) ? (uint32_t)__ldg(&p.scales[rows[j]]) * 0x00010001u : 0u;
+            s8[j] = (BITS == 8 && valid[j]) ? (uint32_t)__ldg(&p.scales[rows[j]]) * 0x00010001u
+                                            : 0u;
         }
-        // the row whose scale and zero words this lane copies
-        const int row_c = n0 + g + 8 * t;
-        const bool valid_c = RING_SZ && row_c < p.N;
-        const int64_t entry_c = (int64_t)(valid_c ? row_c : 0) * gpr;
-        const uint32_t sz_dst = kCodeBytes<BITS> + 4u * (uint32_t)(4 * g + t);
-
-        auto issue = [&](int kb, uint32_t slot) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                if (!valid[j]) continue;
-#pragma unroll
-                for (int h = 0; h < kLaneRowBytes<BITS> / 16; ++h)
-                    cp_async16(slot + piece_offset<BITS>(j, h, lane),
-                               rowp[j] + kb * (BITS == 4 ? 64 : 128) + 16 * h);
-            }
-            if (RING_SZ && valid_c) {
-                const int64_t e = entry_c + group_of_block(p, kb);
-                cp_async4(slot + sz_dst, scale_words + (e >> 1));
-                cp_async4(slot + sz_dst + 128u, zero_words + (e >> 2));
-            }
-        };
-
         float acc[2][MB][4];
 #pragma unroll
         for (int rt = 0; rt < 2; ++rt)
@@ -447,58 +517,43 @@ gemv_kernel(const GemvArgs p) {
 #pragma unroll
                 for (int j = 0; j < 4; ++j) acc[rt][mb][j] = 0.0f;
 
-#pragma unroll
-        for (int q = 0; q < S - 1; ++q) {
-            if (q < nkb) issue(kb_begin + q, ring_u32 + q * kSlot);
-            cp_async_commit();
-        }
-        if (!waited) {
-            wait_for_previous_grid();
-            waited = true;
-        }
-        int slot = 0;
-#pragma unroll 2
-        for (int ii = 0; ii < nkb; ++ii) {
-            cp_async_wait<S - 2>();                  // block ii has landed in its slot
-            if (RING_SZ) __syncwarp();               // ... every lane's copies of it, too
-            const int refill = ii + S - 1;           // into the slot read one block ago
-            const int rslot = slot == 0 ? S - 1 : slot - 1;
-            if (refill < nkb) issue(kb_begin + refill, ring_u32 + rslot * kSlot);
-            cp_async_commit();
-            const int kb = kb_begin + ii;
-            const uint8_t *cur = ring + slot * kSlot;
+        for (int kb = kb0; kb < kb_end; ++kb) {
             Act<MB> ac;
             load_act(ac, p, kb, g, t);
+            if (!mbar_wait(full_bar(s), r & 1, p.wait_limit, abort_flag, p.err_word)) return;
+            const uint32_t stage = sbase + L::codes + s * kCodeStage<BITS>;
             RowWords<BITS> rw;
-            read_block<BITS>(rw, cur, lane);
+            read_codes<BITS>(rw, stage, w * kRowsPerWarp + g, g, t);
             RowParams rp;
-            if (BITS == 4) {
-                if (RING_SZ) {
-                    const uint4 ws = *reinterpret_cast<const uint4 *>(cur + kCodeBytes<BITS> + 16 * g);
-                    const uint4 wz =
-                        *reinterpret_cast<const uint4 *>(cur + kCodeBytes<BITS> + 128 + 16 * g);
-                    const int phase = word_phase + group_of_block(p, kb);
-                    const uint32_t os = (uint32_t)(phase & 1) * 2u, oz = (uint32_t)(phase & 3);
-                    const uint32_t sel_s = os * 0x0101u + (os + 1u) * 0x1010u;   // (S, S)
-                    const uint32_t sel_z = oz * 0x0101u + 0x4040u;               // (0xC3, Z) x 2
-                    const uint32_t wsv[4] = {ws.x, ws.y, ws.z, ws.w};
-                    const uint32_t wzv[4] = {wz.x, wz.y, wz.z, wz.w};
+            if (BITS == 4 && RING_SZ) {
+                const uint32_t sz = sbase + L::sz + s * kSzStage + 16u * (8 * w + g);
+                const uint4 ws = lds128(sz);
+                const uint4 wz = lds128(sz + 512u);
+                const int phase = word_phase + (kb >> p.bpg_shift);
+                const uint32_t os = (uint32_t)(phase & 1) * 2u, oz = (uint32_t)(phase & 3);
+                const uint32_t sel_s = os * 0x0101u + (os + 1u) * 0x1010u;   // (S, S)
+                const uint32_t sel_z = oz * 0x0101u + 0x4040u;               // (0xC3, Z) x 2
+                const uint32_t wsv[4] = {ws.x, ws.y, ws.z, ws.w};
+                const uint32_t wzv[4] = {wz.x, wz.y, wz.z, wz.w};
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        rp.s2[j] = dev::prmt(wsv[j], 0u, sel_s);
-                        rp.z2[j] = dev::prmt(wzv[j], 0xC3C3C3C3u, sel_z);
-                    }
-                } else {
-                    load_params_direct(rp, p, valid, rows, kb, t);
+                for (int j = 0; j < 4; ++j) {
+                    rp.s2[j] = dev::prmt(wsv[j], 0u, sel_s);
+                    rp.z2[j] = dev::prmt(wzv[j], 0xC3C3C3C3u, sel_z);
                 }
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty_bar(s));   // the stage's data is in registers
+            if (BITS == 4 && !RING_SZ) load_params_direct(rp, p, valid, rows, kb, t);
             compute_block<BITS, MB>(rp, ac, rw, s8, acc);
-            slot = slot == S - 1 ? 0 : slot + 1;
+            if (++s == S) {
+                s = 0;
+                ++r;
+            }
         }
-        cp_async_wait<0>();
-        __syncwarp();                                // the ring is reused by the next task
-        gemv_flush<MB>(acc, p, task, nkb == p.kblocks, w, lane);
+        gemv_flush<MB>(acc, p, task, w, nkb == KB, cta, lane);
         u += nkb;
+        ++task;
+        kb0 = 0;
     }
 }
 
@@ -510,8 +565,9 @@ int log2_exact(int64_t v) {
 }
 
 template <int BITS, int MB, bool RING_SZ>
-qz_status launch_variant(const GemvArgs &args, dim3 grid, int overlap, cudaStream_t st) {
-    constexpr int smem = kGemvSmemBytes<BITS>;
+qz_status launch_variant(const CUtensorMap &map, const GemvArgs &args, dim3 grid, int overlap,
+                         cudaStream_t st) {
+    constexpr int smem = Layout<BITS>::bytes;
     static DeviceOnce attr_once;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -519,8 +575,15 @@ qz_status launch_variant(const GemvArgs &args, dim3 grid, int overlap, cudaStrea
         return QZ_ERR_CUDA;
     }
     if (attr_once.run(dev, [] {
-            return cudaFuncSetAttribute(gemv_kernel<BITS, MB, RING_SZ>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            cudaError_t e = cudaFuncSetAttribute(gemv_kernel<BITS, MB, RING_SZ>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 smem);
+            // three rings per SM need (nearly) all of the unified memory as
+            // shared memory
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(gemv_kernel<BITS, MB, RING_SZ>,
+                                         cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+            return e;
         }) != cudaSuccess)
         return QZ_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
@@ -533,7 +596,7 @@ qz_status launch_variant(const GemvArgs &args, dim3 grid, int overlap, cudaStrea
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = overlap > 0 ? 1 : 0;
-    cudaLaunchKernelEx(&cfg, gemv_kernel<BITS, MB, RING_SZ>, args);
+    cudaLaunchKernelEx(&cfg, gemv_kernel<BITS, MB, RING_SZ>, map, args);
     return launch_status();
 }
 
@@ -543,13 +606,13 @@ qz_status launch_gemv(const void *a, const void *codes, const void *scales, cons
                       void *workspace, const GemvPlan &plan, int overlap, cudaStream_t st) {
     GemvArgs args;
     args.a = static_cast<const uint16_t *>(a);
-    args.codes = static_cast<const uint8_t *>(codes);
     args.scales = static_cast<const uint16_t *>(scales);
     args.zeros = static_cast<const uint8_t *>(zeros);
     args.M = (int)M; args.N = (int)N; args.K = (int)K;
     args.group_size = (int)group_size;
     args.group_shift = log2_exact(group_size);
-    args.bpg_shift = group_size % 128 == 0 ? log2_exact(group_size / 128) : -1;
+    args.bpg_shift = group_size % kBlockK == 0 ? log2_exact(group_size / kBlockK) : -1;
+    args.kblocks = (int)(K / kBlockK);
     args.y = static_cast<uint16_t *>(y);
     args.partials = nullptr;
     args.counters = nullptr;
@@ -559,85 +622,75 @@ qz_status launch_gemv(const void *a, const void *codes, const void *scales, cons
             reinterpret_cast<uint32_t *>(static_cast<char *>(workspace) + plan.partial_bytes);
     }
     args.units = plan.tasks * plan.kblocks;
-    args.warps = plan.warps;
-    args.kblocks = (int)plan.kblocks;
+    args.ctas = plan.ctas;
     args.slots = (int)plan.slots;
     args.prefetch_early = overlap;
-    const dim3 grid((unsigned)ceil_div(plan.warps, (int64_t)kWarpsPerCta));
+    args.wait_limit = device_wait_limit();
+    args.err_word = device_error_word();
+    if (args.err_word == nullptr) return QZ_ERR_CUDA;
 
-    // The ring copies the aligned 4-byte words holding each scale and zero;
+    CUtensorMap map;
+    const uint64_t row_bytes = (uint64_t)K * BITS / 8;
+    if (!make_map_2d(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, row_bytes, (uint64_t)N,
+                     row_bytes, kRowBytes<BITS>, kTileRows,
+                     BITS == 4 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B))
+        return QZ_ERR_CUDA;
+    const dim3 grid((unsigned)plan.ctas);
+
+    // The ring gathers the aligned 4-byte words holding each scale and zero;
     // they stay inside the arrays when N * K / g is a multiple of 4.
     if constexpr (BITS == 4) {
         const int64_t entries = N * (K / group_size);
         const bool ring_sz = args.bpg_shift >= 0 && aligned(scales, 4) && aligned(zeros, 4) &&
                              entries % 4 == 0;
         if (M <= 8)
-            return ring_sz ? launch_variant<4, 1, true>(args, grid, overlap, st)
-                           : launch_variant<4, 1, false>(args, grid, overlap, st);
-        return ring_sz ? launch_variant<4, 2, true>(args, grid, overlap, st)
-                       : launch_variant<4, 2, false>(args, grid, overlap, st);
+            return ring_sz ? launch_variant<4, 1, true>(map, args, grid, overlap, st)
+                           : launch_variant<4, 1, false>(map, args, grid, overlap, st);
+        return ring_sz ? launch_variant<4, 2, true>(map, args, grid, overlap, st)
+                       : launch_variant<4, 2, false>(map, args, grid, overlap, st);
     } else {
-        return M <= 8 ? launch_variant<8, 1, false>(args, grid, overlap, st)
-                      : launch_variant<8, 2, false>(args, grid, overlap, st);
+        return M <= 8 ? launch_variant<8, 1, false>(map, args, grid, overlap, st)
+                      : launch_variant<8, 2, false>(map, args, grid, overlap, st);
     }
 }
 
 }  // namespace
 
-// Stream-K plan.  Up to kCtasPerSm 4-warp CTAs are resident on an SM (the
-// ring of a CTA takes 36 KB (int4) or 48 KB (int8) of shared memory), and
-// the same number k runs on every SM.
-//   M = 1: a warp streams its ceil(U / W) K blocks one after another, and a
-//   block takes longer the more warps share an SM sub-partition: about
-//   (0.40 + 0.33 k) us with k CTAs per SM, fitted to the decode layers.  k
-//   minimises ceil(U / W) * (40 + 33 k); ties go to the smaller k.
-//   M > 1: the split-K partials grow with M, so k is the largest that gives
-//   each warp at least kGemvMinBlocksPerWarp blocks (fewer contributors).
-constexpr int kBlockCostBase = 40, kBlockCostPerCta = 33;
-constexpr int kGemvMinBlocksPerWarp = 4;
+// Stream-K plan.  Units are (128-row task x 128-wide K block); up to
+// kMaxCtasPerSm CTAs run on an SM (their rings take 74 KB (int4) or 66 KB
+// (int8) of shared memory each), and the same number k runs on every SM.
+// k is the largest that still gives each CTA at least kMinUnitsPerCta units
+// (more CTAs per SM keep more consumer warps issuing; fewer keep short
+// layers from splitting every task over many CTAs).
+constexpr int64_t kMinUnitsPerCta = 4;
 
 GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K, int bits, int sms) {
+    (void)bits;
     GemvPlan p{};
-    p.tasks = ceil_div(N, kRowsPerWarp);
-    p.kblocks = K / 128;
+    p.tasks = ceil_div(N, kTileRows);
+    p.kblocks = K / kBlockK;
     const int64_t units = p.tasks * p.kblocks;
-    const int64_t max_per_sm = M <= 8 ? (bits == 4 ? kCtasPerSm<4, 1> : kCtasPerSm<8, 1>)
-                                      : kCtasPerSm<4, 2>;
-    int64_t per_sm = 1;
-    if (M == 1) {
-        int64_t best_cost = -1;
-        for (int64_t k = 1; k <= max_per_sm; ++k) {
-            const int64_t cost = ceil_div(units, (int64_t)sms * kWarpsPerCta * k) *
-                                 (kBlockCostBase + kBlockCostPerCta * k);
-            if (best_cost < 0 || cost < best_cost) {
-                best_cost = cost;
-                per_sm = k;
-            }
-        }
-    } else {
-        per_sm = units / ((int64_t)sms * kWarpsPerCta * kGemvMinBlocksPerWarp);
-        if (per_sm > max_per_sm) per_sm = max_per_sm;
-        if (per_sm < 1) per_sm = 1;
-    }
-    p.warps = (int64_t)sms * per_sm * kWarpsPerCta;
-    // Fewer units than warps: one unit per warp.  Every warp must own at
-    // least one unit, or a split task would count a contributor that never
+    int64_t per_sm = kMaxCtasPerSm;
+    while (per_sm > 1 && units < (int64_t)sms * per_sm * kMinUnitsPerCta) --per_sm;
+    p.ctas = (int64_t)sms * per_sm;
+    // Fewer units than CTAs: one unit per CTA.  Every CTA must own at least
+    // one unit, or a split task would count a contributor that never
     // arrives.
-    if (p.warps > units) p.warps = units;
-    // contributors of one task: at most ceil(KB / floor(U/W)) + 1
-    const int64_t per_warp = units / p.warps;
-    p.slots = per_warp >= 1 ? ceil_div(p.kblocks, per_warp) + 1 : p.kblocks + 1;
+    if (p.ctas > units) p.ctas = units;
+    // contributors of one task: at most ceil(KB / floor(U/C)) + 1
+    const int64_t per_cta = units / p.ctas;
+    p.slots = per_cta >= 1 ? ceil_div(p.kblocks, per_cta) + 1 : p.kblocks + 1;
     if (p.slots > p.kblocks) p.slots = p.kblocks;
-    p.partial_bytes = (size_t)p.tasks * p.slots * (size_t)M * kRowsPerWarp * sizeof(float);
+    const int64_t subtasks = p.tasks * kConsumerWarps;
+    p.partial_bytes = (size_t)subtasks * p.slots * (size_t)M * kRowsPerWarp * sizeof(float);
     p.partial_bytes = (p.partial_bytes + 255) & ~(size_t)255;
-    p.counter_bytes = (size_t)ceil_div(p.tasks, 64) * 64 * sizeof(uint32_t);
+    p.counter_bytes = (size_t)ceil_div(subtasks, 64) * 64 * sizeof(uint32_t);
     p.total_bytes = p.partial_bytes + p.counter_bytes;
     return p;
 }
 
-// The plan's workspace is not monotone in the SM count (fewer SMs can pick
-// more CTAs per SM), so the size callers allocate is the largest over every
-// count up to kSmCount.
+// The plan's workspace is not monotone in the SM count, so the size callers
+// allocate is the largest over every count up to kSmCount.
 size_t gemv_workspace_bound(int64_t M, int64_t N, int64_t K, int bits) {
     size_t most = 0;
     for (int sms = 1; sms <= kSmCount; ++sms) {

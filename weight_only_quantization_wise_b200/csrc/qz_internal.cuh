@@ -91,19 +91,21 @@ qz_status launch_dequantize(const void *codes, const void *scales, const void *z
                             int64_t N, int64_t K, int bits, int symmetric,
                             int64_t group_size, void *w_hat, cudaStream_t stream);
 
-// GEMV work plan (stream-K): the (32-row task x 128-wide K block) units are
-// split into equal contiguous ranges, one per launched warp; a task whose
-// units span several warps is reduced through per-task partial slots.
+// GEMV work plan (stream-K): the (128-row task x 128-wide K block) units
+// are split into equal contiguous ranges, one per launched CTA; each of a
+// CTA's four consumer warps owns 32 rows of every unit (a subtask), and a
+// subtask whose units span several CTAs is reduced through per-subtask
+// partial slots.
 struct GemvPlan {
-    int64_t tasks;        // 32-row tasks
+    int64_t tasks;        // 128-row tasks
     int64_t kblocks;      // 128-wide K blocks per task
-    int64_t warps;        // launched warps (each owns at least one unit)
-    int64_t slots;        // partial slots per task (max contributors)
-    size_t partial_bytes; // fp32 partials [tasks][slots][M][32]
-    size_t counter_bytes; // uint32 arrival counter per task
+    int64_t ctas;         // launched CTAs (each owns at least one unit)
+    int64_t slots;        // partial slots per subtask (max contributors)
+    size_t partial_bytes; // fp32 partials [tasks * 4][slots][M][32]
+    size_t counter_bytes; // uint32 arrival counter per 32-row subtask
     size_t total_bytes;
 };
-// Workspace: fp32 partials at offset 0, then one uint32 counter per task.
+// Workspace: fp32 partials at offset 0, then one uint32 counter per subtask.
 // `sms`: the SMs the grid is sized for (device_sm_count() at launch).
 GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K, int bits, int sms);
 // Workspace bytes that serve the plan of every SM count up to kSmCount.
@@ -128,6 +130,13 @@ qz_status launch_w4a16_gemm(const void *a, const void *codes, const void *scales
                             cudaStream_t stream);
 qz_status launch_w8a16_gemm(const void *a, const void *codes, const void *scales, int64_t M,
                             int64_t N, int64_t K, void *y, void *workspace, cudaStream_t stream);
+
+// GPTQ (qz_gptq.cu): fp64 workspace of the damped Hessian factor, its
+// inverse, the working weights and one block of scaled errors.
+size_t gptq_workspace_bytes(int64_t N, int64_t K);
+qz_status launch_gptq(const void *w, const void *x, int64_t N, int64_t K, int64_t n_samples,
+                      int bits, int symmetric, int64_t group_size, double damp, void *codes,
+                      void *scales, void *zeros, void *workspace, cudaStream_t stream);
 
 uint64_t device_wait_limit();
 // qz_set_launch_overlap mode (0 or 1) for the decode GEMV launches.

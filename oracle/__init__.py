@@ -48,6 +48,16 @@ def load(path: str):
     L.qzo_gptq_quantize.argtypes = [_p, _p, _i64, _i64, _i64, ctypes.c_double, _i64, _int,
                                     _int, _i64, _p, _p, _p]
     L.qzo_gptq_quantize.restype = _int
+    L.qzo_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+    L.qzo_e4m3_to_f64.restype = ctypes.c_double
+    L.qzo_e2m1_to_f64.argtypes = [ctypes.c_uint8]
+    L.qzo_e2m1_to_f64.restype = ctypes.c_double
+    L.qzo_fp4_quantize.argtypes = [_p, _i64, _i64, _int, _p, _p, _p]
+    L.qzo_fp4_quantize.restype = _int
+    L.qzo_fp4_dequantize.argtypes = [_p, _p, _p, _i64, _i64, _int, _p, _p]
+    L.qzo_fp4_dequantize.restype = _int
+    L.qzo_matmul_f64_exact.argtypes = [_p, _p, _i64, _i64, _i64, _p, _p]
+    L.qzo_matmul_f64_exact.restype = _int
     L.qzo_set_threads.argtypes = [_int]
     L.qzo_set_threads.restype = None
     L.qzo_max_threads.argtypes = []
@@ -144,6 +154,56 @@ def dequantize(codes, scales, zeros, N: int, K: int, bits: int = 4,
     if rc != 0:
         raise ValueError("qzo_dequantize rejected the arguments")
     return out
+
+
+FP4_MX, FP4_NV = 0, 1                      # MXFP4 (block 32, E8M0), NVFP4 (block 16, E4M3)
+FP4_BLOCK = {FP4_MX: 32, FP4_NV: 16}
+
+
+def e4m3_to_f64(b: int) -> float:
+    return float(lib().qzo_e4m3_to_f64(int(b)))
+
+
+def e2m1_to_f64(code: int) -> float:
+    return float(lib().qzo_e2m1_to_f64(int(code)))
+
+
+def fp4_quantize(w, kind: int):
+    """FP4 with block scales: returns (codes uint8 N x K/2, block scales
+    uint8 N x K/block, tensor scale float (NVFP4) or None)."""
+    wf = _weights_f32(w)
+    N, K = wf.shape
+    codes = np.zeros((N, K // 2), dtype=np.uint8)
+    scales = np.zeros((N, K // FP4_BLOCK[kind]), dtype=np.uint8)
+    ts = np.zeros(1, dtype=np.float32)
+    if lib().qzo_fp4_quantize(_ptr(wf), N, K, kind, _ptr(codes), _ptr(scales), _ptr(ts)) != 0:
+        raise ValueError("qzo_fp4_quantize rejected the arguments")
+    return codes, scales, (float(ts[0]) if kind == FP4_NV else None)
+
+
+def fp4_dequantize(codes, scales, tensor_scale, N: int, K: int, kind: int):
+    """(bf16 bits of the dequantized weights, their exact values in fp64)."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    ts = np.array([tensor_scale if tensor_scale is not None else 1.0], dtype=np.float32)
+    w_hat = np.zeros((N, K), dtype=np.uint16)
+    w_exact = np.zeros((N, K), dtype=np.float64)
+    if lib().qzo_fp4_dequantize(_ptr(codes), _ptr(scales), _ptr(ts), N, K, kind, _ptr(w_hat),
+                                _ptr(w_exact)) != 0:
+        raise ValueError("qzo_fp4_dequantize rejected the arguments")
+    return w_hat, w_exact
+
+
+def matmul_f64_exact(a_bits, w_exact):
+    """fp64 y = a @ w^T and sum_k |a w| for bf16 activations and fp64 weights."""
+    a = np.ascontiguousarray(a_bits, dtype=np.uint16)
+    w = np.ascontiguousarray(w_exact, dtype=np.float64)
+    M, K = a.shape
+    N = w.shape[0]
+    y = np.zeros((M, N), dtype=np.float64)
+    ya = np.zeros((M, N), dtype=np.float64)
+    lib().qzo_matmul_f64_exact(_ptr(a), _ptr(w), M, N, K, _ptr(y), _ptr(ya))
+    return y, ya
 
 
 GPTQ_BLOCK = 128      # the GPTQ explainer's lazy-batch width

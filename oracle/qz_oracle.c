@@ -314,6 +314,198 @@ int qzo_matmul_f64(const uint16_t *a, const uint16_t *w_hat, int64_t M, int64_t 
 }
 
 /* ------------------------------------------------------------------ */
+/* FP4 with block scales (quantization concepts guide, section "FP4 with */
+/* block scales"; the FP8 section for E4M3).                              */
+/*   E2M1: 1 sign, 2 exponent, 1 mantissa bit; the magnitudes 0, 0.5, 1,  */
+/*   1.5, 2, 3, 4, 6 (codes 0..7 in that order, sign in bit 3).           */
+/*   MXFP4: a power-of-two scale per block (only the exponent shifts).    */
+/*   NVFP4: smaller blocks with an FP8 (E4M3) scale, plus one scale for   */
+/*   the tensor that keeps the block scales in range.                     */
+/* Readings (the page gives no block sizes and no rule for choosing a     */
+/* scale):                                                                */
+/*   - MXFP4 blocks are 32 values, NVFP4 blocks 16 (NVFP4's are the       */
+/*     smaller), consecutive along a row;                                 */
+/*   - MXFP4 scale: 2^e with e the smallest integer such that             */
+/*     max|x| / 2^e <= 6 (no value saturates), clamped to [-127, 127],    */
+/*     stored as the E8M0 byte e + 127; an all-zero block has e = -127;   */
+/*   - NVFP4 tensor scale: s_t = fp32(amax / 2688) (2688 = 6 x 448, the    */
+/*     largest E2M1 value times the largest E4M3 value), 1 for an all-    */
+/*     zero tensor; block scale: the smallest E4M3 value >= fp32(amax_b / */
+/*     fp32(6 s_t)) (rounded up, like the bf16 scales of the integer      */
+/*     formats), at most 448, 0 for an all-zero block;                    */
+/*   - element codes: x divided by the block's effective scale (2^e, or    */
+/*     fp32(E4M3(s_b) x s_t)) in fp32, then rounded to the nearest E2M1   */
+/*     magnitude, ties to the even mantissa bit, saturating at 6;          */
+/*   - dequantized weight (bf16 output): MXFP4 e2m1 x 2^e; NVFP4           */
+/*     bf16_rne(fp32(fp32(e2m1 x E4M3(s_b)) x s_t)) (the inner product is  */
+/*     exact);                                                            */
+/*   - the matmul reference uses the exact product e2m1 x scale(s) in fp64.*/
+/* ------------------------------------------------------------------ */
+
+static const double e2m1_mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+/* Nearest E2M1 code (sign in bit 3) of v, ties to the even mantissa bit
+ * (codes with an even index), saturating at 6. */
+static uint8_t e2m1_code(float v)
+{
+    double a = fabs((double)v);
+    int best = 0;
+    for (int i = 1; i < 8; ++i) {
+        double di = fabs(a - e2m1_mag[i]), db = fabs(a - e2m1_mag[best]);
+        if (di < db || (di == db && (i % 2) == 0 && (best % 2) == 1)) best = i;
+    }
+    if (a > 6.0) best = 7;
+    uint8_t code = (uint8_t)best;
+    if (v < 0.0f && best != 0) code |= 0x8;
+    return code;
+}
+
+/* E4M3 (FP8, 4 exponent bits with bias 7, 3 mantissa bits, finite max 448)
+ * byte -> value. */
+double qzo_e4m3_to_f64(uint8_t b)
+{
+    int s = (b >> 7) & 1, e = (b >> 3) & 0xF, m = b & 7;
+    double v = (e == 0) ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* The smallest non-negative E4M3 value >= t (t >= 0), capped at 448. */
+static uint8_t e4m3_round_up(float t)
+{
+    if (!(t > 0.0f)) return 0;
+    for (int b = 1; b <= 0x7E; ++b)               /* 0x7E = 448, 0x7F is NaN */
+        if (qzo_e4m3_to_f64((uint8_t)b) >= (double)t) return (uint8_t)b;
+    return 0x7E;
+}
+
+double qzo_e2m1_to_f64(uint8_t code)
+{
+    double v = e2m1_mag[code & 7];
+    return (code & 8) ? -v : v;
+}
+
+/* kind 0 = MXFP4 (block 32, E8M0), 1 = NVFP4 (block 16, E4M3 + tensor scale). */
+static int fp4_block(int kind) { return kind == 0 ? 32 : 16; }
+
+int qzo_fp4_quantize(const float *w, int64_t N, int64_t K, int kind, uint8_t *codes,
+                     uint8_t *block_scales, float *tensor_scale)
+{
+    if ((kind != 0 && kind != 1) || N < 1 || K < 1) return -1;
+    const int bs = fp4_block(kind);
+    if (K % bs != 0) return -1;
+    float s_t = 1.0f;
+    if (kind == 1) {
+        float amax = 0.0f;
+        for (int64_t i = 0; i < N * K; ++i)
+            if (fabsf(w[i]) > amax) amax = fabsf(w[i]);
+        s_t = amax > 0.0f ? amax / 2688.0f : 1.0f;
+        *tensor_scale = s_t;
+    }
+    const int64_t bpr = K / bs;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t b = 0; b < bpr; ++b) {
+            const float *x = &w[n * K + b * bs];
+            float amax = 0.0f;
+            for (int i = 0; i < bs; ++i)
+                if (fabsf(x[i]) > amax) amax = fabsf(x[i]);
+            float scale;
+            uint8_t sb;
+            if (kind == 0) {
+                int e = -127;
+                if (amax > 0.0f) {
+                    e = (int)floor(log2((double)amax / 6.0)) - 1;
+                    while ((double)amax > 6.0 * ldexp(1.0, e)) ++e;   /* smallest e */
+                    if (e < -127) e = -127;
+                    if (e > 127) e = 127;
+                }
+                sb = (uint8_t)(e + 127);
+                scale = (float)ldexp(1.0, e);
+            } else {
+                float t = amax / (6.0f * s_t);
+                sb = e4m3_round_up(t);
+                scale = (float)qzo_e4m3_to_f64(sb) * s_t;
+            }
+            block_scales[n * bpr + b] = sb;
+            for (int i = 0; i < bs; ++i) {
+                const int64_t k = b * bs + i;
+                uint8_t c = scale > 0.0f ? e2m1_code(x[i] / scale) : 0;
+                uint8_t *byte = &codes[n * (K / 2) + k / 2];
+                if ((k & 1) == 0) *byte = (uint8_t)((*byte & 0xF0) | c);
+                else              *byte = (uint8_t)((*byte & 0x0F) | (c << 4));
+            }
+        }
+    }
+    return 0;
+}
+
+/* Exact dequantized value (fp64) of element (n, k), and its bf16 output. */
+static double fp4_value(const uint8_t *codes, const uint8_t *block_scales, float s_t,
+                        int64_t K, int kind, int64_t n, int64_t k)
+{
+    const int bs = fp4_block(kind);
+    uint8_t byte = codes[n * (K / 2) + k / 2];
+    uint8_t c = (k & 1) ? (byte >> 4) : (byte & 0xF);
+    uint8_t sb = block_scales[n * (K / bs) + k / bs];
+    double q = qzo_e2m1_to_f64(c);
+    if (kind == 0) return q * ldexp(1.0, (int)sb - 127);
+    return q * qzo_e4m3_to_f64(sb) * (double)s_t;
+}
+
+int qzo_fp4_dequantize(const uint8_t *codes, const uint8_t *block_scales, const float *tensor_scale,
+                       int64_t N, int64_t K, int kind, uint16_t *w_hat, double *w_exact)
+{
+    if ((kind != 0 && kind != 1) || N < 1 || K < 1 || K % fp4_block(kind) != 0) return -1;
+    const float s_t = kind == 1 ? *tensor_scale : 1.0f;
+    const int bs = fp4_block(kind);
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            if (w_exact) w_exact[n * K + k] = fp4_value(codes, block_scales, s_t, K, kind, n, k);
+            if (w_hat) {
+                uint8_t byte = codes[n * (K / 2) + k / 2];
+                uint8_t c = (k & 1) ? (byte >> 4) : (byte & 0xF);
+                uint8_t sb = block_scales[n * (K / bs) + k / bs];
+                float v;
+                if (kind == 0) {
+                    v = (float)(qzo_e2m1_to_f64(c) * ldexp(1.0, (int)sb - 127));
+                } else {
+                    float p = (float)qzo_e2m1_to_f64(c) * (float)qzo_e4m3_to_f64(sb);  /* exact */
+                    v = p * s_t;
+                }
+                w_hat[n * K + k] = qzo_f32_to_bf16_rne(v);
+            }
+        }
+    return 0;
+}
+
+/* fp64 reference matmul over exact dequantized weights (N x K fp64):
+ * y[m][n] = sum_k a[m][k] w[n][k] and sum_k |a w|. */
+int qzo_matmul_f64_exact(const uint16_t *a, const double *w, int64_t M, int64_t N, int64_t K,
+                         double *y, double *abs_y)
+{
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t m = 0; m < M; ++m) {
+            double acc = 0.0, acc_abs = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double p = (double)qzo_bf16_to_f32(a[m * K + k]) * w[n * K + k];
+                acc += p;
+                acc_abs += fabs(p);
+            }
+            y[m * N + n] = acc;
+            abs_y[m * N + n] = acc_abs;
+        }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
 /* GPTQ layer-wise quantizer (GPTQ explainer, azimuth.plus/paper/gptq).  */
 /*                                                                        */
 /* The page's steps, in its order:                                        */
@@ -353,7 +545,8 @@ int qzo_matmul_f64(const uint16_t *a, const uint16_t *w_hat, int64_t M, int64_t 
 
 /* In-place Cholesky A = L L^T of an n x n symmetric positive definite
  * matrix (row-major fp64); on return the lower triangle holds L and the
- * strict upper triangle is zero.  Returns -1 if A is not positive definite. */
+ * strict upper triangle is zero.  Returns -1 if A is not positive definite.
+ * (Rows below the pivot are independent: OpenMP over them.) */
 static int cholesky_lower(double *A, int64_t n)
 {
     for (int64_t j = 0; j < n; ++j) {
@@ -362,6 +555,9 @@ static int cholesky_lower(double *A, int64_t n)
         if (!(d > 0.0)) return -1;
         double ljj = sqrt(d);
         A[j * n + j] = ljj;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
         for (int64_t i = j + 1; i < n; ++i) {
             double v = A[i * n + j];
             for (int64_t k = 0; k < j; ++k) v -= A[i * n + k] * A[j * n + k];
@@ -373,44 +569,62 @@ static int cholesky_lower(double *A, int64_t n)
 }
 
 /* Inverse of an SPD matrix from its Cholesky factor: A^-1 = L^-T L^-1.
- * Li = L^-1 by forward substitution, then the product. */
+ * L^-1 by forward substitution, one column c at a time (stored transposed:
+ * LiT[c][i] = (L^-1)[i][c], so the sums run over contiguous memory), then
+ * the product (A^-1)[i][j] = sum_k (L^-1)[k][i] (L^-1)[k][j]. */
 static void spd_inverse_from_cholesky(const double *L, double *Ainv, int64_t n)
 {
-    double *Li = (double *)calloc((size_t)(n * n), sizeof(double));
+    double *LiT = (double *)calloc((size_t)(n * n), sizeof(double));
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 8)
+#endif
     for (int64_t c = 0; c < n; ++c) {             /* column c of L^-1 */
+        double *col = &LiT[c * n];
         for (int64_t i = c; i < n; ++i) {
             double v = (i == c) ? 1.0 : 0.0;
-            for (int64_t k = c; k < i; ++k) v -= L[i * n + k] * Li[k * n + c];
-            Li[i * n + c] = v / L[i * n + i];
+            for (int64_t k = c; k < i; ++k) v -= L[i * n + k] * col[k];
+            col[i] = v / L[i * n + i];
         }
     }
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 8)
+#endif
     for (int64_t i = 0; i < n; ++i)
         for (int64_t j = 0; j < n; ++j) {
             double v = 0.0;
             int64_t k0 = i > j ? i : j;
-            for (int64_t k = k0; k < n; ++k) v += Li[k * n + i] * Li[k * n + j];
+            for (int64_t k = k0; k < n; ++k) v += LiT[i * n + k] * LiT[j * n + k];
             Ainv[i * n + j] = v;
         }
-    free(Li);
+    free(LiT);
 }
 
-/* Upper Cholesky factor: A = U^T U (U upper, positive diagonal). */
+/* Upper Cholesky factor: A = U^T U (U upper, positive diagonal).  Built in
+ * the transposed array UT[j][i] = U[i][j] so the sums are contiguous. */
 static int cholesky_upper(const double *A, double *U, int64_t n)
 {
-    for (int64_t i = 0; i < n; ++i) {
+    double *UT = (double *)calloc((size_t)(n * n), sizeof(double));
+    if (!UT) return -1;
+    int rc = 0;
+    for (int64_t i = 0; i < n && rc == 0; ++i) {
         double d = A[i * n + i];
-        for (int64_t k = 0; k < i; ++k) d -= U[k * n + i] * U[k * n + i];
-        if (!(d > 0.0)) return -1;
+        for (int64_t k = 0; k < i; ++k) d -= UT[i * n + k] * UT[i * n + k];
+        if (!(d > 0.0)) { rc = -1; break; }
         double uii = sqrt(d);
-        U[i * n + i] = uii;
+        UT[i * n + i] = uii;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
         for (int64_t j = i + 1; j < n; ++j) {
             double v = A[i * n + j];
-            for (int64_t k = 0; k < i; ++k) v -= U[k * n + i] * U[k * n + j];
-            U[i * n + j] = v / uii;
+            for (int64_t k = 0; k < i; ++k) v -= UT[i * n + k] * UT[j * n + k];
+            UT[j * n + i] = v / uii;
         }
-        for (int64_t j = 0; j < i; ++j) U[i * n + j] = 0.0;
     }
-    return 0;
+    for (int64_t i = 0; i < n; ++i)
+        for (int64_t j = 0; j < n; ++j) U[i * n + j] = j >= i ? UT[j * n + i] : 0.0;
+    free(UT);
+    return rc;
 }
 
 /* The damped Hessian H = 2 X X^T + lambda I and the upper Cholesky factor U

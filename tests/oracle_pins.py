@@ -523,4 +523,141 @@ def pin_gptq_lowers_the_layer_error():
         assert errs[0] < 0.5 * errs[1], errs
 
 
+
+
+# --------------------------------------------------------------------------
+# FP4 with block scales (guide, section "FP4 with block scales")
+# --------------------------------------------------------------------------
+
+E2M1_PAGE_VALUES = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def pin_e2m1_values_and_layout():
+    """Every code decodes to the page's list of values, and to the value the
+    stated layout (1 sign, 2 exponent, 1 mantissa bit; exponent bias 1,
+    subnormal when the exponent field is 0) gives."""
+    for code in range(16):
+        s, e, m = code >> 3, (code >> 1) & 3, code & 1
+        layout = (m * 0.5) if e == 0 else 2.0 ** (e - 1) * (1 + m / 2)
+        layout = -layout if s else layout
+        v = oracle.e2m1_to_f64(code)
+        assert v == layout, (code, v, layout)
+        assert abs(v) == E2M1_PAGE_VALUES[code & 7]
+
+
+def pin_e4m3_matches_torch():
+    """E4M3 (guide, FP8 section: 4 exponent bits, 3 mantissa bits) decodes
+    like torch's float8_e4m3fn for every finite byte."""
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    for b in range(256):
+        if np.isnan(ref[b]):
+            continue
+        assert oracle.e4m3_to_f64(b) == ref[b], b
+
+
+def _fp4_blocks(w, codes, scales, ts, kind):
+    N, K = w.shape
+    bs = oracle.FP4_BLOCK[kind]
+    x = oracle.bf16_bits_to_f32(w).astype(np.float64) if w.dtype == np.uint16 else w.astype(np.float64)
+    q = np.zeros((N, K), np.float64)
+    lo, hi = codes & 0xF, codes >> 4
+    cod = np.empty((N, K), np.uint8)
+    cod[:, 0::2], cod[:, 1::2] = lo, hi
+    table = np.array([oracle.e2m1_to_f64(c) for c in range(16)])
+    q = table[cod]
+    if kind == oracle.FP4_MX:
+        scale = np.ldexp(1.0, scales.astype(np.int64) - 127)
+    else:
+        e4 = torch.from_numpy(scales.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+        scale = (e4.astype(np.float32) * np.float32(ts)).astype(np.float64)   # fp32 product
+    return x.reshape(N, K // bs, bs), q.reshape(N, K // bs, bs), scale, cod.reshape(N, K // bs, bs)
+
+
+def pin_fp4_scales():
+    """MXFP4: the scale is a power of two (E8M0, read by torch), the smallest
+    that keeps the block's max |x| within 6.  NVFP4: s_t = amax / (6 x 448)
+    and the block scale the smallest E4M3 value >= amax_b / (6 s_t)."""
+    w = _random_bf16((24, 256), 0.02, 700)
+    codes, scales, ts = oracle.fp4_quantize(w, oracle.FP4_MX)
+    x, _, _, _ = _fp4_blocks(w, codes, scales, ts, oracle.FP4_MX)
+    e8 = torch.from_numpy(scales.copy()).view(torch.float8_e8m0fnu).to(torch.float64).numpy()
+    amax = np.abs(x).max(axis=-1)
+    assert (amax <= 6 * e8).all() and (amax > 3 * e8).all()
+    codes, scales, ts = oracle.fp4_quantize(w, oracle.FP4_NV)
+    x, _, _, _ = _fp4_blocks(w, codes, scales, ts, oracle.FP4_NV)
+    amax_t = np.float32(np.abs(x).max())
+    assert ts == float(amax_t / np.float32(2688.0))
+    e4 = torch.from_numpy(scales.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    grid = np.sort(np.unique(torch.arange(0, 127, dtype=torch.uint8).view(torch.float8_e4m3fn)
+                             .to(torch.float64).numpy()))
+    t = (np.abs(x).max(axis=-1).astype(np.float32) / np.float32(6.0 * np.float32(ts))).astype(np.float64)
+    idx = np.searchsorted(grid, t, side="left")           # first grid value >= t
+    assert np.array_equal(e4, grid[np.minimum(idx, len(grid) - 1)])
+
+
+def pin_fp4_codes_nearest_and_roundtrip():
+    """Every code is the nearest E2M1 value to x / scale (exact arithmetic,
+    ties to the even mantissa bit), so |x - q scale| is at most half the gap
+    between neighbouring E2M1 values times the scale."""
+    w = _random_bf16((16, 512), 0.02, 710)
+    vals = np.array(E2M1_PAGE_VALUES)
+    for kind in (oracle.FP4_MX, oracle.FP4_NV):
+        codes, scales, ts = oracle.fp4_quantize(w, kind)
+        x, q, scale, cod = _fp4_blocks(w, codes, scales, ts, kind)
+        u = x / scale[..., None]
+        for i in np.ndindex(u.shape):
+            a = abs(u[i])
+            d = np.abs(vals - a)
+            order = np.argsort(d, kind="stable")
+            if d[order[1]] - d[order[0]] > 1e-6:
+                assert abs(q[i]) == vals[order[0]], (kind, i, u[i], q[i])
+            if a != 0 and q[i] != 0:
+                assert np.sign(q[i]) == np.sign(u[i])
+        gap = np.where(np.abs(q) < 2, 0.5, np.where(np.abs(q) < 4, 1.0, 2.0))
+        assert (np.abs(u - q) <= gap / 2 + 1e-9).all()
+
+
+def pin_fp4_ties_to_even():
+    """x / scale exactly half-way: 0.25 -> 0, 0.75 -> 1, 1.25 -> 1, 1.75 -> 2,
+    2.5 -> 2, 3.5 -> 4, 5 -> 4 (MXFP4 block with max 6 so the scale is 1)."""
+    row = np.zeros((1, 32), np.float32)
+    row[0, :8] = [6.0, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]
+    codes, scales, _ = oracle.fp4_quantize(row, oracle.FP4_MX)
+    assert scales[0, 0] == 127                                  # 2^0
+    got = [oracle.e2m1_to_f64((codes[0, k // 2] >> (4 * (k % 2))) & 0xF) for k in range(8)]
+    assert got == [6.0, 0.0, 1.0, 1.0, 2.0, 2.0, 4.0, 4.0], got
+
+
+def pin_fp4_sizes():
+    """Half a byte per weight plus one scale byte per block: 4.25 bits per
+    weight for MXFP4, 4.5 for NVFP4 (plus one fp32 per tensor)."""
+    N, K = 8, 256
+    w = _random_bf16((N, K), 0.02, 720)
+    for kind, bits in ((oracle.FP4_MX, 4.25), (oracle.FP4_NV, 4.5)):
+        codes, scales, _ = oracle.fp4_quantize(w, kind)
+        assert (codes.size + scales.size) * 8 / (N * K) == bits
+
+
+def pin_fp4_dequant_closed_form():
+    """The bf16 output is torch's bf16 rounding of the fp32 value of the
+    definition; the exact values are code x scale(s)."""
+    w = _random_bf16((8, 256), 0.02, 730)
+    for kind in (oracle.FP4_MX, oracle.FP4_NV):
+        codes, scales, ts = oracle.fp4_quantize(w, kind)
+        w_hat, w_exact = oracle.fp4_dequantize(codes, scales, ts, 8, 256, kind)
+        x, q, scale, _ = _fp4_blocks(w, codes, scales, ts, kind)
+        if kind == oracle.FP4_MX:
+            v32 = (q * scale[..., None]).astype(np.float32)
+            exact = q * scale[..., None]
+        else:
+            e4 = torch.from_numpy(scales.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+            p = (q * e4[..., None]).astype(np.float32)                      # exact
+            v32 = (p * np.float32(ts)).astype(np.float32)
+            exact = q * e4[..., None] * np.float64(np.float32(ts))
+        ref = torch.from_numpy(v32.reshape(8, 256)).to(torch.bfloat16).view(torch.int16).numpy()
+        assert np.array_equal(w_hat, ref.view(np.uint16))
+        assert np.array_equal(w_exact, exact.reshape(8, 256))
+
+
+# every pin_* function of this module (defined last, after all of them)
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -56,6 +56,16 @@ MUTANTS = {
                                "for (int64_t k = j + 1; k < end; ++k) W[k] -= e * U[k * K + j];"),
     "gptq_group_scale_from_original_weights": ("for (int64_t k = 0; k < g; ++k) grp[k] = (float)W[j + k];",
                                                "for (int64_t k = 0; k < g; ++k) grp[k] = w[n * K + j + k];"),
+    # FP4 with block scales
+    "fp4_ties_away_from_zero": ("if (di < db || (di == db && (i % 2) == 0 && (best % 2) == 1)) best = i;",
+                                "if (di <= db) best = i;"),
+    "fp4_mx_scale_one_too_small": ("while ((double)amax > 6.0 * ldexp(1.0, e)) ++e;   /* smallest e */",
+                                   "while ((double)amax > 12.0 * ldexp(1.0, e)) ++e;"),
+    "fp4_nv_scale_rounded_down": ("if (qzo_e4m3_to_f64((uint8_t)b) >= (double)t) return (uint8_t)b;",
+                                  "if (qzo_e4m3_to_f64((uint8_t)b) > (double)t) return (uint8_t)(b - 1);"),
+    "fp4_nv_tensor_scale_without_fp8_range": ("s_t = amax > 0.0f ? amax / 2688.0f : 1.0f;",
+                                              "s_t = amax > 0.0f ? amax / 6.0f : 1.0f;"),
+    "fp4_e4m3_bias_off_by_one": ("ldexp(1.0 + m / 8.0, e - 7)", "ldexp(1.0 + m / 8.0, e - 8)"),
     "gptq_no_damping": ("double lambda = mean > 0.0 ? damp * mean : 1.0;",
                         "double lambda = mean > 0.0 ? 0.0 : 1.0;"),
 }

@@ -86,6 +86,30 @@ def gemm_flops(M, N, K):
     return 2 * M * N * K
 
 
+FP4_BLOCK = {0: 32, 1: 16}     # MXFP4, NVFP4 values per block scale
+
+
+def fp4_gemv_bytes(M, N, K, kind):
+    return N * K // 2 + N * K // FP4_BLOCK[kind] + (4 if kind == 1 else 0) + 2 * M * K + 2 * M * N
+
+
+def fp4_quant_bytes(N, K, kind):
+    return 2 * N * K + N * K // 2 + N * K // FP4_BLOCK[kind]
+
+
+def gptq_flops(N, K, n):
+    """fp64 flops of one GPTQ call: H = 2 X X^T (2 n K^2), the Cholesky of the
+    damped H (K^3 / 3), the triangular inverse (K^3 / 3), the in-block and
+    lazy weight updates (2 N K^2 / 2 each way: N K^2 in all, 2 per FMA)."""
+    return 2 * n * K * K + (2 * K ** 3) // 3 + 2 * N * K * K
+
+
+# fp64 peak of a B200 derived from its unit counts and clock (the pages and
+# the measured-peaks file give none): 148 SMs x 64 fp64 FMA lanes x 2 flops
+# x 1.965 GHz.
+FP64_PEAK_TFLOPS = 148 * 64 * 2 * 1.965e9 / 1e12
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -339,6 +363,14 @@ def roofline_obj(part, work, ms_per_launch_set, launches, bound, pk, traffic, su
             "algorithmic": work, "launches": launches}
 
 
+def qz_gemm_kernel_for(M):
+    """Which kernel qz_w4a16_gemm / qz_w8a16_gemm run for M tokens."""
+    return "decode GEMV" if M <= GEMM_ROUTES_TO_GEMV_UP_TO else "tcgen05 GEMM"
+
+
+GEMM_ROUTES_TO_GEMV_UP_TO = 16
+
+
 def run_extras(qz, dev, pk, stream):
     """Configurations outside the step, each timed with CUDA events on graphs."""
     out = {}
@@ -415,8 +447,30 @@ def run_extras(qz, dev, pk, stream):
             ms4 = time_graph(capture(f4, stream)) / len(packs4)
             ms8 = time_graph(capture(f8, stream)) / len(packs8)
             b4, b8 = w4_gemv_bytes(Ms, N, K), w8_gemv_bytes(Ms, N, K)
+            if 16 < Ms <= 64:
+                # the same tokens through the decode GEMV (up to 64 tokens)
+                wsg = torch.zeros(max(256, qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMV, Ms, N, K,
+                                                                 GROUP),
+                                      qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMV, Ms, N, K, K)),
+                                  dtype=torch.uint8, device=dev)
+
+                def g4():
+                    for c, s, z in packs4:
+                        qz.qz_w4a16_gemv(a, c, s, z, N, K, GROUP, y=y, workspace=wsg)
+
+                def g8():
+                    for c, s, _ in packs8:
+                        qz.qz_w8a16_gemv(a, c, s, N, K, y=y, workspace=wsg)
+
+                g4(); g8()
+                gm4 = time_graph(capture(g4, stream)) / len(packs4)
+                gm8 = time_graph(capture(g8, stream)) / len(packs8)
+                sweep[f"M{Ms}_decode_gemv"] = {
+                    "w4_us": round(gm4 * 1e3, 2), "w4_frac_hbm": round(b4 / gm4 / 1e6 / pk["hbm_gbs"], 4),
+                    "w8_us": round(gm8 * 1e3, 2), "w8_frac_hbm": round(b8 / gm8 / 1e6 / pk["hbm_gbs"], 4)}
+                del wsg
             sweep[f"M{Ms}"] = {
-                "kernel": "decode GEMV" if Ms <= 16 else "tcgen05 GEMM",
+                "kernel": qz_gemm_kernel_for(Ms),
                 "w4_us": round(ms4 * 1e3, 2), "w4_GB/s": round(b4 / ms4 / 1e6, 1),
                 "w4_frac_hbm": round(b4 / ms4 / 1e6 / pk["hbm_gbs"], 4),
                 "w4_TFLOP/s": round(gemm_flops(Ms, N, K) / (ms4 * 1e-3) / 1e12, 1),
@@ -459,6 +513,68 @@ def run_extras(qz, dev, pk, stream):
             del packs4, packs8
         out["decode_70b"] = d70
 
+        # FP4 with block scales (MXFP4, NVFP4) on the 70B decode layers, M = 1
+        # and 16, weights rotating over two copies; the quantizer on the same
+        # layers
+        fp4 = {}
+        for li, (N, K) in enumerate(synthetic.DECODE_70B):
+            w = synthetic.weights(N, K, sigma=0.015, seed=4 + li, device=dev)
+            for kind, name in ((0, "mxfp4"), (1, "nvfp4")):
+                packs = [qz.qz_fp4_quantize(w if r == 0 else w.clone(), kind) for r in range(2)]
+                c0, s0, t0 = packs[0]
+
+                def fq():
+                    qz.qz_fp4_quantize(w, kind, codes=c0, scales=s0, tensor_scale=t0)
+
+                fq()
+                msq = time_graph(capture(fq, stream))
+                qb = fp4_quant_bytes(N, K, kind)
+                fp4[f"{name}_quantize_N{N}_K{K}"] = {
+                    "us": round(msq * 1e3, 2), "GB/s": round(qb / msq / 1e6, 1),
+                    "frac_hbm": round(qb / msq / 1e6 / pk["hbm_gbs"], 4)}
+                for M in (1, 16):
+                    a = synthetic.activations(M, K, seed=M, device=dev)
+                    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+                    ws = torch.zeros(max(256, qz.qz_workspace_bytes(qz.QZ_OP_FP4A16_GEMV, M, N, K,
+                                                                    0)),
+                                     dtype=torch.uint8, device=dev)
+
+                    def fg():
+                        for c, sc, ts in packs:
+                            qz.qz_fp4a16_gemv(a, c, sc, ts, N, K, kind, y=y, workspace=ws)
+
+                    fg()
+                    ms = time_graph(capture(fg, stream)) / len(packs)
+                    b = fp4_gemv_bytes(M, N, K, kind)
+                    fp4[f"{name}_gemv_N{N}_K{K}_M{M}"] = {
+                        "us": round(ms * 1e3, 2), "GB/s": round(b / ms / 1e6, 1),
+                        "frac_hbm": round(b / ms / 1e6 / pk["hbm_gbs"], 4)}
+                del packs, c0, s0, t0
+            del w
+        out["fp4_decode_70b"] = fp4
+
+        # GPTQ of one 7B-class layer (4096 x 4096), 128 calibration samples
+        N, K, n = 4096, 4096, 128
+        w = synthetic.weights(N, K, sigma=0.02, seed=1, device=dev)
+        x = synthetic.activations(n, K, seed=77, device=dev)
+        gws = torch.empty(qz.qz_workspace_bytes(qz.QZ_OP_GPTQ, 1, N, K, GROUP), dtype=torch.uint8,
+                          device=dev)
+        gc, gsc, gz = qz.qz_gptq_quantize(w, x, 4, False, GROUP, workspace=gws)
+
+        def fgptq():
+            qz.qz_gptq_quantize(w, x, 4, False, GROUP, codes=gc, scales=gsc, zeros=gz,
+                                workspace=gws)
+
+        fgptq()
+        ms = time_graph(capture(fgptq, stream), reps=5, warm=1)
+        fl = gptq_flops(N, K, n)
+        out["gptq_4096x4096"] = {
+            "ms": round(ms, 3), "fp64_GFLOP/s": round(fl / (ms * 1e-3) / 1e9, 1),
+            "frac_fp64_peak": round(fl / (ms * 1e-3) / 1e12 / FP64_PEAK_TFLOPS, 4),
+            "fp64_peak_TFLOP/s_derived": round(FP64_PEAK_TFLOPS, 2),
+            "calibration_samples": n}
+        del w, x, gws, gc, gsc, gz
+
         # bulk quantization: 32 layer sets, 7.785e9 parameters
         total_params, b4, b8 = 0, 0, 0
         for N, K in synthetic.BULK_LAYER_SET:
@@ -499,6 +615,9 @@ def run_extras(qz, dev, pk, stream):
             "int8_pc_ms": round(ms8, 3), "int8_pc_GB/s": round(b8 * sets / ms8 / 1e6, 1),
             "int8_frac_hbm": round(b8 * sets / ms8 / 1e6 / pk["hbm_gbs"], 4)}
         del layers, outs4, outs8
+    torch.cuda.synchronize()
+    # a bounded device-side wait that ran out makes every figure above void
+    assert qz.qz_device_status() == 0, "a bounded device-side wait ran out in the extras"
     torch.cuda.empty_cache()
     return out
 
@@ -639,6 +758,9 @@ PROFILE_CASES = {
     "gemm8_prefill": ("gemm8", 2048, 8192, 8192),
     "gemm_m32": ("gemm", 32, 8192, 8192),
     "quant_int4": ("quant4", 0, 28672, 8192),
+    "gemv_nvfp4_70b": ("gemv_nv", 1, 28672, 8192),
+    "gemv_mxfp4_70b": ("gemv_mx", 1, 28672, 8192),
+    "gptq_4096": ("gptq", 128, 4096, 4096),
     "quant_int8": ("quant8", 0, 28672, 8192),
     "dequant_int4": ("dequant", 0, 28672, 8192),
 }
@@ -656,6 +778,9 @@ def run_kernel_case(name, reps):
         c, s, z = qz.qz_quantize_pack(w, 4, False, GROUP)
     if kind in ("gemv8", "gemm8"):
         c, s, _ = qz.qz_quantize_pack(w, 8, True, K)
+    if kind in ("gemv_nv", "gemv_mx"):
+        fk = qz.QZ_FP4_NV if kind == "gemv_nv" else qz.QZ_FP4_MX
+        c, s, ts = qz.qz_fp4_quantize(w, fk)
     a = synthetic.activations(max(M, 1), K, seed=5, device=dev)
     torch.cuda.synchronize()
     for _ in range(reps):
@@ -673,6 +798,11 @@ def run_kernel_case(name, reps):
             qz.qz_quantize_pack(w, 8, True, K)
         elif kind == "dequant":
             qz.qz_dequantize(c, s, z, N, K, 4, False, GROUP)
+        elif kind in ("gemv_nv", "gemv_mx"):
+            qz.qz_fp4a16_gemv(a, c, s, ts, N, K, fk, workspace=ws)
+        elif kind == "gptq":
+            x = synthetic.activations(M, K, seed=77, device=dev)
+            qz.qz_gptq_quantize(w, x, 4, False, GROUP)
     torch.cuda.synchronize()
     assert qz.qz_device_status() == 0
     print(f"{name}: {reps} launches ok")
@@ -834,13 +964,23 @@ def main():
     h2d = host_a_all.numel() * 2
     d2h = host_y_all.numel() * 2
 
+    def e2e_body(p):
+        dev_a_all.copy_(host_a_all, non_blocking=True)
+        for li, (N, K) in enumerate(LAYERS):
+            qz.qz_w4a16_gemv(dev_a[li], ls.c4[p][li], ls.s4[p][li], ls.z4[p][li], N, K, GROUP,
+                             y=dev_y[li], workspace=ls.ws)
+        host_y_all.copy_(dev_y_all, non_blocking=True)
+
+    # each decode step (copy in, the three GEMVs through the public API, copy
+    # out) is one captured CUDA graph, replayed and waited for on the host
+    with torch.cuda.stream(stream):
+        e2e_body(0)
+    stream.synchronize()
+    e2e_graphs = [capture(lambda p=p: e2e_body(p), stream) for p in range(ROT)]
+
     def e2e_step(p):
         with torch.cuda.stream(stream):
-            dev_a_all.copy_(host_a_all, non_blocking=True)
-            for li, (N, K) in enumerate(LAYERS):
-                qz.qz_w4a16_gemv(dev_a[li], ls.c4[p][li], ls.s4[p][li], ls.z4[p][li], N, K, GROUP,
-                                 y=dev_y[li], workspace=ls.ws)
-            host_y_all.copy_(dev_y_all, non_blocking=True)
+            e2e_graphs[p].replay()
         stream.synchronize()
 
     for i in range(args.warmup):
@@ -851,11 +991,13 @@ def main():
     for i in range(args.steps):
         e2e_step(i % ROT)
     el = max_over_ranks([time.perf_counter() - t0], dist, dev)[0]
+    del e2e_graphs
     e2e = {"value": round(replica_rate(gemv_bytes * args.steps, el, world) / 1e9, 3), "unit": "GB/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
            "note": "decode step through qz_w4a16_gemv: the three activation vectors copied in "
-                   "from one pinned host buffer, the three outputs copied out to one, one host "
-                   "sync per step; weights resident"}
+                   "from one pinned host buffer, the three outputs copied out to one, captured "
+                   "with the three public-API calls as one CUDA graph per step, replayed and "
+                   "synchronized on the host every step; weights resident"}
 
     extras = None
     if rank == 0 and not args.no_extras:

@@ -83,7 +83,15 @@ enum {
     QZ_OP_W4A16_GEMV = 2,
     QZ_OP_W4A16_GEMM = 3,
     QZ_OP_W8A16_GEMV = 4,
-    QZ_OP_W8A16_GEMM = 5
+    QZ_OP_W8A16_GEMM = 5,
+    QZ_OP_GPTQ = 6,
+    QZ_OP_FP4A16_GEMV = 7
+};
+
+/* FP4 formats (kind argument of the qz_fp4_* entry points). */
+enum {
+    QZ_FP4_MX = 0,   /* MXFP4: blocks of 32, E8M0 (power-of-two) block scales */
+    QZ_FP4_NV = 1    /* NVFP4: blocks of 16, E4M3 block scales, one fp32 tensor scale */
 };
 
 /* Static description of a status code (never NULL). */
@@ -158,8 +166,10 @@ QZ_API qz_status qz_dequantize(const void *codes, const void *scales, const void
  * before each matmul; decoding one token at a time is bound by reading the
  * weights) and the GPTQ explainer's fused dequantize-in-matmul kernels.
  * Each w_hat is formed exactly as qz_dequantize forms it, products are
- * accumulated in fp32, y is rounded to bf16.  Requirements: 1 <= M <= 16;
- * N >= 1; K % 128 == 0; group_size a multiple of 32 dividing K.  Workspace:
+ * accumulated in fp32, y is rounded to bf16.  Requirements: 1 <= M <= 64
+ * (batched decode; 17..64 tokens take a variant that keeps the activations
+ * in shared memory); N >= 1; K % 128 == 0; group_size a multiple of 32
+ * dividing K.  Workspace:
  * qz_workspace_bytes(QZ_OP_W4A16_GEMV, M, N, K, group_size) bytes,
  * zero-filled before first use (0 bytes means workspace may be NULL).
  */
@@ -195,7 +205,7 @@ QZ_API qz_status qz_w4a16_gemm(const void *a, const void *codes, const void *sca
  * W8A16 decode GEMV: y = a * w_hat^T for the int8 symmetric per-channel
  * weight (bits 8, symmetric 1, group_size K; codes N x K int8, scales N bf16;
  * taqaniya.com IBM absmax example).  w_hat = bf16_rne(S * q), fp32
- * accumulation, bf16 y.  Requirements: 1 <= M <= 16; N >= 1; K % 128 == 0.
+ * accumulation, bf16 y.  Requirements: 1 <= M <= 64; N >= 1; K % 128 == 0.
  * Workspace as for qz_w4a16_gemv with QZ_OP_W8A16_GEMV.
  */
 QZ_API qz_status qz_w8a16_gemv(const void *a, const void *codes, const void *scales,
@@ -227,6 +237,86 @@ QZ_API qz_status qz_w8a16_gemm(const void *a, const void *codes, const void *sca
                         size_t workspace_bytes, void *stream);
 
 /*
+ * GPTQ layer-wise quantization (GPTQ explainer, azimuth.plus/paper/gptq:
+ * sections on OBQ's error-compensating updates, the fixed column order, the
+ * lazy batched updates and the Cholesky decomposition of the inverse
+ * Hessian, and the algorithm paragraph with H = 2 X X^T).
+ *   w        N x K bf16 weights (row-major; rows are outputs);
+ *   x        n_samples x K bf16 calibration samples (one per row), so the
+ *            page's X (one sample per column) is x^T and H = 2 x^T x;
+ *   damp     the damping term is lambda = damp * mean(diag H) (1 if that
+ *            mean is 0); 0.01 is the customary value (the page gives none);
+ *   codes, scales, zeros: the packed format of qz_quantize_pack for the
+ *            same bits / symmetric / group_size, consumed unchanged by the
+ *            decode GEMVs and the prefill GEMMs.
+ * The columns are quantized in their natural order, in lazy blocks of 128.
+ * Each group's scale and zero come from the group's weights as they stand
+ * (already compensated) when its first column is reached; every code is the
+ * round-to-nearest code of that column's compensated weight, computed in
+ * fp32 exactly as qz_quantize_pack computes codes.  The Hessian, its factor
+ * and the compensation run in fp64.  Requirements: N >= 1; n_samples >= 1;
+ * K % 8 == 0; group_size a multiple of 32 dividing K with group_size % 128
+ * == 0 or 128 % group_size == 0 (so groups and blocks nest); damp >= 0.
+ * Workspace: qz_workspace_bytes(QZ_OP_GPTQ, 1, N, K, group_size) bytes
+ * (fp64: two K x K matrices, the N x K working weights and N x 128 errors),
+ * any contents.  Inputs must be finite.
+ */
+QZ_API qz_status qz_gptq_quantize(const void *w, const void *x, int64_t N, int64_t K,
+                                  int64_t n_samples, int32_t bits, int32_t symmetric,
+                                  int64_t group_size, double damp, void *codes, void *scales,
+                                  void *zeros, void *workspace, size_t workspace_bytes,
+                                  void *stream);
+
+/*
+ * FP4 with block scales (Quantization concepts guide, section "FP4 with
+ * block scales"; section "FP8" for E4M3).  An FP4 (E2M1) code has 1 sign,
+ * 2 exponent and 1 mantissa bit and stands for 0, 0.5, 1, 1.5, 2, 3, 4 or 6
+ * (or its negative): code = sign << 3 | index of the magnitude in that list.
+ * Layouts: codes N x K/2 bytes, packed as the int4 format (value k in the
+ * low nibble of byte k/2 when k is even); block scales N x K/B bytes, one per
+ * B consecutive values of a row (MXFP4: B = 32, the E8M0 byte e + 127 of the
+ * scale 2^e; NVFP4: B = 16, an E4M3 byte); NVFP4 also has one fp32 tensor
+ * scale.  Readings of this library (the page fixes neither the block sizes
+ * nor how scales are chosen): MXFP4 e is the smallest integer with
+ * max|x| <= 6 * 2^e; NVFP4 s_t = amax / 2688 (6 x 448) in fp32 and the block
+ * scale is the smallest E4M3 value >= fp32(amax_b / fp32(6 s_t)); each code
+ * is the nearest E2M1 value to x / scale (fp32; NVFP4 scale fp32(s_b * s_t)),
+ * ties to the even mantissa bit.  Dequantized bf16: MXFP4 e2m1 * 2^e (exact),
+ * NVFP4 bf16_rne(fp32(fp32(e2m1 * s_b) * s_t)).
+ */
+QZ_API qz_status qz_fp4_packed_bytes(int64_t N, int64_t K, int32_t kind, size_t *codes_bytes,
+                                     size_t *scales_bytes);
+
+/*
+ * FP4 quantize: w (N x K bf16, 16-byte aligned) -> codes (16-byte aligned),
+ * block scales and, for NVFP4, *tensor_scale (one fp32 in device memory,
+ * 4-byte aligned; it also holds the tensor's amax while the call runs; must
+ * be NULL for MXFP4).  Requirements: K a multiple of the block size.
+ */
+QZ_API qz_status qz_fp4_quantize(const void *w, int64_t N, int64_t K, int32_t kind, void *codes,
+                                 void *block_scales, void *tensor_scale, void *stream);
+
+/* FP4 dequantize to N x K bf16 (w_hat 16-byte aligned, codes 4-byte aligned). */
+QZ_API qz_status qz_fp4_dequantize(const void *codes, const void *block_scales,
+                                   const void *tensor_scale, int64_t N, int64_t K, int32_t kind,
+                                   void *w_hat, void *stream);
+
+/*
+ * FP4A16 decode GEMV: y (M x N bf16) = a (M x K bf16) * w_hat^T for FP4
+ * weights with block scales ("Quantize weights or activations": NVFP4 runs a
+ * matmul with 4-bit weights and 16-bit activations for decoding).  Each
+ * weight enters the fp32-accumulated product as e2m1 * s_b exactly (bf16
+ * holds it without rounding) and NVFP4's tensor scale multiplies the sums
+ * before y is rounded to bf16.  Requirements: 1 <= M <= 16; N >= 1;
+ * K % 128 == 0.  Workspace: qz_workspace_bytes(QZ_OP_FP4A16_GEMV, M, N, K,
+ * 0) bytes, zero-filled before first use (0 bytes means NULL is allowed).
+ */
+QZ_API qz_status qz_fp4a16_gemv(const void *a, const void *codes, const void *block_scales,
+                                const void *tensor_scale, int64_t M, int64_t N, int64_t K,
+                                int32_t kind, void *y, void *workspace, size_t workspace_bytes,
+                                void *stream);
+
+/*
  * Size of the scratch array built into the library for
  * qz_w4a16_gemv_noalloc (8 MiB, held on every GPU that loads the library).
  */
@@ -239,7 +329,7 @@ QZ_API qz_status qz_w8a16_gemm(const void *a, const void *codes, const void *sca
  * host application that owns all device memory and offers no allocator, or
  * latency-critical code that cannot afford cudaMalloc (which may synchronize
  * the device).  Arguments, requirements and results are those of
- * qz_w4a16_gemv; the split-K scratch lives in a fixed array of
+ * qz_w4a16_gemv for 1 <= M <= 16; the split-K scratch lives in a fixed array of
  * QZ_GEMV_NOALLOC_SCRATCH_BYTES inside the library.
  *   - Sizes whose scratch need (qz_workspace_bytes(QZ_OP_W4A16_GEMV, ...))
  *     exceeds that maximum are rejected with QZ_ERR_WORKSPACE before any

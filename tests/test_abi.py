@@ -63,8 +63,12 @@ def test_workspace_bytes():
     big = qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMV, 1, 1024, 1024, 128)
     assert big > 0 and big % 4 == 0
     assert qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMV, 16, 1024, 1024, 128) >= big
+    # the integer decode GEMVs take up to 64 tokens, the FP4A16 GEMV up to 16
+    assert qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMV, 64, 1024, 1024, 128) > 0
     with pytest.raises(qz.QzError):
-        qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMV, 17, 1024, 1024, 128)
+        qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMV, 65, 1024, 1024, 128)
+    with pytest.raises(qz.QzError):
+        qz.qz_workspace_bytes(qz.QZ_OP_FP4A16_GEMV, 17, 1024, 1024, 0)
     with pytest.raises(qz.QzError):
         qz.qz_workspace_bytes(99, 1, 8, 128, 128)
 
@@ -101,7 +105,7 @@ def test_dequantize_rejects(args, expect):
 
 @pytest.mark.parametrize("args,expect", [
     ((A, B, C, D, 0, 64, 128, 128, Y, None, 0, None), INVALID),          # M = 0
-    ((A, B, C, D, 17, 64, 128, 128, Y, None, 0, None), UNSUP),           # M > 16
+    ((A, B, C, D, 65, 64, 128, 128, Y, None, 0, None), UNSUP),           # M > 64
     ((A, B, C, D, 1, 64, 192, 64, Y, None, 0, None), UNSUP),             # K % 128
     ((A, B, C, D, 1, 64, 256, 48, Y, None, 0, None), INVALID),           # K % g
     ((A, B, C, D, 1, 64, 256, 16, Y, None, 0, None), UNSUP),             # g % 32
@@ -115,7 +119,7 @@ def test_w4a16_gemv_rejects(args, expect):
 
 @pytest.mark.parametrize("args,expect", [
     ((A, B, C, 0, 64, 128, Y, None, 0, None), INVALID),
-    ((A, B, C, 17, 64, 128, Y, None, 0, None), UNSUP),
+    ((A, B, C, 65, 64, 128, Y, None, 0, None), UNSUP),           # M > 64
     ((A, B, None, 1, 64, 128, Y, None, 0, None), INVALID),
     ((A, MIS, C, 1, 64, 128, Y, None, 0, None), ALIGN),
     ((A, B, C, 1, 4096, 4096, Y, None, 0, None), WS),
@@ -247,3 +251,25 @@ def test_gptq_workspace_bytes():
     assert qz.qz_workspace_bytes(qz.QZ_OP_GPTQ, 1, N, K, 128) == \
         2 * K * K * 8 + N * K * 8 + N * 128 * 8
     assert qz.qz_workspace_bytes(qz.QZ_OP_GPTQ, 1, 37, 384, 128) >= 2 * 384 * 384 * 8 + 37 * 384 * 8
+
+
+@pytest.mark.parametrize("kind,ts,K,expect", [
+    (2, None, 256, UNSUP), (0, None, 100, INVALID), (1, None, 256, INVALID),   # NV needs a tensor scale
+    (0, C, 256, INVALID), (1, C, 24, INVALID),                                # MX takes none; K % 16
+])
+def test_fp4_quantize_rejects(kind, ts, K, expect):
+    assert L().qz_fp4_quantize(A, 8, K, kind, B, D, ts, None) == expect
+
+
+def test_fp4_gemv_rejects_and_workspace():
+    ts = C
+    assert L().qz_fp4a16_gemv(A, B, D, ts, 17, 64, 256, 1, Y, None, 0, None) == UNSUP     # M > 16
+    assert L().qz_fp4a16_gemv(A, B, D, ts, 1, 64, 192, 1, Y, None, 0, None) == UNSUP     # K % 128
+    assert L().qz_fp4a16_gemv(A, B, D, None, 1, 64, 256, 1, Y, None, 0, None) == INVALID
+    assert L().qz_fp4a16_gemv(MIS, B, D, ts, 1, 64, 256, 1, Y, None, 0, None) == ALIGN
+    assert L().qz_fp4a16_gemv(A, B, D, ts, 4, 4096, 4096, 1, Y, None, 0, None) == WS
+    # the same stream-K plan as the W4A16 GEMV
+    assert qz.qz_workspace_bytes(qz.QZ_OP_FP4A16_GEMV, 4, 4096, 4096, 0) == \
+        qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMV, 4, 4096, 4096, 128)
+    assert qz.qz_fp4_packed_bytes(64, 1024, qz.QZ_FP4_MX) == (64 * 512, 64 * 32)
+    assert qz.qz_fp4_packed_bytes(64, 1024, qz.QZ_FP4_NV) == (64 * 512, 64 * 64)

@@ -112,3 +112,22 @@ def test_traffic_record_dropped_when_source_changes(tmp_path, monkeypatch):
     assert bench.ncu_traffic() == {}
     os.remove(tmp_path / "profiles" / "traffic.json")
     assert bench.ncu_traffic() == {}
+
+
+def test_fp4_gemv_and_quantize_bytes():
+    # half a byte per code plus one scale byte per 32 (MXFP4) or 16 (NVFP4)
+    # values, bf16 activations and outputs; NVFP4 adds its fp32 tensor scale
+    N, K = 28672, 8192
+    assert bench.fp4_gemv_bytes(1, N, K, 0) == N * K // 2 + N * K // 32 + 2 * K + 2 * N
+    assert bench.fp4_gemv_bytes(1, N, K, 1) == N * K // 2 + N * K // 16 + 4 + 2 * K + 2 * N
+    assert abs(bench.fp4_gemv_bytes(1, N, K, 0) / MB - 124.85) <= 0.005   # 4.25 bits per weight
+    assert abs(bench.fp4_gemv_bytes(1, N, K, 1) / MB - 132.19) <= 0.005   # 4.5 bits per weight
+    assert bench.fp4_quant_bytes(N, K, 1) == 2 * N * K + N * K // 2 + N * K // 16
+
+
+def test_gptq_flops_and_fp64_peak():
+    # 4096 x 4096 with 128 samples: 2 n K^2 + 2/3 K^3 + 2 N K^2
+    f = bench.gptq_flops(4096, 4096, 128)
+    assert f == 2 * 128 * 4096 ** 2 + (2 * 4096 ** 3) // 3 + 2 * 4096 ** 3
+    assert abs(f / 1e9 - 187.55) <= 0.005    # 4.29 + 45.81 + 137.44
+    assert abs(bench.FP64_PEAK_TFLOPS - 37.23) <= 0.01

@@ -240,6 +240,51 @@ def test_w8a16_gemv_tolerance(dev, N, K, M):
     assert np.array_equal(u16(y1), w_hat[:, ks].T)
 
 
+@pytest.mark.parametrize("N,K,g", [(1024, 1024, 128), (1000, 384, 128), (4100, 1152, 128),
+                                   (256, 2048, 256), (96, 512, 64)])
+@pytest.mark.parametrize("M", [17, 32, 33, 64])
+@pytest.mark.parametrize("bits", [4, 8])
+def test_gemv_wide_tolerance(dev, N, K, g, M, bits):
+    """17..64 tokens: the decode GEMV keeps the activations in shared memory
+    and reads them per code word (MB = 4 or 8 token groups)."""
+    w = synthetic.weights(N, K, sigma=0.02, seed=N + K + M)
+    a = synthetic.activations(M, K, seed=M + 7)
+    if bits == 4:
+        c, s, z, w_hat = oracle_w4(u16(w), g)
+        y = qz.qz_w4a16_gemv(a.to(dev), to_dev_u8(c, dev), to_dev_bf16(s, dev),
+                             to_dev_u8(z, dev), N, K, g)
+    else:
+        c, s, _ = oracle.quantize_pack(u16(w), 8, True, K)
+        w_hat = oracle.dequantize(c, s, None, N, K, 8, True, K)
+        y = qz.qz_w8a16_gemv(a.to(dev), to_dev_u8(c, dev), to_dev_bf16(s, dev), N, K)
+    torch.cuda.synchronize()
+    assert qz.qz_device_status() == 0
+    y_ref, abs_ref = oracle.matmul_f64(u16(a), w_hat)
+    check_tolerance(u16(y), y_ref, abs_ref, f"wide gemv bits={bits} M={M} N={N} K={K}")
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_gemv_wide_onehot_is_exact(dev, bits):
+    """64 one-hot token rows read back 64 dequantized weights exactly."""
+    N, K, g, M = 300, 1024, 128, 64
+    w = synthetic.weights(N, K, sigma=0.02, seed=15)
+    if bits == 4:
+        c, s, z, w_hat = oracle_w4(u16(w), g)
+    else:
+        c, s, z = oracle.quantize_pack(u16(w), 8, True, K)
+        w_hat = oracle.dequantize(c, s, None, N, K, 8, True, K)
+    ks = np.random.default_rng(2).choice(K, size=M, replace=False)
+    a = np.zeros((M, K), np.uint16)
+    a[np.arange(M), ks] = 0x3F80
+    if bits == 4:
+        y = qz.qz_w4a16_gemv(to_dev_bf16(a, dev), to_dev_u8(c, dev), to_dev_bf16(s, dev),
+                             to_dev_u8(z, dev), N, K, g)
+    else:
+        y = qz.qz_w8a16_gemv(to_dev_bf16(a, dev), to_dev_u8(c, dev), to_dev_bf16(s, dev), N, K)
+    torch.cuda.synchronize()
+    assert np.array_equal(u16(y), w_hat[:, ks].T)
+
+
 def test_gemv_workspace_is_left_zeroed_and_results_repeat(dev):
     N, K, g, M = 4096, 4096, 128, 4
     nbytes = qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMV, M, N, K, g)

@@ -19,7 +19,9 @@ __all__ = [
     "qz_workspace_bytes", "qz_workspace_bytes_for_sms", "qz_quantize_pack", "qz_dequantize",
     "qz_w4a16_gemv",
     "qz_w4a16_gemm", "qz_w8a16_gemv", "qz_w8a16_gemm", "qz_set_device_wait_limit",
-    "qz_set_launch_overlap", "qz_device_status",
+    "qz_set_launch_overlap", "qz_device_status", "qz_gptq_quantize", "QZ_OP_GPTQ",
+    "qz_fp4_packed_bytes", "qz_fp4_quantize", "qz_fp4_dequantize", "qz_fp4a16_gemv",
+    "QZ_OP_FP4A16_GEMV", "QZ_FP4_MX", "QZ_FP4_NV",
     "Workspace", "QZ_OP_QUANTIZE_PACK", "QZ_OP_DEQUANTIZE", "QZ_OP_W4A16_GEMV",
     "QZ_OP_W4A16_GEMM", "QZ_OP_W8A16_GEMV", "QZ_OP_W8A16_GEMM", "EXPORTED_SYMBOLS",
 ]
@@ -29,7 +31,9 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqz.so")
 QZ_OK = 0
 QZ_ERR_DEVICE_TIMEOUT = 6
 (QZ_OP_QUANTIZE_PACK, QZ_OP_DEQUANTIZE, QZ_OP_W4A16_GEMV, QZ_OP_W4A16_GEMM, QZ_OP_W8A16_GEMV,
- QZ_OP_W8A16_GEMM) = range(6)
+ QZ_OP_W8A16_GEMM, QZ_OP_GPTQ, QZ_OP_FP4A16_GEMV) = range(8)
+QZ_FP4_MX, QZ_FP4_NV = 0, 1
+FP4_BLOCK = {QZ_FP4_MX: 32, QZ_FP4_NV: 16}
 
 _i32, _i64, _sz, _p = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p
 _SIGS = {
@@ -47,6 +51,13 @@ _SIGS = {
     "qz_w8a16_gemv": ([_p, _p, _p, _i64, _i64, _i64, _p, _p, _sz, _p], ctypes.c_int),
     "qz_w8a16_gemm": ([_p, _p, _p, _i64, _i64, _i64, _p, _p, _sz, _p], ctypes.c_int),
     "qz_w4a16_gemv_noalloc": ([_p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _p], ctypes.c_int),
+    "qz_gptq_quantize": ([_p, _p, _i64, _i64, _i64, _i32, _i32, _i64, ctypes.c_double, _p, _p, _p,
+                          _p, _sz, _p], ctypes.c_int),
+    "qz_fp4_packed_bytes": ([_i64, _i64, _i32, ctypes.POINTER(_sz), ctypes.POINTER(_sz)],
+                            ctypes.c_int),
+    "qz_fp4_quantize": ([_p, _i64, _i64, _i32, _p, _p, _p, _p], ctypes.c_int),
+    "qz_fp4_dequantize": ([_p, _p, _p, _i64, _i64, _i32, _p, _p], ctypes.c_int),
+    "qz_fp4a16_gemv": ([_p, _p, _p, _p, _i64, _i64, _i64, _i32, _p, _p, _sz, _p], ctypes.c_int),
     "qz_set_device_wait_limit": ([ctypes.c_uint64], None),
     "qz_set_launch_overlap": ([ctypes.c_int32], ctypes.c_int),
     "qz_device_status": ([], ctypes.c_int),
@@ -276,6 +287,96 @@ def qz_w8a16_gemm(a, codes, scales, N, K, y=None, workspace=None, stream=None):
         ws_ptr, ws_bytes = _ws_args(workspace, nbytes, a.device)
         _check(lib.qz_w8a16_gemm(_ptr(a), _ptr(codes), _ptr(scales), M, N, K, _ptr(y),
                                  ws_ptr, ws_bytes, _handle(st)), "qz_w8a16_gemm")
+    return y
+
+
+def qz_gptq_quantize(w, x, bits=4, symmetric=False, group_size=128, damp=0.01, codes=None,
+                     scales=None, zeros=None, workspace=None, stream=None):
+    """GPTQ of one layer: ``w`` (N x K bf16) with calibration samples ``x``
+    (n x K bf16); returns (codes, scales, zeros | None) in the packed format
+    of :func:`qz_quantize_pack`."""
+    if w.dtype != torch.bfloat16 or w.dim() != 2 or x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise ValueError("w and x must be 2-D bf16 tensors")
+    N, K = w.shape
+    if x.shape[1] != K:
+        raise ValueError("x must have K columns")
+    qz_packed_bytes(N, K, bits, symmetric, group_size)      # validates the format
+    dev = w.device
+    st = _launch_stream(stream, dev)
+    with _on(stream):
+        if codes is None:
+            codes = torch.empty((N, K // 2) if bits == 4 else (N, K), dtype=torch.uint8,
+                                device=dev)
+        if scales is None:
+            scales = torch.empty((N, K // group_size), dtype=torch.bfloat16, device=dev)
+        if zeros is None and not symmetric:
+            zeros = torch.empty((N, K // group_size), dtype=torch.uint8, device=dev)
+        nbytes = qz_workspace_bytes(QZ_OP_GPTQ, 1, N, K, group_size)
+        if workspace is None:
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        elif isinstance(workspace, Workspace):
+            workspace = workspace.get(nbytes)
+        _check(lib.qz_gptq_quantize(_ptr(w), _ptr(x), N, K, x.shape[0], bits, int(symmetric),
+                                    group_size, float(damp), _ptr(codes), _ptr(scales),
+                                    _ptr(zeros) if not symmetric else None, _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _handle(st)),
+               "qz_gptq_quantize")
+    return codes, scales, (None if symmetric else zeros)
+
+
+def qz_fp4_packed_bytes(N, K, kind):
+    c, s = _sz(), _sz()
+    _check(lib.qz_fp4_packed_bytes(N, K, kind, ctypes.byref(c), ctypes.byref(s)),
+           "qz_fp4_packed_bytes")
+    return c.value, s.value
+
+
+def qz_fp4_quantize(w, kind, codes=None, scales=None, tensor_scale=None, stream=None):
+    """FP4 with block scales: returns (codes uint8 N x K/2, block scales uint8,
+    tensor scale fp32 tensor of one element (NVFP4) or None)."""
+    if w.dtype != torch.bfloat16 or w.dim() != 2:
+        raise ValueError("w must be a 2-D bf16 tensor")
+    N, K = w.shape
+    qz_fp4_packed_bytes(N, K, kind)                      # validates the shape
+    dev = w.device
+    st = _launch_stream(stream, dev)
+    with _on(stream):
+        if codes is None:
+            codes = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+        if scales is None:
+            scales = torch.empty((N, K // FP4_BLOCK[kind]), dtype=torch.uint8, device=dev)
+        if tensor_scale is None and kind == QZ_FP4_NV:
+            tensor_scale = torch.empty(1, dtype=torch.float32, device=dev)
+        _check(lib.qz_fp4_quantize(_ptr(w), N, K, kind, _ptr(codes), _ptr(scales),
+                                   _ptr(tensor_scale) if kind == QZ_FP4_NV else None,
+                                   _handle(st)), "qz_fp4_quantize")
+    return codes, scales, (tensor_scale if kind == QZ_FP4_NV else None)
+
+
+def qz_fp4_dequantize(codes, scales, tensor_scale, N, K, kind, out=None, stream=None):
+    """The dequantized FP4 weights as an N x K bf16 tensor."""
+    dev = codes.device
+    st = _launch_stream(stream, dev)
+    with _on(stream):
+        if out is None:
+            out = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+        _check(lib.qz_fp4_dequantize(_ptr(codes), _ptr(scales), _ptr(tensor_scale), N, K, kind,
+                                     _ptr(out), _handle(st)), "qz_fp4_dequantize")
+    return out
+
+
+def qz_fp4a16_gemv(a, codes, scales, tensor_scale, N, K, kind, y=None, workspace=None,
+                   stream=None):
+    """y = a * w_hat^T for FP4 weights with block scales, M <= 16."""
+    st = _launch_stream(stream, a.device)
+    M = a.shape[0]
+    with _on(stream):
+        y = _matmul_out(a, N, y)
+        nbytes = qz_workspace_bytes(QZ_OP_FP4A16_GEMV, M, N, K, 0)
+        ws_ptr, ws_bytes = _ws_args(workspace, nbytes, a.device)
+        _check(lib.qz_fp4a16_gemv(_ptr(a), _ptr(codes), _ptr(scales), _ptr(tensor_scale), M, N,
+                                  K, kind, _ptr(y), ws_ptr, ws_bytes, _handle(st)),
+               "qz_fp4a16_gemv")
     return y
 
 

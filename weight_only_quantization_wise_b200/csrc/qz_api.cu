@@ -59,9 +59,13 @@ qz_status check_matrix_format(int64_t N, int64_t K, int32_t bits, int32_t symmet
     return QZ_OK;
 }
 
-qz_status check_gemv_shape(int64_t M, int64_t N, int64_t K) {
+// The integer decode GEMVs take up to 64 tokens; the FP4A16 GEMV up to 16.
+constexpr int64_t kGemvMaxM = 64;
+constexpr int64_t kFp4GemvMaxM = 16;
+
+qz_status check_gemv_shape(int64_t M, int64_t N, int64_t K, int64_t max_m = kGemvMaxM) {
     if (M < 1 || N < 1 || K < 1 || N > kMaxDim || K > kMaxDim) return QZ_ERR_INVALID_ARG;
-    if (M > 16) return QZ_ERR_UNSUPPORTED;
+    if (M > max_m) return QZ_ERR_UNSUPPORTED;
     if (K % 128 != 0) return QZ_ERR_UNSUPPORTED;
     if ((int64_t)N * K > kMaxElems) return QZ_ERR_INVALID_ARG;
     return QZ_OK;
@@ -138,6 +142,16 @@ QZ_API qz_status qz_workspace_bytes(int32_t op, int64_t M, int64_t N, int64_t K,
                      ? gemv_workspace_bound(M, N, K, op == QZ_OP_W4A16_GEMM ? 4 : 8)
                      : gemm_workspace_bytes(M, N, K);
         return QZ_OK;
+    case QZ_OP_FP4A16_GEMV: {
+        const qz_status s = check_gemv_shape(M, N, K, kFp4GemvMaxM);
+        if (s != QZ_OK) return s;
+        *bytes = gemv_workspace_bound(M, N, K, 4);
+        return QZ_OK;
+    }
+    case QZ_OP_GPTQ:
+        if (N < 1 || K < 1 || N > kMaxDim || K > kMaxDim) return QZ_ERR_INVALID_ARG;
+        *bytes = gptq_workspace_bytes(N, K);
+        return QZ_OK;
     default:
         return QZ_ERR_INVALID_ARG;
     }
@@ -161,6 +175,12 @@ QZ_API qz_status qz_workspace_bytes_for_sms(int32_t op, int64_t M, int64_t N, in
                      ? gemv_plan(M, N, K, op == QZ_OP_W4A16_GEMM ? 4 : 8, sms).total_bytes
                      : gemm_workspace_bytes_for(M, N, K, sms);
         return QZ_OK;
+    case QZ_OP_FP4A16_GEMV: {
+        const qz_status s = check_gemv_shape(M, N, K, kFp4GemvMaxM);
+        if (s != QZ_OK) return s;
+        *bytes = gemv_plan(M, N, K, 4, sms).total_bytes;
+        return QZ_OK;
+    }
     default:
         return qz_workspace_bytes(op, M, N, K, group_size, bytes);
     }
@@ -261,6 +281,95 @@ QZ_API qz_status qz_w8a16_gemm(const void *a, const void *codes, const void *sca
     const qz_status s = check_workspace(gemm_workspace_bytes(M, N, K), workspace, workspace_bytes);
     if (s != QZ_OK) return s;
     return launch_w8a16_gemm(a, codes, scales, M, N, K, y, workspace, as_stream(stream));
+}
+
+QZ_API qz_status qz_gptq_quantize(const void *w, const void *x, int64_t N, int64_t K,
+                                  int64_t n_samples, int32_t bits, int32_t symmetric,
+                                  int64_t group_size, double damp, void *codes, void *scales,
+                                  void *zeros, void *workspace, size_t workspace_bytes,
+                                  void *stream) {
+    if (!format_ok(bits, symmetric)) return QZ_ERR_UNSUPPORTED;
+    if (N < 1 || K < 1 || N > kMaxDim || K > kMaxDim || n_samples < 1) return QZ_ERR_INVALID_ARG;
+    if (N * K > kMaxElems || n_samples * K > kMaxElems) return QZ_ERR_INVALID_ARG;
+    if (!(damp >= 0.0) || !(damp < 1e300)) return QZ_ERR_INVALID_ARG;
+    if (group_size <= 0 || K % group_size != 0) return QZ_ERR_INVALID_ARG;
+    if (K % 8 != 0 || group_size % 32 != 0 || (group_size % 128 != 0 && 128 % group_size != 0))
+        return QZ_ERR_UNSUPPORTED;
+    if (!w || !x || !codes || !scales) return QZ_ERR_INVALID_ARG;
+    if (symmetric ? (zeros != nullptr) : (zeros == nullptr)) return QZ_ERR_INVALID_ARG;
+    if (!aligned(w, 2) || !aligned(x, 2) || !aligned(scales, 2)) return QZ_ERR_ALIGNMENT;
+    const qz_status s = check_workspace(gptq_workspace_bytes(N, K), workspace, workspace_bytes);
+    if (s != QZ_OK) return s;
+    return launch_gptq(w, x, N, K, n_samples, bits, symmetric, group_size, damp, codes, scales,
+                       zeros, workspace, as_stream(stream));
+}
+
+QZ_API qz_status qz_fp4_packed_bytes(int64_t N, int64_t K, int32_t kind, size_t *codes_bytes,
+                                     size_t *scales_bytes) {
+    if (!codes_bytes || !scales_bytes) return QZ_ERR_INVALID_ARG;
+    if (kind != QZ_FP4_MX && kind != QZ_FP4_NV) return QZ_ERR_UNSUPPORTED;
+    if (N < 1 || K < 1 || K % fp4_block_size(kind) != 0) return QZ_ERR_INVALID_ARG;
+    *codes_bytes = (size_t)(N * (K / 2));
+    *scales_bytes = (size_t)(N * (K / fp4_block_size(kind)));
+    return QZ_OK;
+}
+
+namespace {
+qz_status check_fp4(int64_t N, int64_t K, int32_t kind) {
+    if (kind != QZ_FP4_MX && kind != QZ_FP4_NV) return QZ_ERR_UNSUPPORTED;
+    if (N < 1 || K < 1 || N > kMaxDim || K > kMaxDim || N * K > kMaxElems)
+        return QZ_ERR_INVALID_ARG;
+    if (K % fp4_block_size(kind) != 0) return QZ_ERR_INVALID_ARG;
+    return QZ_OK;
+}
+}  // namespace
+
+QZ_API qz_status qz_fp4_quantize(const void *w, int64_t N, int64_t K, int32_t kind, void *codes,
+                                 void *block_scales, void *tensor_scale, void *stream) {
+    const qz_status s = check_fp4(N, K, kind);
+    if (s != QZ_OK) return s;
+    if (!w || !codes || !block_scales) return QZ_ERR_INVALID_ARG;
+    if (kind == QZ_FP4_NV ? tensor_scale == nullptr : tensor_scale != nullptr)
+        return QZ_ERR_INVALID_ARG;
+    if (!aligned(w, 16) || !aligned(codes, 16) || (tensor_scale && !aligned(tensor_scale, 4)))
+        return QZ_ERR_ALIGNMENT;
+    return launch_fp4_quantize(w, N, K, kind, codes, block_scales, tensor_scale,
+                               as_stream(stream));
+}
+
+QZ_API qz_status qz_fp4_dequantize(const void *codes, const void *block_scales,
+                                   const void *tensor_scale, int64_t N, int64_t K, int32_t kind,
+                                   void *w_hat, void *stream) {
+    const qz_status s = check_fp4(N, K, kind);
+    if (s != QZ_OK) return s;
+    if (!codes || !block_scales || !w_hat) return QZ_ERR_INVALID_ARG;
+    if (kind == QZ_FP4_NV ? tensor_scale == nullptr : tensor_scale != nullptr)
+        return QZ_ERR_INVALID_ARG;
+    if (!aligned(codes, 4) || !aligned(w_hat, 16) || (tensor_scale && !aligned(tensor_scale, 4)))
+        return QZ_ERR_ALIGNMENT;
+    return launch_fp4_dequantize(codes, block_scales, tensor_scale, N, K, kind, w_hat,
+                                 as_stream(stream));
+}
+
+QZ_API qz_status qz_fp4a16_gemv(const void *a, const void *codes, const void *block_scales,
+                                const void *tensor_scale, int64_t M, int64_t N, int64_t K,
+                                int32_t kind, void *y, void *workspace, size_t workspace_bytes,
+                                void *stream) {
+    qz_status s = check_gemv_shape(M, N, K, kFp4GemvMaxM);
+    if (s != QZ_OK) return s;
+    s = check_fp4(N, K, kind);
+    if (s != QZ_OK) return s;
+    if (!a || !codes || !block_scales || !y) return QZ_ERR_INVALID_ARG;
+    if (kind == QZ_FP4_NV ? tensor_scale == nullptr : tensor_scale != nullptr)
+        return QZ_ERR_INVALID_ARG;
+    if (!aligned(a, 16) || !aligned(codes, 16) || !aligned(y, 2) ||
+        (tensor_scale && !aligned(tensor_scale, 4)))
+        return QZ_ERR_ALIGNMENT;
+    const GemvPlan plan = gemv_plan(M, N, K, 4, device_sm_count());
+    s = check_workspace(plan.total_bytes, workspace, workspace_bytes);
+    if (s != QZ_OK) return s;
+    return launch_fp4a16_gemv(a, codes, block_scales, tensor_scale, M, N, K, kind, y, workspace,
+                              plan, launch_overlap(), as_stream(stream));
 }
 
 QZ_API void qz_set_device_wait_limit(uint64_t limit) {

@@ -1,0 +1,248 @@
+// qz_fp4.cu -- FP4 (E2M1) weights with block scales: quantize and dequantize.
+//
+// Quantization concepts guide, section "FP4 with block scales": an FP4 value
+// has 1 sign, 2 exponent and 1 mantissa bit and represents only 0, 0.5, 1,
+// 1.5, 2, 3, 4 and 6 (and their negatives), so every small block of values
+// carries its own scale, stored in the format.  MXFP4 (micro-scaling) uses a
+// power-of-two scale, which only shifts exponents; NVFP4 uses smaller blocks
+// with an FP8 (E4M3, section "FP8") scale that can fall between powers of two,
+// plus one scale for the tensor that keeps the FP8 block scales in range.
+//
+// Layouts (this library's readings: the page fixes neither block sizes nor
+// how a scale is chosen):
+//   codes         N x K/2 bytes, value k in the low nibble of byte k/2 when k
+//                 is even (the packing of the int4 format); a code is
+//                 sign << 3 | magnitude index (0, 0.5, 1, 1.5, 2, 3, 4, 6);
+//   block scales  N x K/B bytes: MXFP4 B = 32, the E8M0 byte e + 127 of the
+//                 scale 2^e; NVFP4 B = 16, an E4M3 byte;
+//   tensor scale  NVFP4 only: one fp32.
+// Scales: MXFP4 e is the smallest integer with max|x| <= 6 * 2^e (clamped to
+// [-127, 127]); NVFP4 s_t = fp32(amax / 2688) (6 x 448: the largest E2M1
+// and E4M3 values), s_b = the smallest E4M3 value >= fp32(amax_b /
+// fp32(6 s_t)), at most 448, 0 for an all-zero block.  Codes: x divided by
+// the block's scale (2^e, or fp32(s_b * s_t)) in fp32, rounded to the
+// nearest E2M1 magnitude, ties to the even mantissa bit, saturating at 6.
+// Dequantized bf16: MXFP4 e2m1 * 2^e (exact); NVFP4
+// bf16_rne(fp32(fp32(e2m1 * s_b) * s_t)) (the inner product is exact).
+#include <cuda_runtime.h>
+
+#include "qz_internal.cuh"
+
+namespace qz {
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) { return __uint_as_float(h << 16); }
+
+// E4M3 byte (sign ignored) -> value.
+__device__ __forceinline__ float e4m3_value(uint32_t b) {
+    const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+    if (e == 0) return (float)m * 0.001953125f;                  // m * 2^-9 (exact)
+    return __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+
+// The smallest E4M3 value >= t (t >= 0), at most 448 (byte 0x7E); 0 for t = 0.
+// Bytes 1..0x7E are increasing in value without gaps between the subnormal
+// and normal ranges (m * 2^-9, then (8 + m) * 2^(e - 10)).
+__device__ __forceinline__ uint32_t e4m3_round_up(float t) {
+    if (!(t > 0.0f)) return 0u;
+    if (t >= 448.0f) return 0x7Eu;
+    if (t < 0.015625f) {                                         // below 2^-6: subnormal step 2^-9
+        const float m = ceilf(t * 512.0f);                       // exact scaling
+        return (uint32_t)m;                                      // 8 -> 0x08 = 2^-6
+    }
+    const int E = ilogbf(t);                                     // t in [2^E, 2^(E+1))
+    const float mant = ldexpf(t, -E);                            // [1, 2), exact
+    uint32_t m = (uint32_t)ceilf((mant - 1.0f) * 8.0f);          // exact
+    int e = E + 7;
+    if (m == 8u) {
+        m = 0u;
+        ++e;
+    }
+    const uint32_t b = ((uint32_t)e << 3) | m;
+    return b > 0x7Eu ? 0x7Eu : b;
+}
+
+// Nearest E2M1 code of v (sign in bit 3), ties to the even mantissa bit,
+// saturating at 6: the thresholds between neighbouring magnitudes are 0.25,
+// 0.75, 1.25, 1.75, 2.5, 3.5, 5, and a tie goes to the magnitude with an even
+// index (0, 1, 2, 4 at 0.25, 0.75->1, 1.25->1, 1.75->2, 2.5->2, 3.5->4, 5->4).
+__device__ __forceinline__ uint32_t e2m1_code(float v) {
+    const float a = fabsf(v);
+    uint32_t c = (uint32_t)(a > 0.25f) + (uint32_t)(a >= 0.75f) + (uint32_t)(a > 1.25f) +
+                 (uint32_t)(a >= 1.75f) + (uint32_t)(a > 2.5f) + (uint32_t)(a >= 3.5f) +
+                 (uint32_t)(a > 5.0f);
+    if (v < 0.0f && c != 0u) c |= 8u;
+    return c;
+}
+
+__device__ __forceinline__ float e2m1_value(uint32_t c) {
+    const uint32_t i = c & 7u;
+    const float mag = i < 4 ? 0.5f * (float)i : (i == 4 ? 2.0f : i == 5 ? 3.0f : i == 6 ? 4.0f : 6.0f);
+    return (c & 8u) ? -mag : mag;
+}
+
+__device__ __forceinline__ int64_t grid_stride() { return (int64_t)gridDim.x * blockDim.x; }
+__device__ __forceinline__ int64_t thread_index() {
+    return (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+}
+
+// max |w| over the tensor into *amax (fp32 bits, non-negative: ordered as
+// unsigned integers).
+__global__ void __launch_bounds__(kThreads) fp4_amax_kernel(const uint4 *__restrict__ w,
+                                                           int64_t chunks, unsigned *amax) {
+    float m = 0.0f;
+    for (int64_t c = thread_index(); c < chunks; c += grid_stride()) {
+        const uint4 v = __ldg(w + c);
+        const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            m = fmaxf(m, fmaxf(fabsf(bf16_bits_to_f32(x[i] & 0xFFFFu)),
+                               fabsf(bf16_bits_to_f32(x[i] >> 16))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    __shared__ float part[kThreads / 32];
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int i = 1; i < kThreads / 32; ++i) m = fmaxf(m, part[i]);
+        atomicMax(amax, __float_as_uint(m));
+    }
+}
+
+__device__ __forceinline__ float nv_tensor_scale(float amax) {
+    return amax > 0.0f ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+}
+
+// One thread per block of BS values (BS / 8 chunks of 16 bytes).
+template <int KIND>
+__global__ void __launch_bounds__(kThreads)
+fp4_quantize_kernel(const uint4 *__restrict__ w, int64_t blocks, uint8_t *__restrict__ codes,
+                    uint8_t *__restrict__ scales, const unsigned *__restrict__ amax_bits) {
+    constexpr int BS = KIND == 0 ? 32 : 16;
+    float s_t = 1.0f;
+    if (KIND == 1) s_t = nv_tensor_scale(__uint_as_float(*amax_bits));
+    for (int64_t b = thread_index(); b < blocks; b += grid_stride()) {
+        uint32_t x[BS / 2];
+#pragma unroll
+        for (int c = 0; c < BS / 8; ++c) {
+            const uint4 v = __ldg(w + b * (BS / 8) + c);
+            x[4 * c + 0] = v.x; x[4 * c + 1] = v.y; x[4 * c + 2] = v.z; x[4 * c + 3] = v.w;
+        }
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < BS / 2; ++i)
+            amax = fmaxf(amax, fmaxf(fabsf(bf16_bits_to_f32(x[i] & 0xFFFFu)),
+                                     fabsf(bf16_bits_to_f32(x[i] >> 16))));
+        float scale;
+        uint32_t sb;
+        if (KIND == 0) {
+            int e = -127;
+            if (amax > 0.0f) {
+                e = ilogbf(amax) - 3;
+                while (amax > ldexpf(6.0f, e)) ++e;              // the smallest such e
+                if (e < -127) e = -127;
+                if (e > 127) e = 127;
+            }
+            sb = (uint32_t)(e + 127);
+            scale = ldexpf(1.0f, e);
+        } else {
+            sb = e4m3_round_up(__fdiv_rn(amax, __fmul_rn(6.0f, s_t)));
+            scale = __fmul_rn(e4m3_value(sb), s_t);
+        }
+        scales[b] = (uint8_t)sb;
+        uint32_t packed[BS / 8];
+#pragma unroll
+        for (int i = 0; i < BS / 8; ++i) packed[i] = 0u;
+#pragma unroll
+        for (int i = 0; i < BS; ++i) {
+            const uint32_t h = (i & 1) ? (x[i / 2] >> 16) : (x[i / 2] & 0xFFFFu);
+            const uint32_t c = scale > 0.0f ? e2m1_code(__fdiv_rn(bf16_bits_to_f32(h), scale)) : 0u;
+            packed[i / 8] |= c << (4 * (i % 8));
+        }
+        uint32_t *dst = reinterpret_cast<uint32_t *>(codes + b * (BS / 2));
+#pragma unroll
+        for (int i = 0; i < BS / 8; ++i) dst[i] = packed[i];
+    }
+}
+
+__global__ void fp4_finish_kernel(float *tensor_scale) {
+    *tensor_scale = nv_tensor_scale(*tensor_scale);
+}
+
+// One thread per 8 values (4 code bytes -> 16 bytes of bf16).
+template <int KIND>
+__global__ void __launch_bounds__(kThreads)
+fp4_dequantize_kernel(const uint32_t *__restrict__ codes, const uint8_t *__restrict__ scales,
+                      const float *__restrict__ tensor_scale, int64_t words,
+                      uint4 *__restrict__ out) {
+    constexpr int BS = KIND == 0 ? 32 : 16;
+    const float s_t = KIND == 1 ? *tensor_scale : 1.0f;
+    for (int64_t i = thread_index(); i < words; i += grid_stride()) {
+        const uint32_t cw = __ldg(codes + i);
+        const uint32_t sb = __ldg(scales + (i * 8) / BS);
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float v[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float q = e2m1_value((cw >> (4 * (2 * j + h))) & 0xFu);
+                if (KIND == 0) {
+                    v[h] = q * ldexpf(1.0f, (int)sb - 127);               // exact
+                } else {
+                    v[h] = __fmul_rn(__fmul_rn(q, e4m3_value(sb)), s_t);  // inner product exact
+                }
+            }
+            o[j] = dev::pack_bf16x2(v[0], v[1]);
+        }
+        out[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+unsigned grid_for(int64_t items) {
+    const int64_t cap = (int64_t)device_sm_count() * 16;
+    const int64_t b = (items + kThreads - 1) / kThreads;
+    return (unsigned)(b < 1 ? 1 : (b < cap ? b : cap));
+}
+
+}  // namespace
+
+int fp4_block_size(int kind) { return kind == 0 ? 32 : 16; }
+
+qz_status launch_fp4_quantize(const void *w, int64_t N, int64_t K, int kind, void *codes,
+                              void *scales, void *tensor_scale, cudaStream_t st) {
+    const int64_t blocks = N * K / fp4_block_size(kind);
+    const uint4 *w4 = static_cast<const uint4 *>(w);
+    if (kind == 0) {
+        fp4_quantize_kernel<0><<<grid_for(blocks), kThreads, 0, st>>>(
+            w4, blocks, static_cast<uint8_t *>(codes), static_cast<uint8_t *>(scales), nullptr);
+        return launch_status();
+    }
+    unsigned *amax = static_cast<unsigned *>(tensor_scale);      // amax first, then s_t
+    if (cudaMemsetAsync(amax, 0, sizeof(unsigned), st) != cudaSuccess) return QZ_ERR_CUDA;
+    const int64_t chunks = N * K / 8;
+    fp4_amax_kernel<<<grid_for(chunks), kThreads, 0, st>>>(w4, chunks, amax);
+    fp4_quantize_kernel<1><<<grid_for(blocks), kThreads, 0, st>>>(
+        w4, blocks, static_cast<uint8_t *>(codes), static_cast<uint8_t *>(scales), amax);
+    fp4_finish_kernel<<<1, 1, 0, st>>>(static_cast<float *>(tensor_scale));
+    return launch_status();
+}
+
+qz_status launch_fp4_dequantize(const void *codes, const void *scales, const void *tensor_scale,
+                                int64_t N, int64_t K, int kind, void *w_hat, cudaStream_t st) {
+    const int64_t words = N * K / 8;
+    const uint32_t *c = static_cast<const uint32_t *>(codes);
+    const uint8_t *s = static_cast<const uint8_t *>(scales);
+    uint4 *out = static_cast<uint4 *>(w_hat);
+    if (kind == 0)
+        fp4_dequantize_kernel<0><<<grid_for(words), kThreads, 0, st>>>(c, s, nullptr, words, out);
+    else
+        fp4_dequantize_kernel<1><<<grid_for(words), kThreads, 0, st>>>(
+            c, s, static_cast<const float *>(tensor_scale), words, out);
+    return launch_status();
+}
+
+}  // namespace qz

@@ -122,6 +122,17 @@ qz_status launch_w8a16_gemv(const void *a, const void *codes, const void *scales
 
 // Split-K workspace of the GEMM whose grid is sized for `sms` SMs; the
 // kSmCount figure (gemm_workspace_bytes) bounds every smaller count.
+// FP4 with block scales (qz_fp4.cu, qz_gemv.cu); kind 0 = MXFP4, 1 = NVFP4.
+int fp4_block_size(int kind);
+qz_status launch_fp4_quantize(const void *w, int64_t N, int64_t K, int kind, void *codes,
+                              void *scales, void *tensor_scale, cudaStream_t stream);
+qz_status launch_fp4_dequantize(const void *codes, const void *scales, const void *tensor_scale,
+                                int64_t N, int64_t K, int kind, void *w_hat, cudaStream_t stream);
+qz_status launch_fp4a16_gemv(const void *a, const void *codes, const void *scales,
+                             const void *tensor_scale, int64_t M, int64_t N, int64_t K, int kind,
+                             void *y, void *workspace, const GemvPlan &plan, int overlap,
+                             cudaStream_t stream);
+
 size_t gemm_workspace_bytes_for(int64_t M, int64_t N, int64_t K, int sms);
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 qz_status launch_w4a16_gemm(const void *a, const void *codes, const void *scales,

@@ -216,5 +216,43 @@ inline bool make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *ba
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// make_map_2d through a small process-wide cache: a map depends only on its
+// arguments, so a cached copy for the same arguments is always valid (also
+// when the memory behind `base` was freed and allocated again).  Saves the
+// host time of encoding the maps of every launch in decode loops.
+inline bool make_map_2d_cached(CUtensorMap *map, CUtensorMapDataType dt, const void *base,
+                               uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                               uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+    struct Entry {
+        const void *base;
+        uint64_t inner, outer, row_bytes;
+        uint32_t box_inner, box_outer;
+        int dt, swz;
+        bool used;
+        CUtensorMap map;
+    };
+    constexpr int kEntries = 64;
+    static Entry table[kEntries];
+    static int next = 0;
+    static std::mutex mu;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (const Entry &e : table)
+            if (e.used && e.base == base && e.inner == inner && e.outer == outer &&
+                e.row_bytes == row_bytes && e.box_inner == box_inner && e.box_outer == box_outer &&
+                e.dt == (int)dt && e.swz == (int)swz) {
+                *map = e.map;
+                return true;
+            }
+    }
+    if (!make_map_2d(map, dt, base, inner, outer, row_bytes, box_inner, box_outer, swz))
+        return false;
+    std::lock_guard<std::mutex> lock(mu);
+    Entry &e = table[next];
+    next = (next + 1) % kEntries;
+    e = Entry{base, inner, outer, row_bytes, box_inner, box_outer, (int)dt, (int)swz, true, *map};
+    return true;
+}
+
 }  // namespace sm100
 }  // namespace qz

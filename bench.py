@@ -98,16 +98,22 @@ def fp4_quant_bytes(N, K, kind):
 
 
 def gptq_flops(N, K, n):
-    """fp64 flops of one GPTQ call: H = 2 X X^T (2 n K^2), the Cholesky of the
-    damped H (K^3 / 3), the triangular inverse (K^3 / 3), the in-block and
-    lazy weight updates (2 N K^2 / 2 each way: N K^2 in all, 2 per FMA)."""
-    return 2 * n * K * K + (2 * K ** 3) // 3 + 2 * N * K * K
+    """Algorithmic fp64 flops of one GPTQ call (2 per multiply-add): the
+    symmetric H = 2 X X^T, one triangle of K^2 / 2 entries over n samples
+    (n K^2); the Cholesky of the damped H (K^3 / 3); the triangular inverse
+    (K^3 / 3); the weight updates, where quantizing column j moves every later
+    column k > j of every row once (K^2 / 2 pairs per row, N K^2 in all,
+    whether applied inside a block or by the lazy batch update)."""
+    return n * K * K + (2 * K ** 3) // 3 + N * K * K
 
 
 # fp64 peak of a B200 derived from its unit counts and clock (the pages and
 # the measured-peaks file give none): 148 SMs x 64 fp64 FMA lanes x 2 flops
 # x 1.965 GHz.
 FP64_PEAK_TFLOPS = 148 * 64 * 2 * 1.965e9 / 1e12
+# Dense FP4 tensor-core peak: the measured bf16 peak times the nominal ratio
+# of the two (9 PFLOP/s FP4 to 2.25 PFLOP/s bf16, dense).
+FP4_TO_BF16_NOMINAL = 4.0
 
 
 def peaks():
@@ -421,7 +427,33 @@ def run_extras(qz, dev, pk, stream):
             "ms": round(ms, 4), "TFLOP/s": round(tf, 1),
             "frac_of_burst": round(tf / pk["bf16_tflops"], 4),
             "frac_of_sustained": round(tf / pk["bf16_tflops_sustained"], 4)}
-        del c8, s8, a, y
+        del c8, s8
+        # W4A4 prefill (FP4 weights and activations, the activations quantized
+        # inside the call), same shape; the FP4 peak is the measured bf16 burst
+        # peak times the nominal FP4 : bf16 ratio
+        fp4_peak = pk["bf16_tflops"] * FP4_TO_BF16_NOMINAL
+        for kind, name in ((1, "nvfp4"), (0, "mxfp4")):
+            fc, fs, fts = qz.qz_fp4_quantize(w, kind)
+            fsm = qz.qz_fp4_scales_to_mma(fs, N, K, kind)
+            wsa = torch.empty(qz.qz_workspace_bytes(qz.QZ_OP_FP4A4_GEMM, M, N, K, 0),
+                              dtype=torch.uint8, device=dev)
+            qz.qz_fp4a4_gemm(a, fc, fsm, fts, N, K, kind, y=y, workspace=wsa)
+            ms = time_graph(capture(
+                lambda: qz.qz_fp4a4_gemm(a, fc, fsm, fts, N, K, kind, y=y, workspace=wsa), stream))
+            # the activation quantization alone (row-major scales, same work)
+            aq = qz.qz_fp4_quantize(a, kind)
+            msq = time_graph(capture(lambda: qz.qz_fp4_quantize(
+                a, kind, codes=aq[0], scales=aq[1], tensor_scale=aq[2]), stream))
+            tf = gemm_flops(M, N, K) / (ms * 1e-3) / 1e12
+            out[f"prefill_w4a4_{name}_2048x8192x8192"] = {
+                "ms": round(ms, 4), "TFLOP/s": round(tf, 1),
+                "fp4_peak_TFLOP/s_derived": round(fp4_peak, 1),
+                "frac_of_fp4_peak": round(tf / fp4_peak, 4),
+                "activation_quantize_ms": round(msq, 4),
+                "note": "ms covers the whole call: activation amax and quantization, then the "
+                        "block-scaled tcgen05 GEMM"}
+            del fc, fs, fts, fsm, wsa, aq
+        del a, y
 
         # Small-M crossover on the same layer: M <= 16 runs the decode kernel,
         # larger M the tcgen05 GEMM.  Weights rotate over copies larger than L2.
@@ -761,6 +793,8 @@ PROFILE_CASES = {
     "gemv_nvfp4_70b": ("gemv_nv", 1, 28672, 8192),
     "gemv_mxfp4_70b": ("gemv_mx", 1, 28672, 8192),
     "gptq_4096": ("gptq", 128, 4096, 4096),
+    "gemm_w4a4_nv": ("w4a4_nv", 2048, 8192, 8192),
+    "gemm_w4a4_mx": ("w4a4_mx", 2048, 8192, 8192),
     "quant_int8": ("quant8", 0, 28672, 8192),
     "dequant_int4": ("dequant", 0, 28672, 8192),
 }
@@ -778,9 +812,13 @@ def run_kernel_case(name, reps):
         c, s, z = qz.qz_quantize_pack(w, 4, False, GROUP)
     if kind in ("gemv8", "gemm8"):
         c, s, _ = qz.qz_quantize_pack(w, 8, True, K)
-    if kind in ("gemv_nv", "gemv_mx"):
-        fk = qz.QZ_FP4_NV if kind == "gemv_nv" else qz.QZ_FP4_MX
+    if kind in ("gemv_nv", "gemv_mx", "w4a4_nv", "w4a4_mx"):
+        fk = qz.QZ_FP4_NV if kind in ("gemv_nv", "w4a4_nv") else qz.QZ_FP4_MX
         c, s, ts = qz.qz_fp4_quantize(w, fk)
+        if kind.startswith("w4a4"):
+            s = qz.qz_fp4_scales_to_mma(s, N, K, fk)
+            ws = torch.empty(qz.qz_workspace_bytes(qz.QZ_OP_FP4A4_GEMM, M, N, K, 0),
+                             dtype=torch.uint8, device=dev)
     a = synthetic.activations(max(M, 1), K, seed=5, device=dev)
     torch.cuda.synchronize()
     for _ in range(reps):
@@ -800,6 +838,8 @@ def run_kernel_case(name, reps):
             qz.qz_dequantize(c, s, z, N, K, 4, False, GROUP)
         elif kind in ("gemv_nv", "gemv_mx"):
             qz.qz_fp4a16_gemv(a, c, s, ts, N, K, fk, workspace=ws)
+        elif kind in ("w4a4_nv", "w4a4_mx"):
+            qz.qz_fp4a4_gemm(a, c, s, ts, N, K, fk, workspace=ws)
         elif kind == "gptq":
             x = synthetic.activations(M, K, seed=77, device=dev)
             qz.qz_gptq_quantize(w, x, 4, False, GROUP)

@@ -85,7 +85,8 @@ enum {
     QZ_OP_W8A16_GEMV = 4,
     QZ_OP_W8A16_GEMM = 5,
     QZ_OP_GPTQ = 6,
-    QZ_OP_FP4A16_GEMV = 7
+    QZ_OP_FP4A16_GEMV = 7,
+    QZ_OP_FP4A4_GEMM = 8
 };
 
 /* FP4 formats (kind argument of the qz_fp4_* entry points). */
@@ -315,6 +316,45 @@ QZ_API qz_status qz_fp4a16_gemv(const void *a, const void *codes, const void *bl
                                 const void *tensor_scale, int64_t M, int64_t N, int64_t K,
                                 int32_t kind, void *y, void *workspace, size_t workspace_bytes,
                                 void *stream);
+
+/*
+ * W4A4 prefill GEMM with FP4 weights and activations ("Quantize weights or
+ * activations": for compute-bound prefill, quantizing the activations too lets
+ * the matmul itself run on 4-bit tensor cores, NVFP4 W4A4; section "FP4 with
+ * block scales" for the format).  The tensor cores apply the block scales
+ * inside the MMA, so they need the scales of every 128 rows in the "MMA scale
+ * layout": atoms of 128 rows x 4 consecutive scales of a row (512 bytes),
+ * scale j of row r at byte (r % 32) * 16 + ((r % 128) / 32) * 4 + j % 4 of
+ * atom (r / 128, j / 4), which starts at ((r / 128) * (K / B / 4) + j / 4) *
+ * 512; rows are padded with zero scales to a multiple of 128.
+ *
+ * qz_fp4_mma_scale_bytes: bytes of that layout for `rows` rows.
+ * qz_fp4_scales_to_mma: block scales as written by qz_fp4_quantize (rows x
+ *   K/B bytes, 4-byte aligned) -> the MMA scale layout (16-byte aligned); a
+ *   one-time conversion for weights.
+ * qz_fp4a4_gemm: y (M x N bf16) = a_hat (M x K) * w_hat^T, where a_hat is a
+ *   (M x K bf16, 16-byte aligned) quantized inside the call to the same FP4
+ *   kind exactly as qz_fp4_quantize would (NVFP4 with its own tensor scale
+ *   from max |a|), w_hat the FP4 weights: codes (N x K/2, 16-byte aligned),
+ *   scales_mma (from qz_fp4_scales_to_mma) and, for NVFP4, tensor_scale (one
+ *   fp32 in device memory; NULL for MXFP4).  The sums are fp32; NVFP4 scales
+ *   them by fp32(s_t(a) * s_t(w)) before rounding to bf16.  After the call
+ *   the workspace holds the quantized activations: codes (M x K/2 bytes) at
+ *   offset 0, their scales in the MMA scale layout at offset
+ *   round_up(M * K / 2, 256), and (NVFP4) max |a| as fp32 after those,
+ *   at the next multiple of 256.
+ * Requirements: M, N >= 1; K % 256 == 0.  Workspace: qz_workspace_bytes(
+ * QZ_OP_FP4A4_GEMM, M, N, K, 0) bytes, 256-byte aligned; it need not be
+ * zero-filled and is not left zero-filled, so it must not be a buffer that
+ * the split-K calls above count on.
+ */
+QZ_API qz_status qz_fp4_mma_scale_bytes(int64_t rows, int64_t K, int32_t kind, size_t *bytes);
+QZ_API qz_status qz_fp4_scales_to_mma(const void *block_scales, int64_t rows, int64_t K,
+                                      int32_t kind, void *scales_mma, void *stream);
+QZ_API qz_status qz_fp4a4_gemm(const void *a, const void *codes, const void *scales_mma,
+                               const void *tensor_scale, int64_t M, int64_t N, int64_t K,
+                               int32_t kind, void *y, void *workspace, size_t workspace_bytes,
+                               void *stream);
 
 /*
  * Size of the scratch array built into the library for

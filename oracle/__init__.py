@@ -58,6 +58,8 @@ def load(path: str):
     L.qzo_fp4_dequantize.restype = _int
     L.qzo_matmul_f64_exact.argtypes = [_p, _p, _i64, _i64, _i64, _p, _p]
     L.qzo_matmul_f64_exact.restype = _int
+    L.qzo_matmul_f64_ab.argtypes = [_p, _p, _i64, _i64, _i64, _p, _p]
+    L.qzo_matmul_f64_ab.restype = _int
     L.qzo_set_threads.argtypes = [_int]
     L.qzo_set_threads.restype = None
     L.qzo_max_threads.argtypes = []
@@ -203,6 +205,19 @@ def matmul_f64_exact(a_bits, w_exact):
     y = np.zeros((M, N), dtype=np.float64)
     ya = np.zeros((M, N), dtype=np.float64)
     lib().qzo_matmul_f64_exact(_ptr(a), _ptr(w), M, N, K, _ptr(y), _ptr(ya))
+    return y, ya
+
+
+def matmul_f64_ab(a_exact, w_exact):
+    """fp64 y = a @ w^T and sum_k |a w| for fp64 activations and weights (the
+    W4A4 reference: both are exact dequantized FP4 values)."""
+    a = np.ascontiguousarray(a_exact, dtype=np.float64)
+    w = np.ascontiguousarray(w_exact, dtype=np.float64)
+    M, K = a.shape
+    N = w.shape[0]
+    y = np.zeros((M, N), dtype=np.float64)
+    ya = np.zeros((M, N), dtype=np.float64)
+    lib().qzo_matmul_f64_ab(_ptr(a), _ptr(w), M, N, K, _ptr(y), _ptr(ya))
     return y, ya
 
 

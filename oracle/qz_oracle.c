@@ -505,6 +505,30 @@ int qzo_matmul_f64_exact(const uint16_t *a, const double *w, int64_t M, int64_t 
     return 0;
 }
 
+/* y = a @ w^T and sum_k |a w| in fp64 for fp64 a (M x K) and w (N x K):
+ * the W4A4 reference, both operands already exact dequantized FP4 values
+ * (Quantization concepts guide, "Quantize weights or activations": NVFP4
+ * W4A4 quantizes the activations as well as the weights). */
+int qzo_matmul_f64_ab(const double *a, const double *w, int64_t M, int64_t N, int64_t K,
+                      double *y, double *abs_y)
+{
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t m = 0; m < M; ++m) {
+            double sum = 0.0, sum_abs = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double t = a[m * K + k] * w[n * K + k];
+                sum += t;
+                sum_abs += fabs(t);
+            }
+            y[m * N + n] = sum;
+            abs_y[m * N + n] = sum_abs;
+        }
+    return 0;
+}
+
 /* ------------------------------------------------------------------ */
 /* GPTQ layer-wise quantizer (GPTQ explainer, azimuth.plus/paper/gptq).  */
 /*                                                                        */

@@ -659,5 +659,43 @@ def pin_fp4_dequant_closed_form():
         assert np.array_equal(w_exact, exact.reshape(8, 256))
 
 
+def _exact_int_products(M, N, K, seed):
+    """Integer matrices times powers of two: every product and partial sum is
+    exact in fp64, so the reference must equal integer arithmetic."""
+    rng = np.random.default_rng(seed)
+    ai = rng.integers(-7, 8, (M, K))
+    wi = rng.integers(-6, 7, (N, K))
+    exact = ai.astype(object).dot(wi.T.astype(object))              # Python integers
+    exact_abs = np.abs(ai).astype(object).dot(np.abs(wi).T.astype(object))
+    return ai, wi, np.array(exact, dtype=np.float64), np.array(exact_abs, dtype=np.float64)
+
+
+def pin_matmul_f64_exact_integers():
+    """bf16 activations x fp64 weights: small integers scaled by 2^-3 and 2^-5
+    (exact in bf16 and fp64) give integer arithmetic scaled by 2^-8; the
+    shape is not square, so a transposed operand cannot pass."""
+    M, N, K = 3, 5, 40
+    ai, wi, exact, exact_abs = _exact_int_products(M, N, K, 810)
+    a_bits = (torch.from_numpy(ai * 0.125).to(torch.bfloat16).view(torch.int16).numpy()
+              .view(np.uint16))
+    y, ya = oracle.matmul_f64_exact(a_bits, wi * 0.03125)
+    assert np.array_equal(y, exact / 256.0)
+    assert np.array_equal(ya, exact_abs / 256.0)
+
+
+def pin_matmul_f64_ab_integers():
+    """fp64 x fp64: the same integer check, with fractional power-of-two
+    scales on both operands, and a one-hot row that returns a weight column."""
+    M, N, K = 4, 6, 72
+    ai, wi, exact, exact_abs = _exact_int_products(M, N, K, 811)
+    y, ya = oracle.matmul_f64_ab(ai * 0.5, wi * 0.0625)
+    assert np.array_equal(y, exact / 32.0)
+    assert np.array_equal(ya, exact_abs / 32.0)
+    onehot = np.zeros((1, K))
+    onehot[0, 9] = 1.0
+    y1, _ = oracle.matmul_f64_ab(onehot, wi * 0.0625)
+    assert np.array_equal(y1[0], wi[:, 9] * 0.0625)
+
+
 # every pin_* function of this module (defined last, after all of them)
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -273,3 +273,28 @@ def test_fp4_gemv_rejects_and_workspace():
         qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMV, 4, 4096, 4096, 128)
     assert qz.qz_fp4_packed_bytes(64, 1024, qz.QZ_FP4_MX) == (64 * 512, 64 * 32)
     assert qz.qz_fp4_packed_bytes(64, 1024, qz.QZ_FP4_NV) == (64 * 512, 64 * 64)
+
+
+def test_fp4a4_gemm_rejects_and_workspace():
+    ts = C
+    big = ctypes.c_void_p(0x100000)
+    assert L().qz_fp4a4_gemm(A, B, D, ts, 64, 64, 192, 1, Y, big, 1 << 20, None) == UNSUP  # K % 256
+    assert L().qz_fp4a4_gemm(A, B, D, ts, 64, 64, 256, 2, Y, big, 1 << 20, None) == UNSUP  # kind
+    assert L().qz_fp4a4_gemm(A, B, D, None, 64, 64, 256, 1, Y, big, 1 << 20, None) == INVALID
+    assert L().qz_fp4a4_gemm(A, B, D, ts, 64, 64, 256, 0, Y, big, 1 << 20, None) == INVALID
+    assert L().qz_fp4a4_gemm(A, B, D, ts, 0, 64, 256, 1, Y, big, 1 << 20, None) == INVALID
+    assert L().qz_fp4a4_gemm(MIS, B, D, ts, 64, 64, 256, 1, Y, big, 1 << 20, None) == ALIGN
+    assert L().qz_fp4a4_gemm(A, B, MIS, ts, 64, 64, 256, 1, Y, big, 1 << 20, None) == ALIGN
+    assert L().qz_fp4a4_gemm(A, B, D, ts, 64, 64, 256, 1, Y, None, 0, None) == WS
+    assert L().qz_fp4a4_gemm(A, B, D, ts, 64, 64, 256, 1, Y, MIS, 1 << 20, None) == ALIGN
+    # activation codes, their scales (NVFP4-sized atoms) and one word for max |a|
+    M, K = 2048, 8192
+    assert qz.qz_workspace_bytes(qz.QZ_OP_FP4A4_GEMM, M, 8192, K, 0) == \
+        M * K // 2 + (M // 128) * (K // 64) * 512 + 256
+    assert qz.qz_workspace_bytes(qz.QZ_OP_FP4A4_GEMM, 37, 300, 512, 0) == \
+        37 * 256 + 512 * 8 + 256       # 37 x 256 code bytes are already a multiple of 256
+    assert qz.qz_fp4_mma_scale_bytes(300, 1024, qz.QZ_FP4_NV) == 3 * (1024 // 64) * 512
+    assert qz.qz_fp4_mma_scale_bytes(300, 1024, qz.QZ_FP4_MX) == 3 * (1024 // 128) * 512
+    assert L().qz_fp4_scales_to_mma(A, 300, 1000, 1, B, None) == UNSUP
+    assert L().qz_fp4_scales_to_mma(None, 300, 1024, 1, B, None) == INVALID
+    assert L().qz_fp4_scales_to_mma(A, 300, 1024, 1, MIS, None) == ALIGN

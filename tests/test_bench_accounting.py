@@ -126,8 +126,18 @@ def test_fp4_gemv_and_quantize_bytes():
 
 
 def test_gptq_flops_and_fp64_peak():
-    # 4096 x 4096 with 128 samples: 2 n K^2 + 2/3 K^3 + 2 N K^2
-    f = bench.gptq_flops(4096, 4096, 128)
-    assert f == 2 * 128 * 4096 ** 2 + (2 * 4096 ** 3) // 3 + 2 * 4096 ** 3
-    assert abs(f / 1e9 - 187.55) <= 0.005    # 4.29 + 45.81 + 137.44
+    """The leading-order count against multiply-adds counted one by one
+    (2 flops each): the lower triangle of X^T X over n samples; the Cholesky
+    (column j updates the (K-j-1)(K-j)/2 entries of the trailing triangle);
+    the triangular inverse (entry (i, j), i > j, of L^-1 sums i - j terms);
+    each quantized column j moves every later column of every row once."""
+    N, K, n = 4096, 4096, 128
+    f = bench.gptq_flops(N, K, n)
+    hess = n * K * (K + 1) // 2
+    chol = sum((K - j - 1) * (K - j) // 2 for j in range(K))
+    trinv = sum(d * (K - d) for d in range(1, K))        # K - d entries at distance d
+    updates = N * K * (K - 1) // 2
+    exact = 2 * (hess + chol + trinv + updates)
+    assert abs(f - exact) / exact < 1e-3
+    assert abs(f / 1e9 - 116.68) <= 0.005    # 2.15 + 45.81 + 68.72
     assert abs(bench.FP64_PEAK_TFLOPS - 37.23) <= 0.01

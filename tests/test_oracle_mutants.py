@@ -66,6 +66,11 @@ MUTANTS = {
     "fp4_nv_tensor_scale_without_fp8_range": ("s_t = amax > 0.0f ? amax / 2688.0f : 1.0f;",
                                               "s_t = amax > 0.0f ? amax / 6.0f : 1.0f;"),
     "fp4_e4m3_bias_off_by_one": ("ldexp(1.0 + m / 8.0, e - 7)", "ldexp(1.0 + m / 8.0, e - 8)"),
+    "matmul_exact_transposed_weights": ("* w[n * K + k];\n                acc += p;",
+                                        "* w[k * N + n % K];\n                acc += p;"),
+    "matmul_ab_abs_sum_signed": ("sum_abs += fabs(t);", "sum_abs += t;"),
+    "matmul_ab_transposed_activations": ("double t = a[m * K + k] * w[n * K + k];",
+                                         "double t = a[k * M + m % K] * w[n * K + k];"),
     "gptq_no_damping": ("double lambda = mean > 0.0 ? damp * mean : 1.0;",
                         "double lambda = mean > 0.0 ? 0.0 : 1.0;"),
 }

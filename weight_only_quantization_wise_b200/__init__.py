@@ -21,7 +21,8 @@ __all__ = [
     "qz_w4a16_gemm", "qz_w8a16_gemv", "qz_w8a16_gemm", "qz_set_device_wait_limit",
     "qz_set_launch_overlap", "qz_device_status", "qz_gptq_quantize", "QZ_OP_GPTQ",
     "qz_fp4_packed_bytes", "qz_fp4_quantize", "qz_fp4_dequantize", "qz_fp4a16_gemv",
-    "QZ_OP_FP4A16_GEMV", "QZ_FP4_MX", "QZ_FP4_NV",
+    "QZ_OP_FP4A16_GEMV", "QZ_FP4_MX", "QZ_FP4_NV", "qz_fp4_mma_scale_bytes",
+    "qz_fp4_scales_to_mma", "qz_fp4a4_gemm", "QZ_OP_FP4A4_GEMM",
     "Workspace", "QZ_OP_QUANTIZE_PACK", "QZ_OP_DEQUANTIZE", "QZ_OP_W4A16_GEMV",
     "QZ_OP_W4A16_GEMM", "QZ_OP_W8A16_GEMV", "QZ_OP_W8A16_GEMM", "EXPORTED_SYMBOLS",
 ]
@@ -31,7 +32,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqz.so")
 QZ_OK = 0
 QZ_ERR_DEVICE_TIMEOUT = 6
 (QZ_OP_QUANTIZE_PACK, QZ_OP_DEQUANTIZE, QZ_OP_W4A16_GEMV, QZ_OP_W4A16_GEMM, QZ_OP_W8A16_GEMV,
- QZ_OP_W8A16_GEMM, QZ_OP_GPTQ, QZ_OP_FP4A16_GEMV) = range(8)
+ QZ_OP_W8A16_GEMM, QZ_OP_GPTQ, QZ_OP_FP4A16_GEMV, QZ_OP_FP4A4_GEMM) = range(9)
 QZ_FP4_MX, QZ_FP4_NV = 0, 1
 FP4_BLOCK = {QZ_FP4_MX: 32, QZ_FP4_NV: 16}
 
@@ -58,6 +59,9 @@ _SIGS = {
     "qz_fp4_quantize": ([_p, _i64, _i64, _i32, _p, _p, _p, _p], ctypes.c_int),
     "qz_fp4_dequantize": ([_p, _p, _p, _i64, _i64, _i32, _p, _p], ctypes.c_int),
     "qz_fp4a16_gemv": ([_p, _p, _p, _p, _i64, _i64, _i64, _i32, _p, _p, _sz, _p], ctypes.c_int),
+    "qz_fp4_mma_scale_bytes": ([_i64, _i64, _i32, ctypes.POINTER(_sz)], ctypes.c_int),
+    "qz_fp4_scales_to_mma": ([_p, _i64, _i64, _i32, _p, _p], ctypes.c_int),
+    "qz_fp4a4_gemm": ([_p, _p, _p, _p, _i64, _i64, _i64, _i32, _p, _p, _sz, _p], ctypes.c_int),
     "qz_set_device_wait_limit": ([ctypes.c_uint64], None),
     "qz_set_launch_overlap": ([ctypes.c_int32], ctypes.c_int),
     "qz_device_status": ([], ctypes.c_int),
@@ -167,6 +171,14 @@ class Workspace:
         if self.buf is None or self.buf.numel() < nbytes:
             self.buf = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=self.device)
         return self.buf
+
+    def get_scratch(self, nbytes: int):
+        """A second buffer for calls whose workspace is plain scratch (the
+        W4A4 GEMM's quantized activations): it is not zero-filled and must
+        not be the one the split-K calls count on."""
+        if getattr(self, "scratch", None) is None or self.scratch.numel() < nbytes:
+            self.scratch = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=self.device)
+        return self.scratch
 
 
 def _ws_args(workspace, nbytes, device):
@@ -377,6 +389,47 @@ def qz_fp4a16_gemv(a, codes, scales, tensor_scale, N, K, kind, y=None, workspace
         _check(lib.qz_fp4a16_gemv(_ptr(a), _ptr(codes), _ptr(scales), _ptr(tensor_scale), M, N,
                                   K, kind, _ptr(y), ws_ptr, ws_bytes, _handle(st)),
                "qz_fp4a16_gemv")
+    return y
+
+
+def qz_fp4_mma_scale_bytes(rows, K, kind) -> int:
+    out = _sz()
+    _check(lib.qz_fp4_mma_scale_bytes(rows, K, kind, ctypes.byref(out)), "qz_fp4_mma_scale_bytes")
+    return out.value
+
+
+def qz_fp4_scales_to_mma(scales, rows, K, kind, out=None, stream=None):
+    """Block scales as qz_fp4_quantize writes them -> the MMA scale layout
+    (uint8 tensor of qz_fp4_mma_scale_bytes(rows, K, kind) bytes)."""
+    st = _launch_stream(stream, scales.device)
+    with _on(stream):
+        if out is None:
+            out = torch.empty(qz_fp4_mma_scale_bytes(rows, K, kind), dtype=torch.uint8,
+                              device=scales.device)
+        _check(lib.qz_fp4_scales_to_mma(_ptr(scales), rows, K, kind, _ptr(out), _handle(st)),
+               "qz_fp4_scales_to_mma")
+    return out
+
+
+def qz_fp4a4_gemm(a, codes, scales_mma, tensor_scale, N, K, kind, y=None, workspace=None,
+                  stream=None):
+    """W4A4: y = a_hat * w_hat^T with the activations quantized to the same FP4
+    kind inside the call.  `workspace`: a uint8 tensor, a Workspace (its
+    scratch buffer is used) or None; after the call it holds the quantized
+    activations."""
+    st = _launch_stream(stream, a.device)
+    M = a.shape[0]
+    with _on(stream):
+        y = _matmul_out(a, N, y)
+        nbytes = qz_workspace_bytes(QZ_OP_FP4A4_GEMM, M, N, K, 0)
+        if workspace is None:
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=a.device)
+        elif isinstance(workspace, Workspace):
+            workspace = workspace.get_scratch(nbytes)
+        _check(lib.qz_fp4a4_gemm(_ptr(a), _ptr(codes), _ptr(scales_mma), _ptr(tensor_scale), M,
+                                 N, K, kind, _ptr(y), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _handle(st)),
+               "qz_fp4a4_gemm")
     return y
 
 

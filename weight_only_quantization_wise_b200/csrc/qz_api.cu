@@ -80,6 +80,17 @@ qz_status check_workspace(size_t need, const void *ws, size_t ws_bytes) {
 
 cudaStream_t as_stream(void *s) { return static_cast<cudaStream_t>(s); }
 
+// W4A4 GEMM shapes: whole 256-wide K stages (one 128-byte row of codes per
+// stage, 4 or 2 whole scale atoms).
+qz_status check_fp4a4(int64_t M, int64_t N, int64_t K, int32_t kind) {
+    if (kind != QZ_FP4_MX && kind != QZ_FP4_NV) return QZ_ERR_UNSUPPORTED;
+    if (M < 1 || N < 1 || K < 1 || M > kMaxDim || N > kMaxDim || K > kMaxDim ||
+        M * K > kMaxElems || N * K > kMaxElems || M * N > kMaxElems)
+        return QZ_ERR_INVALID_ARG;
+    if (K % 256 != 0) return QZ_ERR_UNSUPPORTED;
+    return QZ_OK;
+}
+
 }  // namespace
 }  // namespace qz
 
@@ -152,6 +163,12 @@ QZ_API qz_status qz_workspace_bytes(int32_t op, int64_t M, int64_t N, int64_t K,
         if (N < 1 || K < 1 || N > kMaxDim || K > kMaxDim) return QZ_ERR_INVALID_ARG;
         *bytes = gptq_workspace_bytes(N, K);
         return QZ_OK;
+    case QZ_OP_FP4A4_GEMM: {
+        const qz_status s = check_fp4a4(M, N, K, QZ_FP4_NV);
+        if (s != QZ_OK) return s;
+        *bytes = fp4a4_workspace_bytes(M, K);
+        return QZ_OK;
+    }
     default:
         return QZ_ERR_INVALID_ARG;
     }
@@ -380,6 +397,41 @@ QZ_API qz_status qz_set_launch_overlap(int32_t mode) {
     if (mode < 0 || mode > 1) return QZ_ERR_INVALID_ARG;
     g_launch_overlap.store(mode, std::memory_order_relaxed);
     return QZ_OK;
+}
+
+QZ_API qz_status qz_fp4_mma_scale_bytes(int64_t rows, int64_t K, int32_t kind, size_t *bytes) {
+    if (!bytes) return QZ_ERR_INVALID_ARG;
+    const qz_status s = check_fp4a4(rows, 1, K, kind);
+    if (s != QZ_OK) return s;
+    *bytes = fp4_mma_scale_bytes(rows, K, kind);
+    return QZ_OK;
+}
+
+QZ_API qz_status qz_fp4_scales_to_mma(const void *block_scales, int64_t rows, int64_t K,
+                                      int32_t kind, void *scales_mma, void *stream) {
+    const qz_status s = check_fp4a4(rows, 1, K, kind);
+    if (s != QZ_OK) return s;
+    if (!block_scales || !scales_mma) return QZ_ERR_INVALID_ARG;
+    if (!aligned(block_scales, 4) || !aligned(scales_mma, 16)) return QZ_ERR_ALIGNMENT;
+    return launch_fp4_scales_to_mma(block_scales, rows, K, kind, scales_mma, as_stream(stream));
+}
+
+QZ_API qz_status qz_fp4a4_gemm(const void *a, const void *codes, const void *scales_mma,
+                               const void *tensor_scale, int64_t M, int64_t N, int64_t K,
+                               int32_t kind, void *y, void *workspace, size_t workspace_bytes,
+                               void *stream) {
+    qz_status s = check_fp4a4(M, N, K, kind);
+    if (s != QZ_OK) return s;
+    if (!a || !codes || !scales_mma || !y) return QZ_ERR_INVALID_ARG;
+    if (kind == QZ_FP4_NV ? tensor_scale == nullptr : tensor_scale != nullptr)
+        return QZ_ERR_INVALID_ARG;
+    if (!aligned(a, 16) || !aligned(codes, 16) || !aligned(scales_mma, 16) || !aligned(y, 2) ||
+        (tensor_scale && !aligned(tensor_scale, 4)))
+        return QZ_ERR_ALIGNMENT;
+    s = check_workspace(fp4a4_workspace_bytes(M, K), workspace, workspace_bytes);
+    if (s != QZ_OK) return s;
+    return launch_fp4a4_gemm(a, codes, scales_mma, tensor_scale, M, N, K, kind, y, workspace,
+                             as_stream(stream));
 }
 
 }  // extern "C"

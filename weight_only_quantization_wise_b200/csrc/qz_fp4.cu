@@ -116,11 +116,22 @@ __device__ __forceinline__ float nv_tensor_scale(float amax) {
     return amax > 0.0f ? __fdiv_rn(amax, 2688.0f) : 1.0f;
 }
 
-// One thread per block of BS values (BS / 8 chunks of 16 bytes).
-template <int KIND>
+// Byte offset of scale j of row r in the MMA scale layout: atoms of 128
+// rows x 4 scales (512 bytes), row r at (r % 32) * 16 + ((r % 128) / 32) * 4
+// + j % 4 inside its atom, atoms ordered (r / 128, j / 4) with `atoms_k`
+// atoms per 128-row block.
+__device__ __forceinline__ int64_t mma_scale_offset(int64_t r, int64_t j, int64_t atoms_k) {
+    return (((r >> 7) * atoms_k + (j >> 2)) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2) + (j & 3);
+}
+
+// One thread per block of BS values (BS / 8 chunks of 16 bytes).  MMA:
+// scales in the MMA scale layout (blocks_per_row scales per row) instead of
+// row-major.
+template <int KIND, bool MMA = false>
 __global__ void __launch_bounds__(kThreads)
 fp4_quantize_kernel(const uint4 *__restrict__ w, int64_t blocks, uint8_t *__restrict__ codes,
-                    uint8_t *__restrict__ scales, const unsigned *__restrict__ amax_bits) {
+                    uint8_t *__restrict__ scales, const unsigned *__restrict__ amax_bits,
+                    int64_t blocks_per_row = 0) {
     constexpr int BS = KIND == 0 ? 32 : 16;
     float s_t = 1.0f;
     if (KIND == 1) s_t = nv_tensor_scale(__uint_as_float(*amax_bits));
@@ -152,7 +163,12 @@ fp4_quantize_kernel(const uint4 *__restrict__ w, int64_t blocks, uint8_t *__rest
             sb = e4m3_round_up(__fdiv_rn(amax, __fmul_rn(6.0f, s_t)));
             scale = __fmul_rn(e4m3_value(sb), s_t);
         }
-        scales[b] = (uint8_t)sb;
+        if (MMA) {
+            const int64_t r = b / blocks_per_row;
+            scales[mma_scale_offset(r, b - r * blocks_per_row, blocks_per_row >> 2)] = (uint8_t)sb;
+        } else {
+            scales[b] = (uint8_t)sb;
+        }
         uint32_t packed[BS / 8];
 #pragma unroll
         for (int i = 0; i < BS / 8; ++i) packed[i] = 0u;
@@ -165,6 +181,18 @@ fp4_quantize_kernel(const uint4 *__restrict__ w, int64_t blocks, uint8_t *__rest
         uint32_t *dst = reinterpret_cast<uint32_t *>(codes + b * (BS / 2));
 #pragma unroll
         for (int i = 0; i < BS / 8; ++i) dst[i] = packed[i];
+    }
+}
+
+// Row-major block scales (rows x words_per_row 32-bit words of 4 scales) into
+// the MMA scale layout; rows up to the next multiple of 128 get zero scales.
+__global__ void __launch_bounds__(kThreads)
+fp4_scales_to_mma_kernel(const uint32_t *__restrict__ src, int64_t rows, int64_t words_per_row,
+                         int64_t total, uint32_t *__restrict__ dst) {
+    for (int64_t i = thread_index(); i < total; i += grid_stride()) {
+        const int64_t r = i / words_per_row, jw = i - r * words_per_row;
+        const uint32_t v = r < rows ? __ldg(src + i) : 0u;
+        dst[mma_scale_offset(r, 4 * jw, words_per_row) >> 2] = v;
     }
 }
 
@@ -228,6 +256,46 @@ qz_status launch_fp4_quantize(const void *w, int64_t N, int64_t K, int kind, voi
     fp4_quantize_kernel<1><<<grid_for(blocks), kThreads, 0, st>>>(
         w4, blocks, static_cast<uint8_t *>(codes), static_cast<uint8_t *>(scales), amax);
     fp4_finish_kernel<<<1, 1, 0, st>>>(static_cast<float *>(tensor_scale));
+    return launch_status();
+}
+
+// Activations for the W4A4 GEMM: codes row-major, scales in the MMA scale
+// layout (rows beyond M zero), and for NVFP4 max |a| in *amax_word (the GEMM
+// forms the tensor scale from it as qz_fp4_quantize does).
+qz_status launch_fp4_quantize_mma(const void *a, int64_t M, int64_t K, int kind, void *codes,
+                                  void *scales_mma, void *amax_word, cudaStream_t st) {
+    const int bs = fp4_block_size(kind);
+    const int64_t blocks = M * K / bs, per_row = K / bs;
+    const uint4 *a4 = static_cast<const uint4 *>(a);
+    if (M % 128 != 0) {
+        // the last 128-row block holds padding rows: their scales must read 0
+        const int64_t atom_row = (per_row / 4) * 512;
+        if (cudaMemsetAsync(static_cast<uint8_t *>(scales_mma) + (M / 128) * atom_row, 0,
+                            (size_t)atom_row, st) != cudaSuccess)
+            return QZ_ERR_CUDA;
+    }
+    unsigned *amax = static_cast<unsigned *>(amax_word);
+    if (kind == 0) {
+        fp4_quantize_kernel<0, true><<<grid_for(blocks), kThreads, 0, st>>>(
+            a4, blocks, static_cast<uint8_t *>(codes), static_cast<uint8_t *>(scales_mma), nullptr,
+            per_row);
+        return launch_status();
+    }
+    if (cudaMemsetAsync(amax, 0, sizeof(unsigned), st) != cudaSuccess) return QZ_ERR_CUDA;
+    const int64_t chunks = M * K / 8;
+    fp4_amax_kernel<<<grid_for(chunks), kThreads, 0, st>>>(a4, chunks, amax);
+    fp4_quantize_kernel<1, true><<<grid_for(blocks), kThreads, 0, st>>>(
+        a4, blocks, static_cast<uint8_t *>(codes), static_cast<uint8_t *>(scales_mma), amax, per_row);
+    return launch_status();
+}
+
+qz_status launch_fp4_scales_to_mma(const void *scales, int64_t rows, int64_t K, int kind,
+                                   void *scales_mma, cudaStream_t st) {
+    const int64_t words_per_row = K / fp4_block_size(kind) / 4;
+    const int64_t total = ceil_div(rows, 128) * 128 * words_per_row;
+    fp4_scales_to_mma_kernel<<<grid_for(total), kThreads, 0, st>>>(
+        static_cast<const uint32_t *>(scales), rows, words_per_row, total,
+        static_cast<uint32_t *>(scales_mma));
     return launch_status();
 }
 

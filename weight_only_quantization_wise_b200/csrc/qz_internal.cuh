@@ -120,9 +120,8 @@ qz_status launch_w8a16_gemv(const void *a, const void *codes, const void *scales
                             int64_t M, int64_t N, int64_t K, void *y, void *workspace,
                             const GemvPlan &plan, int overlap, cudaStream_t stream);
 
-// Split-K workspace of the GEMM whose grid is sized for `sms` SMs; the
-// kSmCount figure (gemm_workspace_bytes) bounds every smaller count.
-// FP4 with block scales (qz_fp4.cu, qz_gemv.cu); kind 0 = MXFP4, 1 = NVFP4.
+// FP4 with block scales (qz_fp4.cu, qz_gemv.cu, qz_gemm_fp4.cu); kind 0 =
+// MXFP4, 1 = NVFP4.
 int fp4_block_size(int kind);
 qz_status launch_fp4_quantize(const void *w, int64_t N, int64_t K, int kind, void *codes,
                               void *scales, void *tensor_scale, cudaStream_t stream);
@@ -133,6 +132,18 @@ qz_status launch_fp4a16_gemv(const void *a, const void *codes, const void *scale
                              void *y, void *workspace, const GemvPlan &plan, int overlap,
                              cudaStream_t stream);
 
+// W4A4 GEMM: the MMA scale layout (atoms of 128 rows x 4 scales), the
+// in-call activation quantization and the block-scaled tcgen05 GEMM.
+size_t fp4_mma_scale_bytes(int64_t rows, int64_t K, int kind);
+size_t fp4a4_workspace_bytes(int64_t M, int64_t K);
+qz_status launch_fp4_scales_to_mma(const void *scales, int64_t rows, int64_t K, int kind,
+                                   void *scales_mma, cudaStream_t stream);
+qz_status launch_fp4a4_gemm(const void *a, const void *w_codes, const void *w_scales_mma,
+                            const void *w_tensor_scale, int64_t M, int64_t N, int64_t K, int kind,
+                            void *y, void *workspace, cudaStream_t stream);
+
+// Split-K workspace of the GEMM whose grid is sized for `sms` SMs; the
+// kSmCount figure (gemm_workspace_bytes) bounds every smaller count.
 size_t gemm_workspace_bytes_for(int64_t M, int64_t N, int64_t K, int sms);
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 qz_status launch_w4a16_gemm(const void *a, const void *codes, const void *scales,

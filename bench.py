@@ -374,7 +374,7 @@ def qz_gemm_kernel_for(M):
     return "decode GEMV" if M <= GEMM_ROUTES_TO_GEMV_UP_TO else "tcgen05 GEMM"
 
 
-GEMM_ROUTES_TO_GEMV_UP_TO = 16
+GEMM_ROUTES_TO_GEMV_UP_TO = 32
 
 
 def run_extras(qz, dev, pk, stream):
@@ -455,7 +455,7 @@ def run_extras(qz, dev, pk, stream):
             del fc, fs, fts, fsm, wsa, aq
         del a, y
 
-        # Small-M crossover on the same layer: M <= 16 runs the decode kernel,
+        # Small-M crossover on the same layer: M <= 32 runs the decode kernel,
         # larger M the tcgen05 GEMM.  Weights rotate over copies larger than L2.
         packs4 = [qz.qz_quantize_pack(w if r == 0 else w.clone(), 4, False, GROUP) for r in range(4)]
         packs8 = [qz.qz_quantize_pack(w if r == 0 else w.clone(), 8, True, K) for r in range(2)]
@@ -479,7 +479,7 @@ def run_extras(qz, dev, pk, stream):
             ms4 = time_graph(capture(f4, stream)) / len(packs4)
             ms8 = time_graph(capture(f8, stream)) / len(packs8)
             b4, b8 = w4_gemv_bytes(Ms, N, K), w8_gemv_bytes(Ms, N, K)
-            if 16 < Ms <= 64:
+            if GEMM_ROUTES_TO_GEMV_UP_TO < Ms <= 64:
                 # the same tokens through the decode GEMV (up to 64 tokens)
                 wsg = torch.zeros(max(256, qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMV, Ms, N, K,
                                                                  GROUP),

@@ -183,13 +183,13 @@ QZ_API qz_status qz_w4a16_gemv(const void *a, const void *codes, const void *sca
  * W4A16 prefill GEMM: the same product as qz_w4a16_gemv for any M >= 1,
  * dequantizing weight tiles into tensor memory for the tcgen05 tensor cores
  * (guide, "Quantize weights or activations": prefill and large batches are
- * compute-bound).  M <= 16 runs the decode kernel of qz_w4a16_gemv.  Each
+ * compute-bound).  M <= 32 runs the decode kernel of qz_w4a16_gemv (faster there).  Each
  * output tile is 128 weight rows x up to 256 tokens, and the MMAs cover only
  * the tile's tokens (rounded up to 16).  When the tiles are fewer than the
  * SMs, the K range of each tile is split over up to 4 CTAs whose fp32
  * partials meet in the workspace and are added in a fixed order (results do
  * not depend on timing).  Requirements: M >= 1; N >= 1; K % 128 == 0;
- * group_size a multiple of 64 dividing K (32 suffices for M <= 16).
+ * group_size a multiple of 64 dividing K (32 suffices for M <= 32).
  * Workspace: qz_workspace_bytes(QZ_OP_W4A16_GEMM, M, N, K, group_size)
  * bytes, zero-filled before first use, left zero-filled by each call that
  * completes.  A device-side wait that runs out (see qz_set_device_wait_limit)
@@ -220,7 +220,7 @@ QZ_API qz_status qz_w8a16_gemv(const void *a, const void *codes, const void *sca
  * activations": weight-only methods dequantize to the compute dtype before
  * each matmul, and prefill is compute-bound).  Weight tiles are dequantized (w_hat = bf16_rne(S * q), exactly as
  * qz_dequantize forms it) into tensor memory as the A operand of tcgen05
- * BF16 MMAs with fp32 accumulation; y is rounded to bf16.  M <= 16 runs the
+ * BF16 MMAs with fp32 accumulation; y is rounded to bf16.  M <= 32 runs the
  * decode kernel of qz_w8a16_gemv.  Tiles and split-K as for qz_w4a16_gemm.
  * Arguments: a (M x K bf16, row-major), codes (N x K int8, row-major),
  * scales (N bf16), y (M x N bf16, row-major), all device pointers owned by
@@ -399,7 +399,7 @@ QZ_API void qz_set_device_wait_limit(uint64_t limit);
 
 /*
  * How a decode GEMV launch (qz_w4a16_gemv, qz_w8a16_gemv, qz_w4a16_gemm with
- * M <= 16) may overlap the kernel launched before it on the same stream.
+ * M <= 32) may overlap the kernel launched before it on the same stream.
  * Not part of the method: a launch-latency optimisation for decode loops.
  *   0  (default) plain stream order.
  *   1  programmatic dependent launch: the GEMV may start while the previous

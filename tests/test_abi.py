@@ -162,8 +162,13 @@ def test_w8a16_gemm_workspace_follows_the_route():
         2 * 128 * 8192 * 4 + 64 * 4
     assert qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMM, 64, 8192, 8192, 128) == \
         qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMM, 64, 8192, 8192, 8192)
-    assert (qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMM, 16, 4096, 4096, 4096) ==
-            qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMV, 16, 4096, 4096, 4096))
+    for M in (16, 32):      # up to 32 tokens the GEMM entry runs the decode GEMV
+        assert (qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMM, M, 4096, 4096, 4096) ==
+                qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMV, M, 4096, 4096, 4096))
+        assert (qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMM, M, 4096, 4096, 128) ==
+                qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMV, M, 4096, 4096, 128))
+    assert (qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMM, 33, 4096, 4096, 4096) !=
+            qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMV, 33, 4096, 4096, 4096))
 
 
 @pytest.mark.parametrize("op,M,N,K,g,expect", [

@@ -161,11 +161,11 @@ def test_matmuls_on_edge_rows(dev, M):
         if bits == 4:
             zd = to_dev_u8(z, dev)
             outs = [("gemm", qz.qz_w4a16_gemm(ad, cd, sd, zd, N, K, g))]
-            if M <= 16:
+            if M <= 32:
                 outs.append(("gemv", qz.qz_w4a16_gemv(ad, cd, sd, zd, N, K, g)))
         else:
             outs = [("gemm", qz.qz_w8a16_gemm(ad, cd, sd, N, K))]
-            if M <= 16:
+            if M <= 32:
                 outs.append(("gemv", qz.qz_w8a16_gemv(ad, cd, sd, N, K)))
         torch.cuda.synchronize()
         assert qz.qz_device_status() == 0
@@ -548,12 +548,12 @@ def test_w8a16_gemm_onehot_is_exact(dev):
 
 
 def test_w8a16_gemm_small_m_matches_the_gemv(dev):
-    """M <= 16 takes the decode kernel: the same bits as qz_w8a16_gemv."""
+    """M <= 32 takes the decode kernel: the same bits as qz_w8a16_gemv."""
     N, K = 1000, 1024
     w = synthetic.weights(N, K, sigma=0.015, seed=5)
     c, s, _ = oracle.quantize_pack(u16(w), 8, True, K)
     cd, sd = to_dev_u8(c, dev), to_dev_bf16(s, dev)
-    for M in (1, 16):
+    for M in (1, 16, 17, 32):
         a = synthetic.activations(M, K, seed=M).to(dev)
         y1 = qz.qz_w8a16_gemm(a, cd, sd, N, K)
         y2 = qz.qz_w8a16_gemv(a, cd, sd, N, K)

@@ -64,19 +64,6 @@ __device__ __forceinline__ uint32_t e4m3_round_up(float t) {
     return b > 0x7Eu ? 0x7Eu : b;
 }
 
-// Nearest E2M1 code of v (sign in bit 3), ties to the even mantissa bit,
-// saturating at 6: the thresholds between neighbouring magnitudes are 0.25,
-// 0.75, 1.25, 1.75, 2.5, 3.5, 5, and a tie goes to the magnitude with an even
-// index (0, 1, 2, 4 at 0.25, 0.75->1, 1.25->1, 1.75->2, 2.5->2, 3.5->4, 5->4).
-__device__ __forceinline__ uint32_t e2m1_code(float v) {
-    const float a = fabsf(v);
-    uint32_t c = (uint32_t)(a > 0.25f) + (uint32_t)(a >= 0.75f) + (uint32_t)(a > 1.25f) +
-                 (uint32_t)(a >= 1.75f) + (uint32_t)(a > 2.5f) + (uint32_t)(a >= 3.5f) +
-                 (uint32_t)(a > 5.0f);
-    if (v < 0.0f && c != 0u) c |= 8u;
-    return c;
-}
-
 __device__ __forceinline__ float e2m1_value(uint32_t c) {
     const uint32_t i = c & 7u;
     const float mag = i < 4 ? 0.5f * (float)i : (i == 4 ? 2.0f : i == 5 ? 3.0f : i == 6 ? 4.0f : 6.0f);
@@ -88,19 +75,32 @@ __device__ __forceinline__ int64_t thread_index() {
     return (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
 }
 
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a & 0x7FFF7FFFu), "r"(b & 0x7FFF7FFFu));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t chunk_absmax(uint32_t m2, const uint4 &v) {
+    return bf16x2_absmax(m2, bf16x2_absmax(bf16x2_absmax(v.x, v.y), bf16x2_absmax(v.z, v.w)));
+}
+
 // max |w| over the tensor into *amax (fp32 bits, non-negative: ordered as
-// unsigned integers).
+// unsigned integers).  Four 16-byte loads in flight per thread.
 __global__ void __launch_bounds__(kThreads) fp4_amax_kernel(const uint4 *__restrict__ w,
                                                            int64_t chunks, unsigned *amax) {
-    float m = 0.0f;
-    for (int64_t c = thread_index(); c < chunks; c += grid_stride()) {
-        const uint4 v = __ldg(w + c);
-        const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+    uint32_t m2 = 0u;
+    const int64_t stride = grid_stride();
+    int64_t c = thread_index();
+    for (; c + 3 * stride < chunks; c += 4 * stride) {
+        uint4 v[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            m = fmaxf(m, fmaxf(fabsf(bf16_bits_to_f32(x[i] & 0xFFFFu)),
-                               fabsf(bf16_bits_to_f32(x[i] >> 16))));
+        for (int u = 0; u < 4; ++u) v[u] = __ldg(w + c + u * stride);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) m2 = chunk_absmax(m2, v[u]);
     }
+    for (; c < chunks; c += stride) m2 = chunk_absmax(m2, __ldg(w + c));
+    float m = fmaxf(bf16_bits_to_f32(m2 & 0xFFFFu), bf16_bits_to_f32(m2 >> 16));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
     __shared__ float part[kThreads / 32];
@@ -124,9 +124,40 @@ __device__ __forceinline__ int64_t mma_scale_offset(int64_t r, int64_t j, int64_
     return (((r >> 7) * atoms_k + (j >> 2)) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2) + (j & 3);
 }
 
+// Eight values (v[i] -> nibble i) as E2M1 codes: the hardware conversion
+// rounds to the nearest E2M1 value, ties to the even mantissa bit (0.25 -> 0,
+// 0.75 -> 1, 1.25 -> 1, 1.75 -> 2, 2.5 -> 2, 3.5 -> 4, 5 -> 4), and saturates
+// at 6 -- the rounding stated above -- but keeps the sign of a negative value
+// that rounds to zero; such a nibble (8) becomes 0 here, as the oracle writes
+// it.
+__device__ __forceinline__ uint32_t e2m1_pack8(const float (&v)[8]) {
+    uint32_t w;
+    asm("{\n\t.reg .b8 c0, c1, c2, c3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 c0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 c1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 c2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 c3, %8, %7;\n\t"
+        "mov.b32 %0, {c0, c1, c2, c3};\n\t}"
+        : "=r"(w)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]),
+          "f"(v[7]));
+    const uint32_t mag = w & 0x77777777u;
+    const uint32_t nonzero = (mag + 0x77777777u) & 0x88888888u;   // bit 3 set where mag != 0
+    return mag | (w & nonzero);
+}
+
 // One thread per block of BS values (BS / 8 chunks of 16 bytes).  MMA:
 // scales in the MMA scale layout (blocks_per_row scales per row) instead of
 // row-major.
+//
+// x / scale without a division: MXFP4 multiplies by 2^-e (exact).  NVFP4 uses
+// Markstein's correction (Markstein 1990, the theorem on correctly rounded
+// quotients from a correctly rounded reciprocal): with r = RN(1/s) and
+// q0 = RN(x r), the residual x - q0 s is exact under fma and
+// RN(q0 + (x - q0 s) r) = RN(x / s), barring underflow or overflow.  Blocks
+// whose scale is subnormal (or whose reciprocal would overflow) take the IEEE
+// division instead; a quotient that underflows is below 0.25 and codes to 0
+// either way.
 template <int KIND, bool MMA = false>
 __global__ void __launch_bounds__(kThreads)
 fp4_quantize_kernel(const uint4 *__restrict__ w, int64_t blocks, uint8_t *__restrict__ codes,
@@ -142,12 +173,12 @@ fp4_quantize_kernel(const uint4 *__restrict__ w, int64_t blocks, uint8_t *__rest
             const uint4 v = __ldg(w + b * (BS / 8) + c);
             x[4 * c + 0] = v.x; x[4 * c + 1] = v.y; x[4 * c + 2] = v.z; x[4 * c + 3] = v.w;
         }
-        float amax = 0.0f;
+        uint32_t m2 = bf16x2_absmax(x[0], x[1]);
 #pragma unroll
-        for (int i = 0; i < BS / 2; ++i)
-            amax = fmaxf(amax, fmaxf(fabsf(bf16_bits_to_f32(x[i] & 0xFFFFu)),
-                                     fabsf(bf16_bits_to_f32(x[i] >> 16))));
-        float scale;
+        for (int i = 2; i < BS / 2; i += 2) m2 = bf16x2_absmax(m2, bf16x2_absmax(x[i], x[i + 1]));
+        const float amax = fmaxf(bf16_bits_to_f32(m2 & 0xFFFFu), bf16_bits_to_f32(m2 >> 16));
+        float scale, r;
+        bool exact_div = false;
         uint32_t sb;
         if (KIND == 0) {
             int e = -127;
@@ -159,24 +190,40 @@ fp4_quantize_kernel(const uint4 *__restrict__ w, int64_t blocks, uint8_t *__rest
             }
             sb = (uint32_t)(e + 127);
             scale = ldexpf(1.0f, e);
+            r = ldexpf(1.0f, -e);                                // exact: x * r = x / 2^e
         } else {
             sb = e4m3_round_up(__fdiv_rn(amax, __fmul_rn(6.0f, s_t)));
             scale = __fmul_rn(e4m3_value(sb), s_t);
+            r = __frcp_rn(scale);
+            // 2^-96 <= scale <= 2^96 keeps x, r, q0 s and the residual normal
+            // for every quotient of 0.25 or more (smaller ones code to 0)
+            exact_div = !(scale >= 0x1p-96f && scale <= 0x1p96f);
         }
         if (MMA) {
-            const int64_t r = b / blocks_per_row;
-            scales[mma_scale_offset(r, b - r * blocks_per_row, blocks_per_row >> 2)] = (uint8_t)sb;
+            const int64_t row = b / blocks_per_row;
+            scales[mma_scale_offset(row, b - row * blocks_per_row, blocks_per_row >> 2)] =
+                (uint8_t)sb;
         } else {
             scales[b] = (uint8_t)sb;
         }
         uint32_t packed[BS / 8];
 #pragma unroll
-        for (int i = 0; i < BS / 8; ++i) packed[i] = 0u;
+        for (int g = 0; g < BS / 8; ++g) {
+            float u[8];
 #pragma unroll
-        for (int i = 0; i < BS; ++i) {
-            const uint32_t h = (i & 1) ? (x[i / 2] >> 16) : (x[i / 2] & 0xFFFFu);
-            const uint32_t c = scale > 0.0f ? e2m1_code(__fdiv_rn(bf16_bits_to_f32(h), scale)) : 0u;
-            packed[i / 8] |= c << (4 * (i % 8));
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t h = (i & 1) ? (x[(8 * g + i) / 2] >> 16) : (x[(8 * g + i) / 2] & 0xFFFFu);
+                const float xv = bf16_bits_to_f32(h);
+                if (KIND == 0) {
+                    u[i] = xv * r;
+                } else if (!exact_div) {
+                    const float q0 = __fmul_rn(xv, r);
+                    u[i] = __fmaf_rn(__fmaf_rn(-q0, scale, xv), r, q0);
+                } else {
+                    u[i] = scale > 0.0f ? __fdiv_rn(xv, scale) : 0.0f;
+                }
+            }
+            packed[g] = e2m1_pack8(u);
         }
         uint32_t *dst = reinterpret_cast<uint32_t *>(codes + b * (BS / 2));
 #pragma unroll

@@ -289,12 +289,19 @@ w4a4_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
                     const uint32_t wgt = sbase + C::kWgt + s * C::kWgtBytes;
                     const uint32_t sfa_s = sbase + C::kSfa + s * C::kSfaBytes;
                     const uint32_t sfb_s = sbase + C::kSfb + s * C::kSfbBytes;
+                    // the stage's scales first, then its MMAs back to back: an
+                    // MMA waits for the copies before it, so copies interleaved
+                    // with the MMAs would stall every MMA
 #pragma unroll
                     for (int a = 0; a < C::kAtoms; ++a) {
                         const uint32_t col = sf_tmem + (uint32_t)((s * C::kAtoms + a) * C::kSfCols);
                         tc_cp_atom(col, smem_desc_atom(sfa_s + a * kAtomBytes));
                         tc_cp_atom(col + 4, smem_desc_atom(sfb_s + a * kAtomBytes));
                         tc_cp_atom(col + 8, smem_desc_atom(sfb_s + (C::kAtoms + a) * kAtomBytes));
+                    }
+#pragma unroll
+                    for (int a = 0; a < C::kAtoms; ++a) {
+                        const uint32_t col = sf_tmem + (uint32_t)((s * C::kAtoms + a) * C::kSfCols);
 #pragma unroll
                         for (int st = 0; st < C::kStepsPerAtom; ++st) {
                             const int ks = a * C::kStepsPerAtom + st;

@@ -28,9 +28,11 @@
 //      Reversing both indices turns L into an upper V with H = V V^T, so
 //      H^-1 = V^-T V^-1 and V^-1 is upper: it is U.
 //   3. Blocked inverse Li = L^-1: trinv_diag_kernel inverts the diagonal
-//      tiles, trinv_offdiag_kernel fills the tiles at block distance d
-//      (which need only tiles at smaller distances) for d = 1, 2, ...;
-//      reverse_kernel writes U[j][k] = Li[K-1-j][K-1-k].
+//      tiles; then, right-looking, for each block row m trinv_finalize_kernel
+//      completes row m (Li[m,j] = -Li[m,m] sum_{k<m} L[m,k] Li[k,j]) and
+//      trinv_update_kernel adds row m's contribution to every later row, so
+//      each launch has many independent tiles; reverse_kernel writes
+//      U[j][k] = Li[K-1-j][K-1-k].
 //   4. Per block of 128 columns: gptq_block_kernel (one warp per weight row,
 //      the row's 128 block columns in registers, U's block triangle in
 //      shared memory) quantizes the columns in order, applies the
@@ -48,7 +50,7 @@ namespace {
 constexpr int kT = 64;              // tile edge of the factorization kernels
 constexpr int kTileThreads = 256;   // 16 x 16 threads, 4 x 4 outputs each
 constexpr int kGptqBlock = 128;     // the page's lazy-batch width B
-constexpr int kRowsPerCta = 8;      // warps (weight rows) per column-loop CTA
+constexpr int kRowsPerCta = 32;     // warps (weight rows) per column-loop CTA
 
 // ---------------------------------------------------------------------------
 // fp64 tile product helper: acc (4 x 4 per thread of a 16 x 16 layout over a
@@ -129,7 +131,9 @@ __global__ void damp_kernel(double *R, int K, double damp) {
 }
 
 // 2a. Factor the diagonal tile p in place (unblocked Cholesky in shared
-// memory); the strict upper part of the tile is zeroed.
+// memory); the strict upper part of the tile is zeroed.  Thread t owns row
+// t / 4 and, within it, the columns c = t % 4 (mod 4), so each step touches
+// only the trailing triangle.
 __global__ void __launch_bounds__(kTileThreads) chol_diag_kernel(double *R, int K, int p) {
     __shared__ double A[kT][kT + 1];
     const int base = p * kT, n = min(kT, K - base);
@@ -138,16 +142,17 @@ __global__ void __launch_bounds__(kTileThreads) chol_diag_kernel(double *R, int 
         A[r][c] = (r < n && c < n) ? R[(int64_t)(base + r) * K + base + c] : 0.0;
     }
     __syncthreads();
+    const int i = threadIdx.x >> 2, cls = threadIdx.x & 3;
     for (int j = 0; j < n; ++j) {
         if (threadIdx.x == 0) A[j][j] = sqrt(A[j][j]);
         __syncthreads();
-        const double d = A[j][j];
-        for (int i = j + 1 + (int)threadIdx.x; i < n; i += kTileThreads) A[i][j] /= d;
+        if (cls == 0 && i > j && i < n) A[i][j] /= A[j][j];
         __syncthreads();
-        // trailing update of the tile: A[i][c] -= A[i][j] A[c][j], j < c <= i
-        for (int e = threadIdx.x; e < kT * kT; e += kTileThreads) {
-            const int i = e / kT, c = e % kT;
-            if (i < n && c > j && c <= i) A[i][c] -= A[i][j] * A[c][j];
+        // trailing update: A[i][c] -= A[i][j] A[c][j], j < c <= i
+        if (i > j && i < n) {
+            const double aij = A[i][j];
+            int c = j + 1 + ((cls - (j + 1)) & 3);
+            for (; c <= i; c += 4) A[i][c] -= aij * A[c][j];
         }
         __syncthreads();
     }
@@ -157,8 +162,11 @@ __global__ void __launch_bounds__(kTileThreads) chol_diag_kernel(double *R, int 
     }
 }
 
-// 2b. Tiles below the diagonal in panel p: A[i,p] <- A[i,p] L[p,p]^-T (each
-// row by forward substitution against the factored diagonal tile).
+// 2b. Tiles below the diagonal in panel p: A[i,p] <- A[i,p] L[p,p]^-T.  Row r
+// of a tile solves x L^T = b column by column: x_c = b_c / L[c][c], then
+// b_k -= x_c L[k][c] for k > c (the same operations, in the same order, as
+// the forward substitution x_c = (b_c - sum_{k<c} x_k L[c][k]) / L[c][c]).
+// Thread t owns row t % 64 and the columns k = t / 64 (mod 4).
 __global__ void __launch_bounds__(kTileThreads) chol_panel_kernel(double *R, int K, int p) {
     QZ_TWO_TILES(Lp, B);
     const int base = p * kT, n = min(kT, K - base);
@@ -169,19 +177,19 @@ __global__ void __launch_bounds__(kTileThreads) chol_panel_kernel(double *R, int
         B[r][c] = (r < rows && c < n) ? R[(int64_t)(rb + r) * K + base + c] : 0.0;
     }
     __syncthreads();
-    // row r of B solves x L^T = b: x_c = (b_c - sum_{k<c} x_k L[c][k]) / L[c][c]
-    if ((int)threadIdx.x < rows) {
-        const int r = threadIdx.x;
-        for (int c = 0; c < n; ++c) {
-            double v = B[r][c];
-            for (int k = 0; k < c; ++k) v -= B[r][k] * Lp[c][k];
-            B[r][c] = v / Lp[c][c];
+    const int r = threadIdx.x & (kT - 1), cls = threadIdx.x / kT;
+    for (int c = 0; c < n; ++c) {
+        if ((c & 3) == cls && r < rows) B[r][c] /= Lp[c][c];
+        __syncthreads();
+        if (r < rows) {
+            const double x = B[r][c];
+            for (int k = c + 1 + ((cls - (c + 1)) & 3); k < n; k += 4) B[r][k] -= x * Lp[k][c];
         }
+        __syncthreads();
     }
-    __syncthreads();
     for (int e = threadIdx.x; e < kT * kT; e += kTileThreads) {
-        const int r = e / kT, c = e % kT;
-        if (r < rows && c < n) R[(int64_t)(rb + r) * K + base + c] = B[r][c];
+        const int rr = e / kT, c = e % kT;
+        if (rr < rows && c < n) R[(int64_t)(rb + rr) * K + base + c] = B[rr][c];
     }
 }
 
@@ -242,35 +250,22 @@ trinv_diag_kernel(const double *__restrict__ L, double *__restrict__ Li, int K) 
     }
 }
 
-// 3b. Tiles at block distance d: Li[i,j] = -Li[i,i] sum_{m=j}^{i-1} L[i,m] Li[m,j]
-// with i = j + d (every Li[m,j] on the right is at a smaller distance).
+// 3b. Off-diagonal tiles, right-looking: with S[i,j] = sum_{m<i} L[i,m] Li[m,j]
+// accumulated in place of Li[i,j] (zero to start), step m first finalizes
+// block row m, Li[m,j] = -Li[m,m] S[m,j] for j < m (trinv_finalize_kernel),
+// then adds L[i,m] Li[m,j] to S[i,j] for every i > m, j <= m
+// (trinv_update_kernel): all tiles of a step are independent.
 __global__ void __launch_bounds__(kTileThreads)
-trinv_offdiag_kernel(const double *__restrict__ L, double *__restrict__ Li, int K, int d) {
-    const int j = blockIdx.x, i = j + d;
+trinv_finalize_kernel(double *__restrict__ Li, int K, int m) {
+    const int j = blockIdx.x;
     QZ_TWO_TILES(As, Bs);
     const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
-    double acc[4][4] = {};
-    for (int m = j; m < i; ++m) {
-        for (int e = tid; e < kT * kT; e += kTileThreads) {
-            const int r = e / kT, c = e % kT;
-            const int gi = i * kT + r, gm = m * kT + c, gmr = m * kT + r, gj = j * kT + c;
-            As[r][c] = (gi < K && gm < K) ? L[(int64_t)gi * K + gm] : 0.0;
-            Bs[r][c] = (gmr < K && gj < K) ? Li[(int64_t)gmr * K + gj] : 0.0;
-        }
-        __syncthreads();
-        tile_fma(acc, As, Bs, ty, tx, kT);
-        __syncthreads();
-    }
-    // T = acc (sum), then Li[i,j] = -Li[i,i] T
     for (int e = tid; e < kT * kT; e += kTileThreads) {
         const int r = e / kT, c = e % kT;
-        const int gi = i * kT + r, gc = i * kT + c;
-        As[r][c] = (gi < K && gc < K) ? Li[(int64_t)gi * K + gc] : 0.0;
+        const int gr = m * kT + r, gc = m * kT + c, gj = j * kT + c;
+        As[r][c] = (gr < K && gc < K) ? Li[(int64_t)gr * K + gc] : 0.0;
+        Bs[r][c] = (gr < K && gj < K) ? Li[(int64_t)gr * K + gj] : 0.0;
     }
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) Bs[ty + 16 * a][tx + 16 * b] = acc[a][b];
     __syncthreads();
     double out[4][4] = {};
     tile_fma(out, As, Bs, ty, tx, kT);
@@ -278,19 +273,32 @@ trinv_offdiag_kernel(const double *__restrict__ L, double *__restrict__ Li, int 
     for (int a = 0; a < 4; ++a)
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
-            const int gi = i * kT + ty + 16 * a, gj = j * kT + tx + 16 * b;
+            const int gi = m * kT + ty + 16 * a, gj = j * kT + tx + 16 * b;
             if (gi < K && gj < K) Li[(int64_t)gi * K + gj] = -out[a][b];
         }
 }
 
-// Zero the strict upper triangle of Li (never written by the kernels above).
-__global__ void zero_upper_kernel(double *Li, int K) {
-    const int64_t total = (int64_t)K * K;
-    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
-         e += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = e / K, c = e % K;
-        if (c > r) Li[e] = 0.0;
+__global__ void __launch_bounds__(kTileThreads)
+trinv_update_kernel(const double *__restrict__ L, double *__restrict__ Li, int K, int m) {
+    const int j = blockIdx.x, i = m + 1 + blockIdx.y;
+    QZ_TWO_TILES(As, Bs);
+    const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
+    for (int e = tid; e < kT * kT; e += kTileThreads) {
+        const int r = e / kT, c = e % kT;
+        const int gi = i * kT + r, gm = m * kT + c, gmr = m * kT + r, gj = j * kT + c;
+        As[r][c] = (gi < K && gm < K) ? L[(int64_t)gi * K + gm] : 0.0;
+        Bs[r][c] = (gmr < K && gj < K) ? Li[(int64_t)gmr * K + gj] : 0.0;
     }
+    __syncthreads();
+    double acc[4][4] = {};
+    tile_fma(acc, As, Bs, ty, tx, kT);
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const int gi = i * kT + ty + 16 * a, gj = j * kT + tx + 16 * b;
+            if (gi < K && gj < K) Li[(int64_t)gi * K + gj] += acc[a][b];
+        }
 }
 
 // U[j][k] = Li[K-1-j][K-1-k].
@@ -535,7 +543,8 @@ qz_status launch_gptq(const void *w, const void *x, int64_t N, int64_t K, int64_
             if (e == cudaSuccess) e = cudaFuncSetAttribute(chol_update_kernel, a, (int)kTwoTiles);
             if (e == cudaSuccess) e = cudaFuncSetAttribute(trinv_diag_kernel, a, (int)kTwoTiles);
             if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(trinv_offdiag_kernel, a, (int)kTwoTiles);
+                e = cudaFuncSetAttribute(trinv_finalize_kernel, a, (int)kTwoTiles);
+            if (e == cudaSuccess) e = cudaFuncSetAttribute(trinv_update_kernel, a, (int)kTwoTiles);
             if (e == cudaSuccess) e = cudaFuncSetAttribute(lazy_update_kernel, a, (int)kTwoTiles);
             if (e == cudaSuccess) e = cudaFuncSetAttribute(gptq_block_kernel, a, (int)block_smem);
             return e;
@@ -555,10 +564,15 @@ qz_status launch_gptq(const void *w, const void *x, int64_t N, int64_t K, int64_
         }
     }
     // 3. Li = L^-1, then U (reversed)
-    zero_upper_kernel<<<grid_for(K * K), 256, 0, st>>>(ws.Li, Ki);
+    if (cudaMemsetAsync(ws.Li, 0, (size_t)K * K * sizeof(double), st) != cudaSuccess)
+        return QZ_ERR_CUDA;
     trinv_diag_kernel<<<P, kTileThreads, kTwoTiles, st>>>(ws.R, ws.Li, Ki);
-    for (int d = 1; d < P; ++d)
-        trinv_offdiag_kernel<<<P - d, kTileThreads, kTwoTiles, st>>>(ws.R, ws.Li, Ki, d);
+    for (int m = 0; m < P; ++m) {
+        if (m > 0) trinv_finalize_kernel<<<m, kTileThreads, kTwoTiles, st>>>(ws.Li, Ki, m);
+        if (m + 1 < P)
+            trinv_update_kernel<<<dim3(m + 1, P - m - 1), kTileThreads, kTwoTiles, st>>>(
+                ws.R, ws.Li, Ki, m);
+    }
     double *U = ws.R;   // the factor is no longer needed
     reverse_kernel<<<grid_for(K * K), 256, 0, st>>>(ws.Li, U, Ki);
     // 4. column loop

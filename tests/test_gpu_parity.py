@@ -182,6 +182,10 @@ def test_matmuls_on_edge_rows(dev, M):
 GEMV_CASES = [  # (N, K, g)
     (1024, 1024, 128), (1000, 384, 128), (17, 128, 32), (96, 512, 64),
     (256, 2048, 256), (64, 1024, 1024), (4100, 1152, 128),
+    # units of 256 k for M <= 8 (K % 256 == 0, K/g a multiple of 16): groups
+    # of 128 (two per unit), 256 (one) and 512 (a group spans two units),
+    # ragged rows
+    (384, 2048, 128), (130, 4096, 256), (4100, 4096, 128), (256, 8192, 512),
 ]
 
 
@@ -202,6 +206,36 @@ def test_w4a16_gemv_tolerance(dev, N, K, g, M):
                          N, K, g)
     torch.cuda.synchronize()
     check_tolerance(u16(y), y_ref, abs_ref, f"w4a16 M={M} N={N} K={K} g={g}")
+
+
+def test_w4a16_gemv_two_half_units_onehot_and_fallback(dev):
+    """Units of 256 k (up to 8 tokens, scale/zero tiles by TMA): one-hot
+    activations read back the oracle's bf16 weights bit for bit; with a scale
+    array that is not 16-byte aligned the call falls back to units of 128 k,
+    within the bound and inside the workspace qz_workspace_bytes gives."""
+    N, K, g = 300, 2048, 128
+    w = synthetic.weights(N, K, sigma=0.02, seed=25)
+    c, s, z, w_hat = oracle_w4(u16(w), g)
+    rng = np.random.default_rng(3)
+    ks = rng.choice(K, size=8, replace=False)
+    a = np.zeros((8, K), np.uint16)
+    a[np.arange(8), ks] = 0x3F80
+    cd, zd = to_dev_u8(c, dev), to_dev_u8(z, dev)
+    y = qz.qz_w4a16_gemv(to_dev_bf16(a, dev), cd, to_dev_bf16(s, dev), zd, N, K, g)
+    torch.cuda.synchronize()
+    assert np.array_equal(u16(y), w_hat[:, ks].T)
+    # scales at a 2-byte offset inside a larger buffer
+    buf = torch.empty(s.size + 1, dtype=torch.bfloat16, device=dev)
+    s_off = buf[1:].view(s.shape)
+    s_off.copy_(to_dev_bf16(s, dev))
+    assert s_off.data_ptr() % 16 != 0
+    act = synthetic.activations(5, K, seed=26)
+    ws = torch.zeros(qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMV, 5, N, K, g), dtype=torch.uint8,
+                     device=dev)
+    y2 = qz.qz_w4a16_gemv(act.to(dev), cd, s_off, zd, N, K, g, workspace=ws)
+    torch.cuda.synchronize()
+    y_ref, abs_ref = oracle.matmul_f64(u16(act), w_hat)
+    check_tolerance(u16(y2), y_ref, abs_ref, "w4a16 misaligned scales")
 
 
 @pytest.mark.parametrize("N,K,g", [(1024, 1024, 128), (37, 384, 32), (300, 4096, 128)])

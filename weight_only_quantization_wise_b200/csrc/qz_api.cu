@@ -147,14 +147,18 @@ QZ_API qz_status qz_workspace_bytes(int32_t op, int64_t M, int64_t N, int64_t K,
     case QZ_OP_W8A16_GEMV: {
         const qz_status s = check_gemv_shape(M, N, K);
         if (s != QZ_OK) return s;
-        *bytes = gemv_workspace_bound(M, N, K, op == QZ_OP_W4A16_GEMV ? 4 : 8);
+        *bytes = op == QZ_OP_W4A16_GEMV
+                     ? gemv_workspace_bound(M, N, K, 4, gemv_unit_k(4, M, K, group_size))
+                     : gemv_workspace_bound(M, N, K, 8);
         return QZ_OK;
     }
     case QZ_OP_W4A16_GEMM:
     case QZ_OP_W8A16_GEMM:
         if (M < 1 || N < 1 || K < 1) return QZ_ERR_INVALID_ARG;
         *bytes = M <= kGemmToGemvMaxM && K % 128 == 0
-                     ? gemv_workspace_bound(M, N, K, op == QZ_OP_W4A16_GEMM ? 4 : 8)
+                     ? (op == QZ_OP_W4A16_GEMM
+                            ? gemv_workspace_bound(M, N, K, 4, gemv_unit_k(4, M, K, group_size))
+                            : gemv_workspace_bound(M, N, K, 8))
                      : gemm_workspace_bytes(M, N, K);
         return QZ_OK;
     case QZ_OP_FP4A16_GEMV: {
@@ -186,14 +190,18 @@ QZ_API qz_status qz_workspace_bytes_for_sms(int32_t op, int64_t M, int64_t N, in
     case QZ_OP_W8A16_GEMV: {
         const qz_status s = check_gemv_shape(M, N, K);
         if (s != QZ_OK) return s;
-        *bytes = gemv_plan(M, N, K, op == QZ_OP_W4A16_GEMV ? 4 : 8, sms).total_bytes;
+        *bytes = op == QZ_OP_W4A16_GEMV
+                     ? gemv_plan(M, N, K, 4, sms, gemv_unit_k(4, M, K, group_size)).total_bytes
+                     : gemv_plan(M, N, K, 8, sms).total_bytes;
         return QZ_OK;
     }
     case QZ_OP_W4A16_GEMM:
     case QZ_OP_W8A16_GEMM:
         if (M < 1 || N < 1 || K < 1) return QZ_ERR_INVALID_ARG;
         *bytes = M <= kGemmToGemvMaxM && K % 128 == 0
-                     ? gemv_plan(M, N, K, op == QZ_OP_W4A16_GEMM ? 4 : 8, sms).total_bytes
+                     ? (op == QZ_OP_W4A16_GEMM
+                            ? gemv_plan(M, N, K, 4, sms, gemv_unit_k(4, M, K, group_size))
+                            : gemv_plan(M, N, K, 8, sms)).total_bytes
                      : gemm_workspace_bytes_for(M, N, K, sms);
         return QZ_OK;
     case QZ_OP_FP4A16_GEMV: {
@@ -245,7 +253,8 @@ QZ_API qz_status qz_w4a16_gemv(const void *a, const void *codes, const void *sca
     if (!a || !codes || !scales || !zeros || !y) return QZ_ERR_INVALID_ARG;
     if (!aligned(a, 16) || !aligned(codes, 16) || !aligned(scales, 2) || !aligned(y, 2))
         return QZ_ERR_ALIGNMENT;
-    const GemvPlan plan = gemv_plan(M, N, K, 4, device_sm_count());
+    const GemvPlan plan =
+        gemv_plan(M, N, K, 4, device_sm_count(), gemv_unit_k(4, M, K, group_size, scales, zeros));
     s = check_workspace(plan.total_bytes, workspace, workspace_bytes);
     if (s != QZ_OK) return s;
     return launch_w4a16_gemv(a, codes, scales, zeros, M, N, K, group_size, y, workspace, plan,

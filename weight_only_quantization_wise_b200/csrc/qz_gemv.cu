@@ -106,16 +106,17 @@ constexpr int kMetaZeroBytes = kTileRows * 16;                 // 16 zeros per r
 // Shared-memory layout (offsets from the 1024-byte aligned base): S stages
 // of [codes | activations (8 MB rows) | gathered scale/zero words], then the
 // two meta slots [scales | zeros], then the barriers.
-template <int BITS, int MB, int META, int FMT = kFmtInt>
+template <int BITS, int MB, int META, int FMT = kFmtInt, int HALVES = 1>
 struct Layout {
-    static constexpr int act = 8 * MB * kBlockK * 2;                    // bytes per stage
-    static constexpr int stage = kCodeStage<BITS> + act + (META == kMetaGather ? kSzStage : 0);
+    static constexpr int code = kCodeStage<BITS> * HALVES;              // code bytes per stage
+    static constexpr int act = 8 * MB * kBlockK * HALVES * 2;           // bytes per stage
+    static constexpr int stage = code + act + (META == kMetaGather ? kSzStage : 0);
     static constexpr int meta = META == kMetaTma ? 2 * (kMetaScaleBytes + kMetaZeroBytes) : 0;
     static constexpr int lut = FMT == kFmtNv ? 512 : 0;                 // E4M3 -> bf16 table
     static constexpr int S = (kCtaSmemBudget<MB> - meta - lut - 256) / stage;
     static constexpr uint32_t codes = 0;                                 // + s * stage
-    static constexpr uint32_t act_off = kCodeStage<BITS>;                // within a stage
-    static constexpr uint32_t sz_off = kCodeStage<BITS> + act;           // within a stage
+    static constexpr uint32_t act_off = code;                            // within a stage
+    static constexpr uint32_t sz_off = code + act;                       // within a stage
     static constexpr uint32_t meta_base = S * stage;
     static constexpr uint32_t lut_base = meta_base + meta;
     static constexpr uint32_t full = lut_base + lut;
@@ -232,6 +233,19 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     return v;
 }
 
+// int4 units of two 128-wide halves: 128-byte rows stored with the 128-byte
+// swizzle (16-byte chunk c of row r at chunk c ^ (r % 8)); half h of lane t is
+// chunk 4h + t, and r % 8 == g for the lane's four rows.
+__device__ __forceinline__ void read_codes_half(RowWords<4> &rw, uint32_t stage, int row0, int g,
+                                                int t, int h) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t row = stage + (uint32_t)(row0 + 8 * j) * 128u;
+        const uint4 v = lds128(row + 16u * (uint32_t)((4 * h + t) ^ g));
+        rw.w[j][0] = v.x; rw.w[j][1] = v.y; rw.w[j][2] = v.z; rw.w[j][3] = v.w;
+    }
+}
+
 // Codes of the lane's four rows from a stage.  int4: row r at 64 r, lane t
 // reads bytes 16t..16t+15 (rows g and g+1 of an 8-lane phase are adjacent:
 // 128 consecutive bytes).  int8: row r at 128 r with the 128-byte swizzle
@@ -298,11 +312,12 @@ __device__ __forceinline__ void load_params_direct(RowParams &rp, const GemvArgs
 // Activations of one unit for tokens g (and g + 8), clamped to M - 1, from
 // the stage: token rows of 256 bytes, lane t reading bytes 64t..64t+63.
 template <int MB>
-__device__ __forceinline__ void load_act(Act<MB> &ac, uint32_t act, int M, int g, int t) {
+__device__ __forceinline__ void load_act(Act<MB> &ac, uint32_t act, int M, int g, int t,
+                                         uint32_t pitch = kBlockK * 2) {
 #pragma unroll
     for (int mb = 0; mb < MB; ++mb) {
         const int tok = min(8 * mb + g, M - 1);
-        const uint32_t src = act + (uint32_t)tok * (kBlockK * 2) + 64u * t;
+        const uint32_t src = act + (uint32_t)tok * pitch + 64u * t;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             const uint4 v = lds128(src + 16u * q);
@@ -567,14 +582,18 @@ __device__ __forceinline__ void gemv_flush(float (&acc)[2][MB][4], const GemvArg
 }
 
 // The kernel.  META: how int4 scales and zeros arrive (kMetaNone: int8's
-// per-row scales, or int4 groups loaded directly by the consumers).
-template <int BITS, int MB, int META, int FMT>
+// per-row scales, or int4 groups loaded directly by the consumers).  HALVES:
+// 128-wide K blocks per unit (2: int4 units of 128 rows x 256 k, one
+// 128-byte row of codes per weight row, consumed as two halves).
+template <int BITS, int MB, int META, int FMT, int HALVES = 1>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm<MB>)
 gemv_kernel(const __grid_constant__ CUtensorMap code_map,
             const __grid_constant__ CUtensorMap act_map,
             const __grid_constant__ CUtensorMap scale_map,
             const __grid_constant__ CUtensorMap zero_map, const GemvArgs p) {
-    using L = Layout<BITS, MB, META, FMT>;
+    using L = Layout<BITS, MB, META, FMT, HALVES>;
+    static_assert(HALVES == 1 || (BITS == 4 && FMT == kFmtInt && META == kMetaTma && MB == 1),
+                  "two-half units: int4 with scale/zero tiles by TMA, up to 8 tokens");
     constexpr int S = L::S;
     constexpr bool kFp4 = FMT != kFmtInt;
     constexpr uint32_t kMetaBytes = kFp4 ? kFp4MetaBytes : kMetaScaleBytes + kMetaZeroBytes;
@@ -595,7 +614,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap code_map,
     const int64_t u_begin = cta * p.units / p.ctas;
     const int64_t u_end = (cta + 1) * p.units / p.ctas;
     const int KB = p.kblocks;
-    const uint32_t act_bytes = (uint32_t)p.M * kBlockK * 2;
+    const uint32_t act_bytes = (uint32_t)p.M * kBlockK * HALVES * 2;
     // a meta slot holds 8 groups: 8 << bpg_shift units of one task
     const int span_mask = META == kMetaTma ? (1 << p.meta_span_shift) - 1 : 0;
 
@@ -649,8 +668,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap code_map,
             if (lane == 0) {
                 int kb2 = kb_first;
                 for (int64_t i = 0; i < no_act; ++i) {
-                    tma_load_2d(stage_addr((int)i) + L::act_off, &act_map, kb2 * kBlockK, 0,
-                                full_bar((int)i));
+                    tma_load_2d(stage_addr((int)i) + L::act_off, &act_map,
+                                kb2 * kBlockK * HALVES, 0, full_bar((int)i));
                     if (++kb2 == KB) kb2 = 0;
                 }
             }
@@ -674,7 +693,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap code_map,
                         tma_load_2d(meta_addr(m), &scale_map, (kb << p.fp4_bpu_shift) & ~31,
                                     task * kTileRows, meta_full_bar(m));
                     } else {
-                        const int gi = kb >> p.bpg_shift;
+                        const int gi = (kb * HALVES) >> p.bpg_shift;
                         tma_load_2d(meta_addr(m), &scale_map, gi & ~(kMetaGroups - 1),
                                     task * kTileRows, meta_full_bar(m));
                         tma_load_2d(meta_addr(m) + kMetaScaleBytes, &zero_map, gi & ~15,
@@ -691,11 +710,12 @@ gemv_kernel(const __grid_constant__ CUtensorMap code_map,
                 }
             }
             if (lane == 0) {
-                mbar_arrive_expect_tx(full_bar(s), kCodeStage<BITS> + act_bytes);
-                tma_load_2d(stage_addr(s), &code_map, kb * kRowBytes<BITS>, task * kTileRows,
-                            full_bar(s));
+                mbar_arrive_expect_tx(full_bar(s), (uint32_t)L::code + act_bytes);
+                tma_load_2d(stage_addr(s), &code_map, kb * kRowBytes<BITS> * HALVES,
+                            task * kTileRows, full_bar(s));
                 if (!early_phase)
-                    tma_load_2d(stage_addr(s) + L::act_off, &act_map, kb * kBlockK, 0, full_bar(s));
+                    tma_load_2d(stage_addr(s) + L::act_off, &act_map, kb * kBlockK * HALVES, 0,
+                                full_bar(s));
             }
             if (META == kMetaGather) {
                 const uint32_t dst = stage_addr(s) + L::sz_off + 16u * lane;
@@ -784,6 +804,43 @@ gemv_kernel(const __grid_constant__ CUtensorMap code_map,
                 }
             }
             if (!mbar_wait(full_bar(s), r & 1, p.wait_limit, abort_flag, p.err_word)) return;
+            if constexpr (HALVES == 2) {
+                // two 128-wide halves: each its own codes, activations and
+                // group scale/zero; the stage is released once the second
+                // half is in registers
+                const uint32_t stage = stage_addr(s);
+                const uint32_t ms = meta_addr(m) + 16u * (uint32_t)(w * kRowsPerWarp + g);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    Act<MB> ac;
+                    load_act(ac, stage + L::act_off + (uint32_t)h * (kBlockK * 2), p.M, g, t,
+                             kBlockK * 2 * HALVES);
+                    RowWords<4> rw;
+                    read_codes_half(rw, stage, w * kRowsPerWarp + g, g, t, h);
+                    RowParams rp;
+                    const int gi = (kb * 2 + h) >> p.bpg_shift;
+                    const uint32_t sc = ms + 2u * (uint32_t)(gi & (kMetaGroups - 1));
+                    const uint32_t zc = ms + kMetaScaleBytes + (uint32_t)(gi & 15);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        uint32_t sv, zv;
+                        asm volatile("ld.shared.u16 %0, [%1];" : "=r"(sv) : "r"(sc + 128u * j));
+                        asm volatile("ld.shared.u8 %0, [%1];" : "=r"(zv) : "r"(zc + 128u * j));
+                        rp.s2[j] = sv * 0x00010001u;
+                        rp.z2[j] = (0xC300u + zv) * 0x00010001u;
+                    }
+                    if (h == 1) {
+                        __syncwarp();
+                        if (lane == 0) {
+                            mbar_arrive(empty_bar(s));
+                            if (kb + 1 == KB || ((kb + 1) & span_mask) == 0 ||
+                                u + (kb - kb0) + 1 == u_end)
+                                mbar_arrive(meta_empty_bar(m));
+                        }
+                    }
+                    compute_block<4, MB>(rp, ac, rw, s8, acc);
+                }
+            } else {
             const uint32_t stage = stage_addr(s);
             constexpr bool kWide = MB > 2;
             Act<kWide ? 1 : MB> ac;
@@ -870,6 +927,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap code_map,
                 if (BITS == 4 && META == kMetaNone) load_params_direct(rp, p, valid, rows, kb, t);
                 compute_block<BITS, MB>(rp, ac, rw, s8, acc);
             }
+            }
             if (++s == S) {
                 s = 0;
                 ++r;
@@ -902,10 +960,10 @@ struct Maps {
     CUtensorMap code, act, scale, zero;
 };
 
-template <int BITS, int MB, int META, int FMT>
+template <int BITS, int MB, int META, int FMT, int HALVES = 1>
 qz_status launch_variant(const Maps &maps, const GemvArgs &args, dim3 grid, int overlap,
                          cudaStream_t st) {
-    constexpr int smem = Layout<BITS, MB, META, FMT>::bytes;
+    constexpr int smem = Layout<BITS, MB, META, FMT, HALVES>::bytes;
     static DeviceOnce attr_once;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -913,13 +971,13 @@ qz_status launch_variant(const Maps &maps, const GemvArgs &args, dim3 grid, int 
         return QZ_ERR_CUDA;
     }
     if (attr_once.run(dev, [] {
-            cudaError_t e = cudaFuncSetAttribute(gemv_kernel<BITS, MB, META, FMT>,
+            cudaError_t e = cudaFuncSetAttribute(gemv_kernel<BITS, MB, META, FMT, HALVES>,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  smem);
             // three rings per SM need (nearly) all of the unified memory as
             // shared memory
             if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(gemv_kernel<BITS, MB, META, FMT>,
+                e = cudaFuncSetAttribute(gemv_kernel<BITS, MB, META, FMT, HALVES>,
                                          cudaFuncAttributePreferredSharedMemoryCarveout, 100);
             return e;
         }) != cudaSuccess)
@@ -934,8 +992,8 @@ qz_status launch_variant(const Maps &maps, const GemvArgs &args, dim3 grid, int 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = overlap > 0 ? 1 : 0;
-    cudaLaunchKernelEx(&cfg, gemv_kernel<BITS, MB, META, FMT>, maps.code, maps.act, maps.scale,
-                       maps.zero, args);
+    cudaLaunchKernelEx(&cfg, gemv_kernel<BITS, MB, META, FMT, HALVES>, maps.code, maps.act,
+                       maps.scale, maps.zero, args);
     return launch_status();
 }
 
@@ -963,8 +1021,11 @@ qz_status launch_gemv(const void *a, const void *codes, const void *scales, cons
     args.group_size = (int)group_size;
     args.group_shift = log2_exact(group_size);
     args.bpg_shift = group_size % kBlockK == 0 ? log2_exact(group_size / kBlockK) : -1;
-    args.meta_span_shift = args.bpg_shift >= 0 ? args.bpg_shift + 3 : 0;
-    args.kblocks = (int)(K / kBlockK);
+    // a meta slot holds 8 groups: 8 << bpg_shift blocks of 128 k, half as
+    // many units when a unit is two blocks
+    const int halves = plan.unit_k / kBlockK;
+    args.meta_span_shift = args.bpg_shift >= 0 ? args.bpg_shift + 3 - (halves - 1) : 0;
+    args.kblocks = (int)(K / plan.unit_k);
     args.y = static_cast<uint16_t *>(y);
     args.partials = nullptr;
     args.counters = nullptr;
@@ -983,11 +1044,13 @@ qz_status launch_gemv(const void *a, const void *codes, const void *scales, cons
 
     Maps maps;
     const uint64_t row_bytes = (uint64_t)K * BITS / 8;
+    // 128-byte code rows (int8, and int4 two-half units) take the 128-byte swizzle
+    const bool swizzle = BITS == 8 || halves == 2;
     if (!make_map_2d_cached(&maps.code, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, row_bytes,
-                            (uint64_t)N, row_bytes, kRowBytes<BITS>, kTileRows,
-                            BITS == 4 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B) ||
+                            (uint64_t)N, row_bytes, kRowBytes<BITS> * halves, kTileRows,
+                            swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !make_map_2d_cached(&maps.act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a, (uint64_t)K,
-                            (uint64_t)M, (uint64_t)K * 2, kBlockK, (uint32_t)M,
+                            (uint64_t)M, (uint64_t)K * 2, kBlockK * halves, (uint32_t)M,
                             CU_TENSOR_MAP_SWIZZLE_NONE))
         return QZ_ERR_CUDA;
     maps.scale = maps.code;   // unused unless kMetaTma
@@ -1005,8 +1068,11 @@ qz_status launch_gemv(const void *a, const void *codes, const void *scales, cons
                                     (uint64_t)gpr, (uint64_t)N, (uint64_t)gpr, 16, kTileRows,
                                     CU_TENSOR_MAP_SWIZZLE_NONE))
                 return QZ_ERR_CUDA;
+            if (halves == 2)
+                return launch_variant<4, 1, kMetaTma, kFmtInt, 2>(maps, args, grid, overlap, st);
             return launch_mb<4, kMetaTma>(maps, args, grid, overlap, st);
         }
+        if (halves != 1) return QZ_ERR_UNSUPPORTED;   // the plan's unit needs the TMA path
         // The gather path copies the aligned 4-byte words holding each scale
         // and zero; they stay inside the arrays when N * K / g is a multiple
         // of 4.
@@ -1032,6 +1098,7 @@ qz_status launch_fp4_gemv(const void *a, const void *codes, const void *scales,
     args.group_size = (int)K;                           // unused by the FP4 path
     args.group_shift = -1;
     args.bpg_shift = 0;
+    if (plan.unit_k != kBlockK) return QZ_ERR_UNSUPPORTED;
     args.kblocks = (int)(K / kBlockK);
     args.y = static_cast<uint16_t *>(y);
     if (plan.total_bytes > 0) {
@@ -1074,7 +1141,7 @@ qz_status launch_fp4_gemv(const void *a, const void *codes, const void *scales,
 
 }  // namespace
 
-// Stream-K plan.  Units are (128-row task x 128-wide K block); up to
+// Stream-K plan.  Units are (128-row task x unit_k-wide K block); up to
 // kMaxCtasPerSm CTAs run on an SM (their rings take 74 KB (int4) or 66 KB
 // (int8) of shared memory each), and the same number k runs on every SM.
 // k is the largest that still gives each CTA at least kMinUnitsPerCta units
@@ -1082,14 +1149,17 @@ qz_status launch_fp4_gemv(const void *a, const void *codes, const void *scales,
 // layers from splitting every task over many CTAs).
 constexpr int64_t kMinUnitsPerCta = 4;
 
-GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K, int bits, int sms) {
+GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K, int bits, int sms, int unit_k) {
     (void)bits;
     GemvPlan p{};
+    p.unit_k = unit_k;
     p.tasks = ceil_div(N, kTileRows);
-    p.kblocks = K / kBlockK;
+    p.kblocks = K / unit_k;
     const int64_t units = p.tasks * p.kblocks;
+    // the minimum counts 128-wide blocks: two-half units count twice
+    const int64_t min_units = kMinUnitsPerCta * kBlockK / unit_k;
     int64_t per_sm = M <= 16 ? kMaxCtasPerSm : (M <= 32 ? 2 : 1);
-    while (per_sm > 1 && units < (int64_t)sms * per_sm * kMinUnitsPerCta) --per_sm;
+    while (per_sm > 1 && units < (int64_t)sms * per_sm * min_units) --per_sm;
     p.ctas = (int64_t)sms * per_sm;
     // Fewer units than CTAs: one unit per CTA.  Every CTA must own at least
     // one unit, or a split task would count a contributor that never
@@ -1108,14 +1178,33 @@ GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K, int bits, int sms) {
 }
 
 // The plan's workspace is not monotone in the SM count, so the size callers
-// allocate is the largest over every count up to kSmCount.
-size_t gemv_workspace_bound(int64_t M, int64_t N, int64_t K, int bits) {
+// allocate is the largest over every count up to kSmCount, and over the unit
+// widths up to max_unit_k (a call planned for 256-wide units falls back to
+// 128 when its scale or zero array is not 16-byte aligned).
+size_t gemv_workspace_bound(int64_t M, int64_t N, int64_t K, int bits, int max_unit_k) {
+    (void)bits;
     size_t most = 0;
-    for (int sms = 1; sms <= kSmCount; ++sms) {
-        const size_t b = gemv_plan(M, N, K, bits, sms).total_bytes;
-        if (b > most) most = b;
+    for (int unit_k = kBlockK; unit_k <= max_unit_k; unit_k += kBlockK) {
+        for (int sms = 1; sms <= kSmCount; ++sms) {
+            const size_t b = gemv_plan(M, N, K, bits, sms, unit_k).total_bytes;
+            if (b > most) most = b;
+        }
     }
     return most;
+}
+
+// K per unit of the integer decode GEMV: 256 (two 128-wide halves, one
+// 128-byte row of codes per weight row and half the per-unit overhead) for
+// int4 with at most 8 tokens when K is a multiple of 256 and the groups'
+// scales and zeros come as TMA tiles (groups a multiple of 128, K/g a
+// multiple of 16, both arrays 16-byte aligned); otherwise 128.
+int gemv_unit_k(int bits, int64_t M, int64_t K, int64_t group_size, const void *scales,
+                const void *zeros) {
+    if (bits != 4 || M > 8 || K % (2 * kBlockK) != 0 || group_size % kBlockK != 0 ||
+        log2_exact(group_size / kBlockK) < 0 || (K / group_size) % 16 != 0 ||
+        !aligned(scales, 16) || !aligned(zeros, 16))
+        return kBlockK;
+    return 2 * kBlockK;
 }
 
 qz_status launch_w4a16_gemv(const void *a, const void *codes, const void *scales,

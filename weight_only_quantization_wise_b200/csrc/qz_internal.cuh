@@ -97,8 +97,9 @@ qz_status launch_dequantize(const void *codes, const void *scales, const void *z
 // subtask whose units span several CTAs is reduced through per-subtask
 // partial slots.
 struct GemvPlan {
+    int unit_k;           // K per unit: 128, or 256 (int4 two-half units)
     int64_t tasks;        // 128-row tasks
-    int64_t kblocks;      // 128-wide K blocks per task
+    int64_t kblocks;      // units per task (K / unit_k)
     int64_t ctas;         // launched CTAs (each owns at least one unit)
     int64_t slots;        // partial slots per subtask (max contributors)
     size_t partial_bytes; // fp32 partials [tasks * 4][slots][M][32]
@@ -107,9 +108,17 @@ struct GemvPlan {
 };
 // Workspace: fp32 partials at offset 0, then one uint32 counter per subtask.
 // `sms`: the SMs the grid is sized for (device_sm_count() at launch).
-GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K, int bits, int sms);
+GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K, int bits, int sms, int unit_k = 128);
+// K per unit the int4 GEMV takes for these arguments (128 or 256); without
+// pointers, for 16-byte aligned scale and zero arrays.
+int gemv_unit_k(int bits, int64_t M, int64_t K, int64_t group_size, const void *scales,
+                const void *zeros);
+inline int gemv_unit_k(int bits, int64_t M, int64_t K, int64_t group_size) {
+    static const uint4 aligned_probe[1] = {};
+    return gemv_unit_k(bits, M, K, group_size, aligned_probe, aligned_probe);
+}
 // Workspace bytes that serve the plan of every SM count up to kSmCount.
-size_t gemv_workspace_bound(int64_t M, int64_t N, int64_t K, int bits);
+size_t gemv_workspace_bound(int64_t M, int64_t N, int64_t K, int bits, int max_unit_k = 128);
 
 // `overlap`: qz_set_launch_overlap mode for this launch.
 qz_status launch_w4a16_gemv(const void *a, const void *codes, const void *scales,

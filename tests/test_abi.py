@@ -189,11 +189,13 @@ def test_w8a16_gemm_workspace_follows_the_route():
     ("W4A16_GEMV", 8, 11008, 4096, 128, 344 * 7 * 8 * 32 * 4 + 6 * 64 * 4),
     # M = 16: units of 128 k; 14336 -> 444 CTAs, 32 each, ceil(64/32) + 1 = 3
     ("W4A16_GEMV", 16, 28672, 8192, 128, 896 * 3 * 16 * 32 * 4 + 14 * 64 * 4),
-    # one task, K = 8192: 32 units of 256 k -> 32 CTAs, 32 slots; with g = 64
-    # (or M = 9, or K % 256 != 0) units of 128 k -> 64 CTAs and 64 slots
+    # one task, K = 8192: 32 units of 256 k -> 32 CTAs, 32 slots (up to 16
+    # tokens); with g = 64, M = 17 or K % 256 != 0 units of 128 k -> 64 CTAs
+    # and 64 slots
     ("W4A16_GEMV", 1, 128, 8192, 128, 4 * 32 * 1 * 32 * 4 + 64 * 4),
+    ("W4A16_GEMV", 16, 128, 8192, 128, 4 * 32 * 16 * 32 * 4 + 64 * 4),
     ("W4A16_GEMV", 1, 128, 8192, 64, 4 * 64 * 1 * 32 * 4 + 64 * 4),
-    ("W4A16_GEMV", 9, 128, 8192, 128, 4 * 64 * 9 * 32 * 4 + 64 * 4),
+    ("W4A16_GEMV", 17, 128, 8192, 128, 4 * 64 * 17 * 32 * 4 + 64 * 4),
     ("W4A16_GEMV", 1, 128, 8320, 128, 4 * 65 * 1 * 32 * 4 + 64 * 4),
 ])
 def test_gemv_plan_workspace(op, M, N, K, g, expect):
@@ -228,14 +230,14 @@ def test_workspace_bound_serves_every_sm_count(op, M, N, K, g):
     """Grids are sized for the device's own SM count (at most 148), while
     qz_workspace_bytes does not depend on the device: it must be at least the
     workspace of the plan for every count, and equal to the largest.  An int4
-    GEMV planned with 256-wide units (M <= 8, K % 256 == 0, g % 128 == 0)
+    GEMV planned with 256-wide units (M <= 16, K % 256 == 0, g % 128 == 0)
     falls back to 128-wide units when its scale or zero array is not 16-byte
     aligned, so its bound also covers the 128-wide plans, which are the plans
     of the same shape with g = 64 (the plan depends on g only through the
     unit width)."""
     bound = qz.qz_workspace_bytes(op, M, N, K, g)
     per_sms = [qz.qz_workspace_bytes_for_sms(op, M, N, K, g, sms) for sms in range(1, 149)]
-    two_half = (op in (qz.QZ_OP_W4A16_GEMV, qz.QZ_OP_W4A16_GEMM) and M <= 8 and K % 256 == 0
+    two_half = (op in (qz.QZ_OP_W4A16_GEMV, qz.QZ_OP_W4A16_GEMM) and M <= 16 and K % 256 == 0
                 and g % 128 == 0 and (K // g) % 16 == 0)
     if two_half:
         narrow = [qz.qz_workspace_bytes_for_sms(op, M, N, K, 64, sms) for sms in range(1, 149)]

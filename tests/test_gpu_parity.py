@@ -182,7 +182,7 @@ def test_matmuls_on_edge_rows(dev, M):
 GEMV_CASES = [  # (N, K, g)
     (1024, 1024, 128), (1000, 384, 128), (17, 128, 32), (96, 512, 64),
     (256, 2048, 256), (64, 1024, 1024), (4100, 1152, 128),
-    # units of 256 k for M <= 8 (K % 256 == 0, K/g a multiple of 16): groups
+    # units of 256 k for M <= 16 (K % 256 == 0, K/g a multiple of 16): groups
     # of 128 (two per unit), 256 (one) and 512 (a group spans two units),
     # ragged rows
     (384, 2048, 128), (130, 4096, 256), (4100, 4096, 128), (256, 8192, 512),
@@ -209,7 +209,7 @@ def test_w4a16_gemv_tolerance(dev, N, K, g, M):
 
 
 def test_w4a16_gemv_two_half_units_onehot_and_fallback(dev):
-    """Units of 256 k (up to 8 tokens, scale/zero tiles by TMA): one-hot
+    """Units of 256 k (up to 16 tokens, scale/zero tiles by TMA): one-hot
     activations read back the oracle's bf16 weights bit for bit; with a scale
     array that is not 16-byte aligned the call falls back to units of 128 k,
     within the bound and inside the workspace qz_workspace_bytes gives."""

@@ -79,8 +79,9 @@ constexpr int kMaxCtasPerSm = 3;
 // CTAs per SM of a variant: tokens in groups of 8 (MB groups); M > 16
 // (integer formats) takes larger stages and more registers: two CTAs per SM
 // for MB = 4, one for MB = 8 (64 accumulators per thread).
-template <int MB>
-constexpr int kCtasPerSm = MB <= 2 ? kMaxCtasPerSm : (MB == 4 ? 2 : 1);
+template <int MB, int HALVES = 1>
+constexpr int kCtasPerSm = MB <= 2 ? (HALVES == 2 && MB == 2 ? 2 : kMaxCtasPerSm)
+                                   : (MB == 4 ? 2 : 1);
 // Independent MMA accumulator chains per 16-row tile for M <= 8: the MMAs of
 // even and odd code words accumulate separately (summed at the flush), so a
 // warp has twice as many MMAs in flight.
@@ -89,8 +90,8 @@ template <int MB>
 constexpr int kChains = MB == 1 ? kAccChains : 1;
 // Shared memory one CTA may use so that kCtasPerSm fit on an SM (228 KB,
 // 1 KB of it reserved per CTA), less the slack for aligning the base.
-template <int MB>
-constexpr int kCtaSmemBudget = 228 * 1024 / kCtasPerSm<MB> - 1024 - 1024;
+template <int MB, int HALVES = 1>
+constexpr int kCtaSmemBudget = 228 * 1024 / kCtasPerSm<MB, HALVES> - 1024 - 1024;
 
 // How int4 scales and zeros reach shared memory (see the header comment).
 enum Meta { kMetaNone = 0, kMetaGather = 1, kMetaTma = 2 };
@@ -113,7 +114,7 @@ struct Layout {
     static constexpr int stage = code + act + (META == kMetaGather ? kSzStage : 0);
     static constexpr int meta = META == kMetaTma ? 2 * (kMetaScaleBytes + kMetaZeroBytes) : 0;
     static constexpr int lut = FMT == kFmtNv ? 512 : 0;                 // E4M3 -> bf16 table
-    static constexpr int S = (kCtaSmemBudget<MB> - meta - lut - 256) / stage;
+    static constexpr int S = (kCtaSmemBudget<MB, HALVES> - meta - lut - 256) / stage;
     static constexpr uint32_t codes = 0;                                 // + s * stage
     static constexpr uint32_t act_off = code;                            // within a stage
     static constexpr uint32_t sz_off = code + act;                       // within a stage
@@ -128,7 +129,7 @@ struct Layout {
     static constexpr uint32_t bytes = end + 1024;                        // + alignment slack
     static_assert(stage % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled codes");
     static_assert(S >= 3, "at least three stages in flight");
-    static_assert(end + 1024 <= kCtaSmemBudget<MB> + 1024, "the CTAs fit on an SM");
+    static_assert(end + 1024 <= kCtaSmemBudget<MB, HALVES> + 1024, "the CTAs fit on an SM");
 };
 
 // bf16 pair (nibble j, nibble j+4) of a code word: bf16_rne(S * (q - Z)).
@@ -586,14 +587,14 @@ __device__ __forceinline__ void gemv_flush(float (&acc)[2][MB][4], const GemvArg
 // 128-wide K blocks per unit (2: int4 units of 128 rows x 256 k, one
 // 128-byte row of codes per weight row, consumed as two halves).
 template <int BITS, int MB, int META, int FMT, int HALVES = 1>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm<MB>)
+__global__ void __launch_bounds__(kThreads, (kCtasPerSm<MB, HALVES>))
 gemv_kernel(const __grid_constant__ CUtensorMap code_map,
             const __grid_constant__ CUtensorMap act_map,
             const __grid_constant__ CUtensorMap scale_map,
             const __grid_constant__ CUtensorMap zero_map, const GemvArgs p) {
     using L = Layout<BITS, MB, META, FMT, HALVES>;
-    static_assert(HALVES == 1 || (BITS == 4 && FMT == kFmtInt && META == kMetaTma && MB == 1),
-                  "two-half units: int4 with scale/zero tiles by TMA, up to 8 tokens");
+    static_assert(HALVES == 1 || (BITS == 4 && FMT == kFmtInt && META == kMetaTma && MB <= 2),
+                  "two-half units: int4 with scale/zero tiles by TMA, up to 16 tokens");
     constexpr int S = L::S;
     constexpr bool kFp4 = FMT != kFmtInt;
     constexpr uint32_t kMetaBytes = kFp4 ? kFp4MetaBytes : kMetaScaleBytes + kMetaZeroBytes;
@@ -1069,7 +1070,10 @@ qz_status launch_gemv(const void *a, const void *codes, const void *scales, cons
                                     CU_TENSOR_MAP_SWIZZLE_NONE))
                 return QZ_ERR_CUDA;
             if (halves == 2)
-                return launch_variant<4, 1, kMetaTma, kFmtInt, 2>(maps, args, grid, overlap, st);
+                return M <= 8 ? launch_variant<4, 1, kMetaTma, kFmtInt, 2>(maps, args, grid,
+                                                                          overlap, st)
+                              : launch_variant<4, 2, kMetaTma, kFmtInt, 2>(maps, args, grid,
+                                                                          overlap, st);
             return launch_mb<4, kMetaTma>(maps, args, grid, overlap, st);
         }
         if (halves != 1) return QZ_ERR_UNSUPPORTED;   // the plan's unit needs the TMA path
@@ -1158,7 +1162,9 @@ GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K, int bits, int sms, int unit_
     const int64_t units = p.tasks * p.kblocks;
     // the minimum counts 128-wide blocks: two-half units count twice
     const int64_t min_units = kMinUnitsPerCta * kBlockK / unit_k;
-    int64_t per_sm = M <= 16 ? kMaxCtasPerSm : (M <= 32 ? 2 : 1);
+    // (9..16 tokens in two-half units: two CTAs per SM, for four stages)
+    int64_t per_sm = M <= 8 ? kMaxCtasPerSm
+                            : M <= 16 ? (unit_k > kBlockK ? 2 : kMaxCtasPerSm) : (M <= 32 ? 2 : 1);
     while (per_sm > 1 && units < (int64_t)sms * per_sm * min_units) --per_sm;
     p.ctas = (int64_t)sms * per_sm;
     // Fewer units than CTAs: one unit per CTA.  Every CTA must own at least
@@ -1195,12 +1201,12 @@ size_t gemv_workspace_bound(int64_t M, int64_t N, int64_t K, int bits, int max_u
 
 // K per unit of the integer decode GEMV: 256 (two 128-wide halves, one
 // 128-byte row of codes per weight row and half the per-unit overhead) for
-// int4 with at most 8 tokens when K is a multiple of 256 and the groups'
+// int4 with at most 16 tokens when K is a multiple of 256 and the groups'
 // scales and zeros come as TMA tiles (groups a multiple of 128, K/g a
 // multiple of 16, both arrays 16-byte aligned); otherwise 128.
 int gemv_unit_k(int bits, int64_t M, int64_t K, int64_t group_size, const void *scales,
                 const void *zeros) {
-    if (bits != 4 || M > 8 || K % (2 * kBlockK) != 0 || group_size % kBlockK != 0 ||
+    if (bits != 4 || M > 16 || K % (2 * kBlockK) != 0 || group_size % kBlockK != 0 ||
         log2_exact(group_size / kBlockK) < 0 || (K / group_size) % 16 != 0 ||
         !aligned(scales, 16) || !aligned(zeros, 16))
         return kBlockK;

@@ -197,6 +197,9 @@ def test_w8a16_gemm_workspace_follows_the_route():
     ("W4A16_GEMV", 1, 128, 8192, 64, 4 * 64 * 1 * 32 * 4 + 64 * 4),
     ("W4A16_GEMV", 17, 128, 8192, 128, 4 * 64 * 17 * 32 * 4 + 64 * 4),
     ("W4A16_GEMV", 1, 128, 8320, 128, 4 * 65 * 1 * 32 * 4 + 64 * 4),
+    # 4096 x 11008: 86 groups per row (gathered words, an even count): 32
+    # tasks x 43 units = 1376 -> 444 CTAs, 3 units each, ceil(43/3) + 1 = 16
+    ("W4A16_GEMV", 1, 4096, 11008, 128, 128 * 16 * 1 * 32 * 4 + 2 * 64 * 4),
 ])
 def test_gemv_plan_workspace(op, M, N, K, g, expect):
     """The stream-K plan (host logic) on a 148-SM device through the
@@ -222,6 +225,7 @@ WS_SHAPES = [  # (op, M, N, K, g): decode GEMV shapes, short and long layers, sm
     (qz.QZ_OP_W4A16_GEMM, 32, 8192, 8192, 128), (qz.QZ_OP_W8A16_GEMM, 200, 512, 2048, 2048),
     (qz.QZ_OP_W4A16_GEMM, 2048, 8192, 8192, 128), (qz.QZ_OP_W4A16_GEMM, 12, 4096, 4096, 128),
     (qz.QZ_OP_W4A16_GEMM, 8, 4096, 4096, 128), (qz.QZ_OP_W4A16_GEMV, 8, 300, 2048, 128),
+    (qz.QZ_OP_W4A16_GEMV, 1, 4096, 11008, 128), (qz.QZ_OP_W4A16_GEMV, 4, 130, 5632, 256),
 ]
 
 
@@ -230,15 +234,18 @@ def test_workspace_bound_serves_every_sm_count(op, M, N, K, g):
     """Grids are sized for the device's own SM count (at most 148), while
     qz_workspace_bytes does not depend on the device: it must be at least the
     workspace of the plan for every count, and equal to the largest.  An int4
-    GEMV planned with 256-wide units (M <= 16, K % 256 == 0, g % 128 == 0)
-    falls back to 128-wide units when its scale or zero array is not 16-byte
-    aligned, so its bound also covers the 128-wide plans, which are the plans
+    GEMV planned with 256-wide units (M <= 16, K % 256 == 0, scales and zeros
+    through the ring: TMA tiles, or gathered words with the two halves' groups
+    in the same words) falls back to 128-wide units when its scale or zero
+    array is misaligned, so its bound also covers the 128-wide plans, which are the plans
     of the same shape with g = 64 (the plan depends on g only through the
     unit width)."""
     bound = qz.qz_workspace_bytes(op, M, N, K, g)
     per_sms = [qz.qz_workspace_bytes_for_sms(op, M, N, K, g, sms) for sms in range(1, 149)]
+    gpr = K // g
+    ring = g % 128 == 0 and ((g // 128) & (g // 128 - 1)) == 0
     two_half = (op in (qz.QZ_OP_W4A16_GEMV, qz.QZ_OP_W4A16_GEMM) and M <= 16 and K % 256 == 0
-                and g % 128 == 0 and (K // g) % 16 == 0)
+                and ring and (gpr % 16 == 0 or ((N * gpr) % 4 == 0 and (g > 128 or gpr % 2 == 0))))
     if two_half:
         narrow = [qz.qz_workspace_bytes_for_sms(op, M, N, K, 64, sms) for sms in range(1, 149)]
         assert max(max(per_sms), max(narrow)) == bound

@@ -186,6 +186,8 @@ GEMV_CASES = [  # (N, K, g)
     # of 128 (two per unit), 256 (one) and 512 (a group spans two units),
     # ragged rows
     (384, 2048, 128), (130, 4096, 256), (4100, 4096, 128), (256, 8192, 512),
+    # ... with gathered scale/zero words (K/g not a multiple of 16)
+    (300, 2816, 128), (130, 5632, 256),
 ]
 
 

@@ -148,7 +148,7 @@ QZ_API qz_status qz_workspace_bytes(int32_t op, int64_t M, int64_t N, int64_t K,
         const qz_status s = check_gemv_shape(M, N, K);
         if (s != QZ_OK) return s;
         *bytes = op == QZ_OP_W4A16_GEMV
-                     ? gemv_workspace_bound(M, N, K, 4, gemv_unit_k(4, M, K, group_size))
+                     ? gemv_workspace_bound(M, N, K, 4, gemv_unit_k(4, M, N, K, group_size))
                      : gemv_workspace_bound(M, N, K, 8);
         return QZ_OK;
     }
@@ -157,7 +157,7 @@ QZ_API qz_status qz_workspace_bytes(int32_t op, int64_t M, int64_t N, int64_t K,
         if (M < 1 || N < 1 || K < 1) return QZ_ERR_INVALID_ARG;
         *bytes = M <= kGemmToGemvMaxM && K % 128 == 0
                      ? (op == QZ_OP_W4A16_GEMM
-                            ? gemv_workspace_bound(M, N, K, 4, gemv_unit_k(4, M, K, group_size))
+                            ? gemv_workspace_bound(M, N, K, 4, gemv_unit_k(4, M, N, K, group_size))
                             : gemv_workspace_bound(M, N, K, 8))
                      : gemm_workspace_bytes(M, N, K);
         return QZ_OK;
@@ -191,7 +191,7 @@ QZ_API qz_status qz_workspace_bytes_for_sms(int32_t op, int64_t M, int64_t N, in
         const qz_status s = check_gemv_shape(M, N, K);
         if (s != QZ_OK) return s;
         *bytes = op == QZ_OP_W4A16_GEMV
-                     ? gemv_plan(M, N, K, 4, sms, gemv_unit_k(4, M, K, group_size)).total_bytes
+                     ? gemv_plan(M, N, K, 4, sms, gemv_unit_k(4, M, N, K, group_size)).total_bytes
                      : gemv_plan(M, N, K, 8, sms).total_bytes;
         return QZ_OK;
     }
@@ -200,7 +200,7 @@ QZ_API qz_status qz_workspace_bytes_for_sms(int32_t op, int64_t M, int64_t N, in
         if (M < 1 || N < 1 || K < 1) return QZ_ERR_INVALID_ARG;
         *bytes = M <= kGemmToGemvMaxM && K % 128 == 0
                      ? (op == QZ_OP_W4A16_GEMM
-                            ? gemv_plan(M, N, K, 4, sms, gemv_unit_k(4, M, K, group_size))
+                            ? gemv_plan(M, N, K, 4, sms, gemv_unit_k(4, M, N, K, group_size))
                             : gemv_plan(M, N, K, 8, sms)).total_bytes
                      : gemm_workspace_bytes_for(M, N, K, sms);
         return QZ_OK;
@@ -254,7 +254,7 @@ QZ_API qz_status qz_w4a16_gemv(const void *a, const void *codes, const void *sca
     if (!aligned(a, 16) || !aligned(codes, 16) || !aligned(scales, 2) || !aligned(y, 2))
         return QZ_ERR_ALIGNMENT;
     const GemvPlan plan =
-        gemv_plan(M, N, K, 4, device_sm_count(), gemv_unit_k(4, M, K, group_size, scales, zeros));
+        gemv_plan(M, N, K, 4, device_sm_count(), gemv_unit_k(4, M, N, K, group_size, scales, zeros));
     s = check_workspace(plan.total_bytes, workspace, workspace_bytes);
     if (s != QZ_OK) return s;
     return launch_w4a16_gemv(a, codes, scales, zeros, M, N, K, group_size, y, workspace, plan,

@@ -593,8 +593,10 @@ gemv_kernel(const __grid_constant__ CUtensorMap code_map,
             const __grid_constant__ CUtensorMap scale_map,
             const __grid_constant__ CUtensorMap zero_map, const GemvArgs p) {
     using L = Layout<BITS, MB, META, FMT, HALVES>;
-    static_assert(HALVES == 1 || (BITS == 4 && FMT == kFmtInt && META == kMetaTma && MB <= 2),
-                  "two-half units: int4 with scale/zero tiles by TMA, up to 16 tokens");
+    static_assert(HALVES == 1 || (BITS == 4 && FMT == kFmtInt && MB <= 2 &&
+                                  (META == kMetaTma || META == kMetaGather)),
+                  "two-half units: int4 with scale/zero tiles by TMA or gathered words, up to "
+                  "16 tokens");
     constexpr int S = L::S;
     constexpr bool kFp4 = FMT != kFmtInt;
     constexpr uint32_t kMetaBytes = kFp4 ? kFp4MetaBytes : kMetaScaleBytes + kMetaZeroBytes;
@@ -720,7 +722,9 @@ gemv_kernel(const __grid_constant__ CUtensorMap code_map,
             }
             if (META == kMetaGather) {
                 const uint32_t dst = stage_addr(s) + L::sz_off + 16u * lane;
-                const int gi = kb >> p.bpg_shift;
+                // two-half units: the first half's group; the second half's
+                // scale and zero share its words (even groups per row)
+                const int gi = (kb * HALVES) >> p.bpg_shift;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int row = task * kTileRows + prow + 8 * j;
@@ -811,6 +815,12 @@ gemv_kernel(const __grid_constant__ CUtensorMap code_map,
                 // half is in registers
                 const uint32_t stage = stage_addr(s);
                 const uint32_t ms = meta_addr(m) + 16u * (uint32_t)(w * kRowsPerWarp + g);
+                uint4 gs = make_uint4(0u, 0u, 0u, 0u), gz = gs;     // gathered words
+                if constexpr (META == kMetaGather) {
+                    const uint32_t sz = stage + L::sz_off + 16u * (8 * w + g);
+                    gs = lds128(sz);
+                    gz = lds128(sz + 512u);
+                }
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     Act<MB> ac;
@@ -820,22 +830,38 @@ gemv_kernel(const __grid_constant__ CUtensorMap code_map,
                     read_codes_half(rw, stage, w * kRowsPerWarp + g, g, t, h);
                     RowParams rp;
                     const int gi = (kb * 2 + h) >> p.bpg_shift;
-                    const uint32_t sc = ms + 2u * (uint32_t)(gi & (kMetaGroups - 1));
-                    const uint32_t zc = ms + kMetaScaleBytes + (uint32_t)(gi & 15);
+                    if constexpr (META == kMetaGather) {
+                        // the group's position in the words the producer
+                        // gathered for the unit's first group
+                        const int phase = word_phase + gi;
+                        const uint32_t os = (uint32_t)(phase & 1) * 2u, oz = (uint32_t)(phase & 3);
+                        const uint32_t sel_s = os * 0x0101u + (os + 1u) * 0x1010u;   // (S, S)
+                        const uint32_t sel_z = oz * 0x0101u + 0x4040u;               // (0xC3, Z) x 2
+                        const uint32_t wsv[4] = {gs.x, gs.y, gs.z, gs.w};
+                        const uint32_t wzv[4] = {gz.x, gz.y, gz.z, gz.w};
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        uint32_t sv, zv;
-                        asm volatile("ld.shared.u16 %0, [%1];" : "=r"(sv) : "r"(sc + 128u * j));
-                        asm volatile("ld.shared.u8 %0, [%1];" : "=r"(zv) : "r"(zc + 128u * j));
-                        rp.s2[j] = sv * 0x00010001u;
-                        rp.z2[j] = (0xC300u + zv) * 0x00010001u;
+                        for (int j = 0; j < 4; ++j) {
+                            rp.s2[j] = dev::prmt(wsv[j], 0u, sel_s);
+                            rp.z2[j] = dev::prmt(wzv[j], 0xC3C3C3C3u, sel_z);
+                        }
+                    } else {
+                        const uint32_t sc = ms + 2u * (uint32_t)(gi & (kMetaGroups - 1));
+                        const uint32_t zc = ms + kMetaScaleBytes + (uint32_t)(gi & 15);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            uint32_t sv, zv;
+                            asm volatile("ld.shared.u16 %0, [%1];" : "=r"(sv) : "r"(sc + 128u * j));
+                            asm volatile("ld.shared.u8 %0, [%1];" : "=r"(zv) : "r"(zc + 128u * j));
+                            rp.s2[j] = sv * 0x00010001u;
+                            rp.z2[j] = (0xC300u + zv) * 0x00010001u;
+                        }
                     }
                     if (h == 1) {
                         __syncwarp();
                         if (lane == 0) {
                             mbar_arrive(empty_bar(s));
-                            if (kb + 1 == KB || ((kb + 1) & span_mask) == 0 ||
-                                u + (kb - kb0) + 1 == u_end)
+                            if (META == kMetaTma && (kb + 1 == KB || ((kb + 1) & span_mask) == 0 ||
+                                                     u + (kb - kb0) + 1 == u_end))
                                 mbar_arrive(meta_empty_bar(m));
                         }
                     }
@@ -1008,6 +1034,31 @@ qz_status launch_mb(const Maps &maps, const GemvArgs &args, dim3 grid, int overl
     return launch_variant<BITS, 8, META, kFmtInt>(maps, args, grid, overlap, st);
 }
 
+// How the int4 GEMV's scales and zeros reach shared memory: as TMA tiles
+// (groups a multiple of 128, K/g a multiple of 16, both arrays 16-byte
+// aligned), as gathered 4-byte words (groups a multiple of 128, arrays 4-byte
+// aligned, N * K / g a multiple of 4 so every word lies inside its array), or
+// loaded by the consumers.
+int int4_meta(int64_t N, int64_t K, int64_t group_size, const void *scales, const void *zeros) {
+    const int64_t gpr = K / group_size;
+    const bool ring = group_size % kBlockK == 0 && log2_exact(group_size / kBlockK) >= 0;
+    if (ring && gpr % 16 == 0 && aligned(scales, 16) && aligned(zeros, 16)) return kMetaTma;
+    if (ring && aligned(scales, 4) && aligned(zeros, 4) && (N * gpr) % 4 == 0) return kMetaGather;
+    return kMetaNone;
+}
+
+// Two-half units (256 k) need a ring metadata path, K % 256 == 0, and, with
+// gathered words, the second half's scale and zero in the words of the
+// first: the two halves share a group (g >= 256), or the row's group count
+// is even (g = 128: the pair 2j, 2j+1 never straddles a scale or zero word).
+bool two_half_ok(int64_t M, int64_t N, int64_t K, int64_t group_size, const void *scales,
+                 const void *zeros) {
+    if (M > 16 || K % (2 * kBlockK) != 0) return false;
+    const int meta = int4_meta(N, K, group_size, scales, zeros);
+    if (meta == kMetaTma) return true;
+    return meta == kMetaGather && (group_size > kBlockK || (K / group_size) % 2 == 0);
+}
+
 template <int BITS>
 qz_status launch_gemv(const void *a, const void *codes, const void *scales, const void *zeros,
                       int64_t M, int64_t N, int64_t K, int64_t group_size, void *y,
@@ -1060,7 +1111,10 @@ qz_status launch_gemv(const void *a, const void *codes, const void *scales, cons
 
     if constexpr (BITS == 4) {
         const int64_t gpr = K / group_size;
-        if (args.bpg_shift >= 0 && gpr % 16 == 0 && aligned(scales, 16) && aligned(zeros, 16)) {
+        const int meta = int4_meta(N, K, group_size, scales, zeros);
+        if (halves == 2 && !two_half_ok(M, N, K, group_size, scales, zeros))
+            return QZ_ERR_UNSUPPORTED;   // the plan's units need a ring metadata path
+        if (meta == kMetaTma) {
             // eight groups of scales and sixteen of zeros per row, 128 rows
             if (!make_map_2d_cached(&maps.scale, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, scales,
                                     (uint64_t)gpr, (uint64_t)N, (uint64_t)gpr * 2, kMetaGroups,
@@ -1076,13 +1130,16 @@ qz_status launch_gemv(const void *a, const void *codes, const void *scales, cons
                                                                           overlap, st);
             return launch_mb<4, kMetaTma>(maps, args, grid, overlap, st);
         }
-        if (halves != 1) return QZ_ERR_UNSUPPORTED;   // the plan's unit needs the TMA path
         // The gather path copies the aligned 4-byte words holding each scale
-        // and zero; they stay inside the arrays when N * K / g is a multiple
-        // of 4.
-        const int64_t entries = N * gpr;
-        if (args.bpg_shift >= 0 && aligned(scales, 4) && aligned(zeros, 4) && entries % 4 == 0)
+        // and zero.
+        if (meta == kMetaGather) {
+            if (halves == 2)
+                return M <= 8 ? launch_variant<4, 1, kMetaGather, kFmtInt, 2>(maps, args, grid,
+                                                                             overlap, st)
+                              : launch_variant<4, 2, kMetaGather, kFmtInt, 2>(maps, args, grid,
+                                                                             overlap, st);
             return launch_mb<4, kMetaGather>(maps, args, grid, overlap, st);
+        }
         return launch_mb<4, kMetaNone>(maps, args, grid, overlap, st);
     } else {
         return launch_mb<8, kMetaNone>(maps, args, grid, overlap, st);
@@ -1202,15 +1259,11 @@ size_t gemv_workspace_bound(int64_t M, int64_t N, int64_t K, int bits, int max_u
 // K per unit of the integer decode GEMV: 256 (two 128-wide halves, one
 // 128-byte row of codes per weight row and half the per-unit overhead) for
 // int4 with at most 16 tokens when K is a multiple of 256 and the groups'
-// scales and zeros come as TMA tiles (groups a multiple of 128, K/g a
-// multiple of 16, both arrays 16-byte aligned); otherwise 128.
-int gemv_unit_k(int bits, int64_t M, int64_t K, int64_t group_size, const void *scales,
-                const void *zeros) {
-    if (bits != 4 || M > 16 || K % (2 * kBlockK) != 0 || group_size % kBlockK != 0 ||
-        log2_exact(group_size / kBlockK) < 0 || (K / group_size) % 16 != 0 ||
-        !aligned(scales, 16) || !aligned(zeros, 16))
-        return kBlockK;
-    return 2 * kBlockK;
+// scales and zeros come through the ring (two_half_ok); otherwise 128.
+int gemv_unit_k(int bits, int64_t M, int64_t N, int64_t K, int64_t group_size,
+                const void *scales, const void *zeros) {
+    if (bits != 4 || group_size <= 0 || K % group_size != 0) return kBlockK;
+    return two_half_ok(M, N, K, group_size, scales, zeros) ? 2 * kBlockK : kBlockK;
 }
 
 qz_status launch_w4a16_gemv(const void *a, const void *codes, const void *scales,

@@ -67,7 +67,7 @@ extern "C" QZ_API qz_status qz_w4a16_gemv_noalloc(const void *a, const void *cod
         !qz::is_aligned(y, 2))
         return QZ_ERR_ALIGNMENT;
     const qz::GemvPlan plan = qz::gemv_plan(M, N, K, 4, qz::device_sm_count(),
-                                            qz::gemv_unit_k(4, M, K, group_size, scales, zeros));
+                                            qz::gemv_unit_k(4, M, N, K, group_size, scales, zeros));
     if (plan.total_bytes > qz::kScratchBytes) return QZ_ERR_WORKSPACE;   // beyond the built-in maximum
     void *scratch = nullptr;
     if (plan.total_bytes > 0) {

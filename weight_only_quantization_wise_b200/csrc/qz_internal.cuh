@@ -111,11 +111,11 @@ struct GemvPlan {
 GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K, int bits, int sms, int unit_k = 128);
 // K per unit the int4 GEMV takes for these arguments (128 or 256); without
 // pointers, for 16-byte aligned scale and zero arrays.
-int gemv_unit_k(int bits, int64_t M, int64_t K, int64_t group_size, const void *scales,
-                const void *zeros);
-inline int gemv_unit_k(int bits, int64_t M, int64_t K, int64_t group_size) {
+int gemv_unit_k(int bits, int64_t M, int64_t N, int64_t K, int64_t group_size,
+                const void *scales, const void *zeros);
+inline int gemv_unit_k(int bits, int64_t M, int64_t N, int64_t K, int64_t group_size) {
     static const uint4 aligned_probe[1] = {};
-    return gemv_unit_k(bits, M, K, group_size, aligned_probe, aligned_probe);
+    return gemv_unit_k(bits, M, N, K, group_size, aligned_probe, aligned_probe);
 }
 // Workspace bytes that serve the plan of every SM count up to kSmCount.
 size_t gemv_workspace_bound(int64_t M, int64_t N, int64_t K, int bits, int max_unit_k = 128);

@@ -120,7 +120,8 @@ def check_gemv(dev, kind, N, K, M, seed, rows=None):
 
 
 @pytest.mark.parametrize("kind", KINDS)
-@pytest.mark.parametrize("N,K", [(1024, 1024), (1000, 384), (4100, 1152), (17, 128), (256, 2048)])
+@pytest.mark.parametrize("N,K", [(1024, 1024), (1000, 384), (4100, 1152), (17, 128), (256, 2048),
+                                 (4100, 1536)])    # K % 512 == 0: units of 256 k
 @pytest.mark.parametrize("M", [1, 3, 8, 16])
 def test_fp4a16_gemv_tolerance(dev, kind, N, K, M):
     check_gemv(dev, kind, N, K, M, seed=N + K + M)

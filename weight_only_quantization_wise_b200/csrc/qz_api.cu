@@ -164,7 +164,9 @@ QZ_API qz_status qz_workspace_bytes(int32_t op, int64_t M, int64_t N, int64_t K,
     case QZ_OP_FP4A16_GEMV: {
         const qz_status s = check_gemv_shape(M, N, K, kFp4GemvMaxM);
         if (s != QZ_OK) return s;
-        *bytes = gemv_workspace_bound(M, N, K, 4);
+        // 256-wide units when K % 512 == 0 (and the block scales are
+        // 16-byte aligned; 128-wide otherwise): the bound covers both
+        *bytes = gemv_workspace_bound(M, N, K, 4, K % 512 == 0 ? 256 : 128);
         return QZ_OK;
     }
     case QZ_OP_GPTQ:
@@ -207,7 +209,7 @@ QZ_API qz_status qz_workspace_bytes_for_sms(int32_t op, int64_t M, int64_t N, in
     case QZ_OP_FP4A16_GEMV: {
         const qz_status s = check_gemv_shape(M, N, K, kFp4GemvMaxM);
         if (s != QZ_OK) return s;
-        *bytes = gemv_plan(M, N, K, 4, sms).total_bytes;
+        *bytes = gemv_plan(M, N, K, 4, sms, K % 512 == 0 ? 256 : 128).total_bytes;
         return QZ_OK;
     }
     default:
@@ -395,7 +397,8 @@ QZ_API qz_status qz_fp4a16_gemv(const void *a, const void *codes, const void *bl
     if (!aligned(a, 16) || !aligned(codes, 16) || !aligned(y, 2) ||
         (tensor_scale && !aligned(tensor_scale, 4)))
         return QZ_ERR_ALIGNMENT;
-    const GemvPlan plan = gemv_plan(M, N, K, 4, device_sm_count());
+    const GemvPlan plan =
+        gemv_plan(M, N, K, 4, device_sm_count(), gemv_fp4_unit_k(M, K, block_scales));
     s = check_workspace(plan.total_bytes, workspace, workspace_bytes);
     if (s != QZ_OK) return s;
     return launch_fp4a16_gemv(a, codes, block_scales, tensor_scale, M, N, K, kind, y, workspace,

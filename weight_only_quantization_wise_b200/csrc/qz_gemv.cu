@@ -593,10 +593,11 @@ gemv_kernel(const __grid_constant__ CUtensorMap code_map,
             const __grid_constant__ CUtensorMap scale_map,
             const __grid_constant__ CUtensorMap zero_map, const GemvArgs p) {
     using L = Layout<BITS, MB, META, FMT, HALVES>;
-    static_assert(HALVES == 1 || (BITS == 4 && FMT == kFmtInt && MB <= 2 &&
-                                  (META == kMetaTma || META == kMetaGather)),
-                  "two-half units: int4 with scale/zero tiles by TMA or gathered words, up to "
-                  "16 tokens");
+    static_assert(HALVES == 1 ||
+                      (BITS == 4 && MB <= 2 &&
+                       (META == kMetaTma || (FMT == kFmtInt && META == kMetaGather))),
+                  "two-half units: 4-bit codes with scales by TMA (int4 also by gathered "
+                  "words), up to 16 tokens");
     constexpr int S = L::S;
     constexpr bool kFp4 = FMT != kFmtInt;
     constexpr uint32_t kMetaBytes = kFp4 ? kFp4MetaBytes : kMetaScaleBytes + kMetaZeroBytes;
@@ -693,7 +694,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap code_map,
                     mbar_arrive_expect_tx(meta_full_bar(m), kMetaBytes);
                     if (kFp4) {
                         // 32 scale bytes (blocks) of each of the 128 rows
-                        tma_load_2d(meta_addr(m), &scale_map, (kb << p.fp4_bpu_shift) & ~31,
+                        tma_load_2d(meta_addr(m), &scale_map,
+                                    ((kb * HALVES) << p.fp4_bpu_shift) & ~31,
                                     task * kTileRows, meta_full_bar(m));
                     } else {
                         const int gi = (kb * HALVES) >> p.bpg_shift;
@@ -829,8 +831,31 @@ gemv_kernel(const __grid_constant__ CUtensorMap code_map,
                     RowWords<4> rw;
                     read_codes_half(rw, stage, w * kRowsPerWarp + g, g, t, h);
                     RowParams rp;
+                    uint32_t fa[4], fb[4];                   // FP4 block scales, rows g + 8j
                     const int gi = (kb * 2 + h) >> p.bpg_shift;
-                    if constexpr (META == kMetaGather) {
+                    if constexpr (kFp4) {
+                        // the half's blocks in the meta slot (32 scale bytes per row)
+                        const int blk = ((kb * 2 + h) << p.fp4_bpu_shift) +
+                                        (FMT == kFmtMx ? t : 2 * t);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint32_t a = meta_addr(m) +
+                                               32u * (uint32_t)(w * kRowsPerWarp + g + 8 * j) +
+                                               (uint32_t)(blk & 31);
+                            uint32_t b0, b1 = 0u;
+                            asm volatile("ld.shared.u8 %0, [%1];" : "=r"(b0) : "r"(a));
+                            if (FMT == kFmtNv)
+                                asm volatile("ld.shared.u8 %0, [%1];" : "=r"(b1) : "r"(a + 1u));
+                            if (FMT == kFmtMx) {
+                                fa[j] = fb[j] = e8m0_pair(b0);
+                            } else {
+                                const uint16_t *lut =
+                                    reinterpret_cast<const uint16_t *>(smem + L::lut_base);
+                                fa[j] = (uint32_t)lut[b0] * 0x00010001u;
+                                fb[j] = (uint32_t)lut[b1] * 0x00010001u;
+                            }
+                        }
+                    } else if constexpr (META == kMetaGather) {
                         // the group's position in the words the producer
                         // gathered for the unit's first group
                         const int phase = word_phase + gi;
@@ -865,7 +890,10 @@ gemv_kernel(const __grid_constant__ CUtensorMap code_map,
                                 mbar_arrive(meta_empty_bar(m));
                         }
                     }
-                    compute_block<4, MB>(rp, ac, rw, s8, acc);
+                    if constexpr (kFp4)
+                        compute_block_fp4<MB>(fa, fb, ac, rw, acc);
+                    else
+                        compute_block<4, MB>(rp, ac, rw, s8, acc);
                 }
             } else {
             const uint32_t stage = stage_addr(s);
@@ -1154,13 +1182,15 @@ qz_status launch_fp4_gemv(const void *a, const void *codes, const void *scales,
     args.fp4_scales = static_cast<const uint8_t *>(scales);
     args.tensor_scale = static_cast<const float *>(tensor_scale);
     args.fp4_bpu_shift = kind == 0 ? 2 : 3;             // 4 or 8 scale blocks per 128 k
-    args.meta_span_shift = 5 - args.fp4_bpu_shift;      // 32 scale bytes per meta slot
+    const int halves = plan.unit_k / kBlockK;
+    // 32 scale bytes per meta slot: 8 (MXFP4) or 4 (NVFP4) blocks of 128 k,
+    // half as many units when a unit is two blocks
+    args.meta_span_shift = 5 - args.fp4_bpu_shift - (halves - 1);
     args.M = (int)M; args.N = (int)N; args.K = (int)K;
     args.group_size = (int)K;                           // unused by the FP4 path
     args.group_shift = -1;
     args.bpg_shift = 0;
-    if (plan.unit_k != kBlockK) return QZ_ERR_UNSUPPORTED;
-    args.kblocks = (int)(K / kBlockK);
+    args.kblocks = (int)(K / plan.unit_k);
     args.y = static_cast<uint16_t *>(y);
     if (plan.total_bytes > 0) {
         args.partials = static_cast<float *>(workspace);
@@ -1177,10 +1207,10 @@ qz_status launch_fp4_gemv(const void *a, const void *codes, const void *scales,
     Maps maps;
     const uint64_t row_bytes = (uint64_t)K / 2;
     if (!make_map_2d_cached(&maps.code, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, row_bytes,
-                            (uint64_t)N, row_bytes, kRowBytes<4>, kTileRows,
-                            CU_TENSOR_MAP_SWIZZLE_NONE) ||
+                            (uint64_t)N, row_bytes, kRowBytes<4> * halves, kTileRows,
+                            halves == 2 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !make_map_2d_cached(&maps.act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a, (uint64_t)K,
-                            (uint64_t)M, (uint64_t)K * 2, kBlockK, (uint32_t)M,
+                            (uint64_t)M, (uint64_t)K * 2, kBlockK * halves, (uint32_t)M,
                             CU_TENSOR_MAP_SWIZZLE_NONE))
         return QZ_ERR_CUDA;
     maps.scale = maps.code;
@@ -1193,6 +1223,14 @@ qz_status launch_fp4_gemv(const void *a, const void *codes, const void *scales,
                             (uint64_t)blocks_per_row, (uint64_t)N, (uint64_t)blocks_per_row, 32,
                             kTileRows, CU_TENSOR_MAP_SWIZZLE_NONE))
         return QZ_ERR_CUDA;
+    if (halves == 2) {
+        if (!tma_meta || K % (2 * kBlockK) != 0) return QZ_ERR_UNSUPPORTED;
+        if (kind == 0)
+            return M <= 8 ? launch_variant<4, 1, kMetaTma, kFmtMx, 2>(maps, args, grid, overlap, st)
+                          : launch_variant<4, 2, kMetaTma, kFmtMx, 2>(maps, args, grid, overlap, st);
+        return M <= 8 ? launch_variant<4, 1, kMetaTma, kFmtNv, 2>(maps, args, grid, overlap, st)
+                      : launch_variant<4, 2, kMetaTma, kFmtNv, 2>(maps, args, grid, overlap, st);
+    }
     if (kind == 0)
         return tma_meta ? launch_mb<4, kMetaTma, kFmtMx>(maps, args, grid, overlap, st)
                         : launch_mb<4, kMetaNone, kFmtMx>(maps, args, grid, overlap, st);
@@ -1260,6 +1298,13 @@ size_t gemv_workspace_bound(int64_t M, int64_t N, int64_t K, int bits, int max_u
 // 128-byte row of codes per weight row and half the per-unit overhead) for
 // int4 with at most 16 tokens when K is a multiple of 256 and the groups'
 // scales and zeros come through the ring (two_half_ok); otherwise 128.
+// K per unit of the FP4A16 GEMV: 256 when K is a multiple of 512 (both
+// kinds then get their block scales as TMA tiles: K/32 and K/16 multiples of
+// 16) and the block-scale array is 16-byte aligned; otherwise 128.
+int gemv_fp4_unit_k(int64_t M, int64_t K, const void *scales) {
+    return M <= 16 && K % 512 == 0 && aligned(scales, 16) ? 2 * kBlockK : kBlockK;
+}
+
 int gemv_unit_k(int bits, int64_t M, int64_t N, int64_t K, int64_t group_size,
                 const void *scales, const void *zeros) {
     if (bits != 4 || group_size <= 0 || K % group_size != 0) return kBlockK;

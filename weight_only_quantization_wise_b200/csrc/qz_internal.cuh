@@ -113,6 +113,7 @@ GemvPlan gemv_plan(int64_t M, int64_t N, int64_t K, int bits, int sms, int unit_
 // pointers, for 16-byte aligned scale and zero arrays.
 int gemv_unit_k(int bits, int64_t M, int64_t N, int64_t K, int64_t group_size,
                 const void *scales, const void *zeros);
+int gemv_fp4_unit_k(int64_t M, int64_t K, const void *scales);
 inline int gemv_unit_k(int bits, int64_t M, int64_t N, int64_t K, int64_t group_size) {
     static const uint4 aligned_probe[1] = {};
     return gemv_unit_k(bits, M, N, K, group_size, aligned_probe, aligned_probe);

@@ -47,20 +47,16 @@ __device__ __forceinline__ float e4m3_value(uint32_t b) {
 // and normal ranges (m * 2^-9, then (8 + m) * 2^(e - 10)).
 __device__ __forceinline__ uint32_t e4m3_round_up(float t) {
     if (!(t > 0.0f)) return 0u;
-    if (t >= 448.0f) return 0x7Eu;
     if (t < 0.015625f) {                                         // below 2^-6: subnormal step 2^-9
         const float m = ceilf(t * 512.0f);                       // exact scaling
         return (uint32_t)m;                                      // 8 -> 0x08 = 2^-6
     }
-    const int E = ilogbf(t);                                     // t in [2^E, 2^(E+1))
-    const float mant = ldexpf(t, -E);                            // [1, 2), exact
-    uint32_t m = (uint32_t)ceilf((mant - 1.0f) * 8.0f);          // exact
-    int e = E + 7;
-    if (m == 8u) {
-        m = 0u;
-        ++e;
-    }
-    const uint32_t b = ((uint32_t)e << 3) | m;
+    // Normal range: adding 2^20 - 1 to the fp32 bits and dropping the low 20
+    // bits keeps three mantissa bits rounded up (a carry moves into the
+    // exponent), which leaves the biased exponent and mantissa of the E4M3
+    // value shifted by (127 - 7) << 3; anything above 448 (0x7E) is clamped.
+    const uint32_t r = (__float_as_uint(t) + 0x000FFFFFu) >> 20;
+    const uint32_t b = r - 960u;
     return b > 0x7Eu ? 0x7Eu : b;
 }
 
@@ -166,6 +162,12 @@ fp4_quantize_kernel(const uint4 *__restrict__ w, int64_t blocks, uint8_t *__rest
     constexpr int BS = KIND == 0 ? 32 : 16;
     float s_t = 1.0f;
     if (KIND == 1) s_t = nv_tensor_scale(__uint_as_float(*amax_bits));
+    // NVFP4: amax_b / fp32(6 s_t) by Markstein's correction from one
+    // reciprocal per thread (as for the codes below), where every operand
+    // stays normal; otherwise the IEEE division
+    const float d6 = __fmul_rn(6.0f, s_t);
+    const float r6 = __frcp_rn(d6);
+    const bool d6_normal = d6 >= 0x1p-96f && d6 <= 0x1p96f;
     for (int64_t b = thread_index(); b < blocks; b += grid_stride()) {
         uint32_t x[BS / 2];
 #pragma unroll
@@ -192,7 +194,11 @@ fp4_quantize_kernel(const uint4 *__restrict__ w, int64_t blocks, uint8_t *__rest
             scale = ldexpf(1.0f, e);
             r = ldexpf(1.0f, -e);                                // exact: x * r = x / 2^e
         } else {
-            sb = e4m3_round_up(__fdiv_rn(amax, __fmul_rn(6.0f, s_t)));
+            const float q0 = __fmul_rn(amax, r6);
+            const float t = d6_normal && amax >= 0x1p-100f && q0 >= 0x1p-100f
+                                ? __fmaf_rn(__fmaf_rn(-q0, d6, amax), r6, q0)
+                                : __fdiv_rn(amax, d6);
+            sb = e4m3_round_up(t);
             scale = __fmul_rn(e4m3_value(sb), s_t);
             r = __frcp_rn(scale);
             // 2^-96 <= scale <= 2^96 keeps x, r, q0 s and the residual normal
@@ -200,7 +206,9 @@ fp4_quantize_kernel(const uint4 *__restrict__ w, int64_t blocks, uint8_t *__rest
             exact_div = !(scale >= 0x1p-96f && scale <= 0x1p96f);
         }
         if (MMA) {
-            const int64_t row = b / blocks_per_row;
+            const int64_t row = b <= 0xFFFFFFFFll && blocks_per_row <= 0xFFFFFFFFll
+                                    ? (int64_t)((uint32_t)b / (uint32_t)blocks_per_row)
+                                    : b / blocks_per_row;
             scales[mma_scale_offset(row, b - row * blocks_per_row, blocks_per_row >> 2)] =
                 (uint8_t)sb;
         } else {
@@ -277,11 +285,16 @@ fp4_dequantize_kernel(const uint32_t *__restrict__ codes, const uint8_t *__restr
     }
 }
 
-unsigned grid_for(int64_t items) {
-    const int64_t cap = (int64_t)device_sm_count() * 16;
+unsigned grid_for(int64_t items, int per_sm = 16) {
+    const int64_t cap = (int64_t)device_sm_count() * per_sm;
     const int64_t b = (items + kThreads - 1) / kThreads;
     return (unsigned)(b < 1 ? 1 : (b < cap ? b : cap));
 }
+
+// The amax pass ends with one atomicMax per CTA on a single word, which the
+// L2 serialises: four CTAs per SM keep four 16-byte loads per thread in
+// flight with a quarter of the atomics of the quantize grid.
+unsigned amax_grid(int64_t chunks) { return grid_for(chunks, 4); }
 
 }  // namespace
 
@@ -299,7 +312,7 @@ qz_status launch_fp4_quantize(const void *w, int64_t N, int64_t K, int kind, voi
     unsigned *amax = static_cast<unsigned *>(tensor_scale);      // amax first, then s_t
     if (cudaMemsetAsync(amax, 0, sizeof(unsigned), st) != cudaSuccess) return QZ_ERR_CUDA;
     const int64_t chunks = N * K / 8;
-    fp4_amax_kernel<<<grid_for(chunks), kThreads, 0, st>>>(w4, chunks, amax);
+    fp4_amax_kernel<<<amax_grid(chunks), kThreads, 0, st>>>(w4, chunks, amax);
     fp4_quantize_kernel<1><<<grid_for(blocks), kThreads, 0, st>>>(
         w4, blocks, static_cast<uint8_t *>(codes), static_cast<uint8_t *>(scales), amax);
     fp4_finish_kernel<<<1, 1, 0, st>>>(static_cast<float *>(tensor_scale));
@@ -330,7 +343,7 @@ qz_status launch_fp4_quantize_mma(const void *a, int64_t M, int64_t K, int kind,
     }
     if (cudaMemsetAsync(amax, 0, sizeof(unsigned), st) != cudaSuccess) return QZ_ERR_CUDA;
     const int64_t chunks = M * K / 8;
-    fp4_amax_kernel<<<grid_for(chunks), kThreads, 0, st>>>(a4, chunks, amax);
+    fp4_amax_kernel<<<amax_grid(chunks), kThreads, 0, st>>>(a4, chunks, amax);
     fp4_quantize_kernel<1, true><<<grid_for(blocks), kThreads, 0, st>>>(
         a4, blocks, static_cast<uint8_t *>(codes), static_cast<uint8_t *>(scales_mma), amax, per_row);
     return launch_status();

@@ -401,8 +401,11 @@ def run_extras(qz, dev, pk, stream):
         a = synthetic.activations(M, K, seed=cfg["seed"] + 1000, device=dev)
         c, s, z = qz.qz_quantize_pack(w, 4, False, GROUP)
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-        qz.qz_w4a16_gemm(a, c, s, z, N, K, GROUP, y=y)
-        g = capture(lambda: qz.qz_w4a16_gemm(a, c, s, z, N, K, GROUP, y=y), stream)
+        wsp = torch.zeros(max(256, qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMM, M, N, K, GROUP),
+                              qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMM, M, N, K, K)),
+                          dtype=torch.uint8, device=dev)
+        qz.qz_w4a16_gemm(a, c, s, z, N, K, GROUP, y=y, workspace=wsp)
+        g = capture(lambda: qz.qz_w4a16_gemm(a, c, s, z, N, K, GROUP, y=y, workspace=wsp), stream)
         ms = time_graph(g)
         tf = gemm_flops(M, N, K) / (ms * 1e-3) / 1e12
         out["prefill_gemm_2048x8192x8192"] = {
@@ -420,8 +423,9 @@ def run_extras(qz, dev, pk, stream):
         del wb, yb, g, gb, c, s, z
         # W8A16 prefill GEMM, same shape, int8 symmetric per-channel
         c8, s8, _ = qz.qz_quantize_pack(w, 8, True, K)
-        qz.qz_w8a16_gemm(a, c8, s8, N, K, y=y)
-        ms = time_graph(capture(lambda: qz.qz_w8a16_gemm(a, c8, s8, N, K, y=y), stream))
+        qz.qz_w8a16_gemm(a, c8, s8, N, K, y=y, workspace=wsp)
+        ms = time_graph(capture(lambda: qz.qz_w8a16_gemm(a, c8, s8, N, K, y=y, workspace=wsp),
+                                stream))
         tf = gemm_flops(M, N, K) / (ms * 1e-3) / 1e12
         out["prefill_w8a16_gemm_2048x8192x8192"] = {
             "ms": round(ms, 4), "TFLOP/s": round(tf, 1),
@@ -807,7 +811,12 @@ def run_kernel_case(name, reps):
     kind, M, N, K = PROFILE_CASES[name]
     dev = torch.device("cuda", 0)
     w = synthetic.weights(N, K, sigma=0.015, seed=4, device=dev)
-    ws = torch.zeros(1 << 24, dtype=torch.uint8, device=dev)
+    op = {"gemv4": qz.QZ_OP_W4A16_GEMV, "gemv8": qz.QZ_OP_W8A16_GEMV, "gemm": qz.QZ_OP_W4A16_GEMM,
+          "gemm8": qz.QZ_OP_W8A16_GEMM, "gemv_nv": qz.QZ_OP_FP4A16_GEMV,
+          "gemv_mx": qz.QZ_OP_FP4A16_GEMV}.get(kind)
+    g = K if kind in ("gemv8", "gemm8") else GROUP
+    ws = torch.zeros(max(256, qz.qz_workspace_bytes(op, max(M, 1), N, K, g) if op is not None else 0),
+                     dtype=torch.uint8, device=dev)
     if kind in ("gemv4", "gemm", "dequant"):
         c, s, z = qz.qz_quantize_pack(w, 4, False, GROUP)
     if kind in ("gemv8", "gemm8"):

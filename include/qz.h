@@ -114,8 +114,9 @@ QZ_API qz_status qz_packed_bytes(int64_t N, int64_t K, int32_t bits, int32_t sym
 /*
  * Device workspace needed by `op` for the given sizes (0 when none).  The
  * workspace of QZ_OP_QUANTIZE_PACK (per-tensor only) and of the GEMV/GEMM
- * split-K paths must be zero-filled once before its first use; every call
- * leaves it zero-filled again when it completes.  Host-only.  The kernels
+ * paths that share tiles between CTAs must be zero-filled once before its
+ * first use; every call that completes leaves its counters (and the
+ * per-tensor word) at zero again, and the rest is scratch.  Host-only.  The kernels
  * size their grids for the device's SM count (a B200 has 148; a device with
  * more is treated as 148); the size returned here serves every SM count up
  * to 148, so it does not depend on the device.
@@ -185,14 +186,18 @@ QZ_API qz_status qz_w4a16_gemv(const void *a, const void *codes, const void *sca
  * (guide, "Quantize weights or activations": prefill and large batches are
  * compute-bound).  M <= 32 runs the decode kernel of qz_w4a16_gemv (faster there).  Each
  * output tile is 128 weight rows x up to 256 tokens, and the MMAs cover only
- * the tile's tokens (rounded up to 16).  When the tiles are fewer than the
- * SMs, the K range of each tile is split over up to 4 CTAs whose fp32
- * partials meet in the workspace and are added in a fixed order (results do
- * not depend on timing).  Requirements: M >= 1; N >= 1; K % 128 == 0;
+ * the tile's tokens (rounded up to 16).  Persistent CTAs take whole tiles
+ * round robin; when the last, partial wave (or all tiles, when they are fewer
+ * than the CTAs) would leave CTAs idle long enough, its tiles' K steps are
+ * shared evenly by the CTAs instead (stream-K), whose fp32 partials meet in
+ * the workspace and are added in K order (results do not depend on timing;
+ * they depend on the device's SM count through the schedule).
+ * Requirements: M >= 1; N >= 1; K % 128 == 0;
  * group_size a multiple of 64 dividing K (32 suffices for M <= 32).
  * Workspace: qz_workspace_bytes(QZ_OP_W4A16_GEMM, M, N, K, group_size)
- * bytes, zero-filled before first use, left zero-filled by each call that
- * completes.  A device-side wait that runs out (see qz_set_device_wait_limit)
+ * bytes (0 when no tile is shared), zero-filled before first use; each call
+ * that completes leaves its arrival counters at zero again (the partials
+ * are scratch), so the buffer serves the next call unchanged.  A device-side wait that runs out (see qz_set_device_wait_limit)
  * makes the kernel return early and the next qz_device_status call reports
  * QZ_ERR_DEVICE_TIMEOUT; the workspace of that call must then be zero-filled
  * again before reuse.
@@ -221,13 +226,14 @@ QZ_API qz_status qz_w8a16_gemv(const void *a, const void *codes, const void *sca
  * each matmul, and prefill is compute-bound).  Weight tiles are dequantized (w_hat = bf16_rne(S * q), exactly as
  * qz_dequantize forms it) into tensor memory as the A operand of tcgen05
  * BF16 MMAs with fp32 accumulation; y is rounded to bf16.  M <= 32 runs the
- * decode kernel of qz_w8a16_gemv.  Tiles and split-K as for qz_w4a16_gemm.
+ * decode kernel of qz_w8a16_gemv.  Tiles and their schedule as for
+ * qz_w4a16_gemm.
  * Arguments: a (M x K bf16, row-major), codes (N x K int8, row-major),
  * scales (N bf16), y (M x N bf16, row-major), all device pointers owned by
  * the caller; a, codes and y 16-byte aligned, scales 2-byte aligned.
  * Requirements: M >= 1; N >= 1; K % 128 == 0.  Workspace:
  * qz_workspace_bytes(QZ_OP_W8A16_GEMM, M, N, K, K) bytes, zero-filled before
- * first use, left zero-filled by each call that completes.  Errors: argument
+ * first use; each call that completes leaves its counters at zero again.  Errors: argument
  * errors return before any launch; QZ_ERR_CUDA if the launch fails; a
  * device-side wait that runs out makes the kernel return early, the next
  * qz_device_status call reports QZ_ERR_DEVICE_TIMEOUT, and the workspace of

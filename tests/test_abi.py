@@ -151,15 +151,105 @@ def test_w8a16_gemm_rejects(args, expect):
     assert L().qz_w8a16_gemm(*args) == expect
 
 
-def test_w8a16_gemm_workspace_follows_the_route():
-    assert qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMM, 2048, 8192, 8192, 8192) == 0
-    # 64 tiles, two CTAs per SM for 64-token tiles: four K splits, fp32
-    # partials [4][M][N] + counters
-    assert qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMM, 64, 8192, 8192, 8192) == \
-        4 * 64 * 8192 * 4 + 64 * 4
-    # 128-token tiles run one CTA per SM: two splits
-    assert qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMM, 128, 8192, 8192, 8192) == \
-        2 * 128 * 8192 * 4 + 64 * 4
+def gemm_schedule_model(M, N, K, sms):
+    """The prefill GEMM's schedule as the header of qz_gemm_sm100.cu states
+    it: whole 128 x 256 tiles round robin for the full waves, the K steps of
+    the last partial wave (all tiles when they are fewer than the CTAs) laid
+    end to end and cut into equal contiguous ranges, one per tail CTA (at
+    least 4 steps each, at most 6 CTAs per tail tile on average); no tail
+    when the waves are full or sharing would save a CTA fewer than 48 K
+    steps ((grid - tail tiles) * KT / grid).
+    Returns (act_rows, grid CTAs, tiles, tail tiles, tail CTAs, KT)."""
+    act_rows = 256 if M >= 256 else (M + 15) // 16 * 16
+    grid = sms * (2 if act_rows <= 64 else 1)
+    tiles = -(-N // 128) * -(-M // 256)
+    KT = K // 64
+    tail = tiles % grid if tiles >= grid else tiles
+    if (tiles >= grid and tail == 0) or (grid - tail) * KT < 48 * grid:
+        return act_rows, grid, tiles, 0, 0, KT
+    ctas = max(1, min(grid, 6 * tail, tail * KT // 4))
+    return act_rows, grid, tiles, tail, ctas, KT
+
+
+def gemm_workspace_model(M, N, K, sms):
+    """fp32 slots of act_rows x 128 placed 1 KB further apart than that,
+    then one counter per tail tile in blocks of 64."""
+    act_rows, _, _, tail, ctas, _ = gemm_schedule_model(M, N, K, sms)
+    if ctas == 0:
+        return 0
+    slots = ctas + tail - 1
+    return -(-(slots * (act_rows * 128 + 256) * 4) // 256) * 256 + -(-tail // 64) * 64 * 4
+
+
+def tail_segments(tail, KT, ctas):
+    """(cta, tail tile, kt0, kt1, slot) of every tail segment: CTA c takes
+    steps [floor(c S / P), floor((c + 1) S / P)), S = tail * KT, P = ctas."""
+    S = tail * KT
+    out = []
+    for c in range(ctas):
+        b0, b1 = c * S // ctas, (c + 1) * S // ctas
+        for t in range(b0 // KT, (b1 - 1) // KT + 1):
+            out.append((c, t, max(b0, t * KT) - t * KT, min(b1, (t + 1) * KT) - t * KT, c + t))
+    return out
+
+
+@pytest.mark.parametrize("M,N,K,sms", [
+    (2048, 8192, 8192, 148), (2048, 4096, 4096, 148), (2048, 11008, 4096, 148),
+    (2048, 4096, 11008, 148), (64, 8192, 8192, 148), (32, 1024, 4096, 148),
+    (300, 1000, 1024, 148), (17, 128, 128, 148), (2048, 8192, 8192, 97), (257, 130, 640, 5),
+])
+def test_gemm_tail_schedule_invariants(M, N, K, sms):
+    """Every K step of every tail tile is covered once; a tile's segments take
+    consecutive slots in K order (so the last arrival adds them in a fixed
+    order), no slot is used twice and every slot index is below tail CTAs +
+    tail tiles - 1 (the workspace's slot count), and no tail CTA's range is
+    shorter than 4 steps."""
+    _, _, _, tail, ctas, KT = gemm_schedule_model(M, N, K, sms)
+    if ctas == 0:
+        return
+    segs = tail_segments(tail, KT, ctas)
+    assert all(k1 - k0 >= 1 for _, _, k0, k1, _ in segs)
+    for t in range(tail):
+        mine = sorted((k0, k1, slot) for _, tt, k0, k1, slot in segs if tt == t)
+        assert mine[0][0] == 0 and mine[-1][1] == KT
+        assert all(a[1] == b[0] for a, b in zip(mine, mine[1:]))
+        assert [x[2] for x in mine] == list(range(mine[0][2], mine[0][2] + len(mine)))
+    slots = [x[4] for x in segs]
+    assert len(set(slots)) == len(slots) and max(slots) < ctas + tail - 1
+    S = tail * KT
+    assert ctas == 1 or min((c + 1) * S // ctas - c * S // ctas for c in range(ctas)) >= 4
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (2048, 8192, 8192), (2048, 4096, 4096), (2048, 11008, 4096), (2048, 28672, 8192),
+    (64, 8192, 8192), (128, 8192, 8192), (48, 1024, 2048), (200, 512, 2048), (33, 128, 128),
+    (4096, 4096, 4096), (300, 1000, 1024), (257, 130, 640), (16, 256, 192),
+])
+def test_gemm_workspace_matches_the_schedule(M, N, K):
+    """qz_workspace_bytes_for_sms of both GEMMs is the schedule's workspace
+    (fp32 slots of act_rows x 128, then one counter per tail tile) for every
+    SM count, and qz_workspace_bytes the largest of them."""
+    for op, g in ((qz.QZ_OP_W4A16_GEMM, 128 if K % 128 == 0 else 64), (qz.QZ_OP_W8A16_GEMM, K)):
+        want = [gemm_workspace_model(M, N, K, sms) for sms in range(1, 149)]
+        got = [qz.qz_workspace_bytes_for_sms(op, M, N, K, g, sms) for sms in range(1, 149)]
+        assert got == want
+        assert qz.qz_workspace_bytes(op, M, N, K, g) == max(want)
+
+
+def test_gemm_workspace_follows_the_route():
+    # 2048 x 8192 x 8192 on 148 SMs: 512 tiles, 3 whole waves and 68 tail
+    # tiles over 148 CTAs: 215 slots of 256 x 128 fp32 (+ 1 KB apart), 68
+    # counters (two blocks of 64)
+    assert qz.qz_workspace_bytes_for_sms(qz.QZ_OP_W8A16_GEMM, 2048, 8192, 8192, 8192, 148) == \
+        215 * (256 * 128 + 256) * 4 + 2 * 64 * 4
+    # 4096 tokens x 4096 rows: 512 tiles; on 128 SMs four whole waves, no workspace
+    assert qz.qz_workspace_bytes_for_sms(qz.QZ_OP_W4A16_GEMM, 4096, 4096, 4096, 128, 128) == 0
+    # 64 tokens: 64 tiles over 296 CTAs (two per SM): 359 slots of 64 x 128
+    assert qz.qz_workspace_bytes_for_sms(qz.QZ_OP_W8A16_GEMM, 64, 8192, 8192, 8192, 148) == \
+        359 * (64 * 128 + 256) * 4 + 64 * 4
+    # 2048 tokens x 4096 x 4096: 256 tiles, the 108-tile last wave would save
+    # a CTA only 17 K steps: whole tiles, no workspace
+    assert qz.qz_workspace_bytes_for_sms(qz.QZ_OP_W4A16_GEMM, 2048, 4096, 4096, 128, 148) == 0
     assert qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMM, 64, 8192, 8192, 128) == \
         qz.qz_workspace_bytes(qz.QZ_OP_W8A16_GEMM, 64, 8192, 8192, 8192)
     for M in (16, 32):      # up to 32 tokens the GEMM entry runs the decode GEMV

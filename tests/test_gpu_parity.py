@@ -462,11 +462,19 @@ def test_decode_70b_layers(dev, M, li, NK, bits):
 # Prefill GEMM (tcgen05)
 # ---------------------------------------------------------------------------
 
-GEMM_CASES = [  # (M, N, K, g); most have fewer tiles than SMs and run split-K
+GEMM_CASES = [  # (M, N, K, g); most have fewer tiles than CTAs, so CTAs share tiles' K steps
     (17, 128, 128, 128), (100, 200, 256, 64), (256, 128, 1024, 128),
     (300, 1000, 1024, 128), (512, 384, 2048, 256), (257, 130, 640, 128),
     (64, 256, 640, 640), (96, 192, 384, 192),      # groups of 10 and 3 stages
-    (32, 1024, 4096, 128), (200, 512, 2048, 128),  # 2 and 4 splits, partial token tiles
+    (32, 1024, 4096, 128), (200, 512, 2048, 128),  # partial token tiles over many CTAs
+    # on 148 SMs: 158 tiles, the last 10 (one token each) shared by 60 CTAs
+    # after a whole wave; 16 full-token tiles over 148 CTAs; N % 4 == 2
+    # (element-wise stores); 16 tiles of 64 K steps over 96 CTAs; 48 tokens
+    # (paired CTAs: 8 tiles over 296)
+    (257, 10112, 4096, 128), (512, 1024, 4096, 64), (257, 2050, 4096, 128), (300, 1000, 4096, 128),
+    (48, 1024, 4096, 128),
+    # one tile of 80 or 112 tokens shared by six CTAs
+    (80, 100, 8192, 128), (112, 100, 8192, 128),
 ]
 
 
@@ -483,11 +491,13 @@ def test_w4a16_gemm_tolerance(dev, M, N, K, g):
     check_tolerance(u16(y), y_ref, abs_ref, f"gemm M={M} N={N} K={K} g={g}")
 
 
-@pytest.mark.parametrize("bits", [4, 8])
-def test_gemm_split_k_repeats_and_leaves_workspace_zeroed(dev, bits):
-    """Split-K partials are added in split order: the same inputs give the
-    same bits on every call, and each call leaves the workspace zero-filled."""
-    M, N, K, g = 48, 1024, 2048, 128
+@pytest.mark.parametrize("bits,M,N,K", [(4, 48, 1024, 4096), (8, 48, 1024, 4096),
+                                         (4, 257, 10112, 4096), (8, 512, 1024, 4096)])
+def test_gemm_split_k_repeats_and_leaves_workspace_zeroed(dev, bits, M, N, K):
+    """Partials of shared tiles are added in K order: the same inputs give the
+    same bits on every call, and each call leaves the arrival counters at
+    zero (short token tiles over many CTAs; whole waves plus a shared tail)."""
+    g = 128
     assert qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMM, M, N, K, g) > 0
     w = synthetic.weights(N, K, sigma=0.02, seed=41, device=dev)
     a = synthetic.activations(M, K, seed=42, device=dev)
@@ -503,9 +513,13 @@ def test_gemm_split_k_repeats_and_leaves_workspace_zeroed(dev, bits):
     torch.cuda.synchronize()
     assert qz.qz_device_status() == 0
     assert all(torch.equal(ys[0], yi) for yi in ys[1:])
-    # the counters after the partials are back to zero
-    counters = ws[qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMM, M, N, K, g) - 64 * 4:]
-    assert int(counters.count_nonzero()) == 0
+    # the counters after the partials (one block of 64: at most 64 shared
+    # tiles here) are back to zero; the layout is the one for this device's
+    # SM count
+    sms = min(torch.cuda.get_device_properties(dev).multi_processor_count, 148)
+    used = qz.qz_workspace_bytes_for_sms(qz.QZ_OP_W4A16_GEMM, M, N, K, g, sms)
+    assert used > 0
+    assert int(ws[used - 64 * 4:used].count_nonzero()) == 0
 
 
 def test_w4a16_gemm_onehot_is_exact(dev):
@@ -544,7 +558,7 @@ def test_prefill_config_sampled(dev):
 
 W8_GEMM_CASES = [  # (M, N, K): ragged token and row tiles, N % 8 != 0 (direct stores)
     (17, 128, 128), (100, 200, 256), (256, 128, 1024), (300, 1000, 1024),
-    (257, 130, 640), (512, 384, 2048), (64, 36, 384),
+    (257, 130, 640), (512, 384, 2048), (64, 36, 384), (257, 10112, 4096),
 ]
 
 

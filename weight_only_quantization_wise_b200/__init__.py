@@ -156,8 +156,9 @@ def _handle(stream):
 class Workspace:
     """A zero-filled device workspace that grows on demand.
 
-    The library leaves split-K workspaces zero-filled after each call, so one
-    buffer serves every call issued on one stream.  Calls that may run
+    Each call leaves the counters in its workspace at zero again (the rest is
+    scratch that every call writes before it reads), so one buffer serves
+    every call issued on one stream.  Calls that may run
     concurrently need separate Workspace objects.
     """
 

@@ -11,8 +11,10 @@
 // group-wise scales and zeros) or w_hat = bf16_rne(S * q) (int8, symmetric,
 // one scale per weight row).
 //
-// Persistent kernel: each CTA loops over tiles of 128 weight rows x 256
-// tokens (tile t = blockIdx.x + i * gridDim.x).  The roles:
+// Persistent kernel: each CTA loops over work items, each a K range of one
+// tile of 128 weight rows x 256 tokens: whole tiles for the full waves, and
+// the K steps of the last, partial wave spread evenly over the CTAs, whose
+// fp32 partials meet in the workspace (GemmSched).  The roles:
 //   warp 0       TMA producer: per 64-wide K step, the activation tile
 //                (256 tokens x 64 bf16, 128-byte swizzle) and the codes
 //                (128 rows x 32 bytes of int4, or x 64 bytes of int8) into a
@@ -40,6 +42,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "qz_sm100.cuh"
@@ -62,7 +65,6 @@ constexpr int kACols = kTileK / 2;                       // A columns per stage 
 constexpr int kTmemCols = 512;
 constexpr int kDequantWarps = 8;
 constexpr int kMetaFifo = 2;              // groups of scales/zeros loaded ahead
-constexpr int kMaxSplits = 4;             // split-K ranges per tile at most
 constexpr int kMaxStages = 16;            // ring depth at most
 constexpr int kEpilogueWarps = 4;
 constexpr int kFirstEpilogueWarp = 2 + kDequantWarps;
@@ -82,7 +84,7 @@ struct GemmLayout {
     int stages;
     uint32_t act_stage, pack_stage;
     // byte offsets from the 1024-aligned base
-    uint32_t act, pack, staging, full, empty, afull, dfull, dempty, drain, tmem_slot,
+    uint32_t act, pack, staging, full, empty, afull, dfull, dempty, drain, fixbar, tmem_slot,
         abort_flag, epi_decision, epi_last, end;
     uint32_t a_col0;   // first tensor-memory column of the A slots (accumulator at 0)
 };
@@ -101,7 +103,8 @@ __host__ __device__ constexpr GemmLayout gemm_layout(int bits, int act_rows, int
     L.dfull = L.afull + 8 * stages;
     L.dempty = L.dfull + 8;
     L.drain = L.dempty + 8;
-    L.tmem_slot = L.drain + 8;
+    L.fixbar = L.drain + 8;
+    L.tmem_slot = L.fixbar + 8;
     L.abort_flag = L.tmem_slot + 4;
     L.epi_decision = L.abort_flag + 4;
     L.epi_last = L.epi_decision + 4;
@@ -155,6 +158,15 @@ __device__ __forceinline__ void tma_store_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
 __device__ __forceinline__ void epilogue_bar_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpilogueWarps) : "memory");
 }
@@ -170,19 +182,104 @@ __device__ __forceinline__ uint32_t dequant_pair_i8_nat(uint32_t wx, int i, uint
                            s2);
 }
 
-// Work item: one 128-row x 256-token output tile and, when the tiles are
-// fewer than the SMs, one of `splits` equal K ranges of it (split-K).
+// Work item: a K range [kt0, kt1) of one output tile (128 weight rows x up
+// to 256 tokens).  nseg == 1: the whole tile, written directly.  nseg > 1:
+// one of the nseg CTAs that share the tile; its fp32 partial goes to
+// workspace slot `slot`, the tile's slots are slot0 .. slot0 + nseg - 1 in K
+// order, and the last of them to arrive at counter `ctr` adds them.
 struct WorkItem {
-    int tile, split, n0, m0, kt0, kt1;
+    int n0, m0, kt0, kt1, nseg, slot, slot0, ctr;
 };
-__device__ __forceinline__ WorkItem work_item(int item, int splits, int tiles_n, int KT) {
+
+// Schedule of one launch (host-made, passed by value).  Tiles [0, dp_tiles)
+// are whole work items, tile c + i * grid on CTA c.  The K steps of tiles
+// [dp_tiles, tiles) -- the last, partial wave, or all tiles when they are
+// fewer than the CTAs -- are laid end to end, sk_steps = (tiles - dp_tiles)
+// * KT of them, and CTA c < sk_ctas takes steps [b_c, b_{c+1}) with b_c =
+// floor(c * sk_steps / sk_ctas) (at least kMinSegSteps each): every CTA then
+// carries the same work, up to one step.  A CTA's range cut at tile
+// boundaries gives its segments; segment (CTA c, tail tile t) takes slot
+// c + t, which grows with the segment's first step, so the slots are unique,
+// each tile's slots are consecutive, and all are below sk_ctas + tail tiles
+// - 1.
+// A CTA runs its whole tiles first and its segments last.  Every CTA ends
+// its range at about the same time, so the segment that ends a range
+// usually finds the tile's other segments done and adds them at once from
+// its own accumulator, after its main loop, when the CTA's whole ring and
+// staging memory are free to receive them; additions that overlapped other
+// CTAs' main loops (loads competing with the dequantizing warps') slowed
+// those to half speed.
+struct GemmSched {
+    int tiles_n;        // tiles along N
+    int KT;             // 64-wide K steps per tile
+    int tiles;
+    int dp_tiles;
+    int sk_ctas;
+    int64_t sk_steps;
+};
+
+#ifndef QZ_SLOT_SKEW
+#define QZ_SLOT_SKEW 1
+#endif
+#ifndef QZ_LAND_STAGE
+#define QZ_LAND_STAGE 1
+#endif
+// Partial slots are act_rows x 128 fp32 each, placed 1 KB further apart than
+// that, so that CTAs writing or reading the same offset of their slots at
+// the same time do not all meet in the same memory channels.
+constexpr int kSlotSkewFloats = QZ_SLOT_SKEW ? 256 : 0;
+__host__ __device__ constexpr int64_t slot_stride(int act_rows) {
+    return (int64_t)act_rows * kTileN + kSlotSkewFloats;
+}
+constexpr int kMaxSegsPerTile = 6;   // tail CTAs per tail tile, on average, at most
+constexpr int kMinSegSteps = 4;      // K steps of a tail CTA's range, at least
+// Sharing the last wave must save each CTA at least this many K steps: the
+// partial writes, the additions and the slower segments cost 15-25 us, about
+// 48 steps of a full tile (measured: 2048 x 8192 x 8192 gains 3%, 256 and 128
+// tokens over 8192 x 8192 gain 8-9%; savings of 17-35 steps lost 3-20%).
+constexpr int kMinGainSteps = 48;
+
+// The tail CTA whose range holds step p.
+__host__ __device__ __forceinline__ int sched_cta_of(const GemmSched &S, int64_t p) {
+    return (int)(((p + 1) * S.sk_ctas - 1) / S.sk_steps);
+}
+__host__ __device__ __forceinline__ int64_t sched_bound(const GemmSched &S, int c) {
+    return (int64_t)c * S.sk_steps / S.sk_ctas;
+}
+__host__ __device__ __forceinline__ int sched_segments(const GemmSched &S, int c) {
+    if (c >= S.sk_ctas) return 0;
+    const int64_t b0 = sched_bound(S, c), b1 = sched_bound(S, c + 1);
+    return (int)((b1 - 1) / S.KT - b0 / S.KT + 1);
+}
+__host__ __device__ __forceinline__ int sched_count(const GemmSched &S, int c, int grid) {
+    const int whole = c < S.dp_tiles ? (S.dp_tiles - 1 - c) / grid + 1 : 0;
+    return whole + sched_segments(S, c);
+}
+__host__ __device__ __forceinline__ WorkItem sched_item(const GemmSched &S, int c, int grid, int i) {
     WorkItem w;
-    w.tile = item / splits;
-    w.split = item - w.tile * splits;
-    w.n0 = (w.tile % tiles_n) * kTileN;
-    w.m0 = (w.tile / tiles_n) * kTileM;
-    w.kt0 = (int)((int64_t)w.split * KT / splits);
-    w.kt1 = (int)((int64_t)(w.split + 1) * KT / splits);
+    const int whole = c < S.dp_tiles ? (S.dp_tiles - 1 - c) / grid + 1 : 0;
+    int tile;
+    if (i >= whole) {
+        const int64_t b0 = sched_bound(S, c), b1 = sched_bound(S, c + 1);
+        const int t = (int)(b0 / S.KT) + (i - whole);       // tail tile
+        const int64_t t0 = (int64_t)t * S.KT;
+        w.kt0 = (int)((b0 > t0 ? b0 : t0) - t0);
+        w.kt1 = (int)((b1 < t0 + S.KT ? b1 : t0 + S.KT) - t0);
+        const int cf = sched_cta_of(S, t0), cl = sched_cta_of(S, t0 + S.KT - 1);
+        w.nseg = cl - cf + 1;
+        w.slot = c + t;
+        w.slot0 = cf + t;
+        w.ctr = t;
+        tile = S.dp_tiles + t;
+    } else {
+        tile = c + i * grid;
+        w.kt0 = 0;
+        w.kt1 = S.KT;
+        w.nseg = 1;
+        w.slot = w.slot0 = w.ctr = 0;
+    }
+    w.n0 = (tile % S.tiles_n) * kTileN;
+    w.m0 = (tile / S.tiles_n) * kTileM;
     return w;
 }
 
@@ -212,7 +309,7 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
                    const __grid_constant__ CUtensorMap y_map,
                    const uint16_t *__restrict__ scales, const uint8_t *__restrict__ zeros,
                    int M, int N, int K, int group_size, uint16_t *__restrict__ y,
-                   int use_tma_store, int act_rows, int stages_rt, int splits,
+                   int use_tma_store, int act_rows, int stages_rt, const GemmSched sched,
                    float *__restrict__ partials, uint32_t *__restrict__ counters,
                    uint64_t wait_limit) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -220,7 +317,6 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
     const int stages = FIXED_STAGES > 0 ? FIXED_STAGES : stages_rt;
-    if (FIXED_STAGES > 0) splits = 1;             // the host launches it only unsplit
     const GemmLayout SmemLayout = kernel_layout<BITS, FIXED_STAGES>(act_rows, stages_rt);
     constexpr int kPackBytes = kPackStageBytes<BITS>;
     const uint32_t kActStageBytes = SmemLayout.act_stage;
@@ -228,10 +324,7 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SmemLayout.tmem_slot);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int KT = K / kTileK;
-    const int tiles_n = (N + kTileN - 1) / kTileN;
-    const int tiles = tiles_n * ((M + kTileM - 1) / kTileM);
-    const int items = tiles * splits;
+    const int items = sched_count(sched, blockIdx.x, gridDim.x);
     const uint32_t act_bytes = kActStageBytes;                    // one activation box
 
     auto full_bar = [&](int s) { return sbase + SmemLayout.full + 8 * s; };
@@ -250,6 +343,7 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
         mbar_init(dfull_bar, 1);
         mbar_init(dempty_bar, kEpilogueWarps);
         mbar_init(drain_bar, 1);
+        mbar_init(sbase + SmemLayout.fixbar, 1);
         *abort_flag = 0u;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&act_map)) : "memory");
@@ -276,8 +370,8 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
             for (int s = 0; s < kMaxStages; ++s) issued_round[s] = -1;
             int s = 0, r = 0;                         // ring slot and its round
             bool ok = true;
-            for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
-                const WorkItem wk = work_item(item, splits, tiles_n, KT);
+            for (int item = 0; item < items && ok; ++item) {
+                const WorkItem wk = sched_item(sched, blockIdx.x, gridDim.x, item);
                 for (int kt = wk.kt0; kt < wk.kt1; ++kt, s = (s + 1 == stages ? 0 : s + 1),
                          r += (s == 0)) {
                     if (r > 0 && !gemm_wait(empty_bar(s), (r - 1) & 1, wait_limit, abort_flag)) {
@@ -302,8 +396,8 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
         if (lane == 0) {
             bool ok = true;
             int s = 0, r = 0, tcount = 0;
-            for (int item = blockIdx.x; item < items && ok; item += gridDim.x, ++tcount) {
-                const WorkItem wk = work_item(item, splits, tiles_n, KT);
+            for (int item = 0; item < items && ok; ++item, ++tcount) {
+                const WorkItem wk = sched_item(sched, blockIdx.x, gridDim.x, item);
                 const uint32_t idesc = idesc_bf16(kTileN, mma_n(M, wk.m0));
                 if (tcount > 0 && !gemm_wait(dempty_bar, (tcount - 1) & 1, wait_limit, abort_flag)) {
                     ok = false;
@@ -339,8 +433,8 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         int s = 0, r = 0;                             // ring slot and its round
         bool ok = true;
-        for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
-            const WorkItem wk = work_item(item, splits, tiles_n, KT);
+        for (int item = 0; item < items && ok; ++item) {
+            const WorkItem wk = sched_item(sched, blockIdx.x, gridDim.x, item);
             const int n = wk.n0 + row_local;
             // Rows beyond N: the codes are TMA fill (zero) and the scale is
             // taken as 0, so their A entries are +-0 and their outputs are
@@ -504,8 +598,9 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
             reinterpret_cast<volatile uint32_t *>(smem + SmemLayout.epi_decision);
         volatile uint32_t *epi_last = reinterpret_cast<volatile uint32_t *>(smem + SmemLayout.epi_last);
         int tcount = 0;
-        for (int item = blockIdx.x; item < items; item += gridDim.x, ++tcount) {
-            const WorkItem wk = work_item(item, splits, tiles_n, KT);
+        uint32_t fix_phase = 0;      // parity of the addition barrier's next phase
+        for (int item = 0; item < items; ++item, ++tcount) {
+            const WorkItem wk = sched_item(sched, blockIdx.x, gridDim.x, item);
             const int n0 = wk.n0, m0 = wk.m0;
             const int chunks = mma_n(M, m0) / 16;     // accumulator columns the MMAs wrote
             // One decision for the four epilogue warps (they meet at named
@@ -522,97 +617,192 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
             if (*epi_decision) break;
             tc_fence_after();
             const int n = n0 + row_local;
-            if (FIXED_STAGES == 0 && splits > 1) {
-                // split-K: this split's fp32 partial goes to partials[split][m][n]
-                float *part = partials + (int64_t)wk.split * M * N;
+            if (wk.nseg > 1) {
+                // A shared tile.  Its partials live in slots laid out [token -
+                // m0][row - n0] (act_rows x 128 fp32); the last of the nseg
+                // segments to arrive adds them in slot (K) order.
+                // (paired CTAs, with short token tiles and few registers, add
+                // from memory)
+                const bool final_item = CTAS == 1 && item + 1 == items;
+                bool own_tmem = false;        // the sum takes this segment from tensor memory
+                if (final_item) {
+                    // if every other segment has arrived, add straight from
+                    // the accumulator without writing this one out
+                    if (storer)
+                        *epi_last = *reinterpret_cast<volatile uint32_t *>(&counters[wk.ctr]) ==
+                                    (uint32_t)(wk.nseg - 1);
+                    epilogue_bar_sync();
+                    own_tmem = *epi_last;
+                }
+                if (!own_tmem) {
+                    float *part = partials + wk.slot * slot_stride(act_rows);
 #pragma unroll 1
-                for (int c = 0; c < chunks; ++c) {
-                    uint32_t v[16];
-                    tmem_ld_x16(tmem_acc + lane_base + c * 16, v);
-                    if (n < N) {
+                    for (int c = 0; c < chunks; ++c) {
+                        uint32_t v[16];
+                        tmem_ld_x16(tmem_acc + lane_base + c * 16, v);
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int m = m0 + c * 16 + j;
-                            if (m < M) part[(int64_t)m * N + n] = __uint_as_float(v[j]);
-                        }
+                        for (int j = 0; j < 16; ++j)
+                            __stcg(&part[(c * 16 + j) * kTileN + row_local], __uint_as_float(v[j]));
                     }
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(dempty_bar);
-                __threadfence();
-                epilogue_bar_sync();
-                if (storer) *epi_last = atomicAdd(&counters[wk.tile], 1u) == (uint32_t)(splits - 1);
-                epilogue_bar_sync();
-                if (*epi_last) {
-                    // The last split of the tile adds the partials in split
-                    // order.  With N % 4 == 0 thread t takes rows n0 + 4(t%32)
-                    // .. +3 (float4) and tokens m0 + t/32, +4, ...; otherwise
-                    // one row per thread.
                     __threadfence();
-                    const int m_end = M < m0 + kTileM ? M : m0 + kTileM;
-                    const int t = (int)threadIdx.x - 32 * kFirstEpilogueWarp;
-                    if ((N & 3) == 0) {
-                        const int nq = n0 + 4 * (t & 31);
-                        if (nq < N) {
-                            for (int mb = m0 + (t >> 5); mb < m_end; mb += 16) {
-                                float4 acc[4];
-#pragma unroll
-                                for (int j = 0; j < 4; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 2
-                                for (int sp = 0; sp < splits; ++sp) {
-                                    float4 v[4];
-#pragma unroll
-                                    for (int j = 0; j < 4; ++j) {
-                                        const int m = mb + 4 * j;
-                                        v[j] = m < m_end ? __ldcg(reinterpret_cast<const float4 *>(
-                                                               &partials[((int64_t)sp * M + m) * N + nq]))
-                                                         : make_float4(0.f, 0.f, 0.f, 0.f);
-                                    }
-#pragma unroll
-                                    for (int j = 0; j < 4; ++j) {
-                                        acc[j].x += v[j].x;
-                                        acc[j].y += v[j].y;
-                                        acc[j].z += v[j].z;
-                                        acc[j].w += v[j].w;
-                                    }
-                                }
-#pragma unroll
-                                for (int j = 0; j < 4; ++j) {
-                                    const int m = mb + 4 * j;
-                                    if (m < m_end) {
-                                        uint2 o;
-                                        o.x = dev::f32_to_bf16_rne(acc[j].x) | (dev::f32_to_bf16_rne(acc[j].y) << 16);
-                                        o.y = dev::f32_to_bf16_rne(acc[j].z) | (dev::f32_to_bf16_rne(acc[j].w) << 16);
-                                        *reinterpret_cast<uint2 *>(&y[(int64_t)m * N + nq]) = o;
-                                    }
-                                }
+                    epilogue_bar_sync();
+                    if (storer)
+                        *epi_last = atomicAdd(&counters[wk.ctr], 1u) == (uint32_t)(wk.nseg - 1);
+                    epilogue_bar_sync();
+                    const bool last = *epi_last;
+                    own_tmem = last && final_item;
+                    if (!own_tmem) {
+                        // the accumulator is free for the next item's MMAs
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(dempty_bar);
+                    }
+                    if (!last) continue;
+                }
+                __threadfence();
+                const int mt = (M < m0 + kTileM ? M : m0 + kTileM) - m0;
+                const int nread = wk.nseg - (own_tmem ? 1 : 0);
+                // tokens per round when the other slots land in the ring and
+                // staging memory (free: this CTA's main loop is over)
+                const bool stage_y = QZ_LAND_STAGE && use_tma_store;
+                const uint32_t land_bytes = stage_y ? SmemLayout.staging : SmemLayout.full;
+                const int tr = own_tmem ? (int)(land_bytes / ((uint32_t)nread * kTileN * 4)) & ~15 : 0;
+                if (CTAS == 1 && own_tmem && tr >= 16) {
+                    const int own_sg = wk.slot - wk.slot0;
+                    const float *land = reinterpret_cast<const float *>(smem);
+                    const uint32_t bar = sbase + SmemLayout.fixbar;
+                    const int toks = chunks * 16;
+                    for (int r0 = 0; r0 < toks; r0 += tr) {
+                        const int rt = toks - r0 < tr ? toks - r0 : tr;
+                        if (storer) {
+                            // the slots were written through the generic proxy;
+                            // the landing zone was last used by it as well
+                            asm volatile("fence.proxy.async;" ::: "memory");
+                            mbar_arrive_expect_tx(bar, (uint32_t)(nread * rt * kTileN * 4));
+                            for (int sg = 0, k = 0; sg < wk.nseg; ++sg) {
+                                if (sg == own_sg) continue;
+                                bulk_load(sbase + (uint32_t)(k++ * tr * kTileN * 4),
+                                          partials + (wk.slot0 + sg) * slot_stride(act_rows) + r0 * kTileN,
+                                          (uint32_t)(rt * kTileN * 4), bar);
                             }
                         }
-                    } else if (n < N) {
-                        for (int mb = m0; mb < m_end; mb += 8) {
-                            float acc[8];
+                        gemm_wait(bar, fix_phase & 1u, wait_limit, abort_flag);
+                        fix_phase ^= 1u;
+#pragma unroll 1
+                        for (int c = r0 / 16; c < (r0 + rt) / 16; ++c) {
+                            uint32_t own[16];
+                            tmem_ld_x16(tmem_acc + lane_base + c * 16, own);
+                            // 16 tokens of this thread's row, the slots added in
+                            // order, each slot's 16 values loaded together
+                            const float *lc = land + (c * 16 - r0) * kTileN + row_local;
+                            float acc[16];
+#pragma unroll 1
+                            for (int sg = 0, k = 0; sg < wk.nseg; ++sg) {
+                                float v[16];
+                                if (sg == own_sg) {
 #pragma unroll
-                            for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
-#pragma unroll 2
-                            for (int sp = 0; sp < splits; ++sp) {
-                                float v[8];
+                                    for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(own[j]);
+                                } else {
+                                    const float *lk = lc + k++ * tr * kTileN;
 #pragma unroll
-                                for (int j = 0; j < 8; ++j)
-                                    v[j] = mb + j < m_end
-                                               ? __ldcg(&partials[((int64_t)sp * M + mb + j) * N + n])
-                                               : 0.0f;
+                                    for (int j = 0; j < 16; ++j) v[j] = lk[j * kTileN];
+                                }
 #pragma unroll
-                                for (int j = 0; j < 8; ++j) acc[j] += v[j];
+                                for (int j = 0; j < 16; ++j) acc[j] = sg == 0 ? v[j] : acc[j] + v[j];
                             }
 #pragma unroll
-                            for (int j = 0; j < 8; ++j)
-                                if (mb + j < m_end)
-                                    y[(int64_t)(mb + j) * N + n] = (uint16_t)dev::f32_to_bf16_rne(acc[j]);
+                            for (int j = 0; j < 16; ++j) {
+                                if (stage_y)
+                                    staging[(c * 16 + j) * kTileN + row_local] =
+                                        (uint16_t)dev::f32_to_bf16_rne(acc[j]);
+                                else if (n < N && c * 16 + j < mt)
+                                    y[(int64_t)(m0 + c * 16 + j) * N + n] =
+                                        (uint16_t)dev::f32_to_bf16_rne(acc[j]);
+                            }
+                        }
+                        // every thread is done with this round's landing zone
+                        epilogue_bar_sync();
+                    }
+                    // after an abort the copies may still be on their way
+                    if (storer && *abort_flag) gemm_drain(bar, (fix_phase & 1u) ^ 1u);
+                    if (stage_y) {
+                        // one store of the whole tile, as for an unshared one
+                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                        epilogue_bar_sync();
+                        if (storer) tma_store_2d(&y_map, sbase + SmemLayout.staging, n0, m0);
+                    }
+                } else {
+                    // From memory (the rare shared tile whose last segment is
+                    // not this CTA's last item, or slots too large to land):
+                    // thread t adds rows n0 + 4(t%32) .. +3 (float4) of tokens
+                    // m0 + t/32, +4, +8, ..., this segment's slot included.
+                    if (own_tmem) {
+                        // this segment's slot was written unless the check found
+                        // every other segment done: write it now
+                        float *part = partials + wk.slot * slot_stride(act_rows);
+#pragma unroll 1
+                        for (int c = 0; c < chunks; ++c) {
+                            uint32_t v[16];
+                            tmem_ld_x16(tmem_acc + lane_base + c * 16, v);
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                __stcg(&part[(c * 16 + j) * kTileN + row_local], __uint_as_float(v[j]));
+                        }
+                        __threadfence();
+                        epilogue_bar_sync();
+                    }
+                    const int t = (int)threadIdx.x - 32 * kFirstEpilogueWarp;
+                    const int nl = 4 * (t & 31), nq = n0 + nl;
+                    const float *base = partials + wk.slot0 * slot_stride(act_rows) + nl;
+                    const int64_t slot_floats = slot_stride(act_rows);
+                    for (int mb = t >> 5; mb < mt; mb += 16) {
+                        float4 acc[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+                        for (int sg = 0; sg < wk.nseg; ++sg) {
+                            float4 v[4];
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                v[j] = mb + 4 * j < mt
+                                           ? __ldcg(reinterpret_cast<const float4 *>(
+                                                 base + sg * slot_floats + (mb + 4 * j) * kTileN))
+                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                acc[j].x += v[j].x;
+                                acc[j].y += v[j].y;
+                                acc[j].z += v[j].z;
+                                acc[j].w += v[j].w;
+                            }
+                        }
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int m = m0 + mb + 4 * j;
+                            if (mb + 4 * j >= mt) continue;
+                            uint16_t *yr = y + (int64_t)m * N;
+                            if ((N & 3) == 0) {
+                                if (nq < N) {
+                                    uint2 o;
+                                    o.x = dev::f32_to_bf16_rne(acc[j].x) | (dev::f32_to_bf16_rne(acc[j].y) << 16);
+                                    o.y = dev::f32_to_bf16_rne(acc[j].z) | (dev::f32_to_bf16_rne(acc[j].w) << 16);
+                                    *reinterpret_cast<uint2 *>(yr + nq) = o;
+                                }
+                            } else {
+                                const float e[4] = {acc[j].x, acc[j].y, acc[j].z, acc[j].w};
+#pragma unroll
+                                for (int q = 0; q < 4; ++q)
+                                    if (nq + q < N) yr[nq + q] = (uint16_t)dev::f32_to_bf16_rne(e[q]);
+                            }
                         }
                     }
-                    if (storer) counters[wk.tile] = 0u;
                 }
+                if (own_tmem) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(dempty_bar);
+                }
+                if (storer) counters[wk.ctr] = 0u;
                 continue;
             }
 #pragma unroll 1
@@ -659,40 +849,68 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
 
 }  // namespace
 
-// Split-K: when the 128 x 256 output tiles are fewer than the SMs, each
-// tile's K range is divided among up to kMaxSplits CTAs (at least 4 stages
-// each); their fp32 partials meet in the workspace.
 // Tokens per activation box: a whole tile, or all of M rounded up to 16.
 int gemm_act_rows(int64_t M) { return M >= kTileM ? kTileM : (int)((M + 15) & ~int64_t(15)); }
 
-// `sms`: the SMs the grid is sized for (fewer SMs give fewer or equal splits,
-// so a workspace sized for kSmCount serves every device).
-int gemm_splits(int64_t M, int64_t N, int64_t K, int sms) {
-    const int64_t tiles = ceil_div(N, kTileN) * ceil_div(M, kTileM);
-    const int64_t slots = (int64_t)sms * gemm_ctas_per_sm(gemm_act_rows(M));
-    if (tiles >= slots) return 1;
-    int64_t s = slots / tiles;
-    if (s > kMaxSplits) s = kMaxSplits;
-    if (s > K / kTileK / 4) s = K / kTileK / 4;
-    return s < 1 ? 1 : (int)s;
+namespace {
+
+// The schedule for a grid of `sms` SMs (see GemmSched).  The tiles of the
+// last partial wave (all tiles, when they are fewer than the CTAs) share
+// their K steps evenly over up to every CTA, at least kMinSegSteps steps
+// each and at most kMaxSegsPerTile CTAs per tile on average, when that
+// shortens each CTA's work by at least kMinGainSteps K steps ((grid - tail
+// tiles) * KT / grid); otherwise every tile is a whole work item.
+GemmSched gemm_schedule(int64_t M, int64_t N, int64_t K, int sms) {
+    GemmSched S{};
+    S.tiles_n = (int)ceil_div(N, kTileN);
+    S.KT = (int)(K / kTileK);
+    S.tiles = S.tiles_n * (int)ceil_div(M, kTileM);
+    const int grid = sms * gemm_ctas_per_sm(gemm_act_rows(M));
+    const int tail = S.tiles >= grid ? S.tiles % grid : S.tiles;
+    if ((S.tiles >= grid && tail == 0) ||
+        (int64_t)(grid - tail) * S.KT < (int64_t)kMinGainSteps * grid) {
+        S.dp_tiles = S.tiles;
+        return S;
+    }
+    S.dp_tiles = S.tiles - tail;
+    S.sk_steps = (int64_t)tail * S.KT;
+    int64_t p = std::min<int64_t>({(int64_t)grid, (int64_t)kMaxSegsPerTile * tail,
+                                   S.sk_steps / kMinSegSteps});
+    S.sk_ctas = (int)std::max<int64_t>(p, 1);
+    return S;
 }
 
-// fp32 partials [splits][M][N], then one uint32 arrival counter per tile
-size_t gemm_partial_bytes(int64_t M, int64_t N, int64_t K, int sms) {
-    const int s = gemm_splits(M, N, K, sms);
-    if (s == 1) return 0;
-    return (((size_t)s * M * N * sizeof(float)) + 255) & ~(size_t)255;
+// CTAs to launch: every slot when the tiles fill a wave; otherwise one per
+// tile, or one per tail range when the tiles' K steps are shared.
+int gemm_grid(const GemmSched &S, int sms, int ctas) {
+    const int grid = sms * ctas;
+    if (S.tiles >= grid) return grid;
+    return S.sk_ctas > 0 ? S.sk_ctas : S.tiles;
 }
+
+// Workspace of a schedule: fp32 partial slots (sk_ctas + tail tiles - 1 of
+// act_rows x 128), then one uint32 arrival counter per tail tile.
+size_t sched_partial_bytes(const GemmSched &S, int64_t M) {
+    const int64_t slots = S.sk_ctas + (S.tiles - S.dp_tiles) - 1;
+    return ((size_t)slots * slot_stride(gemm_act_rows(M)) * sizeof(float) + 255) & ~(size_t)255;
+}
+
+}  // namespace
 
 size_t gemm_workspace_bytes_for(int64_t M, int64_t N, int64_t K, int sms) {
-    if (gemm_splits(M, N, K, sms) == 1) return 0;
-    const int64_t tiles = ceil_div(N, kTileN) * ceil_div(M, kTileM);
-    return gemm_partial_bytes(M, N, K, sms) +
-           (size_t)ceil_div(tiles, 64) * 64 * sizeof(uint32_t);
+    const GemmSched S = gemm_schedule(M, N, K, sms);
+    if (S.sk_ctas == 0) return 0;
+    return sched_partial_bytes(S, M) +
+           (size_t)ceil_div(S.tiles - S.dp_tiles, 64) * 64 * sizeof(uint32_t);
 }
 
+// The largest workspace over every SM count up to kSmCount (the schedule
+// depends on the grid in no monotone way).
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-    return gemm_workspace_bytes_for(M, N, K, kSmCount);
+    size_t most = 0;
+    for (int sms = 1; sms <= kSmCount; ++sms)
+        most = std::max(most, gemm_workspace_bytes_for(M, N, K, sms));
+    return most;
 }
 
 unsigned int *device_error_word() {
@@ -719,13 +937,13 @@ qz_status launch_gemm(const void *a, const void *codes, const void *scales, cons
     const int act_rows = gemm_act_rows(M);
     const int ctas = gemm_ctas_per_sm(act_rows);
     const int sms = device_sm_count();
-    const int splits = gemm_splits(M, N, K, sms);
+    const GemmSched sched = gemm_schedule(M, N, K, sms);
     float *partials = nullptr;
     uint32_t *counters = nullptr;
-    if (splits > 1) {
+    if (sched.sk_ctas > 0) {
         partials = static_cast<float *>(workspace);
         counters = reinterpret_cast<uint32_t *>(static_cast<char *>(workspace) +
-                                                gemm_partial_bytes(M, N, K, sms));
+                                                sched_partial_bytes(sched, M));
     }
     CUtensorMap act_map, pack_map, y_map;
     if (!make_map_2d(&act_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a, (uint64_t)K, (uint64_t)M,
@@ -769,15 +987,14 @@ qz_status launch_gemm(const void *a, const void *codes, const void *scales, cons
     if (attr_err != cudaSuccess) return QZ_ERR_CUDA;
     const int stages = gemm_stages(BITS, act_rows, ctas);
     const uint32_t smem_bytes = gemm_layout(BITS, act_rows, stages).end + 1024;
-    const int64_t items = ceil_div(N, kTileN) * ceil_div(M, kTileM) * splits;
-    const int grid = (int)std::min<int64_t>(items, (int64_t)sms * ctas);
-    auto kernel = act_rows == kTileM && splits == 1 ? wa16_gemm_tcgen05<BITS, kFullTileStages, 1>
+    const int grid = gemm_grid(sched, sms, ctas);
+    auto kernel = act_rows == kTileM ? wa16_gemm_tcgen05<BITS, kFullTileStages, 1>
                   : ctas == 2                      ? wa16_gemm_tcgen05<BITS, 0, 2>
                                                    : wa16_gemm_tcgen05<BITS, 0, 1>;
     kernel<<<grid, kThreads, smem_bytes, st>>>(
         act_map, pack_map, y_map, static_cast<const uint16_t *>(scales),
         static_cast<const uint8_t *>(zeros), (int)M, (int)N, (int)K, (int)group_size,
-        static_cast<uint16_t *>(y), use_tma_store, act_rows, stages, splits, partials, counters,
+        static_cast<uint16_t *>(y), use_tma_store, act_rows, stages, sched, partials, counters,
         device_wait_limit());
     return launch_status();
 }

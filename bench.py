@@ -377,6 +377,60 @@ def qz_gemm_kernel_for(M):
 GEMM_ROUTES_TO_GEMV_UP_TO = 32
 
 
+def read_floor(ls, stream, pk, parts):
+    """The floor of the decode GEMV parts: a plain streaming read (torch.sum,
+    a library reduction, over the same packed codes, scales and zeros as fp32
+    words) of
+    each step's layers, in the same harness as the step (one CUDA graph per
+    rotation of the same resident copies, replayed back to back, timed with
+    events).  For the short 7B layers it is a latency floor, not HBM."""
+    sink = torch.zeros(16, dtype=torch.float32, device=ls.dev)
+
+    def reads(tensors):
+        def f(p):
+            for i, t in enumerate(tensors(p)):
+                # the bytes as fp32 words (the sum's value is irrelevant):
+                # torch's fastest reduction, no conversion pass
+                v = t.reshape(-1).view(torch.float32)
+                sink[i % 16] += torch.sum(v)
+        return f
+
+    sets = {
+        "w4a16_gemv_m1": (reads(lambda p: [x for li in range(len(LAYERS))
+                                           for x in (ls.c4[p][li], ls.s4[p][li], ls.z4[p][li])]),
+                          sum(w4_gemv_bytes(1, N, K) for N, K in LAYERS)),
+        "w4a16_gemv_70b_m1": (reads(lambda p: [x for li in range(len(LAYERS_70B))
+                                               for x in (ls.c4_70[li][p], ls.s4_70[li][p],
+                                                         ls.z4_70[li][p])]),
+                              sum(w4_gemv_bytes(1, N, K) for N, K in LAYERS_70B)),
+    }
+    out = {"method": "torch.sum over the packed codes, scales and zeros of each layer, viewed "
+                     "as fp32 words; one graph per rotation, 40 replays"}
+    with torch.cuda.stream(stream):
+        for name, (f, nbytes) in sets.items():
+            graphs = []
+            for p in range(ROT):
+                f(p)
+                graphs.append(capture(lambda p=p: f(p), stream))
+            for g in graphs[:3]:
+                g.replay()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for i in range(40):
+                graphs[i % ROT].replay()
+            e1.record(stream)
+            e1.synchronize()
+            us = e0.elapsed_time(e1) / 40 * 1e3
+            part_us = parts[name]["ms"] * 1e3
+            out[name] = {"floor_us": round(us, 2), "floor_GB/s": round(nbytes / us / 1e3, 1),
+                         "floor_frac_hbm": round(nbytes / us / 1e3 / pk["hbm_gbs"], 4),
+                         "gemv_us": round(part_us, 2), "gemv_over_floor": round(part_us / us, 3)}
+            del graphs
+    torch.cuda.synchronize()
+    return out
+
+
 def run_extras(qz, dev, pk, stream):
     """Configurations outside the step, each timed with CUDA events on graphs."""
     out = {}
@@ -1053,6 +1107,7 @@ def main():
         del warm, timed                      # the graphs first, then their events
         del warm_ev, ev
         extras = run_extras(qz, dev, pk, stream)
+        extras["decode_read_floor"] = read_floor(ls, stream, pk, parts)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline()

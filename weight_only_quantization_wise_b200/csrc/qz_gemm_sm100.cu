@@ -131,6 +131,7 @@ static_assert(gemm_stages(4, kTileM) == kFullTileStages && gemm_stages(8, kTileM
               "a full token tile keeps four stages");
 static_assert(gemm_stages(4, 16) == kMaxStages - 1 || gemm_stages(4, 16) == kMaxStages,
               "short token tiles get a deep ring");
+static_assert(kTileK == 64, "the MMA issuer writes out the four 16-wide K steps of a stage");
 
 // Bounded waits that report through this file's device error word.
 __device__ __forceinline__ bool gemm_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns,
@@ -404,18 +405,25 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
                     break;
                 }
                 tc_fence_after();
+                // This one thread's instruction stream is the pace of the
+                // whole pipeline (its barriers are found ready): one probe of
+                // both barriers before the bounded waits, one shared-memory
+                // descriptor per stage advanced by 32 bytes (2 in its
+                // 16-byte address field) per 16-wide K step.
                 for (int kt = wk.kt0; kt < wk.kt1;
                      ++kt, s = (s + 1 == stages ? 0 : s + 1), r += (s == 0)) {
-                    ok = gemm_wait(full_bar(s), r & 1, wait_limit, abort_flag) &&
-                         gemm_wait(afull_bar(s), r & 1, wait_limit, abort_flag);
-                    if (!ok) break;
+                    if (!(mbar_try_wait(full_bar(s), r & 1) && mbar_try_wait(afull_bar(s), r & 1))) {
+                        ok = gemm_wait(full_bar(s), r & 1, wait_limit, abort_flag) &&
+                             gemm_wait(afull_bar(s), r & 1, wait_limit, abort_flag);
+                        if (!ok) break;
+                    }
                     tc_fence_after();
-                    const uint32_t act_addr = sbase + SmemLayout.act + s * kActStageBytes;
-#pragma unroll
-                    for (int j = 0; j < kTileK / 16; ++j)
-                        mma_ts(tmem_acc, tmem_a + s * kACols + j * 8,
-                               smem_desc_sw128(act_addr + j * 32), idesc,
-                               (kt > wk.kt0 || j > 0) ? 1u : 0u);
+                    const uint64_t bdesc = smem_desc_sw128(sbase + SmemLayout.act + s * kActStageBytes);
+                    const uint32_t acol = tmem_a + s * kACols;
+                    mma_ts(tmem_acc, acol, bdesc, idesc, kt > wk.kt0 ? 1u : 0u);
+                    mma_ts(tmem_acc, acol + 8, bdesc + 2, idesc, 1u);
+                    mma_ts(tmem_acc, acol + 16, bdesc + 4, idesc, 1u);
+                    mma_ts(tmem_acc, acol + 24, bdesc + 6, idesc, 1u);
                     mma_commit(empty_bar(s));
                 }
                 if (ok) mma_commit(dfull_bar);

@@ -378,34 +378,54 @@ GEMM_ROUTES_TO_GEMV_UP_TO = 32
 
 
 def read_floor(ls, stream, pk, parts):
-    """The floor of the decode GEMV parts: a plain streaming read (torch.sum,
-    a library reduction, over the same packed codes, scales and zeros as fp32
-    words) of
+    """The floor of the decode GEMV parts: a plain streaming read (cuBLAS
+    matrix-vector products over the same packed codes, scales and zeros as
+    fp32 words) of
     each step's layers, in the same harness as the step (one CUDA graph per
     rotation of the same resident copies, replayed back to back, timed with
     events).  For the short 7B layers it is a latency floor, not HBM."""
-    sink = torch.zeros(16, dtype=torch.float32, device=ls.dev)
+    ones = torch.ones(1 << 15, dtype=torch.float32, device=ls.dev)
+    sinks = {}
+
+    def as_matrix(t):
+        # each weight row's bytes as fp32 words (codes: N x K/8); a row whose
+        # bytes are not a multiple of 4 reads the tensor as a flat matrix
+        if t.dim() == 2 and t.shape[1] * t.element_size() % 4 == 0:
+            return t.view(torch.float32)
+        v = t.reshape(-1).view(torch.float32)
+        return v.view(-1, 16 if v.numel() % 16 == 0 else 1)
 
     def reads(tensors):
         def f(p):
             for i, t in enumerate(tensors(p)):
-                # the bytes as fp32 words (the sum's value is irrelevant):
-                # torch's fastest reduction, no conversion pass
-                v = t.reshape(-1).view(torch.float32)
-                sink[i % 16] += torch.sum(v)
+                # the matrix times a ones vector (the values are irrelevant):
+                # cuBLAS's matrix-vector product reads each byte once and
+                # writes one word per row
+                m = as_matrix(t)
+                out = sinks.setdefault((i, m.shape[0]), torch.empty(m.shape[0], dtype=torch.float32,
+                                                                    device=ls.dev))
+                torch.mv(m, ones[:m.shape[1]], out=out)
         return f
 
+    # every byte the GEMV reads (three reads per layer), and the codes alone
+    # (one read per layer, as the GEMV launches once per layer)
     sets = {
         "w4a16_gemv_m1": (reads(lambda p: [x for li in range(len(LAYERS))
                                            for x in (ls.c4[p][li], ls.s4[p][li], ls.z4[p][li])]),
                           sum(w4_gemv_bytes(1, N, K) for N, K in LAYERS)),
+        "w4a16_gemv_m1/codes_only": (reads(lambda p: [ls.c4[p][li] for li in range(len(LAYERS))]),
+                                     sum(N * K // 2 for N, K in LAYERS)),
         "w4a16_gemv_70b_m1": (reads(lambda p: [x for li in range(len(LAYERS_70B))
                                                for x in (ls.c4_70[li][p], ls.s4_70[li][p],
                                                          ls.z4_70[li][p])]),
                               sum(w4_gemv_bytes(1, N, K) for N, K in LAYERS_70B)),
+        "w4a16_gemv_70b_m1/codes_only": (reads(lambda p: [ls.c4_70[li][p]
+                                                          for li in range(len(LAYERS_70B))]),
+                                         sum(N * K // 2 for N, K in LAYERS_70B)),
     }
-    out = {"method": "torch.sum over the packed codes, scales and zeros of each layer, viewed "
-                     "as fp32 words; one graph per rotation, 40 replays"}
+    out = {"method": "cuBLAS matrix-vector product (torch.mv) of the packed codes (N x K/8 fp32 "
+                     "words), scales and zeros of each layer with a ones vector; one graph per "
+                     "rotation, 40 replays"}
     with torch.cuda.stream(stream):
         for name, (f, nbytes) in sets.items():
             graphs = []
@@ -422,7 +442,7 @@ def read_floor(ls, stream, pk, parts):
             e1.record(stream)
             e1.synchronize()
             us = e0.elapsed_time(e1) / 40 * 1e3
-            part_us = parts[name]["ms"] * 1e3
+            part_us = parts[name.split("/")[0]]["ms"] * 1e3
             out[name] = {"floor_us": round(us, 2), "floor_GB/s": round(nbytes / us / 1e3, 1),
                          "floor_frac_hbm": round(nbytes / us / 1e3 / pk["hbm_gbs"], 4),
                          "gemv_us": round(part_us, 2), "gemv_over_floor": round(part_us / us, 3)}

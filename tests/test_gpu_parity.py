@@ -339,6 +339,32 @@ def test_gemv_workspace_is_left_zeroed_and_results_repeat(dev):
     assert int(ws[plan_partials:].count_nonzero()) == 0
 
 
+@pytest.mark.parametrize("overlap", [0, 1])
+def test_gemv_large_layer_results_repeat_back_to_back(dev, overlap):
+    """Decode GEMVs on a 70B-sized layer (28672 x 8192, int4 g128), M = 1
+    and M = 8, launched back to back into separate outputs: the split-K sums
+    are added in a fixed order, so every launch must give the same bits.  A
+    consumer that released a ring stage before its shared-memory loads had
+    returned would let the refill corrupt scattered tasks, differently on
+    every launch."""
+    N, K, g = 28672, 8192, 128
+    w = synthetic.weights(N, K, sigma=0.015, seed=4, device=dev)
+    c, s, z = qz.qz_quantize_pack(w, 4, False, g)
+    qz.qz_set_launch_overlap(overlap)
+    try:
+        for M in (1, 8):
+            a = synthetic.activations(M, K, seed=M, device=dev)
+            nbytes = qz.qz_workspace_bytes(qz.QZ_OP_W4A16_GEMV, M, N, K, g)
+            ws = torch.zeros(max(nbytes, 1), dtype=torch.uint8, device=dev)
+            ys = [qz.qz_w4a16_gemv(a, c, s, z, N, K, g, workspace=ws) for _ in range(6)]
+            torch.cuda.synchronize()
+            for y in ys[1:]:
+                assert torch.equal(y.view(torch.int16), ys[0].view(torch.int16)), M
+    finally:
+        qz.qz_set_launch_overlap(0)              # the library's default
+    assert qz.qz_device_status() == 0
+
+
 def test_explicit_side_stream_with_temporary_workspaces(dev):
     """Calls given an explicit side stream and no workspace: the binding
     allocates and zero-fills each temporary workspace, and the output, on

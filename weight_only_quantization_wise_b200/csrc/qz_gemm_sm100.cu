@@ -464,8 +464,6 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
                     const uint4 p = *reinterpret_cast<const uint4 *>(
                         smem + SmemLayout.pack + s * kPackBytes + row_local * (kTileK / 2) +
                         khalf * 16);
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(empty_bar(s));   // code stage consumed
                     const uint32_t s2 = sb * 0x00010001u;
                     const uint32_t z2 = (0x4300u + zb) * 0x00010001u;
                     const uint32_t words[4] = {p.x, p.y, p.z, p.w};
@@ -481,7 +479,14 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
                     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(afull_bar(s));
+                    // The codes were consumed by the conversion above, so
+                    // their loads have returned; the stage's refill also
+                    // waits for this stage's MMA, which follows afull, so
+                    // releasing it here costs nothing.
+                    if (lane == 0) {
+                        mbar_arrive(empty_bar(s));
+                        mbar_arrive(afull_bar(s));
+                    }
                     ++kt;
                     s = s + 1 == stages ? 0 : s + 1;
                     r += (s == 0);
@@ -575,8 +580,6 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
                         smem + SmemLayout.pack + s * kPackBytes + row_local * kTileK + khalf * 32;
                     const uint4 p0 = *reinterpret_cast<const uint4 *>(src);
                     const uint4 p1 = *reinterpret_cast<const uint4 *>(src + 16);
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(empty_bar(s));   // code stage consumed
                     const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
                     uint32_t a[16];
 #pragma unroll
@@ -590,7 +593,10 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
                     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(afull_bar(s));
+                    if (lane == 0) {                  // codes consumed; A slot written
+                        mbar_arrive(empty_bar(s));
+                        mbar_arrive(afull_bar(s));
+                    }
                 }
             }
         }

@@ -29,8 +29,11 @@
 //     16-byte shared loads (int8 rows are 128 B, loaded with the 128-byte
 //     swizzle so that those loads are free of bank conflicts), its tokens'
 //     activations of the same k, and the four rows' scales and zeros,
-//     releases the stage, and dequantizes in registers to bf16 exactly as
-//     qz_dequantize forms each weight.  int4: a LOP3 builds bf16(128 + q) for
+//     dequantizes in registers to bf16 exactly as qz_dequantize forms each
+//     weight, and releases the stage once its MMAs have consumed every
+//     loaded register (a release right after the loads let a refill
+//     overwrite a stage whose loads had not yet returned, seen with fewer
+//     registers per thread).  int4: a LOP3 builds bf16(128 + q) for
 //     two nibbles, add.rn.bf16x2 of bf16(-(128 + Z)) leaves q - Z exactly,
 //     mul.rn.bf16x2 by the bf16 scale rounds S*(q - Z) once.  int8: the byte
 //     (XOR 0x80) is placed in the mantissa of 2^23, one fp32 subtraction
@@ -813,8 +816,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap code_map,
             if (!mbar_wait(full_bar(s), r & 1, p.wait_limit, abort_flag, p.err_word)) return;
             if constexpr (HALVES == 2) {
                 // two 128-wide halves: each its own codes, activations and
-                // group scale/zero; the stage is released once the second
-                // half is in registers
+                // group scale/zero; the stage is released after both halves'
+                // MMAs
                 const uint32_t stage = stage_addr(s);
                 const uint32_t ms = meta_addr(m) + 16u * (uint32_t)(w * kRowsPerWarp + g);
                 uint4 gs = make_uint4(0u, 0u, 0u, 0u), gz = gs;     // gathered words
@@ -881,19 +884,21 @@ gemv_kernel(const __grid_constant__ CUtensorMap code_map,
                             rp.z2[j] = (0xC300u + zv) * 0x00010001u;
                         }
                     }
-                    if (h == 1) {
-                        __syncwarp();
-                        if (lane == 0) {
-                            mbar_arrive(empty_bar(s));
-                            if (META == kMetaTma && (kb + 1 == KB || ((kb + 1) & span_mask) == 0 ||
-                                                     u + (kb - kb0) + 1 == u_end))
-                                mbar_arrive(meta_empty_bar(m));
-                        }
-                    }
                     if constexpr (kFp4)
                         compute_block_fp4<MB>(fa, fb, ac, rw, acc);
                     else
                         compute_block<4, MB>(rp, ac, rw, s8, acc);
+                }
+                // Both halves' registers have been consumed by their MMAs, so
+                // every shared-memory load of the stage (and of the meta
+                // slot, on its last unit) has returned: only now may the
+                // producer refill them.
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(empty_bar(s));
+                    if (META == kMetaTma && (kb + 1 == KB || ((kb + 1) & span_mask) == 0 ||
+                                             u + (kb - kb0) + 1 == u_end))
+                        mbar_arrive(meta_empty_bar(m));
                 }
             } else {
             const uint32_t stage = stage_addr(s);
@@ -961,26 +966,25 @@ gemv_kernel(const __grid_constant__ CUtensorMap code_map,
                     rp.z2[j] = (0xC300u + zv) * 0x00010001u;          // bf16(-(128 + Z)) twice
                 }
             }
-            __syncwarp();
-            if (lane == 0) {
-                // the stage's data is in registers (wide variants still read
-                // its activations below and release it after the compute)
-                if (!kWide) mbar_arrive(empty_bar(s));
-                // the meta slot's last unit: the next unit starts a new slot
-                if (META == kMetaTma && (kb + 1 == KB || ((kb + 1) & span_mask) == 0 ||
-                                         u + (kb - kb0) + 1 == u_end))
-                    mbar_arrive(meta_empty_bar(m));
-            }
             if constexpr (kFp4) {
                 compute_block_fp4<MB>(fa, fb, ac, rw, acc);
             } else if constexpr (kWide) {
                 if (BITS == 4 && META == kMetaNone) load_params_direct(rp, p, valid, rows, kb, t);
                 compute_block_wide<BITS, MB>(rp, stage + L::act_off, p.M, g, t, rw, s8, acc);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty_bar(s));
             } else {
                 if (BITS == 4 && META == kMetaNone) load_params_direct(rp, p, valid, rows, kb, t);
                 compute_block<BITS, MB>(rp, ac, rw, s8, acc);
+            }
+            // The MMAs have consumed every register loaded from the stage
+            // (and from the meta slot), so those loads have returned: the
+            // producer may refill them.  On the meta slot's last unit the
+            // next unit starts a new slot.
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(empty_bar(s));
+                if (META == kMetaTma && (kb + 1 == KB || ((kb + 1) & span_mask) == 0 ||
+                                         u + (kb - kb0) + 1 == u_end))
+                    mbar_arrive(meta_empty_bar(m));
             }
             }
             if (++s == S) {

@@ -867,6 +867,8 @@ PROFILE_CASES = {
     "gemm_prefill": ("gemm", 2048, 8192, 8192),
     "gemm8_prefill": ("gemm8", 2048, 8192, 8192),
     "gemm_m32": ("gemm", 32, 8192, 8192),
+    "gemm_m64": ("gemm", 64, 8192, 8192),
+    "gemm_m128": ("gemm", 128, 8192, 8192),
     "quant_int4": ("quant4", 0, 28672, 8192),
     "gemv_nvfp4_70b": ("gemv_nv", 1, 28672, 8192),
     "gemv_mxfp4_70b": ("gemv_mx", 1, 28672, 8192),

@@ -203,6 +203,30 @@ __device__ __forceinline__ void act_operand(const uint32_t (&x)[16], int i, int 
     b1 = dev::prmt(lo, hi, 0x7632);
 }
 
+// Activations of one 128-wide half h of a two-half unit for tokens g (and
+// g + 8), clamped to M - 1.  The unit's 256 k arrive as four boxes of 64 k
+// (128-byte token rows, 128-byte swizzle: 16-byte chunk c of token row r at
+// chunk c ^ (r % 8)), box b at act + b * MB KB; lane t reads k = 32t..32t+31
+// of the half: chunks 4(t % 2)..4(t % 2)+3 of box 2h + t / 2.  Tokens g of a
+// warp then spread over all banks (unswizzled 512-byte rows put the eight
+// tokens' chunks in the same banks).
+template <int MB>
+__device__ __forceinline__ void load_act_sw(Act<MB> &ac, uint32_t act, int M, int g, int t,
+                                            int h) {
+    const uint32_t box = act + (uint32_t)(2 * h + (t >> 1)) * (MB * 1024u);
+#pragma unroll
+    for (int mb = 0; mb < MB; ++mb) {
+        const int tok = min(8 * mb + g, M - 1);
+        const uint32_t row = box + (uint32_t)tok * 128u;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint4 v = lds128(row + 16u * (uint32_t)((((t & 1) * 4) + q) ^ (tok & 7)));
+            ac.x[mb][4 * q + 0] = v.x; ac.x[mb][4 * q + 1] = v.y;
+            ac.x[mb][4 * q + 2] = v.z; ac.x[mb][4 * q + 3] = v.w;
+        }
+    }
+}
+
 template <int BITS>
 struct RowWords {
     static constexpr int kWordsPerRow = BITS == 4 ? 4 : 8;
@@ -668,6 +692,18 @@ gemv_kernel(const __grid_constant__ CUtensorMap code_map,
         int64_t no_act = 0;                          // early units without activations
         const int task0 = (int)(u_begin / KB);
         const int kb_first = (int)(u_begin - (int64_t)task0 * KB);
+        // a unit's activations: one box of 128 k, or four swizzled boxes of
+        // 64 k for two-half units (load_act_sw)
+        auto load_unit_act = [&](int st, int kbx) {
+            if constexpr (HALVES == 2) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    tma_load_2d(stage_addr(st) + L::act_off + (uint32_t)i * (MB * 1024u), &act_map,
+                                kbx * kBlockK * HALVES + 64 * i, 0, full_bar(st));
+            } else {
+                tma_load_2d(stage_addr(st) + L::act_off, &act_map, kbx * kBlockK, 0, full_bar(st));
+            }
+        };
         auto finish_early = [&]() {
             if (!early_phase) return;
             early_phase = false;
@@ -675,8 +711,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap code_map,
             if (lane == 0) {
                 int kb2 = kb_first;
                 for (int64_t i = 0; i < no_act; ++i) {
-                    tma_load_2d(stage_addr((int)i) + L::act_off, &act_map,
-                                kb2 * kBlockK * HALVES, 0, full_bar((int)i));
+                    load_unit_act((int)i, kb2);
                     if (++kb2 == KB) kb2 = 0;
                 }
             }
@@ -721,9 +756,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap code_map,
                 mbar_arrive_expect_tx(full_bar(s), (uint32_t)L::code + act_bytes);
                 tma_load_2d(stage_addr(s), &code_map, kb * kRowBytes<BITS> * HALVES,
                             task * kTileRows, full_bar(s));
-                if (!early_phase)
-                    tma_load_2d(stage_addr(s) + L::act_off, &act_map, kb * kBlockK * HALVES, 0,
-                                full_bar(s));
+                if (!early_phase) load_unit_act(s, kb);
             }
             if (META == kMetaGather) {
                 const uint32_t dst = stage_addr(s) + L::sz_off + 16u * lane;
@@ -829,8 +862,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap code_map,
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     Act<MB> ac;
-                    load_act(ac, stage + L::act_off + (uint32_t)h * (kBlockK * 2), p.M, g, t,
-                             kBlockK * 2 * HALVES);
+                    load_act_sw(ac, stage + L::act_off, p.M, g, t, h);
                     RowWords<4> rw;
                     read_codes_half(rw, stage, w * kRowsPerWarp + g, g, t, h);
                     RowParams rp;
@@ -1134,8 +1166,8 @@ qz_status launch_gemv(const void *a, const void *codes, const void *scales, cons
                             (uint64_t)N, row_bytes, kRowBytes<BITS> * halves, kTileRows,
                             swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !make_map_2d_cached(&maps.act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a, (uint64_t)K,
-                            (uint64_t)M, (uint64_t)K * 2, kBlockK * halves, (uint32_t)M,
-                            CU_TENSOR_MAP_SWIZZLE_NONE))
+                            (uint64_t)M, (uint64_t)K * 2, halves == 2 ? 64 : kBlockK, (uint32_t)M,
+                            halves == 2 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE))
         return QZ_ERR_CUDA;
     maps.scale = maps.code;   // unused unless kMetaTma
     maps.zero = maps.code;
@@ -1214,8 +1246,8 @@ qz_status launch_fp4_gemv(const void *a, const void *codes, const void *scales,
                             (uint64_t)N, row_bytes, kRowBytes<4> * halves, kTileRows,
                             halves == 2 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !make_map_2d_cached(&maps.act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a, (uint64_t)K,
-                            (uint64_t)M, (uint64_t)K * 2, kBlockK * halves, (uint32_t)M,
-                            CU_TENSOR_MAP_SWIZZLE_NONE))
+                            (uint64_t)M, (uint64_t)K * 2, halves == 2 ? 64 : kBlockK, (uint32_t)M,
+                            halves == 2 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE))
         return QZ_ERR_CUDA;
     maps.scale = maps.code;
     maps.zero = maps.code;

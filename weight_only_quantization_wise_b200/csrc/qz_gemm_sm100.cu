@@ -173,14 +173,12 @@ __device__ __forceinline__ void epilogue_bar_sync() {
 }
 
 // int8 codes: bf16 pair (byte 2i, byte 2i+1) of word wx (the code word XOR
-// 0x80808080).  Bits 0x4B000000 | byte form the fp32 2^23 + q + 128; one
-// subtraction leaves q exactly, the pair packs to bf16 exactly (|q| <= 127)
-// and mul.rn.bf16x2 by (S, S) rounds S*q once, as qz_dequantize does.
-__device__ __forceinline__ uint32_t dequant_pair_i8_nat(uint32_t wx, int i, uint32_t s2) {
-    const float f0 = __uint_as_float(dev::prmt(wx, 0x4B000000u, (uint32_t)(2 * i) | 0x7540u));
-    const float f1 = __uint_as_float(dev::prmt(wx, 0x4B000000u, (uint32_t)(2 * i + 1) | 0x7540u));
-    return dev::bf16x2_mul(dev::pack_bf16x2(__fsub_rn(f0, 8388736.0f), __fsub_rn(f1, 8388736.0f)),
-                           s2);
+// 0x80808080).  One fma per value gives S*q exactly (dev::I8Scale) and the
+// pack rounds it to bf16 once, as qz_dequantize does.
+__device__ __forceinline__ uint32_t dequant_pair_i8_nat(uint32_t wx, int i, dev::I8Scale sc) {
+    const float f0 = __uint_as_float(dev::prmt(wx, 0x4B000000u, ((uint32_t)(2 * i) << 4) | 0x7504u));
+    const float f1 = __uint_as_float(dev::prmt(wx, 0x4B000000u, ((uint32_t)(2 * i + 1) << 4) | 0x7504u));
+    return dev::pack_bf16x2(__fmaf_rn(f0, sc.s, sc.c), __fmaf_rn(f1, sc.s, sc.c));
 }
 
 // Work item: a K range [kt0, kt1) of one output tile (128 weight rows x up
@@ -568,7 +566,7 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
                 }
             } else {
                 // one scale per weight row for the whole K
-                const uint32_t s2 = valid ? (uint32_t)__ldg(&scales[n]) * 0x00010001u : 0u;
+                const dev::I8Scale s2 = valid ? dev::i8_scale(__ldg(&scales[n])) : dev::I8Scale{0.0f, 0.0f};
                 for (int kt = wk.kt0; kt < wk.kt1;
                      ++kt, s = (s + 1 == stages ? 0 : s + 1), r += (s == 0)) {
                     if (!__all_sync(0xFFFFFFFFu,

@@ -197,6 +197,20 @@ __device__ __forceinline__ uint32_t f32_to_bf16_rne(float x) {
     return r;
 }
 
+// Exact int8 dequantization by one fused multiply-add per value.  For a code
+// byte b (q = (int8)b, u = b ^ 0x80 = q + 128) the fp32 with bits
+// 0x4B000000 | u << 8 is m = 2^23 + 256 u; with s = S / 256 (exact: a power
+// of two times a bf16) and c = -(2^23 + 2^15) s (9 x 8 significant bits,
+// exact), fma(m, s, c) = 256 (u - 128) s = q S exactly (at most 16
+// significant bits), so rounding it to bf16 gives bf16(S q) as one rounding.
+struct I8Scale {
+    float s, c;
+};
+__device__ __forceinline__ I8Scale i8_scale(uint32_t s_bits) {
+    const float s = __fmul_rn(__uint_as_float(s_bits << 16), 0.00390625f);   // S / 256
+    return {s, __fmul_rn(s, -8421376.0f)};                                   // -(2^23 + 2^15) s
+}
+
 // Two fp32 -> packed bf16x2 (lo in bits 0..15), round to nearest even.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;

@@ -876,6 +876,8 @@ PROFILE_CASES = {
     "gemm_w4a4_nv": ("w4a4_nv", 2048, 8192, 8192),
     "gemm_w4a4_mx": ("w4a4_mx", 2048, 8192, 8192),
     "quant_int8": ("quant8", 0, 28672, 8192),
+    "quant_nvfp4": ("quant_nv", 0, 28672, 8192),
+    "quant_mxfp4": ("quant_mx", 0, 28672, 8192),
     "dequant_int4": ("dequant", 0, 28672, 8192),
 }
 
@@ -919,6 +921,8 @@ def run_kernel_case(name, reps):
             qz.qz_quantize_pack(w, 4, False, GROUP)
         elif kind == "quant8":
             qz.qz_quantize_pack(w, 8, True, K)
+        elif kind in ("quant_nv", "quant_mx"):
+            qz.qz_fp4_quantize(w, qz.QZ_FP4_NV if kind == "quant_nv" else qz.QZ_FP4_MX)
         elif kind == "dequant":
             qz.qz_dequantize(c, s, z, N, K, 4, False, GROUP)
         elif kind in ("gemv_nv", "gemv_mx"):

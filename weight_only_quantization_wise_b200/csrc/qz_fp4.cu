@@ -142,6 +142,27 @@ __device__ __forceinline__ uint32_t e2m1_pack8(const float (&v)[8]) {
     return mag | (w & nonzero);
 }
 
+// Markstein's corrected quotients of two values at once with the packed
+// fp32x2 operations (each lane rounds exactly as the scalar fma and mul do):
+// q0 = RN(x r), e = fma(q0, -s, x) = x - q0 s (exact), u = RN(q0 + e r).
+// xlo, xhi: the two values' fp32 bits; r = RN(1 / s).
+__device__ __forceinline__ void quotient2(uint32_t xlo, uint32_t xhi, float r, float s,
+                                          float &ulo, float &uhi) {
+    uint32_t lo, hi;
+    asm("{\n\t.reg .b64 x, rr, ns, q, e, u;\n\t"
+        "mov.b64 x, {%2, %3};\n\t"
+        "mov.b64 rr, {%4, %4};\n\t"
+        "mov.b64 ns, {%5, %5};\n\t"
+        "mul.rn.f32x2 q, x, rr;\n\t"
+        "fma.rn.f32x2 e, q, ns, x;\n\t"
+        "fma.rn.f32x2 u, e, rr, q;\n\t"
+        "mov.b64 {%0, %1}, u;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(xlo), "r"(xhi), "r"(__float_as_uint(r)), "r"(__float_as_uint(-s)));
+    ulo = __uint_as_float(lo);
+    uhi = __uint_as_float(hi);
+}
+
 // One thread per block of BS values (BS / 8 chunks of 16 bytes).  MMA:
 // scales in the MMA scale layout (blocks_per_row scales per row) instead of
 // row-major.
@@ -168,12 +189,25 @@ fp4_quantize_kernel(const uint4 *__restrict__ w, int64_t blocks, uint8_t *__rest
     const float d6 = __fmul_rn(6.0f, s_t);
     const float r6 = __frcp_rn(d6);
     const bool d6_normal = d6 >= 0x1p-96f && d6 <= 0x1p96f;
-    for (int64_t b = thread_index(); b < blocks; b += grid_stride()) {
+    // The next block's loads are issued before this block is converted, so
+    // each thread keeps a load in flight while it computes.
+    const int64_t stride = grid_stride();
+    int64_t b = thread_index();
+    uint4 nxt[BS / 8];
+    if (b < blocks) {
+#pragma unroll
+        for (int c = 0; c < BS / 8; ++c) nxt[c] = __ldg(w + b * (BS / 8) + c);
+    }
+    for (; b < blocks; b += stride) {
         uint32_t x[BS / 2];
 #pragma unroll
         for (int c = 0; c < BS / 8; ++c) {
-            const uint4 v = __ldg(w + b * (BS / 8) + c);
-            x[4 * c + 0] = v.x; x[4 * c + 1] = v.y; x[4 * c + 2] = v.z; x[4 * c + 3] = v.w;
+            x[4 * c + 0] = nxt[c].x; x[4 * c + 1] = nxt[c].y;
+            x[4 * c + 2] = nxt[c].z; x[4 * c + 3] = nxt[c].w;
+        }
+        if (b + stride < blocks) {
+#pragma unroll
+            for (int c = 0; c < BS / 8; ++c) nxt[c] = __ldg(w + (b + stride) * (BS / 8) + c);
         }
         uint32_t m2 = bf16x2_absmax(x[0], x[1]);
 #pragma unroll
@@ -218,17 +252,22 @@ fp4_quantize_kernel(const uint4 *__restrict__ w, int64_t blocks, uint8_t *__rest
 #pragma unroll
         for (int g = 0; g < BS / 8; ++g) {
             float u[8];
+            if (KIND == 1 && !exact_div) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const uint32_t h = (i & 1) ? (x[(8 * g + i) / 2] >> 16) : (x[(8 * g + i) / 2] & 0xFFFFu);
-                const float xv = bf16_bits_to_f32(h);
-                if (KIND == 0) {
-                    u[i] = xv * r;
-                } else if (!exact_div) {
-                    const float q0 = __fmul_rn(xv, r);
-                    u[i] = __fmaf_rn(__fmaf_rn(-q0, scale, xv), r, q0);
-                } else {
-                    u[i] = scale > 0.0f ? __fdiv_rn(xv, scale) : 0.0f;
+                for (int i = 0; i < 8; i += 2) {      // values i, i + 1: one bf16 pair
+                    const uint32_t wv = x[(8 * g + i) / 2];
+                    quotient2(wv << 16, wv & 0xFFFF0000u, r, scale, u[i], u[i + 1]);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint32_t h =
+                        (i & 1) ? (x[(8 * g + i) / 2] >> 16) : (x[(8 * g + i) / 2] & 0xFFFFu);
+                    const float xv = bf16_bits_to_f32(h);
+                    if (KIND == 0)
+                        u[i] = xv * r;
+                    else
+                        u[i] = scale > 0.0f ? __fdiv_rn(xv, scale) : 0.0f;
                 }
             }
             packed[g] = e2m1_pack8(u);

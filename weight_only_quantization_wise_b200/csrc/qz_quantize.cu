@@ -133,10 +133,25 @@ __device__ __forceinline__ uint2 chunk_codes(const float (&x)[8], float s_f, flo
     if (!(r < __int_as_float(0x7F800000))) return chunk_codes_exact<BITS, SYM>(x, s_f, z);
     const float zc = __fadd_rn((float)z, kC);          // exact (small integers)
     uint32_t b[8];
+    // two values per instruction: fma.rn.f32x2 and add.rn.f32x2 round each
+    // lane exactly as the scalar fma and add do
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        b[i] = __float_as_uint(__fadd_rn(__fmaf_rn(x[i], r, zc), kRound));
-        if (!SYM && CLAMP) b[i] = min(b[i], kTop);
+    for (int i = 0; i < 8; i += 2) {
+        asm("{\n\t.reg .b64 xx, rr, zz, kk, yy, uu;\n\t"
+            "mov.b64 xx, {%2, %3};\n\t"
+            "mov.b64 rr, {%4, %4};\n\t"
+            "mov.b64 zz, {%5, %5};\n\t"
+            "mov.b64 kk, {%6, %6};\n\t"
+            "fma.rn.f32x2 yy, xx, rr, zz;\n\t"
+            "add.rn.f32x2 uu, yy, kk;\n\t"
+            "mov.b64 {%0, %1}, uu;\n\t}"
+            : "=r"(b[i]), "=r"(b[i + 1])
+            : "r"(__float_as_uint(x[i])), "r"(__float_as_uint(x[i + 1])), "r"(__float_as_uint(r)),
+              "r"(__float_as_uint(zc)), "r"(__float_as_uint(kRound)));
+    }
+    if (!SYM && CLAMP) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) b[i] = min(b[i], kTop);
     }
     if (BITS == 4) {
         uint32_t p[4];

@@ -176,9 +176,8 @@ __device__ __forceinline__ void epilogue_bar_sync() {
 // 0x80808080).  One fma per value gives S*q exactly (dev::I8Scale) and the
 // pack rounds it to bf16 once, as qz_dequantize does.
 __device__ __forceinline__ uint32_t dequant_pair_i8_nat(uint32_t wx, int i, dev::I8Scale sc) {
-    const float f0 = __uint_as_float(dev::prmt(wx, 0x4B000000u, ((uint32_t)(2 * i) << 4) | 0x7504u));
-    const float f1 = __uint_as_float(dev::prmt(wx, 0x4B000000u, ((uint32_t)(2 * i + 1) << 4) | 0x7504u));
-    return dev::pack_bf16x2(__fmaf_rn(f0, sc.s, sc.c), __fmaf_rn(f1, sc.s, sc.c));
+    return dev::i8_fma2_bf16x2(dev::prmt(wx, 0x4B000000u, ((uint32_t)(2 * i) << 4) | 0x7504u),
+                               dev::prmt(wx, 0x4B000000u, ((uint32_t)(2 * i + 1) << 4) | 0x7504u), sc);
 }
 
 // Work item: a K range [kt0, kt1) of one output tile (128 weight rows x up

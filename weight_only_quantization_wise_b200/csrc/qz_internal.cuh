@@ -211,6 +211,23 @@ __device__ __forceinline__ I8Scale i8_scale(uint32_t s_bits) {
     return {s, __fmul_rn(s, -8421376.0f)};                                   // -(2^23 + 2^15) s
 }
 
+// fma(m, s, c) for two values at once (fma.rn.f32x2), packed to bf16x2 with
+// round to nearest even: the low lane from mlo, the high lane from mhi.
+__device__ __forceinline__ uint32_t i8_fma2_bf16x2(uint32_t mlo, uint32_t mhi, I8Scale sc) {
+    uint32_t lo, hi;
+    asm("{\n\t.reg .b64 mm, ss, cc, uu;\n\t"
+        "mov.b64 mm, {%2, %3};\n\t"
+        "mov.b64 ss, {%4, %4};\n\t"
+        "mov.b64 cc, {%5, %5};\n\t"
+        "fma.rn.f32x2 uu, mm, ss, cc;\n\t"
+        "mov.b64 {%0, %1}, uu;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(mlo), "r"(mhi), "r"(__float_as_uint(sc.s)), "r"(__float_as_uint(sc.c)));
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(__uint_as_float(hi)), "f"(__uint_as_float(lo)));
+    return r;
+}
+
 // Two fp32 -> packed bf16x2 (lo in bits 0..15), round to nearest even.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;

@@ -610,8 +610,10 @@ __device__ __forceinline__ void gemv_flush(float (&acc)[2][MB][4], const GemvArg
 // The kernel.  META: how int4 scales and zeros arrive (kMetaNone: int8's
 // per-row scales, or int4 groups loaded directly by the consumers).  HALVES:
 // 128-wide K blocks per unit (2: int4 units of 128 rows x 256 k, one
-// 128-byte row of codes per weight row, consumed as two halves).
-template <int BITS, int MB, int META, int FMT, int HALVES = 1>
+// 128-byte row of codes per weight row, consumed as two halves).  ACTSW
+// (two-half units): activations as four swizzled 64-k boxes (load_act_sw),
+// else one box of 256 k (one token: its lanes of equal t read the same words).
+template <int BITS, int MB, int META, int FMT, int HALVES = 1, bool ACTSW = true>
 __global__ void __launch_bounds__(kThreads, (kCtasPerSm<MB, HALVES>))
 gemv_kernel(const __grid_constant__ CUtensorMap code_map,
             const __grid_constant__ CUtensorMap act_map,
@@ -690,16 +692,17 @@ gemv_kernel(const __grid_constant__ CUtensorMap code_map,
         int64_t no_act = 0;                          // early units without activations
         const int task0 = (int)(u_begin / KB);
         const int kb_first = (int)(u_begin - (int64_t)task0 * KB);
-        // a unit's activations: one box of 128 k, or four swizzled boxes of
-        // 64 k for two-half units (load_act_sw)
+        // a unit's activations: one box of 128 k (256 k: two-half units
+        // without ACTSW), or four swizzled boxes of 64 k (load_act_sw)
         auto load_unit_act = [&](int st, int kbx) {
-            if constexpr (HALVES == 2) {
+            if constexpr (HALVES == 2 && ACTSW) {
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
                     tma_load_2d(stage_addr(st) + L::act_off + (uint32_t)i * (MB * 1024u), &act_map,
                                 kbx * kBlockK * HALVES + 64 * i, 0, full_bar(st));
             } else {
-                tma_load_2d(stage_addr(st) + L::act_off, &act_map, kbx * kBlockK, 0, full_bar(st));
+                tma_load_2d(stage_addr(st) + L::act_off, &act_map, kbx * kBlockK * HALVES, 0,
+                            full_bar(st));
             }
         };
         auto finish_early = [&]() {
@@ -860,7 +863,11 @@ gemv_kernel(const __grid_constant__ CUtensorMap code_map,
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     Act<MB> ac;
-                    load_act_sw(ac, stage + L::act_off, p.M, g, t, h);
+                    if constexpr (ACTSW)
+                        load_act_sw(ac, stage + L::act_off, p.M, g, t, h);
+                    else
+                        load_act(ac, stage + L::act_off + (uint32_t)h * (kBlockK * 2), p.M, g, t,
+                                 kBlockK * 2 * HALVES);
                     RowWords<4> rw;
                     read_codes_half(rw, stage, w * kRowsPerWarp + g, g, t, h);
                     RowParams rp;
@@ -1049,7 +1056,7 @@ struct Maps {
     CUtensorMap code, act, scale, zero;
 };
 
-template <int BITS, int MB, int META, int FMT, int HALVES = 1>
+template <int BITS, int MB, int META, int FMT, int HALVES = 1, bool ACTSW = true>
 qz_status launch_variant(const Maps &maps, const GemvArgs &args, dim3 grid, int overlap,
                          cudaStream_t st) {
     constexpr int smem = Layout<BITS, MB, META, FMT, HALVES>::bytes;
@@ -1060,13 +1067,13 @@ qz_status launch_variant(const Maps &maps, const GemvArgs &args, dim3 grid, int 
         return QZ_ERR_CUDA;
     }
     if (attr_once.run(dev, [] {
-            cudaError_t e = cudaFuncSetAttribute(gemv_kernel<BITS, MB, META, FMT, HALVES>,
+            cudaError_t e = cudaFuncSetAttribute(gemv_kernel<BITS, MB, META, FMT, HALVES, ACTSW>,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  smem);
             // three rings per SM need (nearly) all of the unified memory as
             // shared memory
             if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(gemv_kernel<BITS, MB, META, FMT, HALVES>,
+                e = cudaFuncSetAttribute(gemv_kernel<BITS, MB, META, FMT, HALVES, ACTSW>,
                                          cudaFuncAttributePreferredSharedMemoryCarveout, 100);
             return e;
         }) != cudaSuccess)
@@ -1081,7 +1088,7 @@ qz_status launch_variant(const Maps &maps, const GemvArgs &args, dim3 grid, int 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = overlap > 0 ? 1 : 0;
-    cudaLaunchKernelEx(&cfg, gemv_kernel<BITS, MB, META, FMT, HALVES>, maps.code, maps.act,
+    cudaLaunchKernelEx(&cfg, gemv_kernel<BITS, MB, META, FMT, HALVES, ACTSW>, maps.code, maps.act,
                        maps.scale, maps.zero, args);
     return launch_status();
 }
@@ -1157,6 +1164,7 @@ qz_status launch_gemv(const void *a, const void *codes, const void *scales, cons
     if (args.err_word == nullptr) return QZ_ERR_CUDA;
 
     Maps maps;
+    const bool act_sw = halves == 2 && M > 1;      // see gemv_kernel's ACTSW
     const uint64_t row_bytes = (uint64_t)K * BITS / 8;
     // 128-byte code rows (int8, and int4 two-half units) take the 128-byte swizzle
     const bool swizzle = BITS == 8 || halves == 2;
@@ -1164,8 +1172,9 @@ qz_status launch_gemv(const void *a, const void *codes, const void *scales, cons
                             (uint64_t)N, row_bytes, kRowBytes<BITS> * halves, kTileRows,
                             swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !make_map_2d_cached(&maps.act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a, (uint64_t)K,
-                            (uint64_t)M, (uint64_t)K * 2, halves == 2 ? 64 : kBlockK, (uint32_t)M,
-                            halves == 2 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE))
+                            (uint64_t)M, (uint64_t)K * 2, act_sw ? 64 : kBlockK * halves,
+                            (uint32_t)M,
+                            act_sw ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE))
         return QZ_ERR_CUDA;
     maps.scale = maps.code;   // unused unless kMetaTma
     maps.zero = maps.code;
@@ -1186,7 +1195,9 @@ qz_status launch_gemv(const void *a, const void *codes, const void *scales, cons
                                     CU_TENSOR_MAP_SWIZZLE_NONE))
                 return QZ_ERR_CUDA;
             if (halves == 2)
-                return M <= 8 ? launch_variant<4, 1, kMetaTma, kFmtInt, 2>(maps, args, grid,
+                return M == 1   ? launch_variant<4, 1, kMetaTma, kFmtInt, 2, false>(maps, args, grid,
+                                                                                   overlap, st)
+                       : M <= 8 ? launch_variant<4, 1, kMetaTma, kFmtInt, 2>(maps, args, grid,
                                                                           overlap, st)
                               : launch_variant<4, 2, kMetaTma, kFmtInt, 2>(maps, args, grid,
                                                                           overlap, st);
@@ -1196,8 +1207,10 @@ qz_status launch_gemv(const void *a, const void *codes, const void *scales, cons
         // and zero.
         if (meta == kMetaGather) {
             if (halves == 2)
-                return M <= 8 ? launch_variant<4, 1, kMetaGather, kFmtInt, 2>(maps, args, grid,
-                                                                             overlap, st)
+                return M == 1   ? launch_variant<4, 1, kMetaGather, kFmtInt, 2, false>(maps, args, grid,
+                                                                                   overlap, st)
+                       : M <= 8 ? launch_variant<4, 1, kMetaGather, kFmtInt, 2>(maps, args, grid,
+                                                                          overlap, st)
                               : launch_variant<4, 2, kMetaGather, kFmtInt, 2>(maps, args, grid,
                                                                              overlap, st);
             return launch_mb<4, kMetaGather>(maps, args, grid, overlap, st);
@@ -1239,13 +1252,15 @@ qz_status launch_fp4_gemv(const void *a, const void *codes, const void *scales,
     args.err_word = device_error_word();
     if (args.err_word == nullptr) return QZ_ERR_CUDA;
     Maps maps;
+    const bool act_sw = halves == 2 && M > 1;      // see gemv_kernel's ACTSW
     const uint64_t row_bytes = (uint64_t)K / 2;
     if (!make_map_2d_cached(&maps.code, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, row_bytes,
                             (uint64_t)N, row_bytes, kRowBytes<4> * halves, kTileRows,
                             halves == 2 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !make_map_2d_cached(&maps.act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a, (uint64_t)K,
-                            (uint64_t)M, (uint64_t)K * 2, halves == 2 ? 64 : kBlockK, (uint32_t)M,
-                            halves == 2 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE))
+                            (uint64_t)M, (uint64_t)K * 2, act_sw ? 64 : kBlockK * halves,
+                            (uint32_t)M,
+                            act_sw ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE))
         return QZ_ERR_CUDA;
     maps.scale = maps.code;
     maps.zero = maps.code;
@@ -1260,9 +1275,11 @@ qz_status launch_fp4_gemv(const void *a, const void *codes, const void *scales,
     if (halves == 2) {
         if (!tma_meta || K % (2 * kBlockK) != 0) return QZ_ERR_UNSUPPORTED;
         if (kind == 0)
-            return M <= 8 ? launch_variant<4, 1, kMetaTma, kFmtMx, 2>(maps, args, grid, overlap, st)
+            return M == 1   ? launch_variant<4, 1, kMetaTma, kFmtMx, 2, false>(maps, args, grid, overlap, st)
+                   : M <= 8 ? launch_variant<4, 1, kMetaTma, kFmtMx, 2>(maps, args, grid, overlap, st)
                           : launch_variant<4, 2, kMetaTma, kFmtMx, 2>(maps, args, grid, overlap, st);
-        return M <= 8 ? launch_variant<4, 1, kMetaTma, kFmtNv, 2>(maps, args, grid, overlap, st)
+        return M == 1   ? launch_variant<4, 1, kMetaTma, kFmtNv, 2, false>(maps, args, grid, overlap, st)
+                   : M <= 8 ? launch_variant<4, 1, kMetaTma, kFmtNv, 2>(maps, args, grid, overlap, st)
                       : launch_variant<4, 2, kMetaTma, kFmtNv, 2>(maps, args, grid, overlap, st);
     }
     if (kind == 0)

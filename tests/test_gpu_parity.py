@@ -623,6 +623,30 @@ def test_w8a16_gemm_onehot_is_exact(dev):
     assert np.array_equal(u16(y2), w_hat[:, kx].T)
 
 
+@pytest.mark.parametrize("M", [1, 8, 256])
+def test_w8a16_onehot_exact_across_the_scale_range(dev, M):
+    """int8 scales from the smallest to the largest a finite bf16 weight can
+    give (S = absmax / 127 up to about 2.7e36, down to subnormal bf16): the
+    dequantized weight S*q is formed exactly and rounded once for every row,
+    with no overflow of an intermediate, in the decode GEMV (M <= 32) and the
+    tcgen05 GEMM."""
+    N, K = 256, 512
+    w = synthetic.weights(N, K, sigma=0.5, seed=91).float().numpy().astype(np.float64)
+    # row magnitudes spread over the whole bf16 exponent range
+    exps = np.linspace(-128, 126, N)
+    w = np.clip(w * np.exp2(exps)[:, None], -3.3e38, 3.3e38)
+    w = u16(torch.tensor(w, dtype=torch.float32).to(torch.bfloat16))
+    c, s, _ = oracle.quantize_pack(w, 8, True, K)
+    w_hat = oracle.dequantize(c, s, None, N, K, 8, True, K)
+    ks = (np.arange(M) * 37) % K
+    a = np.zeros((M, K), np.uint16)
+    a[np.arange(M), ks] = 0x3F80
+    fn = qz.qz_w8a16_gemv if M <= 32 else qz.qz_w8a16_gemm
+    y = fn(to_dev_bf16(a, dev), to_dev_u8(c, dev), to_dev_bf16(s, dev), N, K)
+    torch.cuda.synchronize()
+    assert np.array_equal(u16(y), w_hat[:, ks].T)
+
+
 def test_w8a16_gemm_small_m_matches_the_gemv(dev):
     """M <= 32 takes the decode kernel: the same bits as qz_w8a16_gemv."""
     N, K = 1000, 1024

@@ -173,11 +173,13 @@ __device__ __forceinline__ void epilogue_bar_sync() {
 }
 
 // int8 codes: bf16 pair (byte 2i, byte 2i+1) of word wx (the code word XOR
-// 0x80808080).  One fma per value gives S*q exactly (dev::I8Scale) and the
-// pack rounds it to bf16 once, as qz_dequantize does.
-__device__ __forceinline__ uint32_t dequant_pair_i8_nat(uint32_t wx, int i, dev::I8Scale sc) {
-    return dev::i8_fma2_bf16x2(dev::prmt(wx, 0x4B000000u, ((uint32_t)(2 * i) << 4) | 0x7504u),
-                               dev::prmt(wx, 0x4B000000u, ((uint32_t)(2 * i + 1) << 4) | 0x7504u), sc);
+// 0x80808080): one packed subtraction gives the pair of q exactly
+// (dev::i8_codes_bf16x2) and mul.rn.bf16x2 by (S, S) rounds S*q once, as
+// qz_dequantize does.
+__device__ __forceinline__ uint32_t dequant_pair_i8_nat(uint32_t wx, int i, uint32_t s2) {
+    return dev::bf16x2_mul(dev::i8_codes_bf16x2(dev::prmt(wx, 0x4B000000u, (uint32_t)(2 * i) | 0x7540u),
+                                                dev::prmt(wx, 0x4B000000u, (uint32_t)(2 * i + 1) | 0x7540u)),
+                           s2);
 }
 
 // Work item: a K range [kt0, kt1) of one output tile (128 weight rows x up
@@ -565,7 +567,7 @@ wa16_gemm_tcgen05(const __grid_constant__ CUtensorMap act_map,
                 }
             } else {
                 // one scale per weight row for the whole K
-                const dev::I8Scale s2 = valid ? dev::i8_scale(__ldg(&scales[n])) : dev::I8Scale{0.0f, 0.0f};
+                const uint32_t s2 = valid ? (uint32_t)__ldg(&scales[n]) * 0x00010001u : 0u;
                 for (int kt = wk.kt0; kt < wk.kt1;
                      ++kt, s = (s + 1 == stages ? 0 : s + 1), r += (s == 0)) {
                     if (!__all_sync(0xFFFFFFFFu,

@@ -36,8 +36,9 @@
 //     registers per thread).  int4: a LOP3 builds bf16(128 + q) for
 //     two nibbles, add.rn.bf16x2 of bf16(-(128 + Z)) leaves q - Z exactly,
 //     mul.rn.bf16x2 by the bf16 scale rounds S*(q - Z) once.  int8: the byte
-//     (XOR 0x80) goes to bits 8..15 of the fp32 2^23, one packed fp32 fma
-//     per pair gives S*q exactly and the bf16 pack rounds it once.
+//     (XOR 0x80) is placed in the mantissa of 2^23, one packed fp32
+//     subtraction gives a pair of q exactly, the pair is packed to bf16
+//     exactly and mul.rn.bf16x2 rounds S*q once.
 //   * A byte of codes yields the pairs (q_j, q_{j+4}), so the K axis is
 //     permuted consistently for both MMA operands: the pairs are the A
 //     operand (16 rows x 16 k) of mma.sync m16n8k16 with fp32 accumulation
@@ -143,16 +144,14 @@ __device__ __forceinline__ uint32_t dequant_pair_u4(uint32_t word, int j, uint32
 }
 
 // bf16 pair (code c_j, code c_{j+4}) of 8 consecutive int8 codes held in
-// words lo (c0..c3) and hi (c4..c7), already XORed with 0x80808080: each
-// byte goes to bits 8..15 under 0x4B, one packed fma gives S*q exactly for
-// both (dev::I8Scale, dev::i8_fma2_bf16x2) and the bf16 pack rounds each
-// once, as qz_dequantize does.  (A subtraction, a pack of q and a bf16
-// multiply took 6 instructions per pair; scalar fmas, 5, measured 3.5%
-// slower; the packed fma, 4, measured 1-6% faster.)
-__device__ __forceinline__ uint32_t dequant_pair_i8(uint32_t lo, uint32_t hi, int j,
-                                                    dev::I8Scale sc) {
-    const uint32_t sel = ((uint32_t)j << 4) | 0x7504u;     // bytes 0x4B, 0, byte j, 0
-    return dev::i8_fma2_bf16x2(dev::prmt(lo, 0x4B000000u, sel), dev::prmt(hi, 0x4B000000u, sel), sc);
+// words lo (c0..c3) and hi (c4..c7), already XORed with 0x80808080: both
+// bytes go into the mantissa of 2^23, one packed subtraction gives the pair
+// of q exactly (dev::i8_codes_bf16x2), and mul.rn.bf16x2 by (S, S) rounds
+// S*q once, as qz_dequantize does.
+__device__ __forceinline__ uint32_t dequant_pair_i8(uint32_t lo, uint32_t hi, int j, uint32_t s2) {
+    const uint32_t sel = (uint32_t)j | 0x7540u;            // bytes: byte j, 0, 0, 0x4B
+    return dev::bf16x2_mul(
+        dev::i8_codes_bf16x2(dev::prmt(lo, 0x4B000000u, sel), dev::prmt(hi, 0x4B000000u, sel)), s2);
 }
 
 // FP4: the four natural-order bf16 pairs (q0,q1), (q2,q3), (q4,q5), (q6,q7)
@@ -355,7 +354,7 @@ __device__ __forceinline__ void load_act(Act<MB> &ac, uint32_t act, int M, int g
 
 template <int BITS, int MB>
 __device__ __forceinline__ void compute_block(const RowParams &rp, const Act<MB> &ac,
-                                              const RowWords<BITS> &rw, const dev::I8Scale (&s8)[4],
+                                              const RowWords<BITS> &rw, const uint32_t (&s8)[4],
                                               float (&acc)[kChains<MB>][2][MB][4]) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -404,7 +403,7 @@ __device__ __forceinline__ void compute_block(const RowParams &rp, const Act<MB>
 template <int BITS, int MB>
 __device__ __forceinline__ void compute_block_wide(const RowParams &rp, uint32_t act, int M,
                                                    int g, int t, const RowWords<BITS> &rw,
-                                                   const dev::I8Scale (&s8)[4],
+                                                   const uint32_t (&s8)[4],
                                                    float (&acc)[1][2][MB][4]) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -817,13 +816,13 @@ gemv_kernel(const __grid_constant__ CUtensorMap code_map,
         const int n0 = task * kTileRows + w * kRowsPerWarp;
         int rows[4];
         bool valid[4];
-        dev::I8Scale s8[4];
+        uint32_t s8[4];                              // int8: (S, S) of rows g + 8j
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             rows[j] = n0 + g + 8 * j;
             valid[j] = rows[j] < p.N;
-            s8[j] = (BITS == 8 && valid[j]) ? dev::i8_scale(__ldg(&p.scales[rows[j]]))
-                                            : dev::I8Scale{0.0f, 0.0f};
+            s8[j] = (BITS == 8 && valid[j]) ? (uint32_t)__ldg(&p.scales[rows[j]]) * 0x00010001u
+                                            : 0u;
         }
         float acc[kChains<MB>][2][MB][4];
 #pragma unroll

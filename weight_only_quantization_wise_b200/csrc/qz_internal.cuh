@@ -197,32 +197,21 @@ __device__ __forceinline__ uint32_t f32_to_bf16_rne(float x) {
     return r;
 }
 
-// Exact int8 dequantization by one fused multiply-add per value.  For a code
-// byte b (q = (int8)b, u = b ^ 0x80 = q + 128) the fp32 with bits
-// 0x4B000000 | u << 8 is m = 2^23 + 256 u; with s = S / 256 (exact: a power
-// of two times a bf16) and c = -(2^23 + 2^15) s (9 x 8 significant bits,
-// exact), fma(m, s, c) = 256 (u - 128) s = q S exactly (at most 16
-// significant bits), so rounding it to bf16 gives bf16(S q) as one rounding.
-struct I8Scale {
-    float s, c;
-};
-__device__ __forceinline__ I8Scale i8_scale(uint32_t s_bits) {
-    const float s = __fmul_rn(__uint_as_float(s_bits << 16), 0.00390625f);   // S / 256
-    return {s, __fmul_rn(s, -8421376.0f)};                                   // -(2^23 + 2^15) s
-}
-
-// fma(m, s, c) for two values at once (fma.rn.f32x2), packed to bf16x2 with
-// round to nearest even: the low lane from mlo, the high lane from mhi.
-__device__ __forceinline__ uint32_t i8_fma2_bf16x2(uint32_t mlo, uint32_t mhi, I8Scale sc) {
+// Exact int8 code pair to bf16x2 (q_lo, q_hi): the code bytes u = b ^ 0x80
+// sit in bits 0..7 of the fp32 2^23 (mlo, mhi: 2^23 + q + 128), and one
+// sub.rn.f32x2 of 2^23 + 128 leaves both q exactly; the pack is exact
+// (|q| <= 128).  A bf16 multiply by (S, S) then rounds S*q once.  (One fma
+// per value forming S*q directly would overflow its intermediate 2^15 S for
+// scales above 2^113, which finite bf16 weights can reach.)
+__device__ __forceinline__ uint32_t i8_codes_bf16x2(uint32_t mlo, uint32_t mhi) {
     uint32_t lo, hi;
-    asm("{\n\t.reg .b64 mm, ss, cc, uu;\n\t"
+    asm("{\n\t.reg .b64 mm, kk, qq;\n\t"
         "mov.b64 mm, {%2, %3};\n\t"
-        "mov.b64 ss, {%4, %4};\n\t"
-        "mov.b64 cc, {%5, %5};\n\t"
-        "fma.rn.f32x2 uu, mm, ss, cc;\n\t"
-        "mov.b64 {%0, %1}, uu;\n\t}"
+        "mov.b64 kk, {%4, %4};\n\t"
+        "sub.rn.f32x2 qq, mm, kk;\n\t"
+        "mov.b64 {%0, %1}, qq;\n\t}"
         : "=r"(lo), "=r"(hi)
-        : "r"(mlo), "r"(mhi), "r"(__float_as_uint(sc.s)), "r"(__float_as_uint(sc.c)));
+        : "r"(mlo), "r"(mhi), "r"(0x4B000080u));       // 2^23 + 128
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(__uint_as_float(hi)), "f"(__uint_as_float(lo)));
     return r;
